@@ -1,0 +1,193 @@
+"""Seeded synthetic activations shaped like the pages' Llama-class workloads.
+
+This module holds input recipes only -- no rotation or quantization
+arithmetic -- so both the CUDA path and the float64 oracle can consume the
+same bit patterns.  Every tensor is generated in chunks of ``CHUNK_ROWS``
+rows from a counter-keyed numpy ``PCG64`` stream, so any row range can be
+regenerated on its own (row sampling for the oracle, per-rank shards) and
+gives the same bits as the whole tensor.
+
+Recipes (seed 0 everywhere; an "outlier set" is the first k entries of a
+permutation drawn from a ``seed + 1`` stream):
+
+* ``c1``  64 x 1024 fp32 ~ N(0, 1); full 1024-point rotation; int4, group 128.
+* ``c2``  R1 residual stream: 4096 tokens x 4096 bf16 ~ N(0, 1), 41 outlier
+  channels (1 %) scaled x50; full 4096-point rotation; int4, group 128.
+* ``c3``  R4 down_proj input: 8192 x 14336 bf16 = SiLU(a) * b with a, b ~
+  N(0, 1), 72 outlier channels (0.5 %) scaled x30; block 128; int8 per token.
+* ``c4q`` / ``c4k``  R3 Q and K after RoPE: [16, 32, 4096, 128] bf16 ~ N(0, 1),
+  two outlier dims per head (per-head seeded choice) scaled x20 before RoPE
+  (rotate-half pairing (i, i + 64), theta_i = 10000^(-i/64), position = s);
+  per-head 128-point rotation; Q -> bf16, K -> int4 group 128.
+* ``c5``  65536 x 8192 bf16 Student-t(3); full 8192-point rotation; MXFP4.
+
+Values are drawn in float64, rounded to float32 (nearest even) and, for
+bf16 tensors, to bfloat16 (nearest even).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+CHUNK_ROWS = 1024
+SEED = 0
+
+
+@dataclass(frozen=True)
+class Workload:
+    key: str
+    name: str
+    rows: int
+    n: int
+    block: int          # applied rotation block; == n for a full rotation
+    x_dtype: str        # "f32" | "bf16"
+    fmt: str | None     # "int4" | "int8" | "mxfp4" | None (rotation only)
+    group: int          # quant group (0 = per token for int8)
+    out_dtype: str | None = None   # rotation-only output dtype
+
+    @property
+    def in_bytes(self) -> int:
+        return self.rows * self.n * (4 if self.x_dtype == "f32" else 2)
+
+    @property
+    def out_bytes(self) -> int:
+        r, n = self.rows, self.n
+        if self.fmt is None:
+            return r * n * (4 if self.out_dtype == "f32" else 2)
+        if self.fmt == "int4":
+            return r * n // 2 + r * (n // self.group) * 2
+        if self.fmt == "int8":
+            return r * n + r * 4
+        if self.fmt == "mxfp4":
+            return r * n // 2 + r * (n // 32)
+        raise ValueError(self.fmt)
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """Input read once plus outputs written once."""
+        return self.in_bytes + self.out_bytes
+
+
+WORKLOADS = {
+    "c1": Workload("c1", "64x1024 fp32, full 1024-point Hadamard, int4 sym g128 fp16 scales",
+                   64, 1024, 1024, "f32", "int4", 128),
+    "c2": Workload("c2", "R1 4096 tokens x hidden 4096 bf16, full 4096-point Hadamard, int4 sym g128 fp16 scales",
+                   4096, 4096, 4096, "bf16", "int4", 128),
+    "c3": Workload("c3", "R4 8192 tokens x intermediate 14336 bf16, block 128 (112 blocks), int8 per token",
+                   8192, 14336, 128, "bf16", "int8", 0),
+    "c4q": Workload("c4q", "R3 Q [16,32,4096,128] bf16 after RoPE, per-head 128-point Hadamard -> bf16",
+                    16 * 32 * 4096, 128, 128, "bf16", None, 0, "bf16"),
+    "c4k": Workload("c4k", "R3 K [16,32,4096,128] bf16 after RoPE, per-head 128-point Hadamard, int4 g128",
+                    16 * 32 * 4096, 128, 128, "bf16", "int4", 128),
+    "c5": Workload("c5", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point Hadamard, MXFP4",
+                   65536, 8192, 8192, "bf16", "mxfp4", 32),
+}
+
+_STREAM = {"c1": 1, "c2": 2, "c3": 3, "c4q": 4, "c4k": 5, "c5": 6}
+
+
+def _rng(seed: int, stream: int, chunk: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(entropy=seed, spawn_key=(stream, chunk))))
+
+
+def _outlier_set(seed: int, stream: int, n: int, k: int) -> np.ndarray:
+    return _rng(seed + 1, stream, 0).permutation(n)[:k]
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns, round half to even (finite inputs)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def bits_to_float64(x: np.ndarray, x_dtype: str) -> np.ndarray:
+    """Exact float64 value of stored fp32 values or bf16 bit patterns."""
+    if x_dtype == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    if x_dtype == "bf16":
+        return (np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    raise ValueError(x_dtype)
+
+
+def _chunk_values(key: str, chunk: int, seed: int) -> np.ndarray:
+    w = WORKLOADS[key]
+    r0 = chunk * CHUNK_ROWS
+    nr = min(CHUNK_ROWS, w.rows - r0)
+    g = _rng(seed, _STREAM[key], chunk)
+    if key == "c1":
+        return g.standard_normal((nr, w.n))
+    if key == "c2":
+        v = g.standard_normal((nr, w.n))
+        v[:, _outlier_set(seed, _STREAM[key], w.n, round(0.01 * w.n))] *= 50.0
+        return v
+    if key == "c3":
+        a = g.standard_normal((nr, w.n))
+        b = g.standard_normal((nr, w.n))
+        v = a / (1.0 + np.exp(-a)) * b
+        v[:, _outlier_set(seed, _STREAM[key], w.n, round(0.005 * w.n))] *= 30.0
+        return v
+    if key in ("c4q", "c4k"):
+        seq, heads, d = 4096, 32, 128
+        rows = np.arange(r0, r0 + nr)
+        head = (rows // seq) % heads
+        pos = (rows % seq).astype(np.float64)
+        v = g.standard_normal((nr, d))
+        for h in np.unique(head):
+            dims = _rng(seed + 1, _STREAM[key], 1000 + int(h)).choice(d, 2, replace=False)
+            sel = head == h
+            v[np.ix_(sel, dims)] *= 20.0
+        half = d // 2
+        theta = 10000.0 ** (-np.arange(half) / half)
+        ang = pos[:, None] * theta[None, :]
+        c, s = np.cos(ang), np.sin(ang)
+        x1, x2 = v[:, :half], v[:, half:]
+        return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)
+    if key == "c5":
+        return g.standard_t(3, (nr, w.n))
+    raise KeyError(key)
+
+
+def generate(key: str, rows: slice | None = None, seed: int = SEED) -> np.ndarray:
+    """Stored input for rows ``rows`` of workload ``key``.
+
+    Returns float32 values for fp32 workloads and uint16 bf16 bit patterns for
+    bf16 workloads, shape (len(rows), n), row-major.
+    """
+    w = WORKLOADS[key]
+    r = range(w.rows)[rows if rows is not None else slice(None)]
+    if r.step != 1:
+        raise ValueError("row ranges must be contiguous")
+    out = np.empty((len(r), w.n), dtype=np.float32 if w.x_dtype == "f32" else np.uint16)
+    if len(r) == 0:
+        return out
+    c0, c1 = r.start // CHUNK_ROWS, (r.stop - 1) // CHUNK_ROWS
+    for c in range(c0, c1 + 1):
+        vals = _chunk_values(key, c, seed).astype(np.float32)
+        lo = max(r.start, c * CHUNK_ROWS)
+        hi = min(r.stop, c * CHUNK_ROWS + vals.shape[0])
+        part = vals[lo - c * CHUNK_ROWS: hi - c * CHUNK_ROWS]
+        out[lo - r.start: hi - r.start] = part if w.x_dtype == "f32" else f32_to_bf16_bits(part)
+    return out
+
+
+def generate_rows(key: str, row_ids, seed: int = SEED) -> np.ndarray:
+    """Stored input for an arbitrary set of rows (sorted or not)."""
+    row_ids = np.asarray(row_ids, dtype=np.int64)
+    w = WORKLOADS[key]
+    out = np.empty((len(row_ids), w.n), dtype=np.float32 if w.x_dtype == "f32" else np.uint16)
+    for c in np.unique(row_ids // CHUNK_ROWS):
+        sel = np.nonzero(row_ids // CHUNK_ROWS == c)[0]
+        block = generate(key, slice(int(c) * CHUNK_ROWS, min(w.rows, (int(c) + 1) * CHUNK_ROWS)), seed)
+        out[sel] = block[row_ids[sel] - int(c) * CHUNK_ROWS]
+    return out
+
+
+def rank_seed(rank: int, seed: int = SEED) -> int:
+    """Seed of the batch a rank owns when every rank processes its own full
+    batch of the workload (weak scaling: per-GPU work fixed, no exchange)."""
+    if rank < 0:
+        raise ValueError("rank must be >= 0")
+    return seed + 7919 * rank

@@ -1,0 +1,57 @@
+"""Plain float64 CPU oracle for the fused Hadamard rotation + quantization path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports, links or calls this
+package; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may use it.  It shares no code,
+table or constant generator with the CUDA path.
+
+What it computes, and where the pages define it:
+
+* ``sylvester_hadamard`` / ``rotate`` -- the deterministic Sylvester Hadamard
+  matrix built by the doubling H -> [[H, H], [H, -H]] and normalised by the
+  square root of its size ("Rotation Transform", AutoRound docs, section 1.5
+  "Deterministic vs random Hadamard"), applied to every row as a dense
+  float64 product, full-size or block-diagonal with ``rotation_size`` /
+  ``block_size`` blocks (same page, sections 1.2 and 2.1).  The orthogonality
+  the page states in its introduction (R @ R^T = I) is what lets the rotated
+  activations meet pre-rotated weights.
+* ``quantize_int4_sym`` / ``quantize_int8_per_token`` -- round-to-nearest
+  with symmetric range (the RTN proxy with wbits / groupsize / sym of
+  "Pre-Process (Rotation Preprocessing)", OneCompression docs, Workflow note).
+* ``quantize_mxfp4`` -- the MXFP4 scheme the rotation targets ("Rotation
+  Transform", introduction and section 2.1: MX block 32).  The pages do not
+  define the format's internals; the reading used is the OCP MX v1.0 rule
+  (E2M1 elements, E8M0 shared scale, floor-based exponent).
+
+Readings of points the pages leave open (rounding half to even, the fp16 scale
+used for the codes, the symmetric +/-7 / +/-127 range, zero groups, nibble
+order, non-finite scales) are stated on each function.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+to values the pages or the mathematics fix (hand cases, closed forms, library
+routines, invariants).  End-to-end rotated-and-quantized values have no worked
+example on the pages; they are pinned only through their pinned parts.
+"""
+
+from .hadq_oracle import (  # noqa: F401
+    E2M1_GRID,
+    INT4_QMAX,
+    INT8_QMAX,
+    MX_GROUP,
+    codes_with_scale,
+    e2m1_encode,
+    e8m0_exponent,
+    fp16_scale_midpoint_distance,
+    pack_nibbles,
+    quantize_int4_sym,
+    quantize_int8_per_token,
+    quantize_mxfp4,
+    resolve_block,
+    rotate,
+    rotate_quant,
+    round_to_binary,
+    sylvester_hadamard,
+    to_bf16_bits,
+    to_fp16,
+    to_fp32,
+)

@@ -1,0 +1,295 @@
+"""Float64 reference for rotate / rotate+quantize.  Test infrastructure only.
+
+Every function follows a passage of the pages (cited in its docstring) or,
+where the pages are silent, a reading stated in the docstring.  The code is
+deliberately plain: explicit matrices, dense products, whole-array numpy
+expressions, no blocking or fusion beyond what the definitions state.
+"""
+
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+
+INT4_QMAX = 7      # symmetric int4 range +/-7 (scale = absmax / 7)
+INT8_QMAX = 127    # symmetric int8 range +/-127 (scale = absmax / 127)
+MX_GROUP = 32      # MX block size ("Rotation Transform", section 2.1: 32 for MXFP)
+
+# E2M1 magnitudes indexed by the 3-bit code (exponent 2 bits, mantissa 1 bit).
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Rotation
+# ---------------------------------------------------------------------------
+
+def _is_pow2(v: int) -> bool:
+    return v >= 1 and (v & (v - 1)) == 0
+
+
+@functools.lru_cache(maxsize=6)
+def _sylvester(size: int) -> np.ndarray:
+    h = np.ones((1, 1), dtype=np.float64)
+    while h.shape[0] < size:
+        h = np.block([[h, h], [h, -h]])
+    h.setflags(write=False)
+    return h
+
+
+def sylvester_hadamard(size: int) -> np.ndarray:
+    """Unnormalised Sylvester Hadamard matrix of order ``size`` (entries +/-1).
+
+    "Rotation Transform" (AutoRound docs), section 1.5: the deterministic
+    matrix is built by the doubling H -> [[H, H], [H, -H]]; its size must be a
+    power of 2.  Starting from H_1 = [1] fixes the natural (Hadamard) row
+    order.  The result is read-only and cached.
+    """
+    size = int(size)
+    if not _is_pow2(size):
+        raise ValueError(f"Sylvester Hadamard size must be a power of 2, got {size}")
+    return _sylvester(size)
+
+
+def resolve_block(n: int, block) -> int:
+    """Block size actually applied to a row of length ``n``.
+
+    ``None``, ``-1``, ``0`` and ``n`` all mean the full dimension ("Rotation
+    Transform", section 2.1: block_size None/-1 means full-dimension
+    Hadamard).  Otherwise the block must be a positive power of 2 dividing
+    ``n`` (section 1.2: rotation_size must be a positive power of 2).  A full
+    rotation needs ``n`` itself to be a power of 2 (section 1.5).
+    """
+    n = int(n)
+    if block is None or int(block) in (-1, 0, n):
+        b = n
+    else:
+        b = int(block)
+    if not _is_pow2(b) or n % b != 0:
+        raise ValueError(f"block {block!r} is not a power of 2 dividing n={n}")
+    return b
+
+
+def rotate(x, block=0) -> np.ndarray:
+    """y = x . diag(H_b, ..., H_b) / sqrt(b) for every row of ``x`` (float64).
+
+    The online rotation of "Rotation Transform", section 1.1 (R1 on the
+    residual stream, R3 per head on Q/K, R4 on the down_proj input) and the
+    per-Linear block-diagonal mode of section 2: each row is cut into
+    consecutive blocks of ``b`` elements and each block is multiplied by the
+    normalised Sylvester matrix (section 1.5).  The product is a dense
+    O(b^2)-per-block float64 matmul of the exact upcast input.  H is
+    symmetric, so x . H and H . x agree, and H/sqrt(b) is its own inverse.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if x.ndim != 2:
+        raise ValueError("rotate expects a 2-D (rows, n) array")
+    rows, n = x.shape
+    b = resolve_block(n, block)
+    h = sylvester_hadamard(b)
+    y = (x.reshape(rows * (n // b), b) @ h) / np.sqrt(float(b))
+    return y.reshape(rows, n)
+
+
+# ---------------------------------------------------------------------------
+# Rounding onto binary floating-point grids (scales and outputs)
+# ---------------------------------------------------------------------------
+
+def _floor_log2(a: np.ndarray) -> np.ndarray:
+    """floor(log2(a)) for a > 0, exact (from the binary exponent)."""
+    _, p = np.frexp(a)          # a = f * 2**p with f in [0.5, 1)
+    return p.astype(np.int64) - 1
+
+
+def round_to_binary(v, mant_bits: int, emin: int, max_finite: float) -> np.ndarray:
+    """Round-half-to-even of float64 ``v`` onto a binary floating-point grid.
+
+    The grid has ``mant_bits`` stored mantissa bits and smallest normal
+    exponent ``emin`` (subnormals below it keep the spacing 2**(emin -
+    mant_bits)).  Magnitudes that round above ``max_finite`` become inf, as
+    IEEE rounding does.  Used for fp16 scales (10, -14), fp32 scales (23,
+    -126) and bf16 outputs (7, -126).
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    nz = a > 0
+    e = np.where(nz, _floor_log2(np.where(nz, a, 1.0)), emin)
+    ulp = np.ldexp(1.0, np.maximum(e, emin) - mant_bits)
+    r = np.rint(v / ulp) * ulp          # v/ulp is exact: ulp is a power of 2
+    return np.where(np.abs(r) > max_finite, np.copysign(np.inf, v), r)
+
+
+def to_fp16(v) -> np.ndarray:
+    """float64 -> IEEE binary16, round half to even (returns float64 values)."""
+    return round_to_binary(v, 10, -14, 65504.0)
+
+
+def to_fp32(v) -> np.ndarray:
+    """float64 -> IEEE binary32, round half to even (returns float64 values)."""
+    return round_to_binary(v, 23, -126, float(np.finfo(np.float32).max))
+
+
+def to_bf16_bits(v) -> np.ndarray:
+    """float64 -> bfloat16 bit patterns (uint16), round half to even."""
+    r = round_to_binary(v, 7, -126, (2.0 - 2.0 ** -7) * 2.0 ** 127)
+    return (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def fp16_scale_midpoint_distance(v):
+    """Relative distance of ``v`` to the nearest fp16 rounding midpoint, and
+    the fp16 value the rounding would give on the other side of it.
+
+    Used by the parity checker: a scale whose pre-rounding value lies within
+    1e-6 of a midpoint is a boundary case where either neighbour is valid.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    nz = a > 0
+    e = np.where(nz, _floor_log2(np.where(nz, a, 1.0)), -14)
+    ulp = np.ldexp(1.0, np.maximum(e, -14) - 10)
+    lo = np.floor(a / ulp) * ulp
+    hi = lo + ulp
+    mid = 0.5 * (lo + hi)
+    rounded = np.abs(to_fp16(a))
+    alt = np.where(rounded == lo, hi, lo)
+    rel = np.where(nz, np.abs(a - mid) / np.where(nz, a, 1.0), np.inf)
+    return rel, np.copysign(alt, v)
+
+
+# ---------------------------------------------------------------------------
+# Round-to-nearest quantizers
+# ---------------------------------------------------------------------------
+
+def codes_with_scale(y, s, qmax: int) -> np.ndarray:
+    """q = clamp(round_half_even(y / s), -qmax, qmax); 0 where s is 0 or inf.
+
+    Round-to-nearest with the symmetric range (the RTN proxy of "Pre-Process
+    (Rotation Preprocessing)", Workflow note: wbits, groupsize, sym).
+    Readings: ties round to even; the code uses the stored (rounded) scale,
+    so dequantisation q * s is self-consistent; a zero scale (all-zero group)
+    or an infinite one gives zero codes.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    ok = (s > 0) & np.isfinite(s)
+    safe = np.where(ok, s, 1.0)
+    q = np.clip(np.rint(y / safe), -qmax, qmax)
+    q = np.where(ok, q, 0.0)
+    return q.astype(np.int16)
+
+
+def quantize_int4_sym(y, group: int):
+    """Symmetric int4 RTN per group: scale = fp16(absmax / 7), codes in [-7, 7].
+
+    Returns ``(codes int8 (rows, n), scales float16 (rows, n // group))``.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    rows, n = y.shape
+    if group <= 0 or n % group:
+        raise ValueError(f"group {group} must divide n={n}")
+    g = y.reshape(rows, n // group, group)
+    m = np.abs(g).max(axis=-1)
+    s = to_fp16(m / INT4_QMAX)
+    codes = codes_with_scale(g, s[..., None], INT4_QMAX).reshape(rows, n)
+    return codes.astype(np.int8), s.astype(np.float16)
+
+
+def quantize_int8_per_token(y):
+    """Symmetric int8 RTN per row: scale = fp32(absmax / 127), codes in [-127, 127].
+
+    Returns ``(codes int8 (rows, n), scales float32 (rows,))``.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    m = np.abs(y).max(axis=1)
+    s = to_fp32(m / INT8_QMAX)
+    codes = codes_with_scale(y, s[:, None], INT8_QMAX)
+    return codes.astype(np.int8), s.astype(np.float32)
+
+
+def e8m0_exponent(m) -> np.ndarray:
+    """Shared MX exponent e = floor(log2(m)) - 2, clamped to [-127, 127].
+
+    OCP MX v1.0 reading (the pages name MXFP4 but not its scale rule): the
+    largest E2M1 magnitude is 6 = 1.5 * 2**2, so the exponent is the group
+    absmax's exponent minus 2.  An all-zero group gets -127 (stored byte 0).
+    """
+    m = np.asarray(m, dtype=np.float64)
+    nz = m > 0
+    e = np.where(nz, _floor_log2(np.where(nz, m, 1.0)) - 2, -127)
+    return np.clip(e, -127, 127)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """E2M1 code (sign << 3 | index) of ``v``.
+
+    The index is that of the nearest magnitude in ``E2M1_GRID``; a tie goes
+    to the even index (even mantissa bit), so 0.25 -> 0, 0.75 -> 1.0,
+    1.25 -> 1.0, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4; magnitudes above 6
+    take 6 (saturation).  The sign bit is set for negative values, including
+    those whose magnitude rounds to zero.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    best = np.zeros(a.shape, dtype=np.int64)
+    bestd = np.abs(a - E2M1_GRID[0])
+    for i in range(1, len(E2M1_GRID)):
+        d = np.abs(a - E2M1_GRID[i])
+        better = (d < bestd) | ((d == bestd) & (i % 2 == 0))
+        best = np.where(better, i, best)
+        bestd = np.where(better, d, bestd)
+    sign = (v < 0).astype(np.int64)
+    return (best | (sign << 3)).astype(np.uint8)
+
+
+def quantize_mxfp4(y):
+    """MXFP4: per 32 elements an E8M0 exponent e and E2M1 codes of y / 2**e.
+
+    Returns ``(codes uint8 (rows, n) in [0, 15], scales uint8 (rows, n // 32))``
+    where the stored scale byte is e + 127.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    rows, n = y.shape
+    if n % MX_GROUP:
+        raise ValueError(f"n={n} is not a multiple of {MX_GROUP}")
+    g = y.reshape(rows, n // MX_GROUP, MX_GROUP)
+    m = np.abs(g).max(axis=-1)
+    e = e8m0_exponent(m)
+    v = np.ldexp(g, -e[..., None])
+    codes = e2m1_encode(v).reshape(rows, n)
+    return codes, (e + 127).astype(np.uint8)
+
+
+def pack_nibbles(codes) -> np.ndarray:
+    """Two 4-bit codes per byte, the even-indexed element in the low nibble.
+
+    int4 codes are stored as two's-complement nibbles (q & 0xF).
+    """
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    if c.shape[-1] % 2:
+        raise ValueError("row length must be even to pack nibbles")
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def rotate_quant(x, block, fmt: str, group: int = 0):
+    """Rotate then quantize, as the fused path does in one pass.
+
+    ``fmt`` is ``"int4"`` (codes packed two per byte, fp16 scales per
+    ``group``), ``"int8"`` (per-token; int8 codes, fp32 scale per row) or
+    ``"mxfp4"`` (codes packed two per byte, E8M0 bytes per 32).
+    Returns ``(y, codes_stored, scales)`` where ``y`` is the float64 rotation.
+    """
+    y = rotate(x, block)
+    if fmt == "int4":
+        q, s = quantize_int4_sym(y, group)
+        return y, pack_nibbles(q), s
+    if fmt == "int8":
+        if group not in (0, y.shape[1]):
+            raise ValueError("int8 is per-token: group must be 0 or n")
+        q, s = quantize_int8_per_token(y)
+        return y, q, s
+    if fmt == "mxfp4":
+        if group not in (0, MX_GROUP):
+            raise ValueError("MXFP4 groups are 32 elements")
+        q, s = quantize_mxfp4(y)
+        return y, pack_nibbles(q), s
+    raise ValueError(f"unknown fmt {fmt!r}")

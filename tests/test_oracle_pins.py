@@ -1,0 +1,373 @@
+"""Pins of the float64 oracle to facts the pages or the mathematics fix.
+
+Each test pins one function to something other than itself: hand-worked
+fixtures (tests/golden/, each citing its passage), closed forms, an
+independent library routine, an independent algorithm, or an invariant the
+pages state.  A dropped normalisation, a wrong sign or index, a transposed
+block, a wrong tie rule or nibble order each fails at least one of them.
+"""
+
+import struct
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from tests.conftest import load_golden
+
+SIZES = [2 ** k for k in range(0, 14)]   # 1 .. 8192, every size the path uses
+
+
+# ----------------------------------------------------------------- Hadamard
+
+def test_sylvester_matches_handwritten():
+    g = load_golden("sylvester_small.json")
+    for k in ("H1", "H2", "H4", "H8"):
+        want = np.array(g[k], dtype=np.float64)
+        np.testing.assert_array_equal(oracle.sylvester_hadamard(want.shape[0]), want)
+
+
+@pytest.mark.parametrize("size", [s for s in SIZES if s <= 4096])
+def test_sylvester_matches_scipy(size):
+    # scipy.linalg.hadamard is an independent Sylvester construction (natural order).
+    np.testing.assert_array_equal(oracle.sylvester_hadamard(size), scipy.linalg.hadamard(size))
+
+
+def _popcount(a):
+    c = np.zeros_like(a)
+    while np.any(a):
+        c += a & 1
+        a = a >> 1
+    return c
+
+
+@pytest.mark.parametrize("size", SIZES)
+def test_sylvester_closed_form(size):
+    """H[i, j] = (-1)^popcount(i & j): full check up to 1024, sampled above."""
+    h = oracle.sylvester_hadamard(size)
+    rng = np.random.default_rng(size)
+    if size <= 1024:
+        i, j = np.meshgrid(np.arange(size), np.arange(size), indexing="ij")
+    else:
+        i = rng.integers(0, size, 200_000)
+        j = rng.integers(0, size, 200_000)
+    want = np.where(_popcount(i & j) % 2 == 0, 1.0, -1.0)
+    np.testing.assert_array_equal(h[i, j], want)
+
+
+@pytest.mark.parametrize("size", SIZES)
+def test_hadamard_orthogonal(size):
+    """H . H^T = size . I (full product up to 1024; sampled row pairs above)."""
+    h = oracle.sylvester_hadamard(size)
+    if size <= 1024:
+        np.testing.assert_array_equal(h @ h.T, size * np.eye(size))
+    else:
+        rng = np.random.default_rng(size + 1)
+        a = rng.integers(0, size, 64)
+        b = (a + rng.integers(1, size, 64)) % size
+        np.testing.assert_array_equal(np.einsum("ij,ij->i", h[a], h[b]), 0.0)
+        np.testing.assert_array_equal(np.einsum("ij,ij->i", h[a], h[a]), float(size))
+
+
+# ----------------------------------------------------------------- rotation
+
+def test_rotate_hand_cases():
+    g = load_golden("rotation_hand_cases.json")
+    for c in g["cases"]:
+        x = np.array([c["x"]], dtype=np.float64)
+        want = np.array([c["y_times_sqrt_b"]], dtype=np.float64) / np.sqrt(c["b"])
+        np.testing.assert_allclose(oracle.rotate(x, c["block"]), want, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("n", [s for s in SIZES if s >= 2])
+def test_rotate_basis_vectors(n):
+    """e0 -> (1/sqrt n) * ones and ones -> sqrt(n) * e0 (closed forms of H_n / sqrt(n))."""
+    e0 = np.zeros((1, n))
+    e0[0, 0] = 1.0
+    np.testing.assert_allclose(oracle.rotate(e0), np.full((1, n), 1 / np.sqrt(n)), rtol=1e-15, atol=0)
+    ones = np.ones((1, n))
+    want = np.zeros((1, n))
+    want[0, 0] = np.sqrt(n)
+    np.testing.assert_allclose(oracle.rotate(ones), want, rtol=0, atol=1e-12 * np.sqrt(n))
+
+
+@pytest.mark.parametrize("n,block", [(1024, 0), (4096, 0), (8192, 0), (14336, 128), (4096, 32), (512, 16)])
+def test_rotate_norm_and_involution(n, block):
+    """Orthogonality: norms preserved; H/sqrt(b) is its own inverse."""
+    rng = np.random.default_rng(n + block)
+    x = rng.standard_normal((8, n)) * rng.uniform(0.1, 30.0, (8, 1))
+    y = oracle.rotate(x, block)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(oracle.rotate(y, block), x, rtol=0, atol=1e-12 * np.abs(x).max())
+
+
+@pytest.mark.parametrize("n,block", [(256, 0), (1024, 0), (1024, 128), (896, 128)])
+def test_rotated_activations_meet_rotated_weights(n, block):
+    """x @ R @ R^T @ W^T = x @ W^T ("Rotation Transform", introduction): the
+    online-rotated activation against an offline-rotated weight (W R) gives the
+    unrotated layer output."""
+    rng = np.random.default_rng(7 + n)
+    x = rng.standard_normal((16, n))
+    w = rng.standard_normal((24, n))
+    xr = oracle.rotate(x, block)
+    wr = oracle.rotate(w, block)
+    np.testing.assert_allclose(xr @ wr.T, x @ w.T, rtol=0, atol=1e-10 * np.sqrt(n) * 10)
+
+
+def test_r3_attention_logits_unchanged():
+    """R3 rotates Q and K per head with the same head_dim Hadamard, so the
+    logits q k^T are unchanged ("Rotation Transform" section 1.1 R3; the
+    apply_spinquant docstring: rotated K enters the cache)."""
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((64, 128))
+    k = rng.standard_normal((80, 128))
+    np.testing.assert_allclose(oracle.rotate(q) @ oracle.rotate(k).T, q @ k.T, atol=1e-11)
+
+
+@pytest.mark.parametrize("n,block", [(1024, 128), (14336, 128), (4096, 1024), (256, 16)])
+def test_block_mode_is_per_block_full_transform(n, block):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((5, n))
+    y = oracle.rotate(x, block)
+    for j in range(n // block):
+        sl = slice(j * block, (j + 1) * block)
+        np.testing.assert_allclose(y[:, sl], oracle.rotate(x[:, sl], 0), rtol=0, atol=1e-12)
+
+
+def _fwht_butterflies(x):
+    """Independent fast Walsh-Hadamard transform (iterative butterflies), unnormalised."""
+    a = np.array(x, dtype=np.float64, copy=True)
+    n = a.shape[-1]
+    h = 1
+    while h < n:
+        a = a.reshape(*a.shape[:-1], n // (2 * h), 2, h)
+        u = a[..., 0, :].copy()
+        v = a[..., 1, :].copy()
+        a[..., 0, :] = u + v
+        a[..., 1, :] = u - v
+        a = a.reshape(*a.shape[:-3], n)
+        h *= 2
+    return a
+
+
+@pytest.mark.parametrize("n", [2, 8, 128, 1024, 4096, 8192])
+def test_dense_rotation_equals_fast_transform(n):
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((4, n))
+    want = _fwht_butterflies(x) / np.sqrt(n)
+    np.testing.assert_allclose(oracle.rotate(x), want, rtol=0, atol=1e-12 * np.sqrt(n))
+
+
+def test_block_argument_forms():
+    x = np.arange(16, dtype=np.float64)[None]
+    full = oracle.rotate(x, 16)
+    for b in (0, -1, None):
+        np.testing.assert_array_equal(oracle.rotate(x, b), full)
+    for bad in (3, 12, 32):
+        with pytest.raises(ValueError):
+            oracle.rotate(x, bad)
+    with pytest.raises(ValueError):
+        oracle.rotate(np.zeros((1, 12)), 0)   # full size must be a power of 2
+
+
+# ----------------------------------------------------------- float formats
+
+def _interesting_values(rng):
+    base = np.concatenate([
+        rng.standard_normal(4000) * np.exp(rng.uniform(-25, 12, 4000)),
+        np.ldexp(1.0, np.arange(-30, 17)),
+    ])
+    return base
+
+
+def test_fp16_rounding_matches_numpy_and_struct():
+    rng = np.random.default_rng(0)
+    v = _interesting_values(rng)
+    v = v[np.abs(v) < 65504]
+    # exact fp16 midpoints (ties) and their neighbours
+    grid = np.array([1.0, 1.5, 0.142822265625, 1024.0, 2.0 ** -14, 2.0 ** -20])
+    ulps = np.ldexp(1.0, np.maximum(np.frexp(grid)[1] - 1, -14) - 10)
+    mids = np.concatenate([grid + ulps / 2, grid + 1.5 * ulps])
+    v = np.concatenate([v, mids, -mids])
+    got = oracle.to_fp16(v)
+    np.testing.assert_array_equal(got, v.astype(np.float16).astype(np.float64))
+    for a, b in zip(v[::37], got[::37]):
+        assert struct.unpack("<e", struct.pack("<e", a))[0] == b
+    assert np.isinf(oracle.to_fp16(np.array([65520.0]))[0])
+    assert oracle.to_fp16(np.array([65519.0]))[0] == 65504.0
+
+
+def test_fp32_rounding_matches_numpy_and_struct():
+    rng = np.random.default_rng(1)
+    v = _interesting_values(rng)
+    got = oracle.to_fp32(v)
+    np.testing.assert_array_equal(got, v.astype(np.float32).astype(np.float64))
+    for a, b in zip(v[::41], got[::41]):
+        assert struct.unpack("<f", struct.pack("<f", a))[0] == b
+
+
+def test_bf16_bits_match_torch():
+    rng = np.random.default_rng(2)
+    v = _interesting_values(rng).astype(np.float32).astype(np.float64)   # fp32-exact inputs
+    ties = (np.array([1.0, -3.0, 0.5]) * (1 + 2.0 ** -8)).astype(np.float64)
+    v = np.concatenate([v, ties])
+    want = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.to_bf16_bits(v), want)
+
+
+def test_fp16_midpoint_distance():
+    mid = 1.0 + 2.0 ** -11          # exact midpoint between 1 and 1 + 2^-10
+    rel, alt = oracle.fp16_scale_midpoint_distance(np.array([mid * (1 + 1e-9), mid * (1 - 1e-9), 1.3]))
+    assert rel[0] < 1e-8 and rel[1] < 1e-8 and rel[2] > 1e-4
+    assert alt[0] == 1.0 and alt[1] == 1.0 + 2.0 ** -10     # the neighbour not taken by RNE
+
+
+# -------------------------------------------------------------- quantizers
+
+def test_int4_hand_cases():
+    for c in load_golden("rtn_cases.json")["int4"]:
+        y = np.array([c["y"]])
+        q, s = oracle.quantize_int4_sym(y, c["group"])
+        np.testing.assert_array_equal(q[0], c["codes"])
+        np.testing.assert_array_equal(s[0].astype(np.float64), c["scales"])
+        np.testing.assert_array_equal(oracle.pack_nibbles(q)[0], c["packed"])
+
+
+def test_int8_hand_cases():
+    for c in load_golden("rtn_cases.json")["int8"]:
+        q, s = oracle.quantize_int8_per_token(np.array([c["y"]]))
+        np.testing.assert_array_equal(q[0], c["codes"])
+        assert float(s[0]) == c["scale"]
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_int4_rtn_properties(group):
+    rng = np.random.default_rng(group)
+    y = rng.standard_normal((64, 1024)) * rng.uniform(1e-3, 1e3, (64, 1))
+    q, s = oracle.quantize_int4_sym(y, group)
+    g = y.reshape(64, -1, group)
+    qg = q.reshape(64, -1, group).astype(np.float64)
+    s64 = s.astype(np.float64)[..., None]
+    assert q.min() >= -7 and q.max() <= 7
+    # reconstruction error at most half a step for unclipped elements
+    err = np.abs(g - qg * s64)
+    assert np.all(err <= s64 / 2 * (1 + 1e-12))
+    # the group's absmax element maps to +/-7
+    idx = np.abs(g).argmax(axis=-1)
+    top = np.take_along_axis(qg, idx[..., None], -1)[..., 0]
+    np.testing.assert_array_equal(np.abs(top), 7)
+    # the scale is the fp16 rounding of absmax / 7 (within half an fp16 ulp)
+    m = np.abs(g).max(-1)
+    assert np.all(np.abs(s64[..., 0] - m / 7) <= np.ldexp(1.0, np.frexp(m / 7)[1] - 1 - 11) * (1 + 1e-12))
+
+
+def test_int8_rtn_properties():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((32, 14336)) * rng.uniform(1e-2, 1e2, (32, 1))
+    q, s = oracle.quantize_int8_per_token(y)
+    s64 = s.astype(np.float64)[:, None]
+    assert q.min() >= -127 and q.max() <= 127
+    assert np.all(np.abs(y - q * s64) <= s64 / 2 * (1 + 1e-9))
+    np.testing.assert_array_equal(np.abs(q[np.arange(32), np.abs(y).argmax(1)]), 127)
+
+
+def test_zero_and_nonfinite_scales_give_zero_codes():
+    assert np.all(oracle.codes_with_scale(np.array([1.0, -2.0]), np.array([0.0]), 7) == 0)
+    assert np.all(oracle.codes_with_scale(np.array([1.0, -2.0]), np.array([np.inf]), 7) == 0)
+    # absmax / 7 beyond fp16 range -> infinite scale -> zero codes
+    q, s = oracle.quantize_int4_sym(np.full((1, 32), 1e6), 32)
+    assert np.isinf(s[0, 0]) and np.all(q == 0)
+    # tiny absmax -> subnormal fp16 scale -> codes clamp to +/-7
+    q, s = oracle.quantize_int4_sym(np.array([[5e-7] + [0.0] * 31]), 32)
+    assert 0 < float(s[0, 0]) < 6.2e-5 and q[0, 0] == 7
+
+
+def test_e2m1_table_and_ties():
+    g = load_golden("mxfp4_cases.json")
+    dec = np.array(g["e2m1_decode"])
+    # every code decodes to a grid value that encodes back to itself (except -0 -> +0)
+    for code, val in enumerate(dec):
+        got = int(oracle.e2m1_encode(np.array([val]))[0])
+        assert got == (0 if code == 8 else code)
+    for v, want in g["encode_cases"]:
+        assert int(oracle.e2m1_encode(np.array([v]))[0]) == want, v
+
+
+def test_e2m1_nearest_even_property():
+    """On a dense grid: the code decodes to a nearest E2M1 magnitude (6 above
+    the top), and at an exact tie the chosen code index is even."""
+    dec = np.array(load_golden("mxfp4_cases.json")["e2m1_decode"])
+    v = np.concatenate([np.linspace(-8, 8, 64001), np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])])
+    c = oracle.e2m1_encode(v).astype(np.int64)
+    got = np.abs(dec[c])
+    dist = np.abs(np.abs(v)[:, None] - np.abs(dec[:8])[None, :])
+    best = dist.min(1)
+    assert np.all(np.abs(np.abs(v) - got) == best)
+    tie = (dist == best[:, None]).sum(1) == 2
+    assert np.all((c[tie] & 7) % 2 == 0)
+    assert np.all((c >> 3)[v < 0] == 1) and np.all((c >> 3)[v >= 0] == 0)
+
+
+def test_e8m0_cases_and_bracket():
+    g = load_golden("mxfp4_cases.json")
+    for m, byte in g["e8m0_cases"]:
+        assert int(oracle.e8m0_exponent(np.array([m]))[0]) + 127 == byte, m
+    rng = np.random.default_rng(9)
+    m = np.exp(rng.uniform(-60, 60, 10000))
+    e = oracle.e8m0_exponent(m).astype(np.float64)
+    assert np.all((2.0 ** (e + 2) <= m) & (m < 2.0 ** (e + 3)))
+
+
+def test_mxfp4_block_case():
+    c = load_golden("mxfp4_cases.json")["block_case"]
+    q, s = oracle.quantize_mxfp4(np.array([c["y"]]))
+    assert int(s[0, 0]) == c["scale_byte"]
+    np.testing.assert_array_equal(q[0], c["codes"])
+    np.testing.assert_array_equal(oracle.pack_nibbles(q)[0], c["packed"])
+
+
+def test_mxfp4_dequant_error_bound():
+    """Every unsaturated element is within half an E2M1 step of its value."""
+    rng = np.random.default_rng(12)
+    y = rng.standard_t(3, (16, 8192))
+    q, s = oracle.quantize_mxfp4(y)
+    dec = np.array(load_golden("mxfp4_cases.json")["e2m1_decode"])
+    e = s.astype(np.int64) - 127
+    deq = dec[q.astype(np.int64)].reshape(16, -1, 32) * np.ldexp(1.0, e)[..., None]
+    v = np.abs(y.reshape(16, -1, 32)) / np.ldexp(1.0, e)[..., None]
+    step = np.select([v < 2, v < 4], [0.5, 1.0], 2.0) * np.ldexp(1.0, e)[..., None]
+    unsat = v <= 6
+    assert np.all(np.abs(deq - y.reshape(16, -1, 32))[unsat] <= (step / 2)[unsat] * (1 + 1e-12))
+
+
+def test_rotate_quant_dispatch():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((3, 256))
+    y, c, s = oracle.rotate_quant(x, 0, "int4", 128)
+    assert c.shape == (3, 128) and c.dtype == np.uint8 and s.shape == (3, 2) and s.dtype == np.float16
+    y, c, s = oracle.rotate_quant(x, 128, "int8", 0)
+    assert c.shape == (3, 256) and c.dtype == np.int8 and s.shape == (3,) and s.dtype == np.float32
+    y, c, s = oracle.rotate_quant(x, 64, "mxfp4", 32)
+    assert c.shape == (3, 128) and s.shape == (3, 8) and s.dtype == np.uint8
+    with pytest.raises(ValueError):
+        oracle.rotate_quant(x, 0, "int8", 64)
+
+
+# ------------------------------------------------- incoherence (diagnostic)
+
+def test_rotation_flattens_outliers():
+    """QuIP note, "Incoherence, and the rotation that manufactures it": a
+    rotation takes an outlier-planted matrix's mu down towards the Gaussian
+    floor sqrt(2 ln(mn)).  The deterministic Hadamard does the same to rows
+    with outlier channels (the C2-like input)."""
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((64, 64))
+    x[:, [3, 17]] *= 25.0
+
+    def mu(a):
+        return np.abs(a).max() / np.sqrt((a ** 2).mean())
+    before, after = mu(x), mu(oracle.rotate(x))
+    assert before > 10 and after < 0.5 * before
+    assert after < 1.5 * np.sqrt(2 * np.log(64 * 64))
