@@ -1,0 +1,351 @@
+"""Throughput of the fused Hadamard rotation + int4 quantization (libhadq).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hadq|reference]
+
+One step = one hadq_rotate_quant launch over one batch of the R1 workload:
+4096 tokens x hidden 4096 bf16 (1 % outlier channels x50), full 4096-point
+Sylvester Hadamard, symmetric int4 RTN per group of 128 with fp16 scales.
+The metric is GB/s of algorithmic traffic (input read once + codes and scales
+written once) and its fraction of the measured HBM copy bandwidth.
+
+Timing: inputs resident in HBM; 8 buffer sets (input + outputs) are rotated so
+each step touches data last used 7 steps earlier (336 MB > L2).  The K steps
+are captured in one CUDA graph together with a CUDA event pair around every
+launch; the graph is replayed once untimed and once timed between barriers
+and device synchronisations.  `value` = bytes of all ranks / max-over-ranks
+elapsed time; `roofline.achieved` = bytes per launch / mean event duration.
+`e2e` repeats the metric through hadq_rotate_quant_host (pinned host input,
+copies in and out inside the timed region).
+
+Under torchrun every rank processes its own batch (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+`--impl reference` times the float64 CPU oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hadamard_rotation_bit_b200 import workloads as W  # noqa: E402
+
+WORKLOAD = W.WORKLOADS["c2"]
+METRIC = "fused Hadamard+quant GB/s and % of B200 HBM peak (4096x4096 bf16->int4 g128)"
+UNIT = "GB/s"
+NBUF = 8
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _env_int(k, d):
+    try:
+        return int(os.environ.get(k, d))
+    except ValueError:
+        return d
+
+
+def config_block():
+    w = WORKLOAD
+    return {"workload": w.name, "rows": w.rows, "n": w.n, "block": w.block, "fmt": w.fmt, "group": w.group,
+            "x_dtype": w.x_dtype, "algorithmic_bytes_per_step": w.algorithmic_bytes,
+            "l2": f"{NBUF} rotating buffer sets ({NBUF * w.algorithmic_bytes / 1e6:.0f} MB > L2 126 MB)"}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hadamard_rotation_bit_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic_c2.json")) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    return rec.get("dram_bytes_per_launch") if rec.get("kernel_source_hash") == kernel_source_hash() else None
+
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the timed region runs."""
+
+    NAMES = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+             0x4: "sw_power_cap", 0x1: "gpu_idle", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index, period=0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.nv, self.err = None, str(e)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self.NAMES.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.nv:
+            return {"error": getattr(self, "err", "no NVML")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+def dist_setup():
+    world = _env_int("WORLD_SIZE", 1)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        rank, local = _env_int("RANK", 0), _env_int("LOCAL_RANK", 0)
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, world, local
+    return None, 0, 1, 0
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(dist, v):
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(seconds=12.0):
+    """The float64 oracle, as it stands, on this host's cores: whole C2 batches
+    (or row slices of one) until about `seconds` of CPU work is done."""
+    import oracle
+    w = WORKLOAD
+    rows = 512
+    x = W.bits_to_float64(W.generate("c2", slice(0, rows)), "bf16")
+    oracle.rotate_quant(x[:8], 0, "int4", 128)          # builds and caches H_4096
+    done, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        oracle.rotate_quant(x, 0, "int4", 128)
+        done += rows
+    dt = time.perf_counter() - t0
+    bytes_done = w.algorithmic_bytes * done / w.rows
+    cores = len(os.sched_getaffinity(0))
+    return {"value": bytes_done / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} rows of the 4096x4096 batch in slices of {rows} rows ({dt:.1f} s, float64 numpy/BLAS)"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step a row slice of the workload."""
+    dist, rank, world, _ = dist_setup()
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    import oracle
+    w = WORKLOAD
+    steps, warm = args.steps, args.warmup
+    rows = int(max(1, min(w.rows, 60.0 * 80 / max(1, steps + warm))))   # ~80 rows/s of oracle work
+    x = W.bits_to_float64(W.generate("c2", slice(0, rows)), "bf16")
+    for _ in range(warm):
+        oracle.rotate_quant(x, 0, "int4", 128)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.rotate_quant(x, 0, "int4", 128)
+    dt = time.perf_counter() - t0
+    value = w.algorithmic_bytes * rows / w.rows * steps / dt / 1e9
+    cores = len(os.sched_getaffinity(0))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+            "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": config_block(), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} rows of the 4096x4096 batch per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_hadq(args):
+    from hadamard_rotation_bit_b200 import hadq as H
+    dist, rank, world, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    H.load_library()
+    w = WORKLOAD
+    steps, warm = args.steps, max(3, args.warmup)
+
+    stored = W.generate("c2", seed=W.rank_seed(rank))
+    x0 = torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).to(dev)
+    xs = [x0.clone() for _ in range(NBUF)]
+    outs = [H.hadq_rotate_quant(xs[i], 0, "int4", 128) for i in range(NBUF)]   # allocates outputs, warms caches
+    torch.cuda.synchronize()
+    bytes_step = w.algorithmic_bytes
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        c, s = outs[i % NBUF]
+        H.hadq_rotate_quant(xs[i % NBUF], 0, "int4", 128, codes=c, scales=s, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            step(i)
+    stream.synchronize()
+
+    # K launches with an event pair around each, captured in one graph.
+    ev_s = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            ev_s[i].record(stream)
+            step(i)
+            ev_e[i].record(stream)
+    g.replay()                       # untimed replay (warm-up of the graph itself)
+    stream.synchronize()
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        g.replay()
+        t_end.record(stream)
+        stream.synchronize()
+    barrier(dist)
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    per_launch = [ev_s[i].elapsed_time(ev_e[i]) / 1e3 for i in range(steps)]
+    kernel_s = sum(per_launch) / len(per_launch)
+    elapsed_max = max_over_ranks(dist, elapsed)
+    kernel_max = max_over_ranks(dist, kernel_s)
+
+    # end to end through the host-buffer entry point
+    e2e_steps = max(3, min(steps, 30))
+    xh = torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).pin_memory()
+    ch = torch.empty(outs[0][0].shape, dtype=torch.uint8).pin_memory()
+    sh = torch.empty(outs[0][1].shape, dtype=torch.float16).pin_memory()
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            H.hadq_rotate_quant_host(xh, 0, "int4", 128, ch, sh, xs[0], outs[0][0], outs[0][1], stream=stream)
+    stream.synchronize()
+    barrier(dist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        H.hadq_rotate_quant_host(xh, 0, "int4", 128, ch, sh, xs[i % NBUF], outs[i % NBUF][0], outs[i % NBUF][1],
+                                 stream=stream)
+    e1.record(stream)
+    stream.synchronize()
+    e2e_max = max_over_ranks(dist, e0.elapsed_time(e1) / 1e3)
+    h2d = w.in_bytes
+    d2h = w.out_bytes
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        achieved = bytes_step / kernel_max / 1e9
+        line = {
+            "metric": METRIC,
+            "value": bytes_step * steps * world / elapsed_max / 1e9,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": steps,
+            "warmup": warm,
+            "ms_per_step": elapsed_max / steps * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": config_block(),
+            "impl": "hadq",
+            "rows_per_s": w.rows * steps * world / elapsed_max,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                         "traffic": recorded_traffic(), "kernel_us": kernel_max * 1e6},
+            "e2e": {"value": bytes_step * e2e_steps * world / e2e_max / 1e9, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "path": "hadq_rotate_quant_host (pinned host buffers, copies in the timed region)"},
+            "gpu_launches": steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["hadq", "reference"], default="hadq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_hadq(args)
+
+
+if __name__ == "__main__":
+    main()

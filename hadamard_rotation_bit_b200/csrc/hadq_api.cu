@@ -1,0 +1,433 @@
+// libhadq host side: argument validation, launch planning and the C ABI.
+//
+// Every check runs before the first CUDA call, so a failing call launches
+// nothing and leaves all outputs untouched (validate first, then apply -- the
+// rule the apply_spinquant docstring states for its rotation passes).  There
+// is no CPU path: a missing device or kernel image surfaces as HADQ_ERR_CUDA.
+#include "hadq.h"
+#include "hadq_kernels.cuh"
+
+#include <cmath>
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hadq_status fail(hadq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+bool is_pow2(int64_t v) { return v >= 1 && (v & (v - 1)) == 0; }
+
+int ilog2(int64_t v) {
+  int k = 0;
+  while ((int64_t(1) << k) < v) ++k;
+  return k;
+}
+
+int64_t esize(hadq_dtype d) { return d == HADQ_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Span {
+  uintptr_t lo = 0, hi = 0;
+};
+
+Span span(const void* p, int64_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return Span{a, a + static_cast<uintptr_t>(bytes)};
+}
+
+bool overlaps(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi; }
+
+constexpr int kMaxBlock = 8192;
+constexpr int64_t kMaxInt8N = 32768;
+
+// What the kernels need to know about one call.
+struct Shape {
+  int64_t rows = 0, n = 0, b = 0;
+  int logb = 0;
+  int logs = 0;   // segment kernels: log2 of the per-thread segment
+  float norm = 1.f;
+};
+
+hadq_status check_shape(hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, Shape* sh) {
+  if (x_dtype != HADQ_F32 && x_dtype != HADQ_BF16) return fail(HADQ_ERR_INVALID_ARG, "x_dtype must be HADQ_F32 or HADQ_BF16");
+  if (rows < 0) return fail(HADQ_ERR_INVALID_ARG, "rows must be >= 0");
+  if (n <= 0) return fail(HADQ_ERR_INVALID_ARG, "n must be > 0");
+  if (block < -1) return fail(HADQ_ERR_INVALID_ARG, "block must be -1, 0 (full) or a power of 2 dividing n");
+  const bool full = block == -1 || block == 0 || block == n;
+  const int64_t b = full ? n : block;
+  if (!is_pow2(b))
+    return fail(HADQ_ERR_INVALID_ARG, full ? "a full rotation needs n to be a power of 2" : "block must be a power of 2");
+  if (n % b != 0) return fail(HADQ_ERR_INVALID_ARG, "block must divide n");
+  if (b > kMaxBlock) return fail(HADQ_ERR_UNSUPPORTED, "rotation blocks above 8192 are not supported");
+  if (n % 8 != 0) return fail(HADQ_ERR_UNSUPPORTED, "n must be a multiple of 8");
+  if (rows > (INT64_MAX / 8) / n) return fail(HADQ_ERR_INVALID_ARG, "rows * n overflows");
+  sh->rows = rows;
+  sh->n = n;
+  sh->b = b;
+  sh->logb = ilog2(b);
+  const int64_t low = n & (-n);                 // largest power of 2 dividing n
+  sh->logs = ilog2(low < 128 ? low : 128);
+  sh->norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  return HADQ_OK;
+}
+
+hadq_status check_quant(hadq_fmt fmt, int64_t group, const Shape& sh, int* eff_group) {
+  switch (fmt) {
+    case HADQ_INT4_SYM:
+      if (group != 32 && group != 64 && group != 128) return fail(HADQ_ERR_INVALID_ARG, "int4 group must be 32, 64 or 128");
+      if (sh.n % group != 0) return fail(HADQ_ERR_INVALID_ARG, "int4 group must divide n");
+      *eff_group = static_cast<int>(group);
+      return HADQ_OK;
+    case HADQ_INT8_SYM:
+      if (group != 0 && group != sh.n) return fail(HADQ_ERR_INVALID_ARG, "int8 is per token: group must be 0 or n");
+      if (sh.n > kMaxInt8N) return fail(HADQ_ERR_UNSUPPORTED, "per-token int8 supports n <= 32768");
+      if (sh.b <= 128 && (sh.n >> sh.logs) > 256) return fail(HADQ_ERR_UNSUPPORTED, "per-token int8: n / segment exceeds 256 threads");
+      *eff_group = static_cast<int>(sh.n);
+      return HADQ_OK;
+    case HADQ_MXFP4:
+      if (group != 0 && group != 32) return fail(HADQ_ERR_INVALID_ARG, "MXFP4 group must be 0 or 32");
+      if (sh.n % 32 != 0) return fail(HADQ_ERR_INVALID_ARG, "MXFP4 needs n to be a multiple of 32");
+      *eff_group = 32;
+      return HADQ_OK;
+    default:
+      return fail(HADQ_ERR_INVALID_ARG, "fmt must be HADQ_INT4_SYM, HADQ_INT8_SYM or HADQ_MXFP4");
+  }
+}
+
+int64_t codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt) {
+  return fmt == HADQ_INT8_SYM ? rows * n : rows * n / 2;
+}
+
+int64_t scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int group) {
+  switch (fmt) {
+    case HADQ_INT4_SYM: return rows * (n / group) * 2;
+    case HADQ_INT8_SYM: return rows * 4;
+    default: return rows * (n / 32);
+  }
+}
+
+// ------------------------------------------------------------ kernel tables
+
+using SegFn = void (*)(const void*, int64_t, int, float, int, void*, void*);
+using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, float*);
+using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*);
+using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*);
+
+template <int LOGS, bool BF>
+SegFn seg_fn(int mode) {
+  switch (mode) {
+    case hadq::OUT_F32: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_F32>;
+    case hadq::OUT_BF16: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_BF16>;
+    case hadq::OUT_INT4:
+      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_INT4>;
+      return nullptr;
+    default:
+      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_MXFP4>;
+      return nullptr;
+  }
+}
+
+template <bool BF>
+SegFn seg_fn_logs(int logs, int mode) {
+  switch (logs) {
+    case 3: return seg_fn<3, BF>(mode);
+    case 4: return seg_fn<4, BF>(mode);
+    case 5: return seg_fn<5, BF>(mode);
+    case 6: return seg_fn<6, BF>(mode);
+    default: return seg_fn<7, BF>(mode);
+  }
+}
+
+template <bool BF>
+SegRowFn seg_row_fn(int logs) {
+  switch (logs) {
+    case 3: return &hadq::segment_row_int8_kernel<3, BF>;
+    case 4: return &hadq::segment_row_int8_kernel<4, BF>;
+    case 5: return &hadq::segment_row_int8_kernel<5, BF>;
+    case 6: return &hadq::segment_row_int8_kernel<6, BF>;
+    default: return &hadq::segment_row_int8_kernel<7, BF>;
+  }
+}
+
+template <int LOGB, bool BF>
+TeamFn team_fn(int mode) {
+  switch (mode) {
+    case hadq::OUT_F32: return &hadq::team_kernel<LOGB, BF, hadq::OUT_F32>;
+    case hadq::OUT_BF16: return &hadq::team_kernel<LOGB, BF, hadq::OUT_BF16>;
+    case hadq::OUT_INT4: return &hadq::team_kernel<LOGB, BF, hadq::OUT_INT4>;
+    default: return &hadq::team_kernel<LOGB, BF, hadq::OUT_MXFP4>;
+  }
+}
+
+template <bool BF>
+TeamFn team_fn_logb(int logb, int mode) {
+  switch (logb) {
+    case 8: return team_fn<8, BF>(mode);
+    case 9: return team_fn<9, BF>(mode);
+    case 10: return team_fn<10, BF>(mode);
+    case 11: return team_fn<11, BF>(mode);
+    case 12: return team_fn<12, BF>(mode);
+    default: return team_fn<13, BF>(mode);
+  }
+}
+
+template <bool BF>
+TeamRowFn team_row_fn(int logb) {
+  switch (logb) {
+    case 8: return &hadq::team_row_int8_kernel<8, BF>;
+    case 9: return &hadq::team_row_int8_kernel<9, BF>;
+    case 10: return &hadq::team_row_int8_kernel<10, BF>;
+    case 11: return &hadq::team_row_int8_kernel<11, BF>;
+    case 12: return &hadq::team_row_int8_kernel<12, BF>;
+    default: return &hadq::team_row_int8_kernel<13, BF>;
+  }
+}
+
+// ------------------------------------------------- per-device launch caches
+
+std::mutex g_mu;
+std::map<int, int> g_sms;                                    // device -> SM count
+std::map<std::tuple<int, const void*, int, int>, int> g_occ; // (device, fn, block, smem) -> CTAs/SM
+
+hadq_status device_sms(int* sms, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_sms.find(dev);
+  if (it == g_sms.end()) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
+    it = g_sms.emplace(dev, v).first;
+  }
+  *sms = it->second;
+  *dev_out = dev;
+  return HADQ_OK;
+}
+
+// Resident CTAs per SM for `fn` at this block/smem size; also raises the
+// dynamic shared memory limit of `fn` on this device when it needs > 48 KB.
+hadq_status occupancy(const void* fn, int dev, int block, int smem, int* occ) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const auto key = std::make_tuple(dev, fn, block, smem);
+  auto it = g_occ.find(key);
+  if (it == g_occ.end()) {
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    }
+    int v = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, block, smem);
+    if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(e));
+    if (v < 1) return fail(HADQ_ERR_CUDA, "kernel does not fit on an SM");
+    it = g_occ.emplace(key, v).first;
+  }
+  *occ = it->second;
+  return HADQ_OK;
+}
+
+hadq_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return HADQ_OK;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Launch the kernel for an already validated call.  mode: hadq::OutMode, or
+// -1 for per-token int8.
+hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
+                   cudaStream_t stream) {
+  int sms = 0, dev = 0;
+  hadq_status st = device_sms(&sms, &dev);
+  if (st != HADQ_OK) return st;
+  const bool bf = x_dtype == HADQ_BF16;
+  (void)cudaGetLastError();   // launch errors below must be ours
+  if (mode >= 0) {
+    if (sh.b <= 128) {
+      SegFn fn = bf ? seg_fn_logs<true>(sh.logs, mode) : seg_fn_logs<false>(sh.logs, mode);
+      if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no kernel for this segment size and format");
+      const int64_t segs = sh.rows * (sh.n >> sh.logs);
+      int occ = 0;
+      st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, 0, &occ);
+      if (st != HADQ_OK) return st;
+      const int64_t grid = std::min<int64_t>(ceil_div(segs, hadq::kThreads), int64_t(sms) * occ);
+      fn<<<static_cast<unsigned>(grid), hadq::kThreads, 0, stream>>>(x, segs, sh.logb, sh.norm, group, out0, out1);
+      return check_launch("segment kernel launch");
+    }
+    TeamFn fn = bf ? team_fn_logb<true>(sh.logb, mode) : team_fn_logb<false>(sh.logb, mode);
+    const int smem = hadq::kThreads * 128 * 4;
+    int occ = 0;
+    st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, smem, &occ);
+    if (st != HADQ_OK) return st;
+    const int teams = hadq::kThreads >> (sh.logb - 7);
+    const int64_t units = sh.rows * (sh.n >> sh.logb);
+    const int64_t grid = std::min<int64_t>(ceil_div(units, teams), int64_t(sms) * occ);
+    fn<<<static_cast<unsigned>(grid), hadq::kThreads, smem, stream>>>(x, units, sh.norm, group, out0, out1);
+    return check_launch("team kernel launch");
+  }
+  // per-token int8
+  if (sh.b <= 128) {
+    SegRowFn fn = bf ? seg_row_fn<true>(sh.logs) : seg_row_fn<false>(sh.logs);
+    const int block = static_cast<int>(ceil_div(sh.n >> sh.logs, 32) * 32);
+    int occ = 0;
+    st = occupancy(reinterpret_cast<const void*>(fn), dev, block, 0, &occ);
+    if (st != HADQ_OK) return st;
+    const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
+    fn<<<static_cast<unsigned>(grid), block, 0, stream>>>(x, sh.rows, sh.n, sh.logb, sh.norm,
+                                                           static_cast<int8_t*>(out0), static_cast<float*>(out1));
+    return check_launch("per-token int8 kernel launch");
+  }
+  TeamRowFn fn = bf ? team_row_fn<true>(sh.logb) : team_row_fn<false>(sh.logb);
+  const int block = static_cast<int>(ceil_div(sh.n >> 7, 32) * 32);
+  const int smem = static_cast<int>(sh.n * 4);
+  int occ = 0;
+  st = occupancy(reinterpret_cast<const void*>(fn), dev, block, smem, &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
+  fn<<<static_cast<unsigned>(grid), block, smem, stream>>>(x, sh.rows, sh.n, sh.norm, static_cast<int8_t*>(out0),
+                                                           static_cast<float*>(out1));
+  return check_launch("per-token int8 kernel launch");
+}
+
+hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,
+                        hadq_dtype out_dtype, void* stream) {
+  g_last_error.clear();
+  Shape sh;
+  hadq_status st = check_shape(x_dtype, rows, n, block, &sh);
+  if (st != HADQ_OK) return st;
+  if (out_dtype != HADQ_F32 && out_dtype != HADQ_BF16) return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_F32 or HADQ_BF16");
+  if (rows == 0) return HADQ_OK;
+  if (x == nullptr || out == nullptr) return fail(HADQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(out)) return fail(HADQ_ERR_MISALIGNED, "x and out must be 16-byte aligned");
+  const Span sx = span(x, rows * n * esize(x_dtype));
+  const Span so = span(out, rows * n * esize(out_dtype));
+  if (overlaps(sx, so) && !(x == out && x_dtype == out_dtype))
+    return fail(HADQ_ERR_INVALID_ARG, "out overlaps x (only exact in-place with equal dtypes is allowed)");
+  return launch(x, x_dtype, sh, out_dtype == HADQ_F32 ? hadq::OUT_F32 : hadq::OUT_BF16, 0, out, nullptr,
+                static_cast<cudaStream_t>(stream));
+}
+
+hadq_status quant_checks(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, hadq_fmt fmt,
+                         int64_t group, const void* codes, const void* scales, Shape* sh, int* g) {
+  hadq_status st = check_shape(x_dtype, rows, n, block, sh);
+  if (st != HADQ_OK) return st;
+  st = check_quant(fmt, group, *sh, g);
+  if (st != HADQ_OK) return st;
+  if (rows == 0) return HADQ_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return fail(HADQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales))
+    return fail(HADQ_ERR_MISALIGNED, "x, codes and scales must be 16-byte aligned");
+  const Span sx = span(x, rows * n * esize(x_dtype));
+  const Span sc = span(codes, codes_bytes(rows, n, fmt));
+  const Span ss = span(scales, scales_bytes(rows, n, fmt, *g));
+  if (overlaps(sx, sc) || overlaps(sx, ss) || overlaps(sc, ss))
+    return fail(HADQ_ERR_INVALID_ARG, "x, codes and scales must not overlap");
+  return HADQ_OK;
+}
+
+int quant_mode(hadq_fmt fmt) {
+  return fmt == HADQ_INT4_SYM ? hadq::OUT_INT4 : fmt == HADQ_MXFP4 ? hadq::OUT_MXFP4 : -1;
+}
+
+}  // namespace
+
+extern "C" {
+
+hadq_status hadq_rotate(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,
+                        hadq_dtype out_dtype, void* stream) {
+  return rotate_impl(x, x_dtype, rows, n, block, out, out_dtype, stream);
+}
+
+hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,
+                                hadq_dtype out_dtype, void* stream) {
+  return rotate_impl(x, x_dtype, rows, n, block, out, out_dtype, stream);
+}
+
+hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, hadq_fmt fmt,
+                              int64_t group, void* codes, void* scales, void* stream) {
+  g_last_error.clear();
+  Shape sh;
+  int g = 0;
+  hadq_status st = quant_checks(x, x_dtype, rows, n, block, fmt, group, codes, scales, &sh, &g);
+  if (st != HADQ_OK || rows == 0) return st;
+  return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                   hadq_fmt fmt, int64_t group, void* codes_host, void* scales_host, void* x_dev,
+                                   void* codes_dev, void* scales_dev, void* stream) {
+  g_last_error.clear();
+  Shape sh;
+  int g = 0;
+  hadq_status st = quant_checks(x_dev, x_dtype, rows, n, block, fmt, group, codes_dev, scales_dev, &sh, &g);
+  if (st != HADQ_OK || rows == 0) return st;
+  if (x_host == nullptr || codes_host == nullptr || scales_host == nullptr)
+    return fail(HADQ_ERR_INVALID_ARG, "null host pointer");
+  if (!aligned16(x_host) || !aligned16(codes_host) || !aligned16(scales_host))
+    return fail(HADQ_ERR_MISALIGNED, "host buffers must be 16-byte aligned");
+  const int64_t xb = rows * n * esize(x_dtype), cb = codes_bytes(rows, n, fmt), sb = scales_bytes(rows, n, fmt, g);
+  const Span hx = span(x_host, xb), hc = span(codes_host, cb), hs = span(scales_host, sb);
+  if (overlaps(hx, hc) || overlaps(hx, hs) || overlaps(hc, hs))
+    return fail(HADQ_ERR_INVALID_ARG, "host x, codes and scales must not overlap");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(xb), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy x to device: ") + cudaGetErrorString(e));
+  st = launch(x_dev, x_dtype, sh, quant_mode(fmt), g, codes_dev, scales_dev, s);
+  if (st != HADQ_OK) return st;
+  e = cudaMemcpyAsync(codes_host, codes_dev, static_cast<size_t>(cb), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy codes to host: ") + cudaGetErrorString(e));
+  e = cudaMemcpyAsync(scales_host, scales_dev, static_cast<size_t>(sb), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy scales to host: ") + cudaGetErrorString(e));
+  return HADQ_OK;
+}
+
+int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt) {
+  if (rows < 0 || n <= 0 || n % 2 != 0) return 0;
+  if (fmt != HADQ_INT4_SYM && fmt != HADQ_INT8_SYM && fmt != HADQ_MXFP4) return 0;
+  return codes_bytes(rows, n, fmt);
+}
+
+int64_t hadq_scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int64_t group) {
+  if (rows < 0 || n <= 0) return 0;
+  switch (fmt) {
+    case HADQ_INT4_SYM:
+      if ((group != 32 && group != 64 && group != 128) || n % group != 0) return 0;
+      return scales_bytes(rows, n, fmt, static_cast<int>(group));
+    case HADQ_INT8_SYM:
+      return (group == 0 || group == n) ? rows * 4 : 0;
+    case HADQ_MXFP4:
+      return ((group == 0 || group == 32) && n % 32 == 0) ? rows * (n / 32) : 0;
+    default:
+      return 0;
+  }
+}
+
+const char* hadq_status_string(hadq_status status) {
+  switch (status) {
+    case HADQ_OK: return "ok";
+    case HADQ_ERR_INVALID_ARG: return "invalid argument";
+    case HADQ_ERR_UNSUPPORTED: return "unsupported size or format";
+    case HADQ_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case HADQ_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+const char* hadq_last_error(void) { return g_last_error.c_str(); }
+
+int hadq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+"""ctypes binding for libhadq (include/hadq.h).  Argument marshalling only.
+
+The entry points keep the C names.  Tensors are passed as raw device
+pointers; every step of the rotation and quantization runs in libhadq's CUDA
+kernels.  There is no fallback: if ``libhadq.so`` is missing or the CUDA call
+fails, a ``HadqError`` is raised.
+
+    codes, scales = hadq_rotate_quant(x, block=0, fmt="int4", group=128)
+
+``x`` is any contiguous fp32 / bf16 CUDA tensor; its last dimension is n
+(the rotated dimension), all leading dimensions are rows.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhadq.so")
+
+HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
+HADQ_F32, HADQ_BF16 = 0, 1
+FMTS = {"int4": 0, "int8": 1, "mxfp4": 2}
+EXPORTS = (
+    "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
+    "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class HadqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libhadq status {status}: {message}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libhadq.so once and declare the C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise HadqError(-1, f"{path} is not built; run `python -m hadamard_rotation_bit_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        lib.hadq_rotate.argtypes = [vp, i32, i64, i64, i64, vp, i32, vp]
+        lib.hadq_rotate_inverse.argtypes = [vp, i32, i64, i64, i64, vp, i32, vp]
+        lib.hadq_rotate_quant.argtypes = [vp, i32, i64, i64, i64, i32, i64, vp, vp, vp]
+        lib.hadq_rotate_quant_host.argtypes = [vp, i32, i64, i64, i64, i32, i64, vp, vp, vp, vp, vp, vp]
+        for f in ("hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host"):
+            getattr(lib, f).restype = i32
+        lib.hadq_codes_bytes.argtypes = [i64, i64, i32]
+        lib.hadq_codes_bytes.restype = i64
+        lib.hadq_scales_bytes.argtypes = [i64, i64, i32, i64]
+        lib.hadq_scales_bytes.restype = i64
+        lib.hadq_status_string.argtypes = [i32]
+        lib.hadq_status_string.restype = ctypes.c_char_p
+        lib.hadq_last_error.argtypes = []
+        lib.hadq_last_error.restype = ctypes.c_char_p
+        lib.hadq_version.argtypes = []
+        lib.hadq_version.restype = i32
+        _lib = lib
+        return lib
+
+
+def _check(status: int) -> None:
+    if status != HADQ_OK:
+        lib = load_library()
+        msg = lib.hadq_last_error().decode() or lib.hadq_status_string(status).decode()
+        raise HadqError(status, msg)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return HADQ_F32
+    if t == torch.bfloat16:
+        return HADQ_BF16
+    raise HadqError(HADQ_ERR_INVALID_ARG, f"unsupported dtype {t} (float32 or bfloat16)")
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _rows_n(x: torch.Tensor):
+    if not x.is_contiguous():
+        raise HadqError(HADQ_ERR_INVALID_ARG, "tensors must be contiguous")
+    n = x.shape[-1] if x.dim() else 1
+    return (x.numel() // n if n else 0), n
+
+
+def codes_nbytes(rows: int, n: int, fmt: str) -> int:
+    return int(load_library().hadq_codes_bytes(rows, n, FMTS[fmt]))
+
+
+def scales_nbytes(rows: int, n: int, fmt: str, group: int) -> int:
+    return int(load_library().hadq_scales_bytes(rows, n, FMTS[fmt], group))
+
+
+def output_shapes(rows: int, n: int, fmt: str, group: int):
+    """(codes shape, codes dtype, scales shape, scales dtype) of hadq_rotate_quant."""
+    if fmt == "int4":
+        return (rows, n // 2), torch.uint8, (rows, n // group), torch.float16
+    if fmt == "int8":
+        return (rows, n), torch.int8, (rows,), torch.float32
+    if fmt == "mxfp4":
+        return (rows, n // 2), torch.uint8, (rows, n // 32), torch.uint8
+    raise HadqError(HADQ_ERR_INVALID_ARG, f"unknown fmt {fmt!r}")
+
+
+def hadq_rotate(x: torch.Tensor, block: int = 0, out: torch.Tensor | None = None,
+                out_dtype: torch.dtype | None = None, stream=None) -> torch.Tensor:
+    """out = x . diag(H_b) / sqrt(b) along the last dimension (see include/hadq.h)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _check(lib.hadq_rotate(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, out.data_ptr(),
+                           _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+def hadq_rotate_inverse(x: torch.Tensor, block: int = 0, out: torch.Tensor | None = None,
+                        out_dtype: torch.dtype | None = None, stream=None) -> torch.Tensor:
+    """Inverse rotation (the same symmetric, involutory operation)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _check(lib.hadq_rotate_inverse(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, out.data_ptr(),
+                                   _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+def hadq_rotate_quant(x: torch.Tensor, block: int = 0, fmt: str = "int4", group: int = 128,
+                      codes: torch.Tensor | None = None, scales: torch.Tensor | None = None, stream=None):
+    """Rotate and quantize in one pass; returns (codes, scales) (see include/hadq.h)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    cs, cd, ss, sd = output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=x.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=x.device)
+    _check(lib.hadq_rotate_quant(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, FMTS[fmt], group,
+                                 codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
+    return codes, scales
+
+
+def hadq_rotate_quant_host(x_host: torch.Tensor, block: int, fmt: str, group: int,
+                           codes_host: torch.Tensor, scales_host: torch.Tensor,
+                           x_dev: torch.Tensor, codes_dev: torch.Tensor, scales_dev: torch.Tensor,
+                           stream=None) -> None:
+    """Host-buffer form: copy in, rotate+quantize, copy out, all enqueued on `stream`."""
+    lib = load_library()
+    rows, n = _rows_n(x_host)
+    _check(lib.hadq_rotate_quant_host(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt], group,
+                                      codes_host.data_ptr(), scales_host.data_ptr(), x_dev.data_ptr(),
+                                      codes_dev.data_ptr(), scales_dev.data_ptr(), _stream_handle(stream)))

@@ -150,11 +150,19 @@ def _chunk_values(key: str, chunk: int, seed: int) -> np.ndarray:
     raise KeyError(key)
 
 
-def generate(key: str, rows: slice | None = None, seed: int = SEED) -> np.ndarray:
+def _chunk_stored(key: str, chunk: int, seed: int) -> np.ndarray:
+    vals = _chunk_values(key, chunk, seed).astype(np.float32)
+    return vals if WORKLOADS[key].x_dtype == "f32" else f32_to_bf16_bits(vals)
+
+
+def generate(key: str, rows: slice | None = None, seed: int = SEED, workers: int = 1) -> np.ndarray:
     """Stored input for rows ``rows`` of workload ``key``.
 
     Returns float32 values for fp32 workloads and uint16 bf16 bit patterns for
-    bf16 workloads, shape (len(rows), n), row-major.
+    bf16 workloads, shape (len(rows), n), row-major.  ``workers > 1``
+    generates the chunks in a pool of spawned processes (spawned, not forked,
+    so it is safe after CUDA has been initialised); the bits do not depend on
+    the worker count.
     """
     w = WORKLOADS[key]
     r = range(w.rows)[rows if rows is not None else slice(None)]
@@ -163,13 +171,22 @@ def generate(key: str, rows: slice | None = None, seed: int = SEED) -> np.ndarra
     out = np.empty((len(r), w.n), dtype=np.float32 if w.x_dtype == "f32" else np.uint16)
     if len(r) == 0:
         return out
-    c0, c1 = r.start // CHUNK_ROWS, (r.stop - 1) // CHUNK_ROWS
-    for c in range(c0, c1 + 1):
-        vals = _chunk_values(key, c, seed).astype(np.float32)
+    chunks = list(range(r.start // CHUNK_ROWS, (r.stop - 1) // CHUNK_ROWS + 1))
+
+    def place(c, stored):
         lo = max(r.start, c * CHUNK_ROWS)
-        hi = min(r.stop, c * CHUNK_ROWS + vals.shape[0])
-        part = vals[lo - c * CHUNK_ROWS: hi - c * CHUNK_ROWS]
-        out[lo - r.start: hi - r.start] = part if w.x_dtype == "f32" else f32_to_bf16_bits(part)
+        hi = min(r.stop, c * CHUNK_ROWS + stored.shape[0])
+        out[lo - r.start: hi - r.start] = stored[lo - c * CHUNK_ROWS: hi - c * CHUNK_ROWS]
+
+    if workers > 1 and len(chunks) > 1:
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+        with ProcessPoolExecutor(max_workers=min(workers, len(chunks)), mp_context=mp.get_context("spawn")) as ex:
+            for c, stored in zip(chunks, ex.map(_chunk_stored, [key] * len(chunks), chunks, [seed] * len(chunks))):
+                place(c, stored)
+    else:
+        for c in chunks:
+            place(c, _chunk_stored(key, c, seed))
     return out
 
 

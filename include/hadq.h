@@ -1,0 +1,153 @@
+/*
+ * libhadq -- online Hadamard rotation of activations, fused with the
+ * round-to-nearest quantizer that consumes them.  CUDA, sm_100a (B200).
+ *
+ * Operation (every entry point): each row x of a row-major [rows x n] matrix
+ * becomes y = x . diag(H_b, ..., H_b) / sqrt(b), where H_b is the Sylvester
+ * Hadamard matrix built by the doubling H -> [[H, H], [H, -H]] in natural
+ * order ("Rotation Transform", AutoRound docs, section 1.5 "Deterministic vs
+ * random Hadamard") and b is the rotation block: b = n for a full rotation,
+ * or a power of 2 dividing n for the block-diagonal rotation_size / per-Linear
+ * block_size modes (same page, sections 1.2 and 2.1; block 0 or n means full,
+ * as block_size None / -1 does there).  The positions that apply it online --
+ * R1 residual stream, R3 per-head Q/K after RoPE, R4 down_proj input -- are
+ * section 1.1 of that page; the rows are "arbitrary leading dimensions, final
+ * dimension = in_features" ("orbitquant 0.2.0", Quantize An Instantiated
+ * Module).  H_b / sqrt(b) is symmetric and its own inverse.
+ *
+ * Conventions shared by all entry points
+ *   - Device pointers unless the name says host.  All pointers must be
+ *     16-byte aligned (HADQ_ERR_MISALIGNED otherwise).
+ *   - Rows are contiguous with stride n elements.
+ *   - rows == 0 is a valid empty call: nothing is launched, HADQ_OK.
+ *   - Supported sizes: 1 <= b <= 8192, b a power of 2; n a multiple of 8
+ *     and of b; a full rotation needs n itself to be a power of 2 <= 8192.
+ *     Larger b returns HADQ_ERR_UNSUPPORTED.
+ *   - The caller owns every buffer; the library allocates nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  The caller synchronizes before reading results.
+ *   - All argument checks run on the host before anything is launched.  A
+ *     failing call launches nothing and leaves every output untouched (the
+ *     validate-then-apply rule of the apply_spinquant docstring).  There is
+ *     no CPU fallback and no alternative backend.
+ *   - Non-finite inputs give unspecified (but memory-safe) outputs.
+ *   - hadq_last_error() gives a one-line reason for the calling thread's
+ *     most recent failure.
+ */
+#ifndef HADQ_H
+#define HADQ_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HADQ_API __attribute__((visibility("default")))
+#else
+#define HADQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hadq_status {
+  HADQ_OK = 0,
+  HADQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad block/group, overlapping buffers */
+  HADQ_ERR_UNSUPPORTED = 2,   /* valid by the definition but outside what the kernels cover */
+  HADQ_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+  HADQ_ERR_CUDA = 4           /* the CUDA runtime reported an error at launch or copy */
+} hadq_status;
+
+typedef enum hadq_dtype {
+  HADQ_F32 = 0,               /* IEEE binary32 */
+  HADQ_BF16 = 1               /* bfloat16 (stored as 16-bit patterns) */
+} hadq_dtype;
+
+typedef enum hadq_fmt {
+  HADQ_INT4_SYM = 0,          /* symmetric int4 RTN per group, fp16 scales */
+  HADQ_INT8_SYM = 1,          /* symmetric int8 RTN per token (row), fp32 scale */
+  HADQ_MXFP4 = 2              /* E2M1 codes, E8M0 shared exponent per 32 */
+} hadq_fmt;
+
+/*
+ * hadq_rotate: out = x . diag(H_b) / sqrt(b), rotation only.
+ *   x        [rows x n] of x_dtype (read only)
+ *   out      [rows x n] of out_dtype; out == x (in place) is allowed when the
+ *            dtypes match, any other overlap is HADQ_ERR_INVALID_ARG
+ *   block    0 or n = full rotation, else a power of 2 dividing n
+ * Values are computed in fp32 (butterfly of fp32 adds, one fp32 scaling by
+ * fp32(1/sqrt(b))); bf16 output is rounded to nearest even.
+ */
+HADQ_API hadq_status hadq_rotate(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                        void* out, hadq_dtype out_dtype, void* stream);
+
+/*
+ * hadq_rotate_inverse: the inverse rotation.  H_b / sqrt(b) is symmetric and
+ * involutory (H H^T = b I), so this is the same operation as hadq_rotate;
+ * rotating twice returns x up to fp32 rounding ("Rotation Transform",
+ * introduction: R R^T = I).
+ */
+HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                void* out, hadq_dtype out_dtype, void* stream);
+
+/*
+ * hadq_rotate_quant: rotate, then quantize with round-to-nearest, in one pass
+ * (each input byte read once, codes and scales written once).  The quantizer
+ * is the RTN of "Pre-Process (Rotation Preprocessing)" (Workflow note: wbits,
+ * groupsize, sym) or the MXFP4 target of "Rotation Transform" (introduction,
+ * section 2.1).  With y the rotated row and m the absmax of a group:
+ *
+ *   HADQ_INT4_SYM  group in {32, 64, 128}, group | n.
+ *                  scale s = fp16_rne(m / 7) (fp32 m / 7, then to fp16);
+ *                  q = clamp(rne(y / s), -7, 7); s == 0 or inf -> q = 0.
+ *                  codes:  [rows x n/2] bytes, two's-complement nibbles,
+ *                          element 2i in the low nibble of byte i.
+ *                  scales: [rows x n/group] fp16.
+ *   HADQ_INT8_SYM  per token: group must be 0 or n; n <= 32768.
+ *                  s = fp32(m / 127); q = clamp(rne(y / s), -127, 127).
+ *                  codes:  [rows x n] int8.   scales: [rows] fp32.
+ *   HADQ_MXFP4     group must be 0 or 32; n a multiple of 32.
+ *                  e = clamp(floor(log2 m) - 2, -127, 127) (m == 0 -> -127);
+ *                  code = E2M1 rne(y / 2^e), saturating at +/-6, sign bit 3.
+ *                  codes:  [rows x n/2] bytes, element 2i in the low nibble.
+ *                  scales: [rows x n/32] bytes = e + 127 (E8M0).
+ *
+ * Codes are computed from the fp32 rotation with the stored scale; the
+ * product y * (1/s) is rounded once (fused multiply-add onto the integer grid).
+ * codes and scales must not overlap x or each other.
+ */
+HADQ_API hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                              hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream);
+
+/*
+ * hadq_rotate_quant_host: the same operation on HOST buffers.  Enqueues on
+ * `stream`: copy x_host -> x_dev, hadq_rotate_quant on the device buffers,
+ * copy codes_dev -> codes_host and scales_dev -> scales_host.  The caller
+ * provides the device staging buffers (sizes as for hadq_rotate_quant) and
+ * synchronizes `stream` before reading the host outputs.  Host buffers
+ * should be page-locked for the copies to be asynchronous.  Argument checks
+ * cover both the host and the device buffers and run before anything is
+ * enqueued.
+ */
+HADQ_API hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                   hadq_fmt fmt, int64_t group, void* codes_host, void* scales_host,
+                                   void* x_dev, void* codes_dev, void* scales_dev, void* stream);
+
+/* Bytes of the code and scale outputs of hadq_rotate_quant for these sizes
+ * (0 for an invalid combination). */
+HADQ_API int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt);
+HADQ_API int64_t hadq_scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int64_t group);
+
+/* Static description of a status code. */
+HADQ_API const char* hadq_status_string(hadq_status status);
+
+/* One-line reason for the calling thread's most recent failed call ("" if none). */
+HADQ_API const char* hadq_last_error(void);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+HADQ_API int hadq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HADQ_H */

@@ -1,0 +1,129 @@
+"""libhadq host-side behaviour that needs no GPU.
+
+The library must load, export every function include/hadq.h declares, and
+reject bad arguments on the host -- before any CUDA call -- with the right
+status.  Only argument combinations that fail validation (or are empty) are
+called here, so nothing reaches the device.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from hadamard_rotation_bit_b200 import build as hbuild
+from hadamard_rotation_bit_b200 import hadq as H
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+A = 0x10000          # a fake, 16-byte aligned device address (never dereferenced)
+B = 0x20000000
+C = 0x40000000
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return H.load_library()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "hadq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hadq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 9
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(names) == sorted(H.EXPORTS)
+
+
+def test_status_strings_and_version(lib):
+    for st in range(5):
+        assert lib.hadq_status_string(st)
+    assert lib.hadq_version() == 100
+
+
+def _q(lib, x=A, xd=1, rows=4, n=1024, block=0, fmt=0, group=128, codes=B, scales=C):
+    return lib.hadq_rotate_quant(x, xd, rows, n, block, fmt, group, codes, scales, None)
+
+
+def _r(lib, x=A, xd=1, rows=4, n=1024, block=0, out=B, od=0):
+    return lib.hadq_rotate(x, xd, rows, n, block, out, od, None)
+
+
+def test_empty_calls_are_noops(lib):
+    assert _q(lib, rows=0, x=None, codes=None, scales=None) == H.HADQ_OK
+    assert _r(lib, rows=0, x=None, out=None) == H.HADQ_OK
+    assert lib.hadq_rotate_inverse(None, 0, 0, 64, 0, None, 0, None) == H.HADQ_OK
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(rows=-1), H.HADQ_ERR_INVALID_ARG),
+    (dict(n=0), H.HADQ_ERR_INVALID_ARG),
+    (dict(n=1000), H.HADQ_ERR_INVALID_ARG),              # full rotation of a non-power-of-2
+    (dict(block=96), H.HADQ_ERR_INVALID_ARG),            # block not a power of 2
+    (dict(n=896, block=256), H.HADQ_ERR_INVALID_ARG),    # block does not divide n
+    (dict(n=16384), H.HADQ_ERR_UNSUPPORTED),             # full rotation above 8192
+    (dict(block=-2), H.HADQ_ERR_INVALID_ARG),
+    (dict(xd=7), H.HADQ_ERR_INVALID_ARG),
+    (dict(group=48), H.HADQ_ERR_INVALID_ARG),
+    (dict(group=256), H.HADQ_ERR_INVALID_ARG),
+    (dict(fmt=9), H.HADQ_ERR_INVALID_ARG),
+    (dict(fmt=1, group=64), H.HADQ_ERR_INVALID_ARG),     # int8 is per token
+    (dict(fmt=1, group=0, n=65536, block=128), H.HADQ_ERR_UNSUPPORTED),
+    (dict(fmt=2, group=16), H.HADQ_ERR_INVALID_ARG),
+    (dict(x=None), H.HADQ_ERR_INVALID_ARG),
+    (dict(codes=None), H.HADQ_ERR_INVALID_ARG),
+    (dict(x=A + 8), H.HADQ_ERR_MISALIGNED),
+    (dict(scales=C + 2), H.HADQ_ERR_MISALIGNED),
+    (dict(codes=A + 16), H.HADQ_ERR_INVALID_ARG),        # codes overlap x
+    (dict(scales=B + 64), H.HADQ_ERR_INVALID_ARG),       # scales overlap codes
+    (dict(rows=2 ** 62), H.HADQ_ERR_INVALID_ARG),        # rows * n overflows
+])
+def test_rotate_quant_validation(lib, kw, status):
+    assert _q(lib, **kw) == status
+    assert lib.hadq_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(od=5), H.HADQ_ERR_INVALID_ARG),
+    (dict(out=None), H.HADQ_ERR_INVALID_ARG),
+    (dict(out=A + 64), H.HADQ_ERR_INVALID_ARG),          # partial overlap
+    (dict(out=A, od=0, xd=1), H.HADQ_ERR_INVALID_ARG),   # in place with different dtypes
+    (dict(out=B + 4), H.HADQ_ERR_MISALIGNED),
+    (dict(n=12, block=4), H.HADQ_ERR_UNSUPPORTED),       # n not a multiple of 8
+])
+def test_rotate_validation(lib, kw, status):
+    assert _r(lib, **kw) == status
+
+
+def test_host_entry_point_validation(lib):
+    f = lib.hadq_rotate_quant_host
+    # valid device side, bad host side
+    assert f(None, 1, 4, 1024, 0, 0, 128, A, B, A, B, C, None) == H.HADQ_ERR_INVALID_ARG
+    assert f(A + 4, 1, 4, 1024, 0, 0, 128, B, C, A, B, C, None) == H.HADQ_ERR_MISALIGNED
+    # bad device side
+    assert f(A, 1, 4, 1024, 0, 0, 128, B, C, A + 8, B, C, None) == H.HADQ_ERR_MISALIGNED
+    assert f(A, 1, 0, 1024, 0, 0, 128, B, C, None, None, None, None) == H.HADQ_OK
+
+
+def test_output_size_helpers(lib):
+    assert lib.hadq_codes_bytes(4096, 4096, 0) == 4096 * 2048
+    assert lib.hadq_scales_bytes(4096, 4096, 0, 128) == 4096 * 32 * 2
+    assert lib.hadq_codes_bytes(8192, 14336, 1) == 8192 * 14336
+    assert lib.hadq_scales_bytes(8192, 14336, 1, 0) == 8192 * 4
+    assert lib.hadq_codes_bytes(65536, 8192, 2) == 65536 * 4096
+    assert lib.hadq_scales_bytes(65536, 8192, 2, 32) == 65536 * 256
+    assert lib.hadq_scales_bytes(4, 100, 0, 128) == 0
+    assert lib.hadq_codes_bytes(4, 64, 7) == 0
+
+
+def test_binding_raises_without_cuda_tensor(lib):
+    import torch
+    with pytest.raises(H.HadqError):
+        H.hadq_rotate_quant(torch.zeros(4, 96, dtype=torch.float64), 0, "int4", 32)
