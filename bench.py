@@ -8,12 +8,14 @@ Sylvester Hadamard, symmetric int4 RTN per group of 128 with fp16 scales.
 The metric is GB/s of algorithmic traffic (input read once + codes and scales
 written once) and its fraction of the measured HBM copy bandwidth.
 
-Timing: inputs resident in HBM; 8 buffer sets (input + outputs) are rotated so
-each step touches data last used 7 steps earlier (336 MB > L2).  The K steps
-are captured in one CUDA graph together with a CUDA event pair around every
-launch; the graph is replayed once untimed and once timed between barriers
+Timing: inputs resident in HBM; for C2, 8 buffer sets (input + outputs) are
+rotated so each step touches data last used 7 steps earlier (338 MB > L2).  The K steps
+are captured back to back in one CUDA graph; the graph is replayed once
+untimed and once timed (CUDA events on the launching stream) between barriers
 and device synchronisations.  `value` = bytes of all ranks / max-over-ranks
-elapsed time; `roofline.achieved` = bytes per launch / mean event duration.
+elapsed time; `roofline.achieved` = bytes per launch / mean launch interval
+(kernel plus inter-kernel gap).  A median over per-launch event pairs (queued
+behind a sleep kernel) is reported beside it.
 `e2e` repeats the metric through hadq_rotate_quant_host (pinned host input,
 copies in and out inside the timed region).
 
@@ -41,11 +43,15 @@ sys.path.insert(0, ROOT)
 
 from hadamard_rotation_bit_b200 import workloads as W  # noqa: E402
 
-WORKLOAD = W.WORKLOADS["c2"]
 METRIC = "fused Hadamard+quant GB/s and % of B200 HBM peak (4096x4096 bf16->int4 g128)"
 UNIT = "GB/s"
-NBUF = 8
+L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+
+# A step is one pass of the fused path over one batch of a workload: the
+# launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
+STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"]}
+WORKLOAD = W.WORKLOADS["c2"]
 
 
 def _env_int(k, d):
@@ -55,11 +61,28 @@ def _env_int(k, d):
         return d
 
 
-def config_block():
-    w = WORKLOAD
-    return {"workload": w.name, "rows": w.rows, "n": w.n, "block": w.block, "fmt": w.fmt, "group": w.group,
-            "x_dtype": w.x_dtype, "algorithmic_bytes_per_step": w.algorithmic_bytes,
-            "l2": f"{NBUF} rotating buffer sets ({NBUF * w.algorithmic_bytes / 1e6:.0f} MB > L2 126 MB)"}
+def step_bytes(cfg):
+    return sum(W.WORKLOADS[k].algorithmic_bytes for k in STEP_PARTS[cfg])
+
+
+def n_buffers(cfg):
+    """Distinct buffer sets rotated through so that every step reads data not
+    touched for at least ~3 L2 capacities (or inputs larger than L2)."""
+    return int(max(1, min(8, -(-3 * L2_BYTES // step_bytes(cfg)))))
+
+
+def config_block(cfg="c2"):
+    parts = [W.WORKLOADS[k] for k in STEP_PARTS[cfg]]
+    nb = n_buffers(cfg)
+    d = {"workload": " + ".join(w.name for w in parts), "algorithmic_bytes_per_step": step_bytes(cfg),
+         "l2": (f"inputs larger than L2 ({step_bytes(cfg) / 1e6:.0f} MB per step)" if nb == 1 else
+                f"{nb} rotating buffer sets ({nb * step_bytes(cfg) / 1e6:.0f} MB > L2 126 MB)"
+                if nb * step_bytes(cfg) > L2_BYTES else
+                f"{nb} buffer sets, {nb * step_bytes(cfg) / 1e6:.1f} MB: L2-resident (parity-size config)")}
+    if len(parts) == 1:
+        w = parts[0]
+        d.update({"rows": w.rows, "n": w.n, "block": w.block, "fmt": w.fmt, "group": w.group, "x_dtype": w.x_dtype})
+    return d
 
 
 def measured_peak():
@@ -165,11 +188,18 @@ def barrier(dist):
 
 
 def max_over_ranks(dist, v):
+    """Largest value over all ranks (device timings are reduced with MAX)."""
     if dist is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(bytes_per_step, steps, world, elapsed_max_s):
+    """Whole-job throughput: bytes every rank processed / the slowest rank's time."""
+    return bytes_per_step * steps * world / elapsed_max_s / 1e9
 
 
 def cpu_baseline(seconds=12.0):
@@ -213,7 +243,7 @@ def run_reference(args):
     cores = len(os.sched_getaffinity(0))
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps, "warmup": warm,
             "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "config": config_block(), "impl": "reference",
+            "dtype": "f64", "data": "synthetic", "config": config_block("c2"), "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{rows} rows of the 4096x4096 batch per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -222,87 +252,134 @@ def run_reference(args):
         dist.destroy_process_group()
 
 
+def _device_input(key, seed, dev, workers):
+    w = W.WORKLOADS[key]
+    stored = W.generate(key, seed=seed, workers=workers)
+    if w.x_dtype == "bf16":
+        return stored, torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).to(dev)
+    return stored, torch.from_numpy(stored).to(dev)
+
+
 def run_hadq(args):
     from hadamard_rotation_bit_b200 import hadq as H
     dist, rank, world, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     H.load_library()
-    w = WORKLOAD
+    cfg = args.config
+    keys = STEP_PARTS[cfg]
     steps, warm = args.steps, max(3, args.warmup)
+    nbuf = n_buffers(cfg)
+    workers = max(1, min(16, (os.cpu_count() or 2) // 2))
 
-    stored = W.generate("c2", seed=W.rank_seed(rank))
-    x0 = torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).to(dev)
-    xs = [x0.clone() for _ in range(NBUF)]
-    outs = [H.hadq_rotate_quant(xs[i], 0, "int4", 128) for i in range(NBUF)]   # allocates outputs, warms caches
+    host, bufs = {}, []
+    for k in keys:
+        host[k], x0 = _device_input(k, W.rank_seed(rank), dev, workers)
+        bufs.append([x0] + [x0.clone() for _ in range(nbuf - 1)])
+
+    def launch(j, i, stream=None, outs=None):
+        w = W.WORKLOADS[keys[j]]
+        x = bufs[j][i % nbuf]
+        if w.fmt is None:
+            o = None if outs is None else outs[j][i % nbuf]
+            return H.hadq_rotate(x, w.block, out=o, stream=stream,
+                                 out_dtype=torch.bfloat16 if w.out_dtype == "bf16" else torch.float32)
+        c, sc = (None, None) if outs is None else outs[j][i % nbuf]
+        return H.hadq_rotate_quant(x, w.block, w.fmt, w.group, codes=c, scales=sc, stream=stream)
+
+    outs = [[launch(j, i) for i in range(nbuf)] for j in range(len(keys))]   # allocate outputs, warm caches
     torch.cuda.synchronize()
-    bytes_step = w.algorithmic_bytes
-
+    bytes_step = step_bytes(cfg)
     stream = torch.cuda.Stream(device=dev)
 
     def step(i):
-        c, s = outs[i % NBUF]
-        H.hadq_rotate_quant(xs[i % NBUF], 0, "int4", 128, codes=c, scales=s, stream=stream)
+        for j in range(len(keys)):
+            launch(j, i, stream, outs)
 
     with torch.cuda.stream(stream):
         for i in range(warm):
             step(i)
     stream.synchronize()
 
-    # K launches with an event pair around each, captured in one graph.
-    ev_s = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
+    # K back-to-back steps captured in one CUDA graph, replayed on `stream`.
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for i in range(steps):
-            ev_s[i].record(stream)
             step(i)
-            ev_e[i].record(stream)
-    g.replay()                       # untimed replay (warm-up of the graph itself)
+    with torch.cuda.stream(stream):
+        g.replay()                       # untimed replay (warm-up of the graph itself)
     stream.synchronize()
 
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(dist)
     with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        g.replay()
-        t_end.record(stream)
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            g.replay()
+            t_end.record(stream)
         stream.synchronize()
     barrier(dist)
     elapsed = t_start.elapsed_time(t_end) / 1e3
-    per_launch = [ev_s[i].elapsed_time(ev_e[i]) / 1e3 for i in range(steps)]
-    kernel_s = sum(per_launch) / len(per_launch)
     elapsed_max = max_over_ranks(dist, elapsed)
-    kernel_max = max_over_ranks(dist, kernel_s)
+    interval_max = elapsed_max / steps
 
-    # end to end through the host-buffer entry point
-    e2e_steps = max(3, min(steps, 30))
-    xh = torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).pin_memory()
-    ch = torch.empty(outs[0][0].shape, dtype=torch.uint8).pin_memory()
-    sh = torch.empty(outs[0][1].shape, dtype=torch.float16).pin_memory()
+    # Diagnostic: an event pair around each step, all queued behind a sleep
+    # kernel so the steps run back to back without host gaps.
+    n_ev = min(steps, 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(50_000_000)
+        for i in range(n_ev):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+    stream.synchronize()
+    step_ev = statistics.median(a.elapsed_time(b) / 1e3 for a, b in ev)
+
+    # End to end through the host-buffer entry point (quantizing parts only).
+    e2e = None
+    qkeys = [k for k in keys if W.WORKLOADS[k].fmt is not None]
+    if len(qkeys) == len(keys):
+        e2e_steps = max(3, min(steps, 20))
+        pinned = []
+        for j, k in enumerate(keys):
+            xh = torch.from_numpy(host[k].view(np.int16)).view(torch.bfloat16) if W.WORKLOADS[k].x_dtype == "bf16" \
+                else torch.from_numpy(host[k])
+            c0, s0 = outs[j][0]
+            pinned.append((xh.pin_memory(), torch.empty(c0.shape, dtype=c0.dtype).pin_memory(),
+                           torch.empty(s0.shape, dtype=s0.dtype).pin_memory()))
+
+        def e2e_step(i):
+            for j, k in enumerate(keys):
+                w = W.WORKLOADS[k]
+                xh, ch, sh = pinned[j]
+                c, sc = outs[j][i % nbuf]
+                H.hadq_rotate_quant_host(xh, w.block, w.fmt, w.group, ch, sh, bufs[j][i % nbuf], c, sc, stream=stream)
+
         for i in range(2):
-            H.hadq_rotate_quant_host(xh, 0, "int4", 128, ch, sh, xs[0], outs[0][0], outs[0][1], stream=stream)
-    stream.synchronize()
-    barrier(dist)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        H.hadq_rotate_quant_host(xh, 0, "int4", 128, ch, sh, xs[i % NBUF], outs[i % NBUF][0], outs[i % NBUF][1],
-                                 stream=stream)
-    e1.record(stream)
-    stream.synchronize()
-    e2e_max = max_over_ranks(dist, e0.elapsed_time(e1) / 1e3)
-    h2d = w.in_bytes
-    d2h = w.out_bytes
+            e2e_step(i)
+        stream.synchronize()
+        barrier(dist)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+        stream.synchronize()
+        e2e_max = max_over_ranks(dist, e0.elapsed_time(e1) / 1e3)
+        e2e = {"value": aggregate_gbs(bytes_step, e2e_steps, world, e2e_max), "unit": UNIT,
+               "h2d_bytes_per_step": sum(W.WORKLOADS[k].in_bytes for k in keys),
+               "d2h_bytes_per_step": sum(W.WORKLOADS[k].out_bytes for k in keys),
+               "path": "hadq_rotate_quant_host (pinned host buffers, copies in and out inside the timed region)"}
 
     if rank == 0:
         peak, peak_kind = measured_peak()
-        achieved = bytes_step / kernel_max / 1e9
+        achieved = bytes_step / interval_max / 1e9
+        rows_step = sum(W.WORKLOADS[k].rows for k in keys)
         line = {
-            "metric": METRIC,
-            "value": bytes_step * steps * world / elapsed_max / 1e9,
+            "metric": METRIC if cfg == "c2" else f"fused Hadamard+quant GB/s ({cfg})",
+            "value": aggregate_gbs(bytes_step, steps, world, elapsed_max),
             "unit": UNIT,
             "n_gpus": world,
             "steps": steps,
@@ -313,19 +390,21 @@ def run_hadq(args):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic",
-            "config": config_block(),
+            "config": config_block(cfg),
             "impl": "hadq",
-            "rows_per_s": w.rows * steps * world / elapsed_max,
+            "rows_per_s": rows_step * steps * world / elapsed_max,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
-                         "traffic": recorded_traffic(), "kernel_us": kernel_max * 1e6},
-            "e2e": {"value": bytes_step * e2e_steps * world / e2e_max / 1e9, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "path": "hadq_rotate_quant_host (pinned host buffers, copies in the timed region)"},
-            "gpu_launches": steps,
+                         "traffic": recorded_traffic() if cfg == "c2" else None,
+                         "duration": "mean launch interval of K back-to-back steps in one CUDA graph "
+                                     "(CUDA events on the launching stream around the graph replay)",
+                         "step_interval_us": interval_max * 1e6,
+                         "step_us_event_pairs_median": step_ev * 1e6},
+            "e2e": e2e,
+            "gpu_launches": steps * len(keys),
             "clocks": clocks.summary(),
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and cfg == "c2" and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)
     del g
@@ -340,6 +419,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["hadq", "reference"], default="hadq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", choices=sorted(STEP_PARTS), default="c2",
+                    help="workload (default c2, the metric's configuration; others for reference)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

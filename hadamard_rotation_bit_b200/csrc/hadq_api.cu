@@ -122,40 +122,50 @@ using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, fl
 using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*);
 using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*);
 
-template <int LOGS, bool BF>
+template <int LOGS, bool BF, bool FULL>
 SegFn seg_fn(int mode) {
   switch (mode) {
-    case hadq::OUT_F32: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_F32>;
-    case hadq::OUT_BF16: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_BF16>;
+    case hadq::OUT_F32: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_F32, FULL>;
+    case hadq::OUT_BF16: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_BF16, FULL>;
     case hadq::OUT_INT4:
-      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_INT4>;
+      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_INT4, FULL>;
       return nullptr;
     default:
-      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_MXFP4>;
+      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_MXFP4, FULL>;
       return nullptr;
   }
 }
 
-template <bool BF>
+template <bool BF, bool FULL>
 SegFn seg_fn_logs(int logs, int mode) {
   switch (logs) {
-    case 3: return seg_fn<3, BF>(mode);
-    case 4: return seg_fn<4, BF>(mode);
-    case 5: return seg_fn<5, BF>(mode);
-    case 6: return seg_fn<6, BF>(mode);
-    default: return seg_fn<7, BF>(mode);
+    case 3: return seg_fn<3, BF, FULL>(mode);
+    case 4: return seg_fn<4, BF, FULL>(mode);
+    case 5: return seg_fn<5, BF, FULL>(mode);
+    case 6: return seg_fn<6, BF, FULL>(mode);
+    default: return seg_fn<7, BF, FULL>(mode);
   }
 }
 
-template <bool BF>
+SegFn seg_fn_any(bool bf, bool full, int logs, int mode) {
+  if (bf) return full ? seg_fn_logs<true, true>(logs, mode) : seg_fn_logs<true, false>(logs, mode);
+  return full ? seg_fn_logs<false, true>(logs, mode) : seg_fn_logs<false, false>(logs, mode);
+}
+
+template <bool BF, bool FULL>
 SegRowFn seg_row_fn(int logs) {
   switch (logs) {
-    case 3: return &hadq::segment_row_int8_kernel<3, BF>;
-    case 4: return &hadq::segment_row_int8_kernel<4, BF>;
-    case 5: return &hadq::segment_row_int8_kernel<5, BF>;
-    case 6: return &hadq::segment_row_int8_kernel<6, BF>;
-    default: return &hadq::segment_row_int8_kernel<7, BF>;
+    case 3: return &hadq::segment_row_int8_kernel<3, BF, FULL>;
+    case 4: return &hadq::segment_row_int8_kernel<4, BF, FULL>;
+    case 5: return &hadq::segment_row_int8_kernel<5, BF, FULL>;
+    case 6: return &hadq::segment_row_int8_kernel<6, BF, FULL>;
+    default: return &hadq::segment_row_int8_kernel<7, BF, FULL>;
   }
+}
+
+SegRowFn seg_row_fn_any(bool bf, bool full, int logs) {
+  if (bf) return full ? seg_row_fn<true, true>(logs) : seg_row_fn<true, false>(logs);
+  return full ? seg_row_fn<false, true>(logs) : seg_row_fn<false, false>(logs);
 }
 
 template <int LOGB, bool BF>
@@ -223,7 +233,7 @@ hadq_status occupancy(const void* fn, int dev, int block, int smem, int* occ) {
   auto it = g_occ.find(key);
   if (it == g_occ.end()) {
     cudaError_t e = cudaSuccess;
-    if (smem > 48 * 1024) {
+    if (smem > 0) {   // dynamic + static shared memory above 48 KB needs the opt-in
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
     }
@@ -245,6 +255,29 @@ hadq_status check_launch(const char* what) {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream drains; it waits for that kernel's
+// completion (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*fn)(KArgs...), int64_t grid, int block, int smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, args...);
+}
+
+hadq_status launch_result(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return check_launch(what);
+}
+
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
 // -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
@@ -253,52 +286,53 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   hadq_status st = device_sms(&sms, &dev);
   if (st != HADQ_OK) return st;
   const bool bf = x_dtype == HADQ_BF16;
+  const bool full_seg = sh.logb == sh.logs;
   (void)cudaGetLastError();   // launch errors below must be ours
   if (mode >= 0) {
     if (sh.b <= 128) {
-      SegFn fn = bf ? seg_fn_logs<true>(sh.logs, mode) : seg_fn_logs<false>(sh.logs, mode);
+      SegFn fn = seg_fn_any(bf, full_seg, sh.logs, mode);
       if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no kernel for this segment size and format");
       const int64_t segs = sh.rows * (sh.n >> sh.logs);
       int occ = 0;
       st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, 0, &occ);
       if (st != HADQ_OK) return st;
       const int64_t grid = std::min<int64_t>(ceil_div(segs, hadq::kThreads), int64_t(sms) * occ);
-      fn<<<static_cast<unsigned>(grid), hadq::kThreads, 0, stream>>>(x, segs, sh.logb, sh.norm, group, out0, out1);
-      return check_launch("segment kernel launch");
+      return launch_result(launch_pdl(fn, grid, hadq::kThreads, 0, stream, x, segs, sh.logb, sh.norm, group, out0, out1),
+                           "segment kernel launch");
     }
     TeamFn fn = bf ? team_fn_logb<true>(sh.logb, mode) : team_fn_logb<false>(sh.logb, mode);
-    const int smem = hadq::kThreads * 128 * 4;
+    const int smem = hadq::kThreads * hadq::kRowFloats * 4;
     int occ = 0;
     st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, smem, &occ);
     if (st != HADQ_OK) return st;
     const int teams = hadq::kThreads >> (sh.logb - 7);
     const int64_t units = sh.rows * (sh.n >> sh.logb);
     const int64_t grid = std::min<int64_t>(ceil_div(units, teams), int64_t(sms) * occ);
-    fn<<<static_cast<unsigned>(grid), hadq::kThreads, smem, stream>>>(x, units, sh.norm, group, out0, out1);
-    return check_launch("team kernel launch");
+    return launch_result(launch_pdl(fn, grid, hadq::kThreads, smem, stream, x, units, sh.norm, group, out0, out1),
+                         "team kernel launch");
   }
   // per-token int8
+  int8_t* codes = static_cast<int8_t*>(out0);
+  float* scales = static_cast<float*>(out1);
   if (sh.b <= 128) {
-    SegRowFn fn = bf ? seg_row_fn<true>(sh.logs) : seg_row_fn<false>(sh.logs);
+    SegRowFn fn = seg_row_fn_any(bf, full_seg, sh.logs);
     const int block = static_cast<int>(ceil_div(sh.n >> sh.logs, 32) * 32);
     int occ = 0;
     st = occupancy(reinterpret_cast<const void*>(fn), dev, block, 0, &occ);
     if (st != HADQ_OK) return st;
     const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
-    fn<<<static_cast<unsigned>(grid), block, 0, stream>>>(x, sh.rows, sh.n, sh.logb, sh.norm,
-                                                           static_cast<int8_t*>(out0), static_cast<float*>(out1));
-    return check_launch("per-token int8 kernel launch");
+    return launch_result(launch_pdl(fn, grid, block, 0, stream, x, sh.rows, sh.n, sh.logb, sh.norm, codes, scales),
+                         "per-token int8 kernel launch");
   }
   TeamRowFn fn = bf ? team_row_fn<true>(sh.logb) : team_row_fn<false>(sh.logb);
   const int block = static_cast<int>(ceil_div(sh.n >> 7, 32) * 32);
-  const int smem = static_cast<int>(sh.n * 4);
+  const int smem = static_cast<int>((sh.n >> 7) * hadq::kRowFloats * 4);
   int occ = 0;
   st = occupancy(reinterpret_cast<const void*>(fn), dev, block, smem, &occ);
   if (st != HADQ_OK) return st;
   const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
-  fn<<<static_cast<unsigned>(grid), block, smem, stream>>>(x, sh.rows, sh.n, sh.norm, static_cast<int8_t*>(out0),
-                                                           static_cast<float*>(out1));
-  return check_launch("per-token int8 kernel launch");
+  return launch_result(launch_pdl(fn, grid, block, smem, stream, x, sh.rows, sh.n, sh.norm, codes, scales),
+                       "per-token int8 kernel launch");
 }
 
 hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,

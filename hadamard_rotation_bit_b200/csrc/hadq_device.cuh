@@ -21,7 +21,24 @@ enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3 };
 // mantissa bits (fp32 addition rounds to the nearest representable value, and
 // the spacing at this magnitude is exactly 1).
 constexpr float kRoundMagic = 12582912.0f;
-constexpr int kRoundMagicBits = 0x4B400000;
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// ------------------------------------------------------------ launch control
+
+// Programmatic dependent launch: wait until the previous grid in the stream
+// has completed and its writes are visible (a no-op without the launch
+// attribute), then let the next grid start scheduling its CTAs.  Called
+// before the first global memory access of every kernel.
+__device__ __forceinline__ void grid_dependency_sync() {
+  cudaGridDependencySynchronize();
+  cudaTriggerProgrammaticLaunchCompletion();
+}
+
+// Hint the TMA unit to stage [p, p + bytes) into L2 (16-byte aligned address,
+// size a multiple of 16, range inside the tensor).  Uses no SM resources.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // ---------------------------------------------------------------- butterflies
 
@@ -44,7 +61,9 @@ __device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1
       : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
 }
 
-// H_2 along register-index bit K of an N-element register array.
+// H_2 along register-index bit K of an N-element register array.  Bit 0 pairs
+// the two halves of a packed register pair, so it uses scalar adds; every
+// other bit uses packed f32x2 adds.
 template <int N, int K>
 __device__ __forceinline__ void fwht_stage(float (&v)[N]) {
   static_assert((2 << K) <= N, "stage bit out of range");
@@ -80,8 +99,10 @@ __device__ __forceinline__ void fwht_low(float (&v)[N], int nbits) {
 
 // --------------------------------------------------------------- loads/stores
 
+// bf16 pair -> two fp32 (exact): the low half moved up by a byte permute, the
+// high half masked; both stay off the fp32 pipe.
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
-  lo = __uint_as_float(w << 16);
+  lo = __uint_as_float(__byte_perm(w, 0u, 0x1044));
   hi = __uint_as_float(w & 0xffff0000u);
 }
 
@@ -153,41 +174,93 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return l | (h << 16);
 }
 
+// ----------------------------------------------------------- register orders
+// A thread's register array holds its elements either in element order or,
+// after the team transpose, with the two low element-index bits swapped inside
+// every quad (registers 4q..4q+3 = elements 4q, 4q+2, 4q+1, 4q+3), which lets
+// the element-bit-0 butterfly use packed f32x2 adds.  reg<PERM>(e) maps an
+// element index to its register (the swap is its own inverse).
+
+template <bool PERM>
+__host__ __device__ constexpr int reg(int e) {
+  return PERM ? ((e & ~3) | ((e & 1) << 1) | ((e >> 1) & 1)) : e;
+}
+
 // ------------------------------------------------------------------ quantizers
 
-// Eight int4 codes clamp(rne(v * rn), -7, 7) as two's-complement nibbles,
-// element i in bits [4i, 4i + 4).  The product is rounded once onto the
-// integer grid by the fused multiply-add with the magic constant (+8 keeps
-// the offset code in 1..15 so the clamp is an integer min/max).
-__device__ __forceinline__ uint32_t pack_int4x8(const float* v, float rn) {
+// Absmax of registers [lo, lo + cnt) (cnt a multiple of 4; order does not matter).
+template <int N>
+__device__ __forceinline__ float absmax_regs(const float (&v)[N], int lo, int cnt) {
+  float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < cnt; i += 4) {
+    m0 = fmaxf(m0, fmaxf(fabsf(v[lo + i]), fabsf(v[lo + i + 1])));
+    m1 = fmaxf(m1, fmaxf(fabsf(v[lo + i + 2]), fabsf(v[lo + i + 3])));
+  }
+  return fmaxf(m0, m1);
+}
+
+// Eight int4 codes rne(v * rn) of elements e0..e0+7 (register order PERM), as
+// two's-complement nibbles, element i in bits [4i, 4i + 4).  Valid when every
+// |v * rn| < 7.5 (no clamp needed): each product is rounded once onto the
+// integer grid by a fused multiply-add with 1.5*2^23 + 8, leaving q + 8 in
+// 1..15 in the low bits; the eight words are combined by shift-add (Horner),
+// the constant high parts removed, and the offset-8 nibbles turned into
+// two's complement by flipping their top bits.
+template <bool PERM, int N>
+__device__ __forceinline__ uint32_t pack_int4x8(const float (&v)[N], int e0, float rn) {
+  constexpr float kM = kRoundMagic + 8.0f;
+  const float2 r2 = make_float2(rn, rn), m2 = make_float2(kM, kM);
+  uint32_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = __ffma2_rn(make_float2(v[reg<PERM>(e0 + i)], v[reg<PERM>(e0 + i + 1)]), r2, m2);
+    t[i] = __float_as_uint(p.x);
+    t[i + 1] = __float_as_uint(p.y);
+  }
+  uint32_t w = t[7];
+#pragma unroll
+  for (int i = 6; i >= 0; --i) w = (w << 4) + t[i];
+  constexpr uint32_t kHigh = kRoundMagicBits * 0x11111111u;   // sum of the magic parts, mod 2^32
+  return (w - kHigh) ^ 0x88888888u;
+}
+
+// The same with an explicit clamp to [-7, 7] (subnormal, zero or huge scales).
+template <bool PERM, int N>
+__device__ __forceinline__ uint32_t pack_int4x8_clamped(const float (&v)[N], int e0, float rn) {
   uint32_t w = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    int b = __float_as_int(__fmaf_rn(v[i], rn, kRoundMagic + 8.0f));
-    b = min(max(b, kRoundMagicBits + 1), kRoundMagicBits + 15);
-    w |= static_cast<uint32_t>((b - (kRoundMagicBits + 8)) & 0xF) << (4 * i);
+    const float q = fminf(fmaxf(v[reg<PERM>(e0 + i)] * rn, -7.0f), 7.0f);
+    const uint32_t b = __float_as_uint(__fadd_rn(q, kRoundMagic + 8.0f)) - (kRoundMagicBits + 8u);
+    w |= (b & 0xFu) << (4 * i);
   }
   return w;
 }
 
-// Four int8 codes clamp(rne(v * rn), -127, 127), element i in byte i.
-__device__ __forceinline__ uint32_t pack_int8x4(const float* v, float rn) {
-  int b[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    b[i] = __float_as_int(__fmaf_rn(v[i], rn, kRoundMagic));
-    b[i] = min(max(b[i], kRoundMagicBits - 127), kRoundMagicBits + 127);
-  }
-  const uint32_t lo = __byte_perm(b[0], b[1], 0x5140);
-  const uint32_t hi = __byte_perm(b[2], b[3], 0x5140);
+// Four int8 codes rne(v * rn), element i in byte i (|v * rn| < 127.5).
+template <bool PERM, int N>
+__device__ __forceinline__ uint32_t pack_int8x4(const float (&v)[N], int e0, float rn) {
+  const float2 r2 = make_float2(rn, rn), m2 = make_float2(kRoundMagic, kRoundMagic);
+  const float2 p0 = __ffma2_rn(make_float2(v[reg<PERM>(e0)], v[reg<PERM>(e0 + 1)]), r2, m2);
+  const float2 p1 = __ffma2_rn(make_float2(v[reg<PERM>(e0 + 2)], v[reg<PERM>(e0 + 3)]), r2, m2);
+  const uint32_t lo = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5140);
+  const uint32_t hi = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5140);
   return __byte_perm(lo, hi, 0x5410);
 }
 
 // Eight E2M1 codes (round to nearest even, saturating at +/-6, sign in bit 3)
 // of v * f, element i in bits [4i, 4i + 4).
-__device__ __forceinline__ uint32_t pack_e2m1x8(const float* v, float f) {
-  const float a0 = v[0] * f, a1 = v[1] * f, a2 = v[2] * f, a3 = v[3] * f;
-  const float a4 = v[4] * f, a5 = v[5] * f, a6 = v[6] * f, a7 = v[7] * f;
+template <bool PERM, int N>
+__device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, float f) {
+  const float2 f2 = make_float2(f, f);
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = __fmul2_rn(make_float2(v[reg<PERM>(e0 + i)], v[reg<PERM>(e0 + i + 1)]), f2);
+    a[i] = p.x;
+    a[i + 1] = p.y;
+  }
   uint32_t w;
   asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
@@ -196,61 +269,49 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float* v, float f) {
       "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
       "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
       : "=r"(w)
-      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
   return w;
-}
-
-template <int N>
-__device__ __forceinline__ float absmax32(const float (&v)[N], int j) {
-  float m = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[32 * j + i]));
-  return m;
 }
 
 // --------------------------------------------------------------- epilogues
 // Each epilogue owns N consecutive rotated-but-unnormalised values z of one
-// row, starting at flattened element index e0; y = z * norm is the rotation.
+// row (register order PERM), starting at flattened element index e0;
+// y = z * norm is the rotation.
 
 // Rotation output (fp32 or bf16).
-template <int N, bool OUT_IS_BF16>
+template <bool PERM, int N, bool OUT_IS_BF16>
 __device__ __forceinline__ void store_rotated(const float (&v)[N], float norm, void* __restrict__ out, int64_t e0) {
   if constexpr (OUT_IS_BF16) {
     uint16_t* o = static_cast<uint16_t*>(out) + e0;
-    if constexpr (N % 8 == 0) {
+    static_assert(N % 8 == 0, "bf16 chunk must hold whole 16-byte stores");
 #pragma unroll
-      for (int i = 0; i < N / 8; ++i) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * i + 0] * norm, v[8 * i + 1] * norm);
-        w.y = pack_bf16x2(v[8 * i + 2] * norm, v[8 * i + 3] * norm);
-        w.z = pack_bf16x2(v[8 * i + 4] * norm, v[8 * i + 5] * norm);
-        w.w = pack_bf16x2(v[8 * i + 6] * norm, v[8 * i + 7] * norm);
-        reinterpret_cast<uint4*>(o)[i] = w;
-      }
-    } else {
-      static_assert(N % 2 == 0, "odd bf16 chunk");
-#pragma unroll
-      for (int i = 0; i < N / 2; ++i) reinterpret_cast<uint32_t*>(o)[i] = pack_bf16x2(v[2 * i] * norm, v[2 * i + 1] * norm);
+    for (int i = 0; i < N / 8; ++i) {
+      uint4 w;
+      w.x = pack_bf16x2(v[reg<PERM>(8 * i + 0)] * norm, v[reg<PERM>(8 * i + 1)] * norm);
+      w.y = pack_bf16x2(v[reg<PERM>(8 * i + 2)] * norm, v[reg<PERM>(8 * i + 3)] * norm);
+      w.z = pack_bf16x2(v[reg<PERM>(8 * i + 4)] * norm, v[reg<PERM>(8 * i + 5)] * norm);
+      w.w = pack_bf16x2(v[reg<PERM>(8 * i + 6)] * norm, v[reg<PERM>(8 * i + 7)] * norm);
+      reinterpret_cast<uint4*>(o)[i] = w;
     }
   } else {
     float* o = static_cast<float*>(out) + e0;
     static_assert(N % 4 == 0, "fp32 chunk must hold whole float4s");
 #pragma unroll
     for (int i = 0; i < N / 4; ++i)
-      reinterpret_cast<float4*>(o)[i] =
-          make_float4(v[4 * i] * norm, v[4 * i + 1] * norm, v[4 * i + 2] * norm, v[4 * i + 3] * norm);
+      reinterpret_cast<float4*>(o)[i] = make_float4(v[reg<PERM>(4 * i)] * norm, v[reg<PERM>(4 * i + 1)] * norm,
+                                                    v[reg<PERM>(4 * i + 2)] * norm, v[reg<PERM>(4 * i + 3)] * norm);
   }
 }
 
 // Symmetric int4, group in {32, 64, 128} with group | N: scale fp16(m / 7).
-template <int N>
+template <bool PERM, int N>
 __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int group, uint8_t* __restrict__ codes,
                                            __half* __restrict__ scales, int64_t e0) {
   static_assert(N % 32 == 0, "int4 groups need 32-element sub-blocks");
   constexpr int NS = N / 32;
   float m32[NS];
 #pragma unroll
-  for (int j = 0; j < NS; ++j) m32[j] = absmax32(v, j);
+  for (int j = 0; j < NS; ++j) m32[j] = absmax_regs(v, 32 * j, 32);   // a 32-block is closed under reg<>
   const int spg = group >> 5;  // 32-element sub-blocks per group: 1, 2 or 4
 #pragma unroll
   for (int j = 0; j < NS; ++j) {
@@ -267,23 +328,30 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
     const float r = (s > 0.f && s <= 65504.f) ? __frcp_rn(s) : 0.f;   // zero / inf scale -> zero codes
     const float rn = r * norm;
     uint4 w;
-    w.x = pack_int4x8(&v[32 * j + 0], rn);
-    w.y = pack_int4x8(&v[32 * j + 8], rn);
-    w.z = pack_int4x8(&v[32 * j + 16], rn);
-    w.w = pack_int4x8(&v[32 * j + 24], rn);
+    if (mz * rn < 7.25f) {        // normal scale: every |v * rn| <= 7.0035, no clamp
+      w.x = pack_int4x8<PERM>(v, 32 * j + 0, rn);
+      w.y = pack_int4x8<PERM>(v, 32 * j + 8, rn);
+      w.z = pack_int4x8<PERM>(v, 32 * j + 16, rn);
+      w.w = pack_int4x8<PERM>(v, 32 * j + 24, rn);
+    } else {
+      w.x = pack_int4x8_clamped<PERM>(v, 32 * j + 0, rn);
+      w.y = pack_int4x8_clamped<PERM>(v, 32 * j + 8, rn);
+      w.z = pack_int4x8_clamped<PERM>(v, 32 * j + 16, rn);
+      w.w = pack_int4x8_clamped<PERM>(v, 32 * j + 24, rn);
+    }
     reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
     if ((j & (spg - 1)) == 0) scales[(e0 + 32 * j) / group] = s16;
   }
 }
 
 // MXFP4: per 32 elements an E8M0 exponent e = clamp(floor(log2 m) - 2, -127, 127).
-template <int N>
+template <bool PERM, int N>
 __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales, int64_t e0) {
   static_assert(N % 32 == 0, "MX groups are 32 elements");
 #pragma unroll
   for (int j = 0; j < N / 32; ++j) {
-    const float m = absmax32(v, j) * norm;
+    const float m = absmax_regs(v, 32 * j, 32) * norm;
     // floor(log2 m) is the unbiased exponent field for normal m; zero and
     // subnormal m (and anything below 2^-125) clamp to e = -127, byte 0.
     const int ebits = static_cast<int>((__float_as_uint(m) >> 23) & 0xFF);
@@ -291,48 +359,47 @@ __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uin
     const int e = byte - 127;                         // in [-127, 126]
     const float f = norm * __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // norm * 2^-e, exact
     uint4 w;
-    w.x = pack_e2m1x8(&v[32 * j + 0], f);
-    w.y = pack_e2m1x8(&v[32 * j + 8], f);
-    w.z = pack_e2m1x8(&v[32 * j + 16], f);
-    w.w = pack_e2m1x8(&v[32 * j + 24], f);
+    w.x = pack_e2m1x8<PERM>(v, 32 * j + 0, f);
+    w.y = pack_e2m1x8<PERM>(v, 32 * j + 8, f);
+    w.z = pack_e2m1x8<PERM>(v, 32 * j + 16, f);
+    w.w = pack_e2m1x8<PERM>(v, 32 * j + 24, f);
     reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
     scales[(e0 >> 5) + j] = static_cast<uint8_t>(byte);
   }
 }
 
 // Symmetric int8 with a per-row scale s = fp32(m / 127) (m = the row absmax of y).
-template <int N>
+template <bool PERM, int N>
 __device__ __forceinline__ void store_int8(const float (&v)[N], float norm, float m, int8_t* __restrict__ codes,
                                            int64_t e0) {
   static_assert(N % 8 == 0, "int8 chunk must hold whole 8-byte stores");
   const float s = __fdiv_rn(m, 127.0f);
   const float r = (s > 0.f && s <= 3.0e38f) ? __frcp_rn(s) : 0.f;
-  if (r <= 1.0e30f) {
-    const float rn = r * norm;
+  const float rn = r * norm;
+  if (m * r < 127.25f) {         // normal scale: every |v * rn| < 127.5, no clamp
     if constexpr (N % 16 == 0) {
       uint4* o = reinterpret_cast<uint4*>(codes + e0);
 #pragma unroll
-      for (int i = 0; i < N / 16; ++i) {
-        uint4 w;
-        w.x = pack_int8x4(&v[16 * i + 0], rn);
-        w.y = pack_int8x4(&v[16 * i + 4], rn);
-        w.z = pack_int8x4(&v[16 * i + 8], rn);
-        w.w = pack_int8x4(&v[16 * i + 12], rn);
-        o[i] = w;
-      }
+      for (int i = 0; i < N / 16; ++i)
+        o[i] = make_uint4(pack_int8x4<PERM>(v, 16 * i, rn), pack_int8x4<PERM>(v, 16 * i + 4, rn),
+                          pack_int8x4<PERM>(v, 16 * i + 8, rn), pack_int8x4<PERM>(v, 16 * i + 12, rn));
     } else {
       uint2* o = reinterpret_cast<uint2*>(codes + e0);
 #pragma unroll
-      for (int i = 0; i < N / 8; ++i) o[i] = make_uint2(pack_int8x4(&v[8 * i], rn), pack_int8x4(&v[8 * i + 4], rn));
+      for (int i = 0; i < N / 8; ++i)
+        o[i] = make_uint2(pack_int8x4<PERM>(v, 8 * i, rn), pack_int8x4<PERM>(v, 8 * i + 4, rn));
     }
   } else {
-    // Scale so small that its reciprocal overflows: divide element by element.
+    // Subnormal scale: the reciprocal is inexact or overflows -- divide, clamp.
 #pragma unroll
     for (int i = 0; i < N / 4; ++i) {
-      float q[4];
+      uint32_t w = 0;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) q[k] = fminf(fmaxf(__fdiv_rn(v[4 * i + k] * norm, s), -127.f), 127.f);
-      reinterpret_cast<uint32_t*>(codes + e0)[i] = pack_int8x4(q, 1.0f);
+      for (int k = 0; k < 4; ++k) {
+        const float q = fminf(fmaxf(__fdiv_rn(v[reg<PERM>(4 * i + k)] * norm, s), -127.f), 127.f);
+        w |= ((__float_as_uint(__fadd_rn(q, kRoundMagic)) - kRoundMagicBits) & 0xFFu) << (8 * k);
+      }
+      reinterpret_cast<uint32_t*>(codes + e0)[i] = w;
     }
   }
 }

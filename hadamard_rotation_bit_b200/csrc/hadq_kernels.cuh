@@ -12,12 +12,15 @@
 //    block.  Index bits: e = [hi: t bits | mid: t bits | vec: 7 - t bits],
 //    t = log2 T.  Phase 1: each thread loads, for every hi value, one
 //    contiguous chunk of 2^(7-t) elements (the team reads 128 contiguous
-//    elements per hi value) and runs the 7 stages of its register bits
-//    (vec + hi).  A transpose through shared memory (fp32, XOR-swizzled in
-//    16-byte quads so both sides are bank-conflict free for t >= 3) hands
-//    every thread the 128 consecutive elements with hi = its team index.
-//    Phase 2 runs the remaining t stages (mid bits); the thread then holds a
-//    whole run of 128 consecutive outputs for the quantizer.
+//    elements per hi value) and runs the stages of its register bits (vec +
+//    hi).  A transpose through shared memory (fp32 rows of 128 + 4 pad floats:
+//    conflict-free on both sides for t >= 5, immediate offsets) hands every
+//    thread the 128 consecutive elements with hi = its team index.  Phase 2
+//    runs the remaining stages (mid bits); the thread then holds a whole run of
+//    128 consecutive outputs for the quantizer.  When the chunk holds at least
+//    4 elements, the transpose stores every quad as (e0, e2, e1, e3), so the
+//    element-bit-0 stage runs in phase 2 on packed f32x2 pairs instead of as
+//    scalar adds in phase 1.
 //
 // The per-token int8 format needs the whole row before any code is written,
 // so it has row kernels: one CTA per row, the same two layouts inside, and a
@@ -27,6 +30,10 @@
 // quantized paths: it is folded into the group absmax (fp32 rounding is
 // monotone, so max|fl(z * c)| = fl(max|z| * c)) and into the reciprocal
 // scale.  For even log2(b) it is an exact power of 2.
+//
+// Every kernel starts with the programmatic-dependent-launch handshake (see
+// grid_dependency_sync) and prefetches its next unit of input into L2 while it
+// computes the current one.
 #pragma once
 
 #include "hadq_device.cuh"
@@ -34,56 +41,77 @@
 namespace hadq {
 
 constexpr int kThreads = 128;
+constexpr int kRowFloats = 132;   // transpose row: 128 floats + one quad of padding
 
 // ----------------------------------------------------------- segment kernels
 
-template <int LOGS, bool IN_BF16, int MODE>
+// FULL: b == S, all LOGS stages unconditionally; otherwise the low nbits stages.
+template <int LOGS, bool IN_BF16, int MODE, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, int group,
                void* __restrict__ out0, void* __restrict__ out1) {
   constexpr int S = 1 << LOGS;
+  constexpr uint32_t kSegBytes = S * (IN_BF16 ? 2 : 4);
+  grid_dependency_sync();
   float v[S];
+  const int lane = threadIdx.x & 31;
   for (int64_t s = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; s < segs;
        s += static_cast<int64_t>(gridDim.x) * kThreads) {
+    if (lane == 0) {   // the warp's next 32 segments are contiguous
+      const int64_t nxt = s + static_cast<int64_t>(gridDim.x) * kThreads;
+      if (nxt < segs) {
+        const int64_t cnt = segs - nxt < 32 ? segs - nxt : 32;
+        prefetch_l2(static_cast<const char*>(x) + nxt * kSegBytes, static_cast<uint32_t>(cnt) * kSegBytes);
+      }
+    }
     const int64_t e0 = s << LOGS;
     load_elems<IN_BF16, S>(x, e0, v);
-    fwht_low<S>(v, nbits);
-    if constexpr (MODE == OUT_F32) {
-      store_rotated<S, false>(v, norm, out0, e0);
-    } else if constexpr (MODE == OUT_BF16) {
-      store_rotated<S, true>(v, norm, out0, e0);
-    } else if constexpr (MODE == OUT_INT4) {
-      store_int4<S>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+    if constexpr (FULL) {
+      fwht_bits<S, 0, LOGS>(v);
     } else {
-      store_mxfp4<S>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+      fwht_low<S>(v, nbits);
+    }
+    if constexpr (MODE == OUT_F32) {
+      store_rotated<false, S, false>(v, norm, out0, e0);
+    } else if constexpr (MODE == OUT_BF16) {
+      store_rotated<false, S, true>(v, norm, out0, e0);
+    } else if constexpr (MODE == OUT_INT4) {
+      store_int4<false, S>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+    } else {
+      store_mxfp4<false, S>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
     }
   }
 }
 
 // Per-token int8, b <= 128: one CTA per row, blockDim = n / S rounded up to 32 (<= 256).
-template <int LOGS, bool IN_BF16>
+template <int LOGS, bool IN_BF16, bool FULL>
 __global__ void __launch_bounds__(256)
 segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int nbits, float norm,
                         int8_t* __restrict__ codes, float* __restrict__ scales) {
   constexpr int S = 1 << LOGS;
+  grid_dependency_sync();
   __shared__ float red[32];
   const int segs_row = static_cast<int>(n >> LOGS);
   const bool active = static_cast<int>(threadIdx.x) < segs_row;
+  const int64_t row_bytes = n * (IN_BF16 ? 2 : 4);
   float v[S];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    if (threadIdx.x == 0 && r + gridDim.x < rows)
+      prefetch_l2(static_cast<const char*>(x) + (r + gridDim.x) * row_bytes, static_cast<uint32_t>(row_bytes));
     const int64_t e0 = r * n + (static_cast<int64_t>(threadIdx.x) << LOGS);
     if (active) {
       load_elems<IN_BF16, S>(x, e0, v);
-      fwht_low<S>(v, nbits);
+      if constexpr (FULL) {
+        fwht_bits<S, 0, LOGS>(v);
+      } else {
+        fwht_low<S>(v, nbits);
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < S; ++i) v[i] = 0.f;
     }
-    float mz = 0.f;
-#pragma unroll
-    for (int i = 0; i < S; ++i) mz = fmaxf(mz, fabsf(v[i]));
-    const float m = cta_max(mz, red) * norm;
-    if (active) store_int8<S>(v, norm, m, codes, e0);
+    const float m = cta_max(absmax_regs(v, 0, S), red) * norm;
+    if (active) store_int8<false, S>(v, norm, m, codes, e0);
     if (threadIdx.x == 0) scales[r] = __fdiv_rn(m, 127.0f);
   }
 }
@@ -97,6 +125,7 @@ struct TeamShape {
   static constexpr int V = 7 - t;             // vec bits per phase-1 chunk
   static constexpr int CE = 1 << V;           // elements per phase-1 chunk
   static constexpr int B = 1 << LOGB;
+  static constexpr bool PERM = V >= 2;        // quads transposed as (e0, e2, e1, e3)
   static_assert(LOGB >= 8 && LOGB <= 13, "team kernels cover 256..8192");
 };
 
@@ -110,12 +139,12 @@ __device__ __forceinline__ void team_sync() {
 }
 
 // Rotate one block of 2^LOGB elements (element base `base`) by a team; on
-// return v[0..128) holds the unnormalised outputs base + tau*128 + [0, 128).
-// `rows` points at this team's T x 128-float shared buffer; `grow` is the
-// team's first row in the CTA buffer (the swizzle key).
+// return v[0..128) holds the unnormalised outputs base + tau*128 + [0, 128) in
+// register order TeamShape<LOGB>::PERM.  `rows` is this team's T x kRowFloats
+// shared buffer.
 template <int LOGB, bool IN_BF16>
 __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t base, bool valid, int tau,
-                                            float* __restrict__ rows, int grow, float (&v)[128]) {
+                                            float* __restrict__ rows, float (&v)[128]) {
   using Sh = TeamShape<LOGB>;
   if (valid) {
 #pragma unroll
@@ -124,33 +153,33 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
 #pragma unroll
     for (int i = 0; i < 128; ++i) v[i] = 0.f;
   }
-  // Phase 1: register bits = vec (element bits 0..V-1) and hi (element bits 7..).
-  fwht_bits<128, 0, 7>(v);
-  // Transpose: row h of the team buffer holds elements h*128 + [0, 128).
+  // Phase 1: register index h * CE + j (j = element bits 0..V-1, h = element bits 7..).
+  if constexpr (Sh::PERM) {
+    fwht_bits<128, 1, 7>(v);          // element bit 0 waits for phase 2
+  } else {
+    fwht_bits<128, 0, 7>(v);
+  }
+  // Transpose: buffer row h holds elements h*128 + [0, 128).
 #pragma unroll
   for (int h = 0; h < Sh::T; ++h) {
-    const int g = grow + h;
-    float* rowp = rows + h * 128;
+    float* rowp = rows + h * kRowFloats;
     if constexpr (Sh::CE >= 4) {
 #pragma unroll
       for (int k = 0; k < Sh::CE / 4; ++k) {
-        const int q = tau * (Sh::CE / 4) + k;
-        reinterpret_cast<float4*>(rowp)[q ^ (g & 31)] =
-            make_float4(v[h * Sh::CE + 4 * k], v[h * Sh::CE + 4 * k + 1], v[h * Sh::CE + 4 * k + 2],
-                        v[h * Sh::CE + 4 * k + 3]);
+        const float* s = &v[h * Sh::CE + 4 * k];
+        reinterpret_cast<float4*>(rowp)[tau * (Sh::CE / 4) + k] =
+            Sh::PERM ? make_float4(s[0], s[2], s[1], s[3]) : make_float4(s[0], s[1], s[2], s[3]);
       }
     } else {
-      const int q = tau >> 1;
-      reinterpret_cast<float2*>(rowp)[((q ^ (g & 31)) << 1) + (tau & 1)] = make_float2(v[h * 2], v[h * 2 + 1]);
+      reinterpret_cast<float2*>(rowp)[tau] = make_float2(v[h * 2], v[h * 2 + 1]);
     }
   }
   team_sync<Sh::T>();
   {
-    const int g = grow + tau;
-    const float4* rowp = reinterpret_cast<const float4*>(rows + tau * 128);
+    const float4* rowp = reinterpret_cast<const float4*>(rows + tau * kRowFloats);
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
-      const float4 f = rowp[q ^ (g & 31)];
+      const float4 f = rowp[q];
       v[4 * q] = f.x;
       v[4 * q + 1] = f.y;
       v[4 * q + 2] = f.z;
@@ -158,50 +187,58 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
     }
   }
   team_sync<Sh::T>();
-  // Phase 2: the mid bits (element bits V..6).
+  // Phase 2: the mid bits (element bits V..6), and element bit 0 (register bit 1 under PERM).
+  if constexpr (Sh::PERM) fwht_stage<128, 1>(v);
   fwht_bits<128, Sh::V, 7>(v);
 }
 
 template <int LOGB, bool IN_BF16, int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, void* __restrict__ out0,
             void* __restrict__ out1) {
   using Sh = TeamShape<LOGB>;
   constexpr int TEAMS = kThreads / Sh::T;
+  constexpr uint32_t kUnitBytes = Sh::B * (IN_BF16 ? 2 : 4);
+  grid_dependency_sync();
   extern __shared__ float4 smem_f4[];
   float* buf = reinterpret_cast<float*>(smem_f4);
   const int team = threadIdx.x >> Sh::t;
   const int tau = threadIdx.x & (Sh::T - 1);
-  float* rows = buf + team * Sh::T * 128;
+  float* rows = buf + team * Sh::T * kRowFloats;
   float v[128];
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * TEAMS; u0 < units;
        u0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
     const int64_t u = u0 + team;
+    if (tau == 0) {
+      const int64_t nxt = u + static_cast<int64_t>(gridDim.x) * TEAMS;
+      if (nxt < units) prefetch_l2(static_cast<const char*>(x) + nxt * kUnitBytes, kUnitBytes);
+    }
     const bool valid = u < units;
     const int64_t base = u << LOGB;
-    team_rotate<LOGB, IN_BF16>(x, base, valid, tau, rows, team * Sh::T, v);
+    team_rotate<LOGB, IN_BF16>(x, base, valid, tau, rows, v);
     if (valid) {
       const int64_t e0 = base + tau * 128;
       if constexpr (MODE == OUT_F32) {
-        store_rotated<128, false>(v, norm, out0, e0);
+        store_rotated<Sh::PERM, 128, false>(v, norm, out0, e0);
       } else if constexpr (MODE == OUT_BF16) {
-        store_rotated<128, true>(v, norm, out0, e0);
+        store_rotated<Sh::PERM, 128, true>(v, norm, out0, e0);
       } else if constexpr (MODE == OUT_INT4) {
-        store_int4<128>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+        store_int4<Sh::PERM, 128>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
       } else {
-        store_mxfp4<128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+        store_mxfp4<Sh::PERM, 128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
       }
     }
   }
 }
 
 // Per-token int8, b >= 256: one CTA per row of n elements (n / b teams).
-// blockDim = n / 128 rounded up to 32; dynamic shared memory = n floats.
+// blockDim = n / 128 rounded up to 32; dynamic shared memory = n / 128 rows.
 template <int LOGB, bool IN_BF16>
 __global__ void __launch_bounds__(256)
 team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float norm, int8_t* __restrict__ codes,
                      float* __restrict__ scales) {
   using Sh = TeamShape<LOGB>;
+  grid_dependency_sync();
   extern __shared__ float4 smem_f4[];
   float* buf = reinterpret_cast<float*>(smem_f4);
   __shared__ float red[32];
@@ -209,12 +246,15 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
   const bool active = static_cast<int>(threadIdx.x) < nthreads;
   const int team = threadIdx.x >> Sh::t;
   const int tau = threadIdx.x & (Sh::T - 1);
-  float* team_rows = buf + (active ? team * Sh::T * 128 : 0);
+  float* team_rows = buf + (active ? team * Sh::T * kRowFloats : 0);
+  const int64_t row_bytes = n * (IN_BF16 ? 2 : 4);
   float v[128];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    if (threadIdx.x == 0 && r + gridDim.x < rows)
+      prefetch_l2(static_cast<const char*>(x) + (r + gridDim.x) * row_bytes, static_cast<uint32_t>(row_bytes));
     const int64_t base = r * n + (static_cast<int64_t>(team) << LOGB);
     if (active) {
-      team_rotate<LOGB, IN_BF16>(x, base, true, tau, team_rows, team * Sh::T, v);
+      team_rotate<LOGB, IN_BF16>(x, base, true, tau, team_rows, v);
     } else {
       // Idle threads still take part in every barrier of team_rotate.
 #pragma unroll
@@ -222,11 +262,8 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
       team_sync<Sh::T>();
       team_sync<Sh::T>();
     }
-    float mz = 0.f;
-#pragma unroll
-    for (int i = 0; i < 128; ++i) mz = fmaxf(mz, fabsf(v[i]));
-    const float m = cta_max(mz, red) * norm;
-    if (active) store_int8<128>(v, norm, m, codes, base + tau * 128);
+    const float m = cta_max(absmax_regs(v, 0, 128), red) * norm;
+    if (active) store_int8<Sh::PERM, 128>(v, norm, m, codes, base + tau * 128);
     if (threadIdx.x == 0) scales[r] = __fdiv_rn(m, 127.0f);
   }
 }

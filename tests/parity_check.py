@@ -4,7 +4,8 @@ Tolerances (the benchmark spec of the problem, with the readings listed
 in DESIGN.md):
 
 * rotated fp32: max |gpu - oracle| <= 1e-5 * ||x_row||_2 for every row;
-* rotated bf16: within one bf16 ulp of the oracle rounded to bf16;
+* rotated bf16: the round-to-nearest-even of a value within the fp32
+  tolerance (between bf16(y - d) and bf16(y + d), d = 1e-5 * ||x_row||);
 * codes: bit-exact, except where the oracle's pre-round value lies within a
   window W = 1e-6 * (group absmax) of a rounding boundary; there either
   adjacent code is accepted and the case is counted;
@@ -47,18 +48,30 @@ def check_rotation_f32(x64: np.ndarray, y_gpu: np.ndarray, block: int) -> dict:
     return {"rows": len(rel), "worst_rel_err": float(rel.max())}
 
 
+def _bf16_value(bits):
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def check_rotation_bf16(x64: np.ndarray, y_bits: np.ndarray, block: int) -> dict:
+    """bf16 output = round-to-nearest-even of a value within the fp32 tolerance.
+
+    With d = 1e-5 * ||x_row||, the output must lie between bf16(y - d) and
+    bf16(y + d) (rounding is monotone).  Away from zero this is within one
+    bf16 ulp of bf16(y); near zero the fp32 error bound (relative to the row
+    norm) dominates the ulp of the element.
+    """
     y = oracle.rotate(x64, block)
-    want = oracle.to_bf16_bits(y)
-    wv = (want.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    gv = (np.asarray(y_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    a = np.abs(wv)
+    d = 1e-5 * np.linalg.norm(x64, axis=1, keepdims=True)
+    lo = _bf16_value(oracle.to_bf16_bits(y - d))
+    hi = _bf16_value(oracle.to_bf16_bits(y + d))
+    want = _bf16_value(oracle.to_bf16_bits(y))
+    gv = _bf16_value(y_bits)
+    bad = (gv < lo) | (gv > hi)
+    assert not bad.any(), f"{bad.sum()} bf16 outputs outside bf16([y - d, y + d])"
+    a = np.abs(want)
     ulp = np.ldexp(1.0, np.maximum(np.frexp(np.where(a > 0, a, 1.0))[1] - 1, -126) - 7)
-    ulp = np.where(a > 0, ulp, 2.0 ** -133)
-    diff = np.abs(gv - wv)
-    bad = diff > ulp
-    assert not bad.any(), f"{bad.sum()} bf16 outputs differ by more than one ulp"
-    return {"elements": int(y.size), "not_bit_equal": int((gv != wv).sum())}
+    return {"elements": int(y.size), "not_bit_equal": int((gv != want).sum()),
+            "max_ulps_from_rne_of_oracle": float((np.abs(gv - want) / ulp).max())}
 
 
 def _check_codes(got, v, w, encode):
