@@ -6,9 +6,14 @@
 // is no CPU path: a missing device or kernel image surfaces as HADQ_ERR_CUDA.
 #include "hadq.h"
 #include "hadq_kernels.cuh"
+#include "hadq_tc.cuh"
+
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <string>
@@ -278,6 +283,97 @@ hadq_status launch_result(cudaError_t e, const char* what) {
   return check_launch(what);
 }
 
+// ------------------------------------------------------- tensor-core path
+
+// Which implementation serves full-size bf16 rotations of 4096 and 8192:
+// HADQ_KERNEL = "auto" or unset (the tcgen05 + TMA kernel), "tensor" (the
+// same), or "butterfly" (the CUDA-core team kernel, kept for comparison).
+enum class KernelChoice { Auto, Butterfly, Tensor };
+
+KernelChoice kernel_choice() {
+  const char* v = std::getenv("HADQ_KERNEL");
+  if (v == nullptr || std::strcmp(v, "auto") == 0) return KernelChoice::Auto;
+  if (std::strcmp(v, "butterfly") == 0) return KernelChoice::Butterfly;
+  if (std::strcmp(v, "tensor") == 0) return KernelChoice::Tensor;
+  return KernelChoice::Auto;
+}
+
+bool tc_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
+  return x_dtype == HADQ_BF16 && (sh.logb == 12 || sh.logb == 13) && mode >= 0;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+using TcFn = void (*)(const CUtensorMap, int64_t, int, float, int, void*, void*);
+
+template <class C>
+TcFn tc_fn_mode(int mode) {
+  switch (mode) {
+    case hadq::OUT_F32: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_F32>;
+    case hadq::OUT_BF16: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_BF16>;
+    case hadq::OUT_INT4: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_INT4>;
+    default: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_MXFP4>;
+  }
+}
+
+// Tensor-core kernel configuration: 128-column tiles, 5 operand stages, and
+// 4 (n = 4096) or 2 (n = 8192) epilogue warps per tensor-memory lane quarter
+// -- the fastest of the measured variants for each size.
+struct TcVariant {
+  TcFn fn;
+  int threads, smem, tile_n;
+};
+
+template <int LO, int SPLIT>
+TcVariant tc_variant(int mode) {
+  using C = hadq::tc::TcCfg<LO, 128, 5, SPLIT>;
+  return TcVariant{tc_fn_mode<C>(mode), C::THREADS, C::SMEM_BYTES, C::TILE_N};
+}
+
+TcVariant tc_pick(int lo, int mode) { return lo == 5 ? tc_variant<5, 4>(mode) : tc_variant<6, 2>(mode); }
+
+// Blocks of b = 2^(7 + LO) bf16 elements, each rotated in full: the blocks are
+// the rows of a (rows * n / b) x b matrix.
+hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
+                      cudaStream_t stream, int sms, int dev) {
+  const int lo = sh.logb - 7;
+  const TcVariant v = tc_pick(lo, mode);
+  const int L = 1 << lo, R = v.tile_n / L;
+  const int64_t rows = sh.rows * (sh.n >> sh.logb);
+  if (rows > (int64_t(1) << 31) - R) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many rows");
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (encode == nullptr) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  CUtensorMap map;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(L), 128, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(L) * 2, static_cast<cuuint64_t>(sh.b) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(L), 128, static_cast<cuuint32_t>(R)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            lo == 5 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  int occ = 0;
+  hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t tiles = (rows + R - 1) / R;
+  const int64_t grid = std::min<int64_t>(tiles, sms);
+  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, rows, static_cast<int>(sh.b), sh.norm,
+                                  group, out0, out1),
+                       "tensor-core kernel launch");
+}
+
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
 // -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
@@ -288,6 +384,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   const bool bf = x_dtype == HADQ_BF16;
   const bool full_seg = sh.logb == sh.logs;
   (void)cudaGetLastError();   // launch errors below must be ours
+  if (tc_eligible(x_dtype, sh, mode) && kernel_choice() != KernelChoice::Butterfly)
+    return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev);
   if (mode >= 0) {
     if (sh.b <= 128) {
       SegFn fn = seg_fn_any(bf, full_seg, sh.logs, mode);
@@ -463,5 +561,15 @@ const char* hadq_status_string(hadq_status status) {
 const char* hadq_last_error(void) { return g_last_error.c_str(); }
 
 int hadq_version(void) { return 100; }
+
+int hadq_device_faults(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, hadq::tc::hadq_tc_fault, sizeof(v)) != cudaSuccess) return -1;
+  if (clear && v != 0) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(hadq::tc::hadq_tc_fault, &z, sizeof(z)) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(v);
+}
 
 }  // extern "C"

@@ -218,11 +218,13 @@ __device__ __forceinline__ uint32_t pack_int4x8(const float (&v)[N], int e0, flo
     t[i] = __float_as_uint(p.x);
     t[i + 1] = __float_as_uint(p.y);
   }
-  uint32_t w = t[7];
-#pragma unroll
-  for (int i = 6; i >= 0; --i) w = (w << 4) + t[i];
-  constexpr uint32_t kHigh = kRoundMagicBits * 0x11111111u;   // sum of the magic parts, mod 2^32
-  return (w - kHigh) ^ 0x88888888u;
+  // Low byte of t[i] + (t[i+1] << 4) is the offset nibble pair: t[i] & 0xFF is
+  // 8 + q (no borrow), and the magic part of t[i+1] shifted by 4 has a zero
+  // low byte.  Gather the four low bytes, then flip the nibbles' top bits.
+  const uint32_t p0 = t[0] + (t[1] << 4), p1 = t[2] + (t[3] << 4);
+  const uint32_t p2 = t[4] + (t[5] << 4), p3 = t[6] + (t[7] << 4);
+  const uint32_t w = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040), 0x5410);
+  return w ^ 0x88888888u;
 }
 
 // The same with an explicit clamp to [-7, 7] (subnormal, zero or huge scales).
@@ -272,6 +274,16 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, flo
       : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
   return w;
 }
+
+// Scale arithmetic.  The scales are m / 7 (int4, then rounded to fp16) and
+// m / 127 (int8, fp32); they are formed as m * fp32(1/q) and inverted with the
+// fast reciprocal.  Each step is within 2 ulp (relative error < 3e-7), far
+// inside the 1e-6 window in which a rounding decision may go either way, so
+// the codes and scales equal the exactly rounded ones everywhere else.
+constexpr float kInv7 = 1.0f / 7.0f;
+constexpr float kInv127 = 1.0f / 127.0f;
+
+__device__ __forceinline__ float fast_recip(float s) { return __fdividef(1.0f, s); }
 
 // --------------------------------------------------------------- epilogues
 // Each epilogue owns N consecutive rotated-but-unnormalised values z of one
@@ -323,9 +335,9 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
       if (spg >= 4) mz = fmaxf(mz, fmaxf(m32[j ^ 2], m32[j ^ 3]));
     }
     const float m = mz * norm;                         // absmax of y (rounding is monotone)
-    const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
+    const __half s16 = __float2half_rn(m * kInv7);
     const float s = __half2float(s16);
-    const float r = (s > 0.f && s <= 65504.f) ? __frcp_rn(s) : 0.f;   // zero / inf scale -> zero codes
+    const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;   // zero / inf scale -> zero codes
     const float rn = r * norm;
     uint4 w;
     if (mz * rn < 7.25f) {        // normal scale: every |v * rn| <= 7.0035, no clamp
@@ -340,7 +352,7 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
       w.w = pack_int4x8_clamped<PERM>(v, 32 * j + 24, rn);
     }
     reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
-    if ((j & (spg - 1)) == 0) scales[(e0 + 32 * j) / group] = s16;
+    if ((j & (spg - 1)) == 0) scales[(e0 + 32 * j) >> (__ffs(group) - 1)] = s16;   // group is a power of 2
   }
 }
 
@@ -373,8 +385,8 @@ template <bool PERM, int N>
 __device__ __forceinline__ void store_int8(const float (&v)[N], float norm, float m, int8_t* __restrict__ codes,
                                            int64_t e0) {
   static_assert(N % 8 == 0, "int8 chunk must hold whole 8-byte stores");
-  const float s = __fdiv_rn(m, 127.0f);
-  const float r = (s > 0.f && s <= 3.0e38f) ? __frcp_rn(s) : 0.f;
+  const float s = m * kInv127;
+  const float r = (s >= 1.0e-36f && s <= 3.0e38f) ? fast_recip(s) : (s > 0.f ? __frcp_rn(s) : 0.f);
   const float rn = r * norm;
   if (m * r < 127.25f) {         // normal scale: every |v * rn| < 127.5, no clamp
     if constexpr (N % 16 == 0) {

@@ -14,14 +14,20 @@
 // butterfly stages.  The epilogue reads one TMEM lane (= one hi') per thread,
 // runs the remaining LO butterfly stages over lo in registers and quantizes.
 //
-// Roles (one CTA per SM, persistent over tiles):
+// Roles (one CTA per SM, persistent over tiles; tile = TILE_N columns =
+// TILE_N / 2^LO rows):
 //   warp 0      TMA producer: X tiles (box 2^LO x 128 x R, 64B/128B swizzle,
-//               no multicast) into a ring of kStages shared-memory stages;
-//   warp 1      TMEM allocator and MMA issuer (one thread), double-buffered
-//               accumulators (kAccBufs x 128 columns);
-//   warps 2..5  epilogue, warp w reading TMEM lanes 32 * (w % 4) + [0, 32).
-// Every mbarrier wait is bounded; on timeout the kernel records a fault in
-// hadq_tc_fault and stops issuing work.
+//               no multicast) into a ring of STAGES shared-memory stages;
+//   warp 1      TMEM allocator and MMA issuer (one thread); accumulators in
+//               512 / TILE_N tensor-memory buffers;
+//   warps 2..   4 * SPLIT epilogue warps; warp w reads TMEM lanes
+//               32 * (w % 4) + [0, 32) for the rows r = j (mod SPLIT) of every
+//               tile, j = (w - 2) / 4, so each tile is finished by all of them.
+// The producer starts streaming as soon as the barriers exist; the other
+// warps build H_128 in shared memory and allocate tensor memory meanwhile.
+// Every mbarrier wait gives up after one second (globaltimer); on timeout the
+// kernel records a fault in hadq_tc_fault, stops issuing work and still
+// releases its tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -30,14 +36,33 @@
 namespace hadq {
 namespace tc {
 
-constexpr int kStages = 5;
-constexpr int kAccBufs = 4;
-constexpr int kAccCols = 128;            // fp32 accumulator columns per tile
-constexpr int kTmemCols = kAccBufs * kAccCols;
-constexpr int kTileBytes = 128 * 128 * 2;  // B operand: K = 128 rows x N = 128 bf16
 constexpr int kABytes = 128 * 128 * 2;     // A operand: H_128 in bf16
-constexpr int kThreads = 192;
-constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits (~seconds)
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after 1 s
+
+template <int LO_, int TILE_N_, int STAGES_, int SPLIT_>
+struct TcCfg {
+  static constexpr int LO = LO_, L = 1 << LO;
+  static constexpr int TILE_N = TILE_N_;                  // MMA N: columns per tile
+  static constexpr int R = TILE_N / L;                    // rows per tile
+  static constexpr int STAGES = STAGES_;
+  static constexpr int TILE_BYTES = 128 * TILE_N * 2;     // B operand: K = 128 x N bf16
+  static constexpr int TMEM_COLS = 512;                   // the whole tensor memory of the SM
+  static constexpr int ACC_BUFS = TMEM_COLS / TILE_N;
+  static constexpr int SPLIT = SPLIT_;                    // epilogue warps per TMEM lane quarter
+  static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
+  static_assert(LO == 5 || LO == 6, "tensor-core path covers n = 4096 and 8192");
+  static_assert(R >= 1 && (TILE_N == 64 || TILE_N == 128), "tile of 64 or 128 columns");
+  // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, A K-major,
+  // B MN-major, N = TILE_N, M = 128.
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                    (static_cast<uint32_t>(TILE_N >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  // Shared memory (offsets from a 1024-byte aligned base).
+  static constexpr int SM_A = 0;                          // H_128, 2 K-panels x 16 KB
+  static constexpr int SM_B = SM_A + kABytes;             // STAGES x TILE_BYTES
+  static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
+  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * STAGES + 2 * ACC_BUFS);
+  static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;  // + alignment slack
+};
 
 // Fault codes written to hadq_tc_fault.
 constexpr unsigned kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u;
@@ -58,26 +83,45 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Wait for the phase with parity `parity` to complete; false after kSpinLimit tries.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with parity `parity` to complete; false after kWaitLimitNs.
+// Each try_wait may suspend the warp in hardware for up to kSuspendHintNs (it
+// resumes as soon as the phase completes), so waiting warps do not spin on
+// issue slots the working warps need.
+constexpr uint32_t kSuspendHintNs = 100000;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    uint32_t ok;
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  if (ok) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     if (ok) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
-  return false;
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
       ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
@@ -91,17 +135,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 
 constexpr uint32_t kSwizzle128 = 2, kSwizzle64 = 4;
 
-// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, A K-major,
-// B MN-major, N = 128, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            (static_cast<uint32_t>(kAccCols >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(accumulate));
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -132,16 +172,6 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 __device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits that ran out)
 
-// Shared-memory layout (offsets from a 1024-byte aligned base).
-struct Smem {
-  static constexpr int kA = 0;                                   // H_128, 2 K-panels x 16 KB
-  static constexpr int kB = kA + kABytes;                        // kStages x 32 KB
-  static constexpr int kBars = kB + kStages * kTileBytes;        // mbarriers
-  static constexpr int kTmemSlot = kBars + 8 * (2 * kStages + 2 * kAccBufs);
-  static constexpr int kEnd = kTmemSlot + 16;
-  static constexpr int kDynamicBytes = kEnd + 1024;              // + alignment slack
-};
-
 // Epilogue for one row of one tile: z holds the 2^LO values of TMEM lane hi'
 // (after the tensor-core stage over hi); finish the butterfly over lo and emit.
 template <int LO, int MODE>
@@ -169,9 +199,9 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
 #pragma unroll
     for (int j = 0; j < L / 32; ++j) {
       const float m = (j == 0 ? mz_lo : mz_hi) * norm;
-      const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
+      const __half s16 = __float2half_rn(m * kInv7);
       const float s = __half2float(s16);
-      const float r = (s > 0.f && s <= 65504.f) ? __frcp_rn(s) : 0.f;
+      const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
       const float rn = r * norm;
       uint4 w;
       if ((j == 0 ? mz_lo : mz_hi) * rn < 7.25f) {
@@ -183,7 +213,8 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
       }
       if (row_ok) {
         reinterpret_cast<uint4*>(static_cast<uint8_t*>(out0) + ((e0 + 32 * j) >> 1))[0] = w;
-        if (((e0 + 32 * j) % group) == 0) static_cast<__half*>(out1)[(e0 + 32 * j) / group] = s16;
+        if (((e0 + 32 * j) & (group - 1)) == 0)   // group is a power of 2
+          static_cast<__half*>(out1)[(e0 + 32 * j) >> (__ffs(group) - 1)] = s16;
       }
     }
   } else if constexpr (MODE == OUT_MXFP4) {
@@ -195,139 +226,144 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
   }
 }
 
-template <int LO, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <class C, int MODE>
+__global__ void __launch_bounds__(C::THREADS, 1)
 tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, float norm, int group,
                  void* __restrict__ out0, void* __restrict__ out1) {
-  constexpr int L = 1 << LO;          // lo values per row per TMEM lane
-  constexpr int R = 128 / L;          // rows per tile
-  static_assert(LO == 5 || LO == 6, "tensor-core path covers n = 4096 and 8192");
+  constexpr int LO = C::LO, L = C::L, R = C::R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
-  uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + kAccBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::kTmemSlot);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tiles = (rows + R - 1) / R;
 
-  // A = H_128 (K-major, 128-byte swizzle, two K-panels of 64): element (m, k)
-  // at panel (k / 64) + m * 128 + (k % 64) * 2 bytes, 16-byte chunk index
-  // XOR-ed with (m % 8).
-  for (int i = threadIdx.x; i < 128 * 128 / 8; i += kThreads) {
-    const int m = i >> 4, kc = i & 15;                // 8 consecutive k per 16-byte chunk
-    uint32_t w[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      uint32_t h2 = 0;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int k = kc * 8 + p * 2 + q;
-        const uint32_t neg = __popc(m & k) & 1;
-        h2 |= (neg ? 0xBF80u : 0x3F80u) << (16 * q);  // bf16 -1 / +1
-      }
-      w[p] = h2;
-    }
-    const int panel = kc >> 3, chunk = kc & 7;
-    const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
-    *reinterpret_cast<uint4*>(smem + Smem::kA + off) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < kAccBufs; ++b) {
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);      // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], 4 * C::SPLIT);  // every epilogue warp reads every tile
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // A visible to the tensor core
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  grid_dependency_sync();   // x may be written by the previous kernel in the stream
 
   if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
+      grid_dependency_sync();   // x may be written by the previous kernel in the stream
       uint32_t it = 0;
       for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (it >= kStages && !mbar_wait(&empty[s], ph ^ 1)) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (it >= C::STAGES && !mbar_wait(&empty[s], ph ^ 1)) {
           atomicOr(&hadq_tc_fault, kFaultProducer);
           break;
         }
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
-        tma_load_3d(smem + Smem::kB + s * kTileBytes, &xmap, 0, 0, static_cast<int>(t * R), &full[s]);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t a_base = smem_u32(smem + Smem::kA);
-      uint32_t it = 0;
-      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        const int b = it % kAccBufs;
-        const uint32_t aph = (it / kAccBufs) & 1;
-        if (!mbar_wait(&full[s], ph) || (it >= kAccBufs && !mbar_wait(&acc_empty[b], aph ^ 1))) {
-          atomicOr(&hadq_tc_fault, kFaultMma);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t b_base = smem_u32(smem + Smem::kB + s * kTileBytes);
-        const uint32_t d = tmem_base + b * kAccCols;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // K = 128 in steps of 16
-          const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
-          const uint64_t b_desc = (LO == 5) ? smem_desc(b_base + kk * 1024, 8192, 512, kSwizzle64)
-                                            : smem_desc(b_base + kk * 2048, 16384, 1024, kSwizzle128);
-          mma_bf16(d, a_desc, b_desc, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&empty[s]);      // stage s may be refilled once these MMAs have read it
-        mma_commit(&acc_full[b]);   // accumulator b is ready for the epilogue
+        mbar_arrive_expect_tx(&full[s], C::TILE_BYTES);
+        tma_load_3d(smem + C::SM_B + s * C::TILE_BYTES, &xmap, 0, 0, static_cast<int>(t * R), &full[s]);
       }
     }
   } else {
-    const int quarter = warp & 3;            // TMEM lanes this warp may access
-    const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
-    uint32_t it = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
-      const int b = it % kAccBufs;
-      const uint32_t aph = (it / kAccBufs) & 1;
-      if (!mbar_wait(&acc_full[b], aph)) {
-        atomicOr(&hadq_tc_fault, kFaultEpilogue);
-        ok = false;
-        break;
+    // A = H_128 (K-major, 128-byte swizzle, two K-panels of 64): element (m, k)
+    // at panel (k / 64) + m * 128 + (k % 64) * 2 bytes, 16-byte chunk index
+    // XOR-ed with (m % 8).  Entry (m, k) = (-1)^popcount(m & k) as bf16.
+    for (int i = threadIdx.x - 32; i < 128 * 16; i += C::THREADS - 32) {
+      const int m = i >> 4, kc = i & 15;              // 8 consecutive k per 16-byte chunk
+      uint32_t w[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int k = kc * 8 + 2 * p;
+        w[p] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
       }
-      tc_fence_after();
-      float z[R][L];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * kAccCols;
+      const int panel = kc >> 3, chunk = kc & 7;
+      const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
+      *reinterpret_cast<uint4*>(smem + C::SM_A + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // A visible to the tensor core
+    if (warp == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(C::THREADS - 32) : "memory");   // warps 1.. only
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 1) {
+      // ------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t a_base = smem_u32(smem + C::SM_A);
+        uint32_t it = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          const int b = it % C::ACC_BUFS;
+          const uint32_t aph = (it / C::ACC_BUFS) & 1;
+          if (!mbar_wait(&full[s], ph) || (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
+            atomicOr(&hadq_tc_fault, kFaultMma);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(smem + C::SM_B + s * C::TILE_BYTES);
+          const uint32_t d = tmem_base + b * C::TILE_N;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-#pragma unroll
-        for (int c = 0; c < L; c += 32) tmem_ld32(taddr + r * L + c, &z[r][c]);
+          for (int kk = 0; kk < 8; ++kk) {   // K = 128 in steps of 16
+            const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
+            const uint64_t b_desc = (LO == 5) ? smem_desc(b_base + kk * 1024, 8192, 512, kSwizzle64)
+                                              : smem_desc(b_base + kk * 2048, 16384, 1024, kSwizzle128);
+            mma_bf16(d, a_desc, b_desc, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);      // stage s may be refilled once these MMAs have read it
+          mma_commit(&acc_full[b]);   // accumulator b is ready for the epilogue
+        }
       }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    } else {
+      // --------------------------------------------------------- epilogue
+      grid_dependency_sync();                  // outputs may still be read by the previous kernel
+      const int quarter = warp & 3;            // TMEM lanes this warp may access
+      const int sub = (warp - 2) >> 2;         // rows r = sub (mod SPLIT) of every tile
+      const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int b = it % C::ACC_BUFS;
+        const uint32_t aph = (it / C::ACC_BUFS) & 1;
+        if (!mbar_wait(&acc_full[b], aph)) {
+          atomicOr(&hadq_tc_fault, kFaultEpilogue);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * C::TILE_N;
+        constexpr int RW = (R + C::SPLIT - 1) / C::SPLIT;   // rows per warp per tile (at most)
+        float z[RW][L];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t row = t * R + r;
-        tc_emit_row<LO, MODE>(z[r], hi, row, row < rows, n, norm, group, out0, out1);
+        for (int j = 0; j < RW; ++j) {
+          const int r = sub + C::SPLIT * j;
+          if (r < R) {
+#pragma unroll
+            for (int c = 0; c < L; c += 32) tmem_ld32(taddr + r * L + c, &z[j][c]);
+          }
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+#pragma unroll
+        for (int j = 0; j < RW; ++j) {
+          const int r = sub + C::SPLIT * j;
+          if (r < R) {
+            const int64_t row = t * R + r;
+            tc_emit_row<LO, MODE>(z[j], hi, row, row < rows, n, norm, group, out0, out1);
+          }
+        }
       }
     }
   }
@@ -336,7 +372,8 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+    const uint32_t tmem_base = *tmem_slot;
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
   }
 }
 

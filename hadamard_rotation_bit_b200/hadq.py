@@ -27,6 +27,7 @@ FMTS = {"int4": 0, "int8": 1, "mxfp4": 2}
 EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
+    "hadq_device_faults",
 )
 
 _lock = threading.Lock()
@@ -65,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_last_error.restype = ctypes.c_char_p
         lib.hadq_version.argtypes = []
         lib.hadq_version.restype = i32
+        lib.hadq_device_faults.argtypes = [i32]
+        lib.hadq_device_faults.restype = i32
         _lib = lib
         return lib
 
@@ -95,6 +98,11 @@ def _rows_n(x: torch.Tensor):
         raise HadqError(HADQ_ERR_INVALID_ARG, "tensors must be contiguous")
     n = x.shape[-1] if x.dim() else 1
     return (x.numel() // n if n else 0), n
+
+
+def hadq_device_faults(clear: bool = True) -> int:
+    """Fault bits of kernels whose bounded waits ran out (0 = none)."""
+    return int(load_library().hadq_device_faults(1 if clear else 0))
 
 
 def codes_nbytes(rows: int, n: int, fmt: str) -> int:

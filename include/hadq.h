@@ -143,6 +143,12 @@ HADQ_API const char* hadq_status_string(hadq_status status);
 /* One-line reason for the calling thread's most recent failed call ("" if none). */
 HADQ_API const char* hadq_last_error(void);
 
+/* Fault bits recorded by kernels whose bounded internal waits ran out (0 when
+ * every wait completed; -1 if the flag could not be read).  Synchronous:
+ * call after the work of interest has completed.  `clear` != 0 resets the
+ * flags.  No paper counterpart: a diagnostic of this implementation. */
+HADQ_API int hadq_device_faults(int clear);
+
 /* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
 HADQ_API int hadq_version(void);
 

@@ -1,0 +1,137 @@
+"""GPU parity of the tensor-core (tcgen05 + TMA) path against the float64 oracle.
+
+The path serves full-size rotations of b = 4096 and 8192 with bf16 input and
+is the default there.  Every test runs it (HADQ_KERNEL=tensor), compares with
+the oracle exactly as the butterfly tests do, and checks that no bounded wait
+inside the kernel ran out (hadq_device_faults() == 0).
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from hadamard_rotation_bit_b200 import hadq as H
+from hadamard_rotation_bit_b200 import workloads as W
+from tests import parity_check as pc
+from tests.test_gpu_parity import NPROC, _log, run_quant, run_rotate, synth, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def tensor_path():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    old = os.environ.get("HADQ_KERNEL")
+    os.environ["HADQ_KERNEL"] = "tensor"
+    H.hadq_device_faults(clear=True)
+    yield
+    torch.cuda.synchronize()
+    faults = H.hadq_device_faults(clear=True)
+    if old is None:
+        os.environ.pop("HADQ_KERNEL", None)
+    else:
+        os.environ["HADQ_KERNEL"] = old
+    assert faults == 0, f"tensor-core kernel reported fault bits {faults}"
+
+
+SIZES = [(4, 4096, 0), (19, 4096, 0), (2, 8192, 0), (7, 8192, 0), (3, 12288, 4096), (3, 16384, 8192),
+         (1, 4096, 0), (1, 8192, 0)]
+
+
+@pytest.mark.parametrize("rows,n,block", SIZES)
+def test_tc_rotate(rows, n, block):
+    stored, x64 = synth(rows, n, "bf16", seed=n + rows + 101)
+    _log(f"tc-rot-f32-{rows}x{n}", pc.check_rotation_f32(x64, run_rotate(stored, "bf16", block, "f32"), block))
+    _log(f"tc-rot-bf16-{rows}x{n}", pc.check_rotation_bf16(x64, run_rotate(stored, "bf16", block, "bf16"), block))
+
+
+@pytest.mark.parametrize("rows,n,block", SIZES)
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
+def test_tc_quant(rows, n, block, fmt, group):
+    stored, x64 = synth(rows, n, "bf16", seed=3 * n + rows + group, dist="t" if fmt == "mxfp4" else "normal")
+    codes, scales = run_quant(stored, "bf16", block, fmt, group)
+    _log(f"tc-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, codes, scales, block, group))
+
+
+@pytest.mark.parametrize("rows,n,fmt,group", [(2501, 4096, "int4", 128), (3001, 8192, "mxfp4", 32),
+                                              (1037, 4096, "mxfp4", 32), (999, 8192, "int4", 64)])
+def test_tc_many_tiles_ragged(rows, n, fmt, group):
+    stored, x64 = synth(rows, n, "bf16", seed=rows + 7)
+    codes, scales = run_quant(stored, "bf16", 0, fmt, group)
+    _log(f"tc-grid-{fmt}-{rows}x{n}", pc.check(fmt, x64, codes, scales, 0, group))
+
+
+def test_default_path_is_the_tensor_core_kernel():
+    """With HADQ_KERNEL unset the full-size bf16 rotation takes the tensor-core
+    kernel: same codes as the forced tensor path, bit for bit."""
+    stored, x64 = synth(64, 4096, "bf16", seed=5)
+    c_t, s_t = run_quant(stored, "bf16", 0, "int4", 128)
+    os.environ.pop("HADQ_KERNEL", None)
+    c_d, s_d = run_quant(stored, "bf16", 0, "int4", 128)
+    os.environ["HADQ_KERNEL"] = "tensor"
+    np.testing.assert_array_equal(c_d, c_t)
+    np.testing.assert_array_equal(s_d, s_t)
+
+
+def test_tc_config_c2():
+    w = W.WORKLOADS["c2"]
+    stored = W.generate("c2", workers=NPROC)
+    codes, scales = run_quant(stored, "bf16", w.block, "int4", 128)
+    _log("tc-c2", pc.check_int4(W.bits_to_float64(stored, "bf16"), codes, scales, w.block, 128))
+
+
+def test_tc_config_c5():
+    w = W.WORKLOADS["c5"]
+    stored = W.generate("c5", workers=NPROC)
+    codes, scales = run_quant(stored, "bf16", w.block, "mxfp4", 32)
+    rng = np.random.default_rng(5)
+    ids = np.unique(np.concatenate([np.arange(256), np.arange(w.rows - 256, w.rows),
+                                    rng.choice(w.rows, 2048, replace=False)]))
+    _log("tc-c5", pc.check_mxfp4(W.bits_to_float64(stored[ids], "bf16"), codes[ids], scales[ids], w.block))
+
+
+def test_tc_matches_butterfly_codes():
+    """Both implementations agree with the oracle; here also with each other
+    outside the oracle's boundary window (same C2 slice, same format)."""
+    stored, x64 = synth(512, 4096, "bf16", seed=77)
+    c_tc, s_tc = run_quant(stored, "bf16", 0, "int4", 128)
+    os.environ["HADQ_KERNEL"] = "butterfly"
+    c_bf, s_bf = run_quant(stored, "bf16", 0, "int4", 128)
+    os.environ["HADQ_KERNEL"] = "tensor"
+    pc.check_int4(x64, c_tc, s_tc, 0, 128)
+    pc.check_int4(x64, c_bf, s_bf, 0, 128)
+    differ = (pc.unpack_nibbles(c_tc, True) != pc.unpack_nibbles(c_bf, True)).sum()
+    assert differ <= 64, f"{differ} codes differ between the two implementations"
+
+
+def test_tc_guard_bytes_and_offsets():
+    rows, n = 37, 8192
+    stored, x64 = synth(rows, n, "bf16", seed=12)
+    x = to_dev(stored, "bf16")
+    pad = 4096
+    cbytes, sbytes = rows * n // 2, rows * n // 32
+    cbuf = torch.full((cbytes + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((sbytes + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda")
+    codes = cbuf[pad:pad + cbytes].view(rows, n // 2)
+    scales = sbuf[pad:pad + sbytes].view(rows, n // 32)
+    H.hadq_rotate_quant(x, 0, "mxfp4", 32, codes=codes, scales=scales)
+    torch.cuda.synchronize()
+    cb, sb = cbuf.cpu().numpy(), sbuf.cpu().numpy()
+    assert (cb[:pad] == 0xA5).all() and (cb[pad + cbytes:] == 0xA5).all()
+    assert (sb[:pad] == 0x5A).all() and (sb[pad + sbytes:] == 0x5A).all()
+    pc.check_mxfp4(x64, codes.cpu().numpy(), scales.cpu().numpy(), 0)
+
+
+def test_tc_offsets_beyond_2_31_elements():
+    n = 8192
+    rows = (1 << 31) // n + 64
+    x = torch.zeros((rows, n), dtype=torch.bfloat16, device="cuda")
+    tail, x64 = synth(64, n, "bf16", seed=31)
+    x[-64:] = torch.from_numpy(tail.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales = H.hadq_rotate_quant(x, 0, "mxfp4", 32)
+    torch.cuda.synchronize()
+    pc.check_mxfp4(x64, codes[-64:].cpu().numpy(), scales[-64:].cpu().numpy(), 0)
+    del x, codes, scales
+    torch.cuda.empty_cache()
