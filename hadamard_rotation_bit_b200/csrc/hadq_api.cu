@@ -7,6 +7,7 @@
 #include "hadq.h"
 #include "hadq_kernels.cuh"
 #include "hadq_tc.cuh"
+#include "hadq_tc128.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -285,9 +286,10 @@ hadq_status launch_result(cudaError_t e, const char* what) {
 
 // ------------------------------------------------------- tensor-core path
 
-// Which implementation serves full-size bf16 rotations of 4096 and 8192:
-// HADQ_KERNEL = "auto" or unset (the tcgen05 + TMA kernel), "tensor" (the
-// same), or "butterfly" (the CUDA-core team kernel, kept for comparison).
+// Which implementation serves bf16 rotations the tensor-core kernels cover
+// (full size 4096 / 8192, and block 128): HADQ_KERNEL = "auto" or unset (the
+// tcgen05 + TMA kernels), "tensor" (the same), or "butterfly" (the CUDA-core
+// kernels, kept for comparison).
 enum class KernelChoice { Auto, Butterfly, Tensor };
 
 KernelChoice kernel_choice() {
@@ -374,6 +376,60 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
                        "tensor-core kernel launch");
 }
 
+// Block-128 rotations of bf16 rows on the tensor cores: every 128-element
+// block is a row of the MMA's A operand.  Per-token int8 takes one row per
+// tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
+using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, float, int, void*, void*);
+using Tc128C = hadq::tc::Tc128Cfg<4, 2>;
+
+Tc128Fn tc128_fn(int mode) {
+  switch (mode) {
+    case hadq::OUT_F32: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_F32>;
+    case hadq::OUT_BF16: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_BF16>;
+    case hadq::OUT_INT4: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_INT4>;
+    case hadq::OUT_MXFP4: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_MXFP4>;
+    default: return &hadq::tc::tc128_kernel<Tc128C, -1>;
+  }
+}
+
+bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
+  if (x_dtype != HADQ_BF16 || sh.b != 128) return false;
+  if (mode >= 0) return true;
+  const int64_t bpr = sh.n >> 7;            // whole 8-row swizzle atoms per tile
+  return bpr >= 32 && bpr <= 128 && bpr % 8 == 0;
+}
+
+hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
+                         cudaStream_t stream, int sms, int dev) {
+  const int64_t blocks = sh.rows * (sh.n >> 7);
+  if (blocks > (int64_t(1) << 31) - 256) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many blocks");
+  const int bpt = mode < 0 ? static_cast<int>(sh.n >> 7) : 128;   // blocks per tile
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (encode == nullptr) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  CUtensorMap maps[2];
+  for (int p = 0; p < 2; ++p) {
+    cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(blocks)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(bpt)};
+    cuuint32_t estr[2] = {1, 1};
+    void* base = const_cast<char*>(static_cast<const char*>(x)) + 128 * p;
+    const CUresult r = encode(&maps[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  }
+  Tc128Fn fn = tc128_fn(mode);
+  const int smem = Tc128C::SMEM_BYTES;
+  int occ = 0;
+  hadq_status st = occupancy(reinterpret_cast<const void*>(fn), dev, Tc128C::THREADS, smem, &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t tiles = (blocks + bpt - 1) / bpt;
+  const int64_t grid = std::min<int64_t>(tiles, sms);
+  return launch_result(launch_pdl(fn, grid, Tc128C::THREADS, smem, stream, maps[0], maps[1], blocks, bpt, sh.norm,
+                                  group, out0, out1),
+                       "tensor-core block-128 kernel launch");
+}
+
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
 // -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
@@ -384,8 +440,10 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   const bool bf = x_dtype == HADQ_BF16;
   const bool full_seg = sh.logb == sh.logs;
   (void)cudaGetLastError();   // launch errors below must be ours
-  if (tc_eligible(x_dtype, sh, mode) && kernel_choice() != KernelChoice::Butterfly)
-    return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev);
+  if (kernel_choice() != KernelChoice::Butterfly) {
+    if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev);
+    if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev);
+  }
   if (mode >= 0) {
     if (sh.b <= 128) {
       SegFn fn = seg_fn_any(bf, full_seg, sh.logs, mode);

@@ -1,7 +1,8 @@
 """GPU parity of the tensor-core (tcgen05 + TMA) path against the float64 oracle.
 
-The path serves full-size rotations of b = 4096 and 8192 with bf16 input and
-is the default there.  Every test runs it (HADQ_KERNEL=tensor), compares with
+The path serves full-size rotations of b = 4096 and 8192 and block-128
+rotations (R3 heads, R4 rotation_size 128) with bf16 input and is the
+default there.  Every test runs it (HADQ_KERNEL=tensor), compares with
 the oracle exactly as the butterfly tests do, and checks that no bounded wait
 inside the kernel ran out (hadq_device_faults() == 0).
 """
@@ -135,3 +136,68 @@ def test_tc_offsets_beyond_2_31_elements():
     pc.check_mxfp4(x64, codes[-64:].cpu().numpy(), scales[-64:].cpu().numpy(), 0)
     del x, codes, scales
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------- block-128 kernel
+
+B128 = [(37, 128), (1, 128), (300, 128), (13, 1024), (5, 14336), (129, 4096)]
+
+
+@pytest.mark.parametrize("rows,n", B128)
+def test_tc128_rotate(rows, n):
+    stored, x64 = synth(rows, n, "bf16", seed=n + rows + 5)
+    _log(f"tc128-rot-f32-{rows}x{n}", pc.check_rotation_f32(x64, run_rotate(stored, "bf16", 128, "f32"), 128))
+    _log(f"tc128-rot-bf16-{rows}x{n}", pc.check_rotation_bf16(x64, run_rotate(stored, "bf16", 128, "bf16"), 128))
+
+
+@pytest.mark.parametrize("rows,n", B128)
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
+def test_tc128_quant(rows, n, fmt, group):
+    stored, x64 = synth(rows, n, "bf16", seed=5 * n + rows + group, dist="t" if fmt == "mxfp4" else "normal")
+    codes, scales = run_quant(stored, "bf16", 128, fmt, group)
+    _log(f"tc128-{fmt}{group}-{rows}x{n}", pc.check(fmt, x64, codes, scales, 128, group))
+
+
+@pytest.mark.parametrize("rows,n", [(5, 14336), (77, 4096), (33, 16384), (3, 8192)])
+def test_tc128_int8_per_token(rows, n):
+    stored, x64 = synth(rows, n, "bf16", seed=rows * 3 + n)
+    codes, scales = run_quant(stored, "bf16", 128, "int8", 0)
+    _log(f"tc128-int8-{rows}x{n}", pc.check_int8(x64, codes, scales, 128))
+
+
+def test_tc128_config_c3():
+    w = W.WORKLOADS["c3"]
+    stored = W.generate("c3", workers=NPROC)
+    codes, scales = run_quant(stored, "bf16", w.block, "int8", 0)
+    _log("tc128-c3", pc.check_int8(W.bits_to_float64(stored, "bf16"), codes, scales, w.block))
+
+
+def test_tc128_config_c4():
+    wq = W.WORKLOADS["c4q"]
+    q_stored = W.generate("c4q", workers=NPROC)
+    q_out = run_rotate(q_stored, "bf16", 128, "bf16")
+    k_stored = W.generate("c4k", workers=NPROC)
+    k_codes, k_scales = run_quant(k_stored, "bf16", 128, "int4", 128)
+    rng = np.random.default_rng(4)
+    ids = np.unique(np.concatenate([np.arange(4096), np.arange(wq.rows - 4096, wq.rows),
+                                    rng.choice(wq.rows, 65536, replace=False)]))
+    _log("tc128-c4q", pc.check_rotation_bf16(W.bits_to_float64(q_stored[ids], "bf16"), q_out[ids], 128))
+    _log("tc128-c4k", pc.check_int4(W.bits_to_float64(k_stored[ids], "bf16"), k_codes[ids], k_scales[ids], 128, 128))
+
+
+def test_tc128_guard_bytes_ragged_blocks():
+    rows, n = 301, 128
+    stored, x64 = synth(rows, n, "bf16", seed=19)
+    x = to_dev(stored, "bf16")
+    pad = 4096
+    cbytes, sbytes = rows * n // 2, rows * n // 128 * 2
+    cbuf = torch.full((cbytes + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((sbytes + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda")
+    codes = cbuf[pad:pad + cbytes].view(rows, n // 2)
+    scales = sbuf[pad:pad + sbytes].view(torch.float16).view(rows, 1)
+    H.hadq_rotate_quant(x, 128, "int4", 128, codes=codes, scales=scales)
+    torch.cuda.synchronize()
+    cb, sb = cbuf.cpu().numpy(), sbuf.cpu().numpy()
+    assert (cb[:pad] == 0xA5).all() and (cb[pad + cbytes:] == 0xA5).all()
+    assert (sb[:pad] == 0x5A).all() and (sb[pad + sbytes:] == 0x5A).all()
+    pc.check_int4(x64, codes.cpu().numpy(), scales.cpu().numpy(), 128, 128)
