@@ -531,6 +531,35 @@ int quant_mode(hadq_fmt fmt) {
   return fmt == HADQ_INT4_SYM ? hadq::OUT_INT4 : fmt == HADQ_MXFP4 ? hadq::OUT_MXFP4 : -1;
 }
 
+// ----------------------------------------------- allocation-free host path
+// Device staging for hadq_rotate_quant_host_static: one file-scope array that
+// every GPU loading this library holds until the process exits.  In host code
+// `g_static_scratch` only names the symbol; its device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;   // 32 MiB per GPU
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::map<int, void*> g_static_scratch_ptr;   // device -> device address of g_static_scratch (under g_mu)
+
+hadq_status static_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_static_scratch_ptr.find(dev);
+  if (it == g_static_scratch_ptr.end()) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(HADQ_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") + cudaGetErrorString(e));
+    it = g_static_scratch_ptr.emplace(dev, p).first;
+  }
+  *ptr = it->second;
+  return HADQ_OK;
+}
+
+size_t align256(int64_t v) { return (static_cast<size_t>(v) + 255) & ~size_t(255); }
+
 }  // namespace
 
 extern "C" {
@@ -575,6 +604,48 @@ hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dtype, int64
   (void)cudaGetLastError();
   cudaError_t e = cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(xb), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy x to device: ") + cudaGetErrorString(e));
+  st = launch(x_dev, x_dtype, sh, quant_mode(fmt), g, codes_dev, scales_dev, s);
+  if (st != HADQ_OK) return st;
+  e = cudaMemcpyAsync(codes_host, codes_dev, static_cast<size_t>(cb), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy codes to host: ") + cudaGetErrorString(e));
+  e = cudaMemcpyAsync(scales_host, scales_dev, static_cast<size_t>(sb), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy scales to host: ") + cudaGetErrorString(e));
+  return HADQ_OK;
+}
+
+hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n,
+                                          int64_t block, hadq_fmt fmt, int64_t group, void* codes_host,
+                                          void* scales_host, void* stream) {
+  g_last_error.clear();
+  Shape sh;
+  int g = 0;
+  hadq_status st = check_shape(x_dtype, rows, n, block, &sh);
+  if (st != HADQ_OK) return st;
+  st = check_quant(fmt, group, sh, &g);
+  if (st != HADQ_OK || rows == 0) return st;
+  if (x_host == nullptr || codes_host == nullptr || scales_host == nullptr)
+    return fail(HADQ_ERR_INVALID_ARG, "null host pointer");
+  if (!aligned16(x_host) || !aligned16(codes_host) || !aligned16(scales_host))
+    return fail(HADQ_ERR_MISALIGNED, "host buffers must be 16-byte aligned");
+  const int64_t xb = rows * n * esize(x_dtype), cb = codes_bytes(rows, n, fmt), sb = scales_bytes(rows, n, fmt, g);
+  const Span hx = span(x_host, xb), hc = span(codes_host, cb), hs = span(scales_host, sb);
+  if (overlaps(hx, hc) || overlaps(hx, hs) || overlaps(hc, hs))
+    return fail(HADQ_ERR_INVALID_ARG, "host x, codes and scales must not overlap");
+  if (align256(xb) + align256(cb) + align256(sb) > kStaticScratchBytes)
+    return fail(HADQ_ERR_UNSUPPORTED,
+                "input + codes + scales exceed the 32 MiB static device scratch of hadq_rotate_quant_host_static; "
+                "use hadq_rotate_quant_host with caller-owned device buffers");
+  void* scratch = nullptr;
+  st = static_scratch(&scratch);   // first call on a device: resolve the symbol's device address
+  if (st != HADQ_OK) return st;
+  unsigned char* base = static_cast<unsigned char*>(scratch);
+  void* x_dev = base;
+  void* codes_dev = base + align256(xb);
+  void* scales_dev = base + align256(xb) + align256(cb);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(xb), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("copy x to static scratch: ") + cudaGetErrorString(e));
   st = launch(x_dev, x_dtype, sh, quant_mode(fmt), g, codes_dev, scales_dev, s);
   if (st != HADQ_OK) return st;
   e = cudaMemcpyAsync(codes_host, codes_dev, static_cast<size_t>(cb), cudaMemcpyDeviceToHost, s);

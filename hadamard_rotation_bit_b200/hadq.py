@@ -27,7 +27,7 @@ FMTS = {"int4": 0, "int8": 1, "mxfp4": 2}
 EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
-    "hadq_device_faults",
+    "hadq_device_faults", "hadq_rotate_quant_host_static",
 )
 
 _lock = threading.Lock()
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_version.restype = i32
         lib.hadq_device_faults.argtypes = [i32]
         lib.hadq_device_faults.restype = i32
+        lib.hadq_rotate_quant_host_static.argtypes = [vp, i32, i64, i64, i64, i32, i64, vp, vp, vp]
+        lib.hadq_rotate_quant_host_static.restype = i32
         _lib = lib
         return lib
 
@@ -173,3 +175,14 @@ def hadq_rotate_quant_host(x_host: torch.Tensor, block: int, fmt: str, group: in
     _check(lib.hadq_rotate_quant_host(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt], group,
                                       codes_host.data_ptr(), scales_host.data_ptr(), x_dev.data_ptr(),
                                       codes_dev.data_ptr(), scales_dev.data_ptr(), _stream_handle(stream)))
+
+
+def hadq_rotate_quant_host_static(x_host: torch.Tensor, block: int, fmt: str, group: int,
+                                  codes_host: torch.Tensor, scales_host: torch.Tensor, stream=None) -> None:
+    """Host buffers only: the library stages through its own static device
+    array (32 MiB per GPU), so this call allocates no device memory."""
+    lib = load_library()
+    rows, n = _rows_n(x_host)
+    _check(lib.hadq_rotate_quant_host_static(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt],
+                                             group, codes_host.data_ptr(), scales_host.data_ptr(),
+                                             _stream_handle(stream)))

@@ -132,6 +132,37 @@ HADQ_API hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dty
                                    hadq_fmt fmt, int64_t group, void* codes_host, void* scales_host,
                                    void* x_dev, void* codes_dev, void* scales_dev, void* stream);
 
+/*
+ * hadq_rotate_quant_host_static: hadq_rotate_quant_host for callers that
+ * cannot allocate device memory.  Some callers cannot call cudaMalloc at all:
+ * a host-only C or Fortran application that links libhadq but manages no
+ * device memory, or a plugin inside a framework whose allocator owns every
+ * device byte (allocating behind its back breaks its pooling and budget).
+ * This entry point allocates nothing: it stages x, codes and scales in a
+ * 32 MiB array that the library itself declares as static device memory, so
+ * the caller passes only host buffers (page-locked for asynchronous copies).
+ * There is no counterpart on the pages: it is a deployment variant of the
+ * host-buffer entry point above, with the same operation and results.
+ *
+ *   - Sizes: input bytes + code bytes + scale bytes, each rounded up to 256,
+ *     must not exceed 32 MiB (e.g. 2048 x 4096 bf16 with int4 g128 fits);
+ *     larger calls return HADQ_ERR_UNSUPPORTED and do nothing.
+ *   - The static array exists once per GPU that loads the library and lives
+ *     until the process exits.  The first call on a device looks up its
+ *     device address (a one-time set-up per device, made with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls whose work overlaps
+ *     on the GPU (for example on two streams without ordering between them)
+ *     race on it: order them on one stream or synchronize between them.
+ *     Nothing in the array has to start at zero: each call's copy fills the
+ *     input region and its kernel writes every code and scale byte.
+ *   - Otherwise as hadq_rotate_quant_host: enqueued on `stream`, the caller
+ *     synchronizes before reading codes_host / scales_host.
+ */
+HADQ_API hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n,
+                                                   int64_t block, hadq_fmt fmt, int64_t group, void* codes_host,
+                                                   void* scales_host, void* stream);
+
 /* Bytes of the code and scale outputs of hadq_rotate_quant for these sizes
  * (0 for an invalid combination). */
 HADQ_API int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt);
