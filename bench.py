@@ -22,6 +22,8 @@ copies in and out inside the timed region).
 Under torchrun every rank processes its own batch (weak scaling, no
 collective on the data path); rank 0 prints one JSON line.
 `--impl reference` times the float64 CPU oracle on the host cores instead.
+`--rows R` keeps only the first R rows of every workload part (a smaller case
+of the same kernel, for profiler captures); the default is the full workload.
 """
 
 from __future__ import annotations
@@ -61,27 +63,38 @@ def _env_int(k, d):
         return d
 
 
-def step_bytes(cfg):
-    return sum(W.WORKLOADS[k].algorithmic_bytes for k in STEP_PARTS[cfg])
+def part_rows(key, rows=None):
+    """Rows of one workload part: all of them, or the first `rows`."""
+    w = W.WORKLOADS[key]
+    return w.rows if rows is None else max(1, min(w.rows, rows))
 
 
-def n_buffers(cfg):
+def step_bytes(cfg, rows=None):
+    return sum(W.WORKLOADS[k].algorithmic_bytes * part_rows(k, rows) // W.WORKLOADS[k].rows
+               for k in STEP_PARTS[cfg])
+
+
+def n_buffers(cfg, rows=None):
     """Distinct buffer sets rotated through so that every step reads data not
     touched for at least ~3 L2 capacities (or inputs larger than L2)."""
-    return int(max(1, min(8, -(-3 * L2_BYTES // step_bytes(cfg)))))
+    return int(max(1, min(8, -(-3 * L2_BYTES // step_bytes(cfg, rows)))))
 
 
-def config_block(cfg="c2"):
+def config_block(cfg="c2", rows=None):
     parts = [W.WORKLOADS[k] for k in STEP_PARTS[cfg]]
-    nb = n_buffers(cfg)
-    d = {"workload": " + ".join(w.name for w in parts), "algorithmic_bytes_per_step": step_bytes(cfg),
-         "l2": (f"inputs larger than L2 ({step_bytes(cfg) / 1e6:.0f} MB per step)" if nb == 1 else
-                f"{nb} rotating buffer sets ({nb * step_bytes(cfg) / 1e6:.0f} MB > L2 126 MB)"
-                if nb * step_bytes(cfg) > L2_BYTES else
-                f"{nb} buffer sets, {nb * step_bytes(cfg) / 1e6:.1f} MB: L2-resident (parity-size config)")}
+    nb = n_buffers(cfg, rows)
+    sb = step_bytes(cfg, rows)
+    d = {"workload": " + ".join(w.name for w in parts), "algorithmic_bytes_per_step": sb,
+         "l2": (f"inputs larger than L2 ({sb / 1e6:.0f} MB per step)" if nb == 1 else
+                f"{nb} rotating buffer sets ({nb * sb / 1e6:.0f} MB > L2 126 MB)"
+                if nb * sb > L2_BYTES else
+                f"{nb} buffer sets, {nb * sb / 1e6:.1f} MB: L2-resident (parity-size config)")}
     if len(parts) == 1:
         w = parts[0]
-        d.update({"rows": w.rows, "n": w.n, "block": w.block, "fmt": w.fmt, "group": w.group, "x_dtype": w.x_dtype})
+        d.update({"rows": part_rows(w.key, rows), "n": w.n, "block": w.block, "fmt": w.fmt, "group": w.group,
+                  "x_dtype": w.x_dtype})
+    if rows is not None:
+        d["rows_override"] = rows
     return d
 
 
@@ -94,10 +107,14 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Sources of the C2 kernel and of its launch configuration.
+C2_KERNEL_SOURCES = ("hadq_api.cu", "hadq_device.cuh", "hadq_tc.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_rotation_bit_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in C2_KERNEL_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -252,9 +269,9 @@ def run_reference(args):
         dist.destroy_process_group()
 
 
-def _device_input(key, seed, dev, workers):
+def _device_input(key, seed, dev, workers, rows=None):
     w = W.WORKLOADS[key]
-    stored = W.generate(key, seed=seed, workers=workers)
+    stored = W.generate(key, None if rows is None else slice(0, part_rows(key, rows)), seed=seed, workers=workers)
     if w.x_dtype == "bf16":
         return stored, torch.from_numpy(stored.view(np.int16)).view(torch.bfloat16).to(dev)
     return stored, torch.from_numpy(stored).to(dev)
@@ -269,12 +286,12 @@ def run_hadq(args):
     cfg = args.config
     keys = STEP_PARTS[cfg]
     steps, warm = args.steps, max(3, args.warmup)
-    nbuf = n_buffers(cfg)
+    nbuf = n_buffers(cfg, args.rows)
     workers = max(1, min(16, (os.cpu_count() or 2) // 2))
 
     host, bufs = {}, []
     for k in keys:
-        host[k], x0 = _device_input(k, W.rank_seed(rank), dev, workers)
+        host[k], x0 = _device_input(k, W.rank_seed(rank), dev, workers, args.rows)
         bufs.append([x0] + [x0.clone() for _ in range(nbuf - 1)])
 
     def launch(j, i, stream=None, outs=None):
@@ -289,7 +306,7 @@ def run_hadq(args):
 
     outs = [[launch(j, i) for i in range(nbuf)] for j in range(len(keys))]   # allocate outputs, warm caches
     torch.cuda.synchronize()
-    bytes_step = step_bytes(cfg)
+    bytes_step = step_bytes(cfg, args.rows)
     stream = torch.cuda.Stream(device=dev)
 
     def step(i):
@@ -369,14 +386,16 @@ def run_hadq(args):
         stream.synchronize()
         e2e_max = max_over_ranks(dist, e0.elapsed_time(e1) / 1e3)
         e2e = {"value": aggregate_gbs(bytes_step, e2e_steps, world, e2e_max), "unit": UNIT,
-               "h2d_bytes_per_step": sum(W.WORKLOADS[k].in_bytes for k in keys),
-               "d2h_bytes_per_step": sum(W.WORKLOADS[k].out_bytes for k in keys),
+               "h2d_bytes_per_step": sum(W.WORKLOADS[k].in_bytes * part_rows(k, args.rows) // W.WORKLOADS[k].rows
+                                         for k in keys),
+               "d2h_bytes_per_step": sum(W.WORKLOADS[k].out_bytes * part_rows(k, args.rows) // W.WORKLOADS[k].rows
+                                         for k in keys),
                "path": "hadq_rotate_quant_host (pinned host buffers, copies in and out inside the timed region)"}
 
     if rank == 0:
         peak, peak_kind = measured_peak()
         achieved = bytes_step / interval_max / 1e9
-        rows_step = sum(W.WORKLOADS[k].rows for k in keys)
+        rows_step = sum(part_rows(k, args.rows) for k in keys)
         line = {
             "metric": METRIC if cfg == "c2" else f"fused Hadamard+quant GB/s ({cfg})",
             "value": aggregate_gbs(bytes_step, steps, world, elapsed_max),
@@ -390,12 +409,12 @@ def run_hadq(args):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic",
-            "config": config_block(cfg),
+            "config": config_block(cfg, args.rows),
             "impl": "hadq",
             "rows_per_s": rows_step * steps * world / elapsed_max,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
-                         "traffic": recorded_traffic() if cfg == "c2" else None,
+                         "traffic": recorded_traffic() if cfg == "c2" and args.rows is None else None,
                          "duration": "mean launch interval of K back-to-back steps in one CUDA graph "
                                      "(CUDA events on the launching stream around the graph replay)",
                          "step_interval_us": interval_max * 1e6,
@@ -404,7 +423,7 @@ def run_hadq(args):
             "gpu_launches": steps * len(keys),
             "clocks": clocks.summary(),
         }
-        if world == 1 and cfg == "c2" and not args.no_cpu_baseline:
+        if world == 1 and cfg == "c2" and args.rows is None and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)
     del g
@@ -421,6 +440,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", choices=sorted(STEP_PARTS), default="c2",
                     help="workload (default c2, the metric's configuration; others for reference)")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="only the first ROWS rows of each workload part (smaller case for profiler captures)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -317,17 +317,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-using TcFn = void (*)(const CUtensorMap, int64_t, int, float, int, void*, void*);
+using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*);
 
-template <class C>
-TcFn tc_fn_mode(int mode) {
-  switch (mode) {
-    case hadq::OUT_F32: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_F32>;
-    case hadq::OUT_BF16: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_BF16>;
-    case hadq::OUT_INT4: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_INT4>;
-    default: return &hadq::tc::tc_rotate_kernel<C, hadq::OUT_MXFP4>;
-  }
-}
 
 // Tensor-core kernel configuration: 128-column tiles, 5 operand stages, and
 // 4 (n = 4096) or 2 (n = 8192) epilogue warps per tensor-memory lane quarter
@@ -337,13 +328,26 @@ struct TcVariant {
   int threads, smem, tile_n;
 };
 
-template <int LO, int SPLIT>
-TcVariant tc_variant(int mode) {
-  using C = hadq::tc::TcCfg<LO, 128, 5, SPLIT>;
-  return TcVariant{tc_fn_mode<C>(mode), C::THREADS, C::SMEM_BYTES, C::TILE_N};
+template <class C, int MODE>
+TcVariant tc_variant() {
+  return TcVariant{&hadq::tc::tc_rotate_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::TILE_N};
 }
 
-TcVariant tc_pick(int lo, int mode) { return lo == 5 ? tc_variant<5, 4>(mode) : tc_variant<6, 2>(mode); }
+// n = 4096: 4 rows per tile, one row per epilogue warp, 3 stages.  n = 8192:
+// 2 rows per tile, 4 stages; for int4 (whose epilogue is the heaviest) the
+// MMAs are committed per row so the first row's epilogue starts early.
+TcVariant tc_pick(int lo, int mode) {
+  using hadq::tc::TcCfg;
+  using C5 = TcCfg<5, 128, 3, 4, false>;
+  using C6 = TcCfg<6, 128, 4, 2, false>;
+  using C6H = TcCfg<6, 128, 4, 2, true>;
+  switch (mode) {
+    case hadq::OUT_F32: return lo == 5 ? tc_variant<C5, hadq::OUT_F32>() : tc_variant<C6, hadq::OUT_F32>();
+    case hadq::OUT_BF16: return lo == 5 ? tc_variant<C5, hadq::OUT_BF16>() : tc_variant<C6, hadq::OUT_BF16>();
+    case hadq::OUT_INT4: return lo == 5 ? tc_variant<C5, hadq::OUT_INT4>() : tc_variant<C6H, hadq::OUT_INT4>();
+    default: return lo == 5 ? tc_variant<C5, hadq::OUT_MXFP4>() : tc_variant<C6, hadq::OUT_MXFP4>();
+  }
+}
 
 // Blocks of b = 2^(7 + LO) bf16 elements, each rotated in full: the blocks are
 // the rows of a (rows * n / b) x b matrix.
@@ -371,15 +375,15 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
   if (st != HADQ_OK) return st;
   const int64_t tiles = (rows + R - 1) / R;
   const int64_t grid = std::min<int64_t>(tiles, sms);
-  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, rows, static_cast<int>(sh.b), sh.norm,
-                                  group, out0, out1),
+  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, static_cast<const uint16_t*>(x), rows,
+                                  static_cast<int>(sh.b), sh.norm, group, out0, out1),
                        "tensor-core kernel launch");
 }
 
 // Block-128 rotations of bf16 rows on the tensor cores: every 128-element
 // block is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
-using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, float, int, void*, void*);
+using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*);
 using Tc128C = hadq::tc::Tc128Cfg<4, 2>;
 
 Tc128Fn tc128_fn(int mode) {
@@ -425,8 +429,8 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
   if (st != HADQ_OK) return st;
   const int64_t tiles = (blocks + bpt - 1) / bpt;
   const int64_t grid = std::min<int64_t>(tiles, sms);
-  return launch_result(launch_pdl(fn, grid, Tc128C::THREADS, smem, stream, maps[0], maps[1], blocks, bpt, sh.norm,
-                                  group, out0, out1),
+  return launch_result(launch_pdl(fn, grid, Tc128C::THREADS, smem, stream, maps[0], maps[1],
+                                  static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1),
                        "tensor-core block-128 kernel launch");
 }
 

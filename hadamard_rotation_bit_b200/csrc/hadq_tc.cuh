@@ -15,7 +15,7 @@
 // runs the remaining LO butterfly stages over lo in registers and quantizes.
 //
 // Roles (one CTA per SM, persistent over tiles; tile = TILE_N columns =
-// TILE_N / 2^LO rows):
+// TILE_N / 2^LO rows, contiguous in global memory):
 //   warp 0      TMA producer: X tiles (box 2^LO x 128 x R, 64B/128B swizzle,
 //               no multicast) into a ring of STAGES shared-memory stages;
 //   warp 1      TMEM allocator and MMA issuer (one thread); accumulators in
@@ -25,6 +25,13 @@
 //               tile, j = (w - 2) / 4, so each tile is finished by all of them.
 // The producer starts streaming as soon as the barriers exist; the other
 // warps build H_128 in shared memory and allocate tensor memory meanwhile.
+// Before anything else, thread 0 asks L2 to prefetch the CTA's first
+// kPrefetchTiles tiles.  A prefetch is only a hint (no data reaches the CTA
+// and nothing is observed), so it may precede the wait for the previous
+// kernel in the stream; it lets the first TMA loads after that wait hit L2
+// instead of starting cold from HBM.  With HALF, the MMAs of a tile are issued
+// as two N/2 halves with their own commit, so the epilogue warps of the first
+// half start while the tensor core still works on the second.
 // Every mbarrier wait gives up after one second (globaltimer); on timeout the
 // kernel records a fault in hadq_tc_fault, stops issuing work and still
 // releases its tensor memory.
@@ -39,7 +46,9 @@ namespace tc {
 constexpr int kABytes = 128 * 128 * 2;     // A operand: H_128 in bf16
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after 1 s
 
-template <int LO_, int TILE_N_, int STAGES_, int SPLIT_>
+constexpr int kPrefetchTiles = 2;          // tiles per CTA prefetched into L2 at kernel entry
+
+template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_>
 struct TcCfg {
   static constexpr int LO = LO_, L = 1 << LO;
   static constexpr int TILE_N = TILE_N_;                  // MMA N: columns per tile
@@ -50,17 +59,21 @@ struct TcCfg {
   static constexpr int ACC_BUFS = TMEM_COLS / TILE_N;
   static constexpr int SPLIT = SPLIT_;                    // epilogue warps per TMEM lane quarter
   static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
+  static constexpr bool HALF = HALF_;                      // two N/2 MMA halves per tile, committed apart
+  static_assert(!HALF || (R == SPLIT && R % 2 == 0),
+                "HALF: one row per epilogue sub-group, so each half tile has its own sub-groups");
   static_assert(LO == 5 || LO == 6, "tensor-core path covers n = 4096 and 8192");
   static_assert(R >= 1 && (TILE_N == 64 || TILE_N == 128), "tile of 64 or 128 columns");
   // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, A K-major,
   // B MN-major, N = TILE_N, M = 128.
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                     (static_cast<uint32_t>(TILE_N >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  static constexpr uint32_t IDESC_HALF = (IDESC & ~(63u << 17)) | (static_cast<uint32_t>(TILE_N >> 4) << 17);
   // Shared memory (offsets from a 1024-byte aligned base).
   static constexpr int SM_A = 0;                          // H_128, 2 K-panels x 16 KB
   static constexpr int SM_B = SM_A + kABytes;             // STAGES x TILE_BYTES
   static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
-  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * STAGES + 2 * ACC_BUFS);
+  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * STAGES + 3 * ACC_BUFS);
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;  // + alignment slack
 };
 
@@ -235,8 +248,8 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
 
 template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
-tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, float norm, int group,
-                 void* __restrict__ out0, void* __restrict__ out1) {
+tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
+                 float norm, int group, void* __restrict__ out0, void* __restrict__ out1) {
   constexpr int LO = C::LO, L = C::L, R = C::R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,11 +257,19 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, 
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  uint64_t* acc_full2 = acc_empty + C::ACC_BUFS;   // second half of a tile (HALF)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tiles = (rows + R - 1) / R;
 
+  if (threadIdx.x == 0) {
+    int64_t t = blockIdx.x;
+    for (int i = 0; i < kPrefetchTiles && t < tiles; ++i, t += gridDim.x) {
+      const int64_t r1 = (t + 1) * R < rows ? (t + 1) * R : rows;   // a tile is rows [t R, r1), contiguous
+      prefetch_l2(x + t * R * n, static_cast<uint32_t>((r1 - t * R) * n * 2));
+    }
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -257,6 +278,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, 
     for (int b = 0; b < C::ACC_BUFS; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4 * C::SPLIT);  // every epilogue warp reads every tile
+      mbar_init(&acc_full2[b], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -322,15 +344,24 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, 
           tc_fence_after();
           const uint32_t b_base = smem_u32(smem + C::SM_B + s * C::TILE_BYTES);
           const uint32_t d = tmem_base + b * C::TILE_N;
+          // A half tile is R/2 whole rows: half h starts TILE_BYTES/2 into the
+          // stage (rows are the outermost box dimension) and TILE_N/2 columns
+          // into the accumulator.
+          constexpr int NH = C::HALF ? 2 : 1;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {   // K = 128 in steps of 16
-            const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
-            const uint64_t b_desc = (LO == 5) ? smem_desc(b_base + kk * 1024, 8192, 512, kSwizzle64)
-                                              : smem_desc(b_base + kk * 2048, 16384, 1024, kSwizzle128);
-            mma_bf16(d, a_desc, b_desc, C::IDESC, kk > 0 ? 1u : 0u);
+          for (int h = 0; h < NH; ++h) {
+            const uint32_t bh = b_base + h * (C::TILE_BYTES / 2);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {   // K = 128 in steps of 16
+              const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
+              const uint64_t b_desc = (LO == 5) ? smem_desc(bh + kk * 1024, 8192, 512, kSwizzle64)
+                                                : smem_desc(bh + kk * 2048, 16384, 1024, kSwizzle128);
+              mma_bf16(d + h * (C::TILE_N / 2), a_desc, b_desc, C::HALF ? C::IDESC_HALF : C::IDESC,
+                       kk > 0 ? 1u : 0u);
+            }
+            if (h == NH - 1) mma_commit(&empty[s]);   // stage s may be refilled once these MMAs have read it
+            mma_commit(h == 0 ? &acc_full[b] : &acc_full2[b]);   // (this half of) accumulator b is ready
           }
-          mma_commit(&empty[s]);      // stage s may be refilled once these MMAs have read it
-          mma_commit(&acc_full[b]);   // accumulator b is ready for the epilogue
         }
       }
     } else {
@@ -339,11 +370,13 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows, int n, 
       const int quarter = warp & 3;            // TMEM lanes this warp may access
       const int sub = (warp - 2) >> 2;         // rows r = sub (mod SPLIT) of every tile
       const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
+      // With HALF, sub-groups sub < SPLIT/2 own rows of the first half tile.
+      const bool second_half = C::HALF && 2 * sub >= C::SPLIT;
       uint32_t it = 0;
       for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
         const int b = it % C::ACC_BUFS;
         const uint32_t aph = (it / C::ACC_BUFS) & 1;
-        if (!mbar_wait(&acc_full[b], aph)) {
+        if (!mbar_wait(second_half ? &acc_full2[b] : &acc_full[b], aph)) {
           atomicOr(&hadq_tc_fault, kFaultEpilogue);
           break;
         }

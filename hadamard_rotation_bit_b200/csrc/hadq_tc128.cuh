@@ -20,7 +20,9 @@
 // memory in the same layout.  Roles as in hadq_tc.cuh: warp 0 TMA producer,
 // warp 1 TMEM allocator + single-thread MMA issuer, warps 2.. EPI_GROUPS
 // groups of 4 epilogue warps taking whole tiles round-robin.  Waits are
-// bounded (hadq_tc_fault).
+// bounded (hadq_tc_fault).  As there, thread 0 first asks L2 to prefetch the
+// CTA's first kPrefetchTiles tiles (a hint, so it may precede the wait for
+// the previous kernel).
 #pragma once
 
 #include "hadq_tc.cuh"
@@ -50,8 +52,8 @@ struct Tc128Cfg {
 template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
-             int64_t blocks, int blocks_per_tile, float norm, int group, void* __restrict__ out0,
-             void* __restrict__ out1) {
+             const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
+             void* __restrict__ out0, void* __restrict__ out1) {
   constexpr bool PER_TOKEN = MODE < 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -66,6 +68,14 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
   const int64_t tiles = (blocks + blocks_per_tile - 1) / blocks_per_tile;
   const uint32_t tile_bytes = static_cast<uint32_t>(blocks_per_tile) * 256u;   // both panels
 
+  if (threadIdx.x == 0) {
+    int64_t t = blockIdx.x;
+    for (int i = 0; i < kPrefetchTiles && t < tiles; ++i, t += gridDim.x) {
+      const int64_t b0 = t * blocks_per_tile;   // a tile is blocks [b0, b1), contiguous
+      const int64_t b1 = b0 + blocks_per_tile < blocks ? b0 + blocks_per_tile : blocks;
+      prefetch_l2(x + b0 * 128, static_cast<uint32_t>((b1 - b0) * 256));
+    }
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
