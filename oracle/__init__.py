@@ -15,6 +15,11 @@ What it computes, and where the pages define it:
   ``block_size`` blocks (same page, sections 1.2 and 2.1).  The orthogonality
   the page states in its introduction (R @ R^T = I) is what lets the rotated
   activations meet pre-rotated weights.
+* ``random_hadamard_matrix`` / ``rotate_signed`` -- the random Hadamard
+  matrix H @ diag(+/-1) / sqrt(N) of the same section 1.5 (signs persisted as
+  int8, section 1.7), and its transpose diag(+/-1) @ H / sqrt(N), which is its
+  inverse and puts the signs ahead of the transform as in orbitquant's RPBH
+  ("orbitquant 0.2.0", how it works).
 * ``quantize_int4_sym`` / ``quantize_int8_per_token`` -- round-to-nearest
   with symmetric range (the RTN proxy with wbits / groupsize / sym of
   "Pre-Process (Rotation Preprocessing)", OneCompression docs, Workflow note).
@@ -43,13 +48,18 @@ from .hadq_oracle import (  # noqa: F401
     e8m0_exponent,
     fp16_scale_midpoint_distance,
     pack_nibbles,
+    quantize,
     quantize_int4_sym,
     quantize_int8_per_token,
     quantize_mxfp4,
+    random_hadamard_matrix,
     resolve_block,
     rotate,
     rotate_quant,
+    rotate_quant_signed,
+    rotate_signed,
     round_to_binary,
+    sign_vector,
     sylvester_hadamard,
     to_bf16_bits,
     to_fp16,

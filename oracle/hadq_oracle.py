@@ -91,6 +91,56 @@ def rotate(x, block=0) -> np.ndarray:
     return y.reshape(rows, n)
 
 
+def sign_vector(signs) -> np.ndarray:
+    """The +/-1 diagonal of a random Hadamard rotation as float64.
+
+    The signs are persisted as int8 ("Rotation Transform", section 1.7: a
+    random rotation is stored as an int8 +/-1 matrix); reading: a negative
+    entry is -1, any other entry +1.
+    """
+    return np.where(np.asarray(signs).reshape(-1).astype(np.int64) < 0, -1.0, 1.0)
+
+
+def random_hadamard_matrix(signs, side: str = "after") -> np.ndarray:
+    """Normalised random Hadamard matrix of order b = len(signs).
+
+    "Rotation Transform", section 1.5: random_hadamard_matrix(size) is
+    H @ diag(+/-1) / sqrt(N) -- side ``"after"``.  Side ``"before"`` is
+    diag(+/-1) @ H / sqrt(N), its transpose and so its inverse (H and the
+    diagonal are symmetric); it puts the signs on the input, ahead of the
+    Hadamard transform, in the order of the Rademacher signs and block FWHT
+    of orbitquant's RPBH rotation ("orbitquant 0.2.0", how it works).
+    """
+    d = np.diag(sign_vector(signs))
+    h = sylvester_hadamard(d.shape[0])
+    if side == "after":
+        r = h @ d
+    elif side == "before":
+        r = d @ h
+    else:
+        raise ValueError(f"side must be 'after' or 'before', got {side!r}")
+    return r / np.sqrt(float(d.shape[0]))
+
+
+def rotate_signed(x, block, signs, side: str = "after") -> np.ndarray:
+    """y = x . diag(R, ..., R) with R = random_hadamard_matrix(signs, side).
+
+    The random-Hadamard variant of ``rotate`` ("Rotation Transform", section
+    1.2: random_r1..random_r4 replace the deterministic matrix at a
+    position): each block of b = len(signs) elements is multiplied by the same
+    R, as a dense float64 product.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if x.ndim != 2:
+        raise ValueError("rotate_signed expects a 2-D (rows, n) array")
+    rows, n = x.shape
+    b = resolve_block(n, block)
+    if sign_vector(signs).size != b:
+        raise ValueError(f"need {b} signs (one per column of the {b}-point block)")
+    r = random_hadamard_matrix(signs, side)
+    return (x.reshape(rows * (n // b), b) @ r).reshape(rows, n)
+
+
 # ---------------------------------------------------------------------------
 # Rounding onto binary floating-point grids (scales and outputs)
 # ---------------------------------------------------------------------------
@@ -278,7 +328,17 @@ def rotate_quant(x, block, fmt: str, group: int = 0):
     ``"mxfp4"`` (codes packed two per byte, E8M0 bytes per 32).
     Returns ``(y, codes_stored, scales)`` where ``y`` is the float64 rotation.
     """
-    y = rotate(x, block)
+    return quantize(rotate(x, block), fmt, group)
+
+
+def rotate_quant_signed(x, block, signs, side: str, fmt: str, group: int = 0):
+    """``rotate_signed`` then the quantizer of ``rotate_quant`` (same returns)."""
+    return quantize(rotate_signed(x, block, signs, side), fmt, group)
+
+
+def quantize(y, fmt: str, group: int = 0):
+    """The quantizer step of ``rotate_quant`` applied to a rotated ``y``."""
+    y = np.asarray(y, dtype=np.float64)
     if fmt == "int4":
         q, s = quantize_int4_sym(y, group)
         return y, pack_nibbles(q), s

@@ -371,3 +371,109 @@ def test_rotation_flattens_outliers():
     before, after = mu(x), mu(oracle.rotate(x))
     assert before > 10 and after < 0.5 * before
     assert after < 1.5 * np.sqrt(2 * np.log(64 * 64))
+
+
+# ------------------------------------------------- random Hadamard (signs)
+
+def test_random_hadamard_hand_cases():
+    """Hand-summed cases of both sign sides, full and block-diagonal."""
+    gold = load_golden("random_hadamard_cases.json")
+    assert "section 1.5" in gold["citation"]
+    for c in gold["cases"]:
+        x = np.array([c["x"]], dtype=np.float64)
+        y = oracle.rotate_signed(x, c["block"], np.array(c["signs"], dtype=np.int8), c["side"])
+        np.testing.assert_allclose(y[0] * np.sqrt(c["b"]), c["y_times_sqrt_b"], rtol=0, atol=1e-12)
+
+
+def _rademacher(b, seed):
+    return np.where(np.random.default_rng(seed).random(b) < 0.5, -1, 1).astype(np.int8)
+
+
+@pytest.mark.parametrize("b", [2, 16, 128, 1024])
+def test_random_hadamard_matrix_definition(b):
+    """H @ diag(s): column j of the Sylvester matrix times s_j; the transpose
+    puts s_j on row j.  Checked entry by entry against the closed form
+    (-1)^popcount(i & j) s_j, and the stored int8 matrix's first row is s."""
+    s = _rademacher(b, b)
+    i, j = np.meshgrid(np.arange(b), np.arange(b), indexing="ij")
+    pop = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    closed = np.where(pop % 2 == 0, 1.0, -1.0)
+    after = oracle.random_hadamard_matrix(s, "after") * np.sqrt(b)
+    before = oracle.random_hadamard_matrix(s, "before") * np.sqrt(b)
+    np.testing.assert_array_equal(after, closed * s[None, :])
+    np.testing.assert_array_equal(before, closed * s[:, None])
+    np.testing.assert_array_equal(after[0], s)          # first row of the persisted +/-1 matrix
+    np.testing.assert_array_equal(before, after.T)
+
+
+@pytest.mark.parametrize("b", [2, 8, 256, 2048])
+def test_random_hadamard_orthogonal_and_inverse(b):
+    s = _rademacher(b, 7 + b)
+    r = oracle.random_hadamard_matrix(s, "after")
+    np.testing.assert_allclose(r @ r.T, np.eye(b), rtol=0, atol=1e-12)
+    x = np.random.default_rng(b).standard_normal((3, 4 * b))
+    y = oracle.rotate_signed(x, b, s, "after")
+    np.testing.assert_allclose(oracle.rotate_signed(y, b, s, "before"), x, rtol=0, atol=1e-12 * np.sqrt(b))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+
+
+@pytest.mark.parametrize("n,block", [(64, 0), (256, 32), (4096, 0)])
+def test_random_hadamard_all_plus_is_deterministic(n, block):
+    x = np.random.default_rng(n).standard_normal((5, n))
+    b = oracle.resolve_block(n, block)
+    ones = np.ones(b, dtype=np.int8)
+    for side in ("after", "before"):
+        np.testing.assert_allclose(oracle.rotate_signed(x, block, ones, side), oracle.rotate(x, block),
+                                   rtol=0, atol=1e-12 * np.sqrt(b))
+    # any non-negative int8 is +1, any negative int8 is -1
+    np.testing.assert_array_equal(oracle.sign_vector(np.array([0, 1, 127, -1, -128], np.int8)),
+                                  [1.0, 1.0, 1.0, -1.0, -1.0])
+
+
+@pytest.mark.parametrize("n,block", [(128, 0), (1024, 128), (4096, 0)])
+def test_random_hadamard_equals_signs_around_fast_transform(n, block):
+    """Independent route: butterflies, then the column signs (after), or the
+    signs, then butterflies (before)."""
+    b = oracle.resolve_block(n, block)
+    s = _rademacher(b, n + 3).astype(np.float64)
+    x = np.random.default_rng(n + 1).standard_normal((3, n))
+    xb = x.reshape(-1, b)
+    after = (_fwht_butterflies(xb) * s / np.sqrt(b)).reshape(3, n)
+    before = (_fwht_butterflies(xb * s) / np.sqrt(b)).reshape(3, n)
+    si = s.astype(np.int8)
+    np.testing.assert_allclose(oracle.rotate_signed(x, block, si, "after"), after, rtol=0, atol=1e-12 * np.sqrt(b))
+    np.testing.assert_allclose(oracle.rotate_signed(x, block, si, "before"), before, rtol=0, atol=1e-12 * np.sqrt(b))
+
+
+def test_random_hadamard_quantized_codes_follow_the_signs():
+    """Symmetric RTN is odd (q(-v) = -q(v)) and the absmax ignores signs, so
+    the signed-after int4 / int8 codes are the deterministic codes negated in
+    the negative columns, with the same scales; MXFP4 keeps the exponents
+    and flips the sign bit of the code of every nonzero value there (also
+    where the magnitude rounds to 0: the sign bit follows the value)."""
+    n = 256
+    x = np.random.default_rng(11).standard_normal((6, n))
+    s = _rademacher(n, 5)
+    neg = s < 0
+    for fmt, group in (("int4", 128), ("int4", 32), ("int8", 0), ("mxfp4", 32)):
+        y0, c0, s0 = oracle.rotate_quant(x, 0, fmt, group)
+        _, c1, s1 = oracle.rotate_quant_signed(x, 0, s, "after", fmt, group)
+        np.testing.assert_array_equal(s0, s1)
+        if fmt == "int8":
+            np.testing.assert_array_equal(c1, np.where(neg, -c0, c0))
+            continue
+        lo0, hi0 = (c0 & 0xF).astype(np.int64), (c0 >> 4).astype(np.int64)
+        q0 = np.stack([lo0, hi0], axis=-1).reshape(6, n)
+        lo1, hi1 = (c1 & 0xF).astype(np.int64), (c1 >> 4).astype(np.int64)
+        q1 = np.stack([lo1, hi1], axis=-1).reshape(6, n)
+        if fmt == "int4":
+            v0 = np.where(q0 >= 8, q0 - 16, q0)
+            v1 = np.where(q1 >= 8, q1 - 16, q1)
+            np.testing.assert_array_equal(v1, np.where(neg, -v0, v0))
+        else:
+            flip = neg & (y0 != 0)
+            np.testing.assert_array_equal(q1, np.where(flip, q0 ^ 8, q0))
+    with pytest.raises(ValueError):
+        oracle.rotate_signed(x, 0, s[:128], "after")
+    with pytest.raises(ValueError):
+        oracle.rotate_signed(x, 0, s, "sideways")
