@@ -123,10 +123,11 @@ int64_t scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int group) {
 
 // ------------------------------------------------------------ kernel tables
 
-using SegFn = void (*)(const void*, int64_t, int, float, int, void*, void*);
-using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, float*);
-using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*);
-using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*);
+using hadq::Signs;
+using SegFn = void (*)(const void*, int64_t, int, float, int, void*, void*, Signs);
+using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, float*, Signs);
+using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*, Signs);
+using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*, Signs);
 
 template <int LOGS, bool BF, bool FULL>
 SegFn seg_fn(int mode) {
@@ -317,7 +318,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*);
+using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, Signs);
 
 
 // Tensor-core kernel configuration: 128-column tiles, 5 operand stages, and
@@ -352,7 +353,7 @@ TcVariant tc_pick(int lo, int mode) {
 // Blocks of b = 2^(7 + LO) bf16 elements, each rotated in full: the blocks are
 // the rows of a (rows * n / b) x b matrix.
 hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
-                      cudaStream_t stream, int sms, int dev) {
+                      cudaStream_t stream, int sms, int dev, Signs sg) {
   const int lo = sh.logb - 7;
   const TcVariant v = tc_pick(lo, mode);
   const int L = 1 << lo, R = v.tile_n / L;
@@ -376,14 +377,15 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
   const int64_t tiles = (rows + R - 1) / R;
   const int64_t grid = std::min<int64_t>(tiles, sms);
   return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, static_cast<const uint16_t*>(x), rows,
-                                  static_cast<int>(sh.b), sh.norm, group, out0, out1),
+                                  static_cast<int>(sh.b), sh.norm, group, out0, out1, sg),
                        "tensor-core kernel launch");
 }
 
 // Block-128 rotations of bf16 rows on the tensor cores: every 128-element
 // block is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
-using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*);
+using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*,
+                         Signs);
 using Tc128C = hadq::tc::Tc128Cfg<4, 2>;
 
 Tc128Fn tc128_fn(int mode) {
@@ -404,7 +406,7 @@ bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
 }
 
 hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
-                         cudaStream_t stream, int sms, int dev) {
+                         cudaStream_t stream, int sms, int dev, Signs sg) {
   const int64_t blocks = sh.rows * (sh.n >> 7);
   if (blocks > (int64_t(1) << 31) - 256) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many blocks");
   const int bpt = mode < 0 ? static_cast<int>(sh.n >> 7) : 128;   // blocks per tile
@@ -430,23 +432,24 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
   const int64_t tiles = (blocks + bpt - 1) / bpt;
   const int64_t grid = std::min<int64_t>(tiles, sms);
   return launch_result(launch_pdl(fn, grid, Tc128C::THREADS, smem, stream, maps[0], maps[1],
-                                  static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1),
+                                  static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1, sg),
                        "tensor-core block-128 kernel launch");
 }
 
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
-// -1 for per-token int8.
+// -1 for per-token int8.  Signs on the input side (SIGNS_BEFORE) are applied
+// by the butterfly kernels only; the tensor-core kernels take the others.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, Signs sg = Signs{nullptr, hadq::SIGNS_NONE}) {
   int sms = 0, dev = 0;
   hadq_status st = device_sms(&sms, &dev);
   if (st != HADQ_OK) return st;
   const bool bf = x_dtype == HADQ_BF16;
   const bool full_seg = sh.logb == sh.logs;
   (void)cudaGetLastError();   // launch errors below must be ours
-  if (kernel_choice() != KernelChoice::Butterfly) {
-    if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev);
-    if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev);
+  if (kernel_choice() != KernelChoice::Butterfly && sg.side != hadq::SIGNS_BEFORE) {
+    if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
+    if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
   }
   if (mode >= 0) {
     if (sh.b <= 128) {
@@ -457,7 +460,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
       st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, 0, &occ);
       if (st != HADQ_OK) return st;
       const int64_t grid = std::min<int64_t>(ceil_div(segs, hadq::kThreads), int64_t(sms) * occ);
-      return launch_result(launch_pdl(fn, grid, hadq::kThreads, 0, stream, x, segs, sh.logb, sh.norm, group, out0, out1),
+      return launch_result(launch_pdl(fn, grid, hadq::kThreads, 0, stream, x, segs, sh.logb, sh.norm, group, out0, out1,
+                                      sg),
                            "segment kernel launch");
     }
     TeamFn fn = bf ? team_fn_logb<true>(sh.logb, mode) : team_fn_logb<false>(sh.logb, mode);
@@ -468,7 +472,7 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     const int teams = hadq::kThreads >> (sh.logb - 7);
     const int64_t units = sh.rows * (sh.n >> sh.logb);
     const int64_t grid = std::min<int64_t>(ceil_div(units, teams), int64_t(sms) * occ);
-    return launch_result(launch_pdl(fn, grid, hadq::kThreads, smem, stream, x, units, sh.norm, group, out0, out1),
+    return launch_result(launch_pdl(fn, grid, hadq::kThreads, smem, stream, x, units, sh.norm, group, out0, out1, sg),
                          "team kernel launch");
   }
   // per-token int8
@@ -481,7 +485,7 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     st = occupancy(reinterpret_cast<const void*>(fn), dev, block, 0, &occ);
     if (st != HADQ_OK) return st;
     const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
-    return launch_result(launch_pdl(fn, grid, block, 0, stream, x, sh.rows, sh.n, sh.logb, sh.norm, codes, scales),
+    return launch_result(launch_pdl(fn, grid, block, 0, stream, x, sh.rows, sh.n, sh.logb, sh.norm, codes, scales, sg),
                          "per-token int8 kernel launch");
   }
   TeamRowFn fn = bf ? team_row_fn<true>(sh.logb) : team_row_fn<false>(sh.logb);
@@ -491,17 +495,49 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   st = occupancy(reinterpret_cast<const void*>(fn), dev, block, smem, &occ);
   if (st != HADQ_OK) return st;
   const int64_t grid = std::min<int64_t>(sh.rows, int64_t(sms) * occ);
-  return launch_result(launch_pdl(fn, grid, block, smem, stream, x, sh.rows, sh.n, sh.norm, codes, scales),
+  return launch_result(launch_pdl(fn, grid, block, smem, stream, x, sh.rows, sh.n, sh.norm, codes, scales, sg),
                        "per-token int8 kernel launch");
 }
 
+// Random Hadamard signs: a signed entry point passes its caller's side
+// (which must be HADQ_SIGNS_AFTER or HADQ_SIGNS_BEFORE); the unsigned entry
+// points pass kUnsigned, which no caller value can reach.
+constexpr int kUnsigned = -1;
+
+struct SideArg {
+  bool is_signed;
+  int side;
+};
+
+hadq_status check_side(SideArg a) {
+  if (a.is_signed && a.side != HADQ_SIGNS_AFTER && a.side != HADQ_SIGNS_BEFORE)
+    return fail(HADQ_ERR_INVALID_ARG, "side must be HADQ_SIGNS_AFTER or HADQ_SIGNS_BEFORE");
+  return HADQ_OK;
+}
+
+// For rows > 0: the signs array (b bytes) must exist and must not overlap an
+// output, since every CTA reads it while others may already be writing.
+hadq_status make_signs(const int8_t* signs, SideArg a, const Shape& sh, const Span* outs, int nouts, Signs* sg) {
+  *sg = Signs{nullptr, hadq::SIGNS_NONE};
+  if (!a.is_signed) return HADQ_OK;
+  if (signs == nullptr) return fail(HADQ_ERR_INVALID_ARG, "null signs");
+  const Span ss = span(signs, sh.b);
+  for (int i = 0; i < nouts; ++i)
+    if (overlaps(ss, outs[i])) return fail(HADQ_ERR_INVALID_ARG, "signs must not overlap an output");
+  *sg = Signs{signs, a.side == HADQ_SIGNS_AFTER ? hadq::SIGNS_AFTER : hadq::SIGNS_BEFORE};
+  return HADQ_OK;
+}
+
 hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,
-                        hadq_dtype out_dtype, void* stream) {
+                        hadq_dtype out_dtype, void* stream, const int8_t* signs = nullptr,
+                        SideArg side = SideArg{false, kUnsigned}) {
   g_last_error.clear();
   Shape sh;
   hadq_status st = check_shape(x_dtype, rows, n, block, &sh);
   if (st != HADQ_OK) return st;
   if (out_dtype != HADQ_F32 && out_dtype != HADQ_BF16) return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_F32 or HADQ_BF16");
+  st = check_side(side);
+  if (st != HADQ_OK) return st;
   if (rows == 0) return HADQ_OK;
   if (x == nullptr || out == nullptr) return fail(HADQ_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(x) || !aligned16(out)) return fail(HADQ_ERR_MISALIGNED, "x and out must be 16-byte aligned");
@@ -509,9 +545,13 @@ hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t
   const Span so = span(out, rows * n * esize(out_dtype));
   if (overlaps(sx, so) && !(x == out && x_dtype == out_dtype))
     return fail(HADQ_ERR_INVALID_ARG, "out overlaps x (only exact in-place with equal dtypes is allowed)");
+  Signs sg;
+  st = make_signs(signs, side, sh, &so, 1, &sg);
+  if (st != HADQ_OK) return st;
   return launch(x, x_dtype, sh, out_dtype == HADQ_F32 ? hadq::OUT_F32 : hadq::OUT_BF16, 0, out, nullptr,
-                static_cast<cudaStream_t>(stream));
+                static_cast<cudaStream_t>(stream), sg);
 }
+
 
 hadq_status quant_checks(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, hadq_fmt fmt,
                          int64_t group, const void* codes, const void* scales, Shape* sh, int* g) {
@@ -533,6 +573,23 @@ hadq_status quant_checks(const void* x, hadq_dtype x_dtype, int64_t rows, int64_
 
 int quant_mode(hadq_fmt fmt) {
   return fmt == HADQ_INT4_SYM ? hadq::OUT_INT4 : fmt == HADQ_MXFP4 ? hadq::OUT_MXFP4 : -1;
+}
+
+hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                              hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream,
+                              const int8_t* signs = nullptr, SideArg side = SideArg{false, kUnsigned}) {
+  g_last_error.clear();
+  Shape sh;
+  int g = 0;
+  hadq_status st = check_side(side);
+  if (st != HADQ_OK) return st;
+  st = quant_checks(x, x_dtype, rows, n, block, fmt, group, codes, scales, &sh, &g);
+  if (st != HADQ_OK || rows == 0) return st;
+  const Span outs[2] = {span(codes, codes_bytes(rows, n, fmt)), span(scales, scales_bytes(rows, n, fmt, g))};
+  Signs sg;
+  st = make_signs(signs, side, sh, outs, 2, &sg);
+  if (st != HADQ_OK) return st;
+  return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream), sg);
 }
 
 // ----------------------------------------------- allocation-free host path
@@ -580,12 +637,20 @@ hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int64_t rows,
 
 hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, hadq_fmt fmt,
                               int64_t group, void* codes, void* scales, void* stream) {
-  g_last_error.clear();
-  Shape sh;
-  int g = 0;
-  hadq_status st = quant_checks(x, x_dtype, rows, n, block, fmt, group, codes, scales, &sh, &g);
-  if (st != HADQ_OK || rows == 0) return st;
-  return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream));
+  return rotate_quant_impl(x, x_dtype, rows, n, block, fmt, group, codes, scales, stream);
+}
+
+hadq_status hadq_rotate_signed(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                               const int8_t* signs, hadq_sign_side side, void* out, hadq_dtype out_dtype,
+                               void* stream) {
+  return rotate_impl(x, x_dtype, rows, n, block, out, out_dtype, stream, signs, SideArg{true, static_cast<int>(side)});
+}
+
+hadq_status hadq_rotate_quant_signed(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                     const int8_t* signs, hadq_sign_side side, hadq_fmt fmt, int64_t group,
+                                     void* codes, void* scales, void* stream) {
+  return rotate_quant_impl(x, x_dtype, rows, n, block, fmt, group, codes, scales, stream, signs,
+                           SideArg{true, static_cast<int>(side)});
 }
 
 hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,

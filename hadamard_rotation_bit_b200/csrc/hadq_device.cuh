@@ -17,6 +17,23 @@ namespace hadq {
 
 enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3 };
 
+// Random Hadamard signs ("Rotation Transform", section 1.5: H @ diag(+/-1) /
+// sqrt(N), the signs persisted as int8).  AFTER: output column j of every
+// block is multiplied by s_j (R = H diag(s)); BEFORE: input column j is
+// (R = diag(s) H, the transpose and inverse).  s has one int8 per block
+// column; a negative entry is -1.
+enum SignSide : int { SIGNS_NONE = 0, SIGNS_BEFORE = 1, SIGNS_AFTER = 2 };
+
+struct Signs {
+  const int8_t* s;   // b entries, device memory; unused for SIGNS_NONE
+  int side;
+};
+
+// 1 if block column `col` is negated.
+__device__ __forceinline__ uint32_t neg_bit(const int8_t* __restrict__ s, int col) {
+  return s[col] < 0 ? 1u : 0u;
+}
+
 // 1.5 * 2^23: adding it to |v| < 2^22 leaves round-half-even(v) in the low
 // mantissa bits (fp32 addition rounds to the nearest representable value, and
 // the spacing at this magnitude is exactly 1).
@@ -186,6 +203,16 @@ __host__ __device__ constexpr int reg(int e) {
   return PERM ? ((e & ~3) | ((e & 1) << 1) | ((e >> 1) & 1)) : e;
 }
 
+// Flip the sign of register i where bit i of the mask (word i / 32) is set.
+// Each thread's mask is fixed for a whole launch: a thread always holds the
+// same block columns in the same registers.
+template <int N>
+__device__ __forceinline__ void apply_signs(float (&v)[N], const uint32_t (&m)[(N + 31) / 32]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ ((m[i >> 5] << (31 - (i & 31))) & 0x80000000u));
+}
+
 // ------------------------------------------------------------------ quantizers
 
 // Absmax of registers [lo, lo + cnt) (cnt a multiple of 4; order does not matter).
@@ -252,14 +279,16 @@ __device__ __forceinline__ uint32_t pack_int8x4(const float (&v)[N], int e0, flo
 }
 
 // Eight E2M1 codes (round to nearest even, saturating at +/-6, sign in bit 3)
-// of v * f, element i in bits [4i, 4i + 4).
+// of v * f, element i in bits [4i, 4i + 4).  The product is formed as
+// v * f + 0, which turns a zero of either sign into +0, so an exact zero
+// codes as 0 (only a negative nonzero value sets the sign bit).
 template <bool PERM, int N>
 __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, float f) {
-  const float2 f2 = make_float2(f, f);
+  const float2 f2 = make_float2(f, f), z2 = make_float2(0.f, 0.f);
   float a[8];
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
-    const float2 p = __fmul2_rn(make_float2(v[reg<PERM>(e0 + i)], v[reg<PERM>(e0 + i + 1)]), f2);
+    const float2 p = __ffma2_rn(make_float2(v[reg<PERM>(e0 + i)], v[reg<PERM>(e0 + i + 1)]), f2, z2);
     a[i] = p.x;
     a[i + 1] = p.y;
   }

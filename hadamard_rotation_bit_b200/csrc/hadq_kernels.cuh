@@ -34,6 +34,11 @@
 // Every kernel starts with the programmatic-dependent-launch handshake (see
 // grid_dependency_sync) and prefetches its next unit of input into L2 while it
 // computes the current one.
+//
+// Random Hadamard signs (Signs, SIGNS_BEFORE / SIGNS_AFTER): a thread always
+// owns the same block columns in the same registers, so it reads its signs
+// once into a bit mask and flips the loaded values (before) or the rotated
+// values (after) with one XOR of the sign bit each.
 #pragma once
 
 #include "hadq_device.cuh"
@@ -45,14 +50,27 @@ constexpr int kRowFloats = 132;   // transpose row: 128 floats + one quad of pad
 
 // ----------------------------------------------------------- segment kernels
 
+// A segment of S elements starts on a block boundary (b = 2^nbits divides S),
+// so register i holds block column i mod b in every segment.
+template <int S>
+__device__ __forceinline__ void segment_sign_mask(const Signs& sg, int nbits, uint32_t (&sm)[(S + 31) / 32]) {
+#pragma unroll
+  for (int w = 0; w < (S + 31) / 32; ++w) sm[w] = 0u;
+  if (sg.side == SIGNS_NONE) return;
+  const int bmask = (1 << nbits) - 1;
+  for (int i = 0; i < S; ++i) sm[i >> 5] |= neg_bit(sg.s, i & bmask) << (i & 31);
+}
+
 // FULL: b == S, all LOGS stages unconditionally; otherwise the low nbits stages.
 template <int LOGS, bool IN_BF16, int MODE, bool FULL>
 __global__ void __launch_bounds__(kThreads)
 segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, int group,
-               void* __restrict__ out0, void* __restrict__ out1) {
+               void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
   constexpr int S = 1 << LOGS;
   constexpr uint32_t kSegBytes = S * (IN_BF16 ? 2 : 4);
   grid_dependency_sync();
+  uint32_t sm[(S + 31) / 32];
+  segment_sign_mask<S>(sg, nbits, sm);
   float v[S];
   const int lane = threadIdx.x & 31;
   for (int64_t s = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; s < segs;
@@ -66,11 +84,13 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
     }
     const int64_t e0 = s << LOGS;
     load_elems<IN_BF16, S>(x, e0, v);
+    if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
     if constexpr (FULL) {
       fwht_bits<S, 0, LOGS>(v);
     } else {
       fwht_low<S>(v, nbits);
     }
+    if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
     if constexpr (MODE == OUT_F32) {
       store_rotated<false, S, false>(v, norm, out0, e0);
     } else if constexpr (MODE == OUT_BF16) {
@@ -87,9 +107,11 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
 template <int LOGS, bool IN_BF16, bool FULL>
 __global__ void __launch_bounds__(256)
 segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int nbits, float norm,
-                        int8_t* __restrict__ codes, float* __restrict__ scales) {
+                        int8_t* __restrict__ codes, float* __restrict__ scales, Signs sg) {
   constexpr int S = 1 << LOGS;
   grid_dependency_sync();
+  uint32_t sm[(S + 31) / 32];
+  segment_sign_mask<S>(sg, nbits, sm);
   __shared__ float red[32];
   const int segs_row = static_cast<int>(n >> LOGS);
   const bool active = static_cast<int>(threadIdx.x) < segs_row;
@@ -101,11 +123,13 @@ segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int
     const int64_t e0 = r * n + (static_cast<int64_t>(threadIdx.x) << LOGS);
     if (active) {
       load_elems<IN_BF16, S>(x, e0, v);
+      if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
       if constexpr (FULL) {
         fwht_bits<S, 0, LOGS>(v);
       } else {
         fwht_low<S>(v, nbits);
       }
+      if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
     } else {
 #pragma unroll
       for (int i = 0; i < S; ++i) v[i] = 0.f;
@@ -138,17 +162,36 @@ __device__ __forceinline__ void team_sync() {
   }
 }
 
+// Sign mask of team thread tau.  BEFORE: phase-1 register h * CE + j holds
+// block column h * 128 + tau * CE + j.  AFTER: register i holds output column
+// tau * 128 + reg<PERM>(i).
+template <int LOGB>
+__device__ __forceinline__ void team_sign_mask(const Signs& sg, int tau, uint32_t (&sm)[4]) {
+  using Sh = TeamShape<LOGB>;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) sm[w] = 0u;
+  if (sg.side == SIGNS_NONE) return;
+  for (int i = 0; i < 128; ++i) {
+    const int col = sg.side == SIGNS_BEFORE ? (i / Sh::CE) * 128 + tau * Sh::CE + (i % Sh::CE)
+                                            : tau * 128 + reg<Sh::PERM>(i);
+    sm[i >> 5] |= neg_bit(sg.s, col) << (i & 31);
+  }
+}
+
 // Rotate one block of 2^LOGB elements (element base `base`) by a team; on
 // return v[0..128) holds the unnormalised outputs base + tau*128 + [0, 128) in
 // register order TeamShape<LOGB>::PERM.  `rows` is this team's T x kRowFloats
-// shared buffer.
+// shared buffer.  With `before`, the loaded values are first multiplied by
+// the signs in `sm` (team_sign_mask, BEFORE layout).
 template <int LOGB, bool IN_BF16>
 __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t base, bool valid, int tau,
-                                            float* __restrict__ rows, float (&v)[128]) {
+                                            float* __restrict__ rows, float (&v)[128], bool before,
+                                            const uint32_t (&sm)[4]) {
   using Sh = TeamShape<LOGB>;
   if (valid) {
 #pragma unroll
     for (int h = 0; h < Sh::T; ++h) load_elems<IN_BF16, Sh::CE>(x, base + h * 128 + tau * Sh::CE, &v[h * Sh::CE]);
+    if (before) apply_signs<128>(v, sm);
   } else {
 #pragma unroll
     for (int i = 0; i < 128; ++i) v[i] = 0.f;
@@ -195,7 +238,7 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
 template <int LOGB, bool IN_BF16, int MODE>
 __global__ void __launch_bounds__(kThreads, 3)
 team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, void* __restrict__ out0,
-            void* __restrict__ out1) {
+            void* __restrict__ out1, Signs sg) {
   using Sh = TeamShape<LOGB>;
   constexpr int TEAMS = kThreads / Sh::T;
   constexpr uint32_t kUnitBytes = Sh::B * (IN_BF16 ? 2 : 4);
@@ -205,6 +248,8 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
   const int team = threadIdx.x >> Sh::t;
   const int tau = threadIdx.x & (Sh::T - 1);
   float* rows = buf + team * Sh::T * kRowFloats;
+  uint32_t sm[4];
+  team_sign_mask<LOGB>(sg, tau, sm);
   float v[128];
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * TEAMS; u0 < units;
        u0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
@@ -215,8 +260,9 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
     }
     const bool valid = u < units;
     const int64_t base = u << LOGB;
-    team_rotate<LOGB, IN_BF16>(x, base, valid, tau, rows, v);
+    team_rotate<LOGB, IN_BF16>(x, base, valid, tau, rows, v, sg.side == SIGNS_BEFORE, sm);
     if (valid) {
+      if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
       const int64_t e0 = base + tau * 128;
       if constexpr (MODE == OUT_F32) {
         store_rotated<Sh::PERM, 128, false>(v, norm, out0, e0);
@@ -236,7 +282,7 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
 template <int LOGB, bool IN_BF16>
 __global__ void __launch_bounds__(256)
 team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float norm, int8_t* __restrict__ codes,
-                     float* __restrict__ scales) {
+                     float* __restrict__ scales, Signs sg) {
   using Sh = TeamShape<LOGB>;
   grid_dependency_sync();
   extern __shared__ float4 smem_f4[];
@@ -248,13 +294,16 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
   const int tau = threadIdx.x & (Sh::T - 1);
   float* team_rows = buf + (active ? team * Sh::T * kRowFloats : 0);
   const int64_t row_bytes = n * (IN_BF16 ? 2 : 4);
+  uint32_t sm[4];
+  team_sign_mask<LOGB>(sg, tau, sm);
   float v[128];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     if (threadIdx.x == 0 && r + gridDim.x < rows)
       prefetch_l2(static_cast<const char*>(x) + (r + gridDim.x) * row_bytes, static_cast<uint32_t>(row_bytes));
     const int64_t base = r * n + (static_cast<int64_t>(team) << LOGB);
     if (active) {
-      team_rotate<LOGB, IN_BF16>(x, base, true, tau, team_rows, v);
+      team_rotate<LOGB, IN_BF16>(x, base, true, tau, team_rows, v, sg.side == SIGNS_BEFORE, sm);
+      if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
     } else {
       // Idle threads still take part in every barrier of team_rotate.
 #pragma unroll

@@ -194,11 +194,15 @@ __device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits tha
 
 // Epilogue for one row of one tile: z holds the 2^LO values of TMEM lane hi'
 // (after the tensor-core stage over hi); finish the butterfly over lo and emit.
+// With `flip`, output column hi * 2^LO + c is negated where bit c of `sm` is
+// set (random Hadamard, signs after the rotation).
 template <int LO, int MODE>
 __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t row, bool row_ok, int n, float norm,
-                                            int group, void* __restrict__ out0, void* __restrict__ out1) {
+                                            int group, void* __restrict__ out0, void* __restrict__ out1, bool flip,
+                                            const uint32_t (&sm)[(1 << LO) / 32]) {
   constexpr int L = 1 << LO;
   fwht_bits<L, 0, LO>(z);
+  if (flip) apply_signs<L>(z, sm);
   const int64_t e0 = row * n + static_cast<int64_t>(hi) * L;   // first output element of this thread
   if constexpr (MODE == OUT_INT4) {
     // Groups of `group` outputs = L values x (group / L) consecutive lanes.
@@ -249,7 +253,7 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
 template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
-                 float norm, int group, void* __restrict__ out0, void* __restrict__ out1) {
+                 float norm, int group, void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
   constexpr int LO = C::LO, L = C::L, R = C::R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -370,6 +374,14 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
       const int quarter = warp & 3;            // TMEM lanes this warp may access
       const int sub = (warp - 2) >> 2;         // rows r = sub (mod SPLIT) of every tile
       const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
+      // Signs after the rotation (the launcher never passes SIGNS_BEFORE here):
+      // this thread's outputs are block columns hi * L + [0, L).
+      const bool flip = sg.side == SIGNS_AFTER;
+      uint32_t sm[L / 32];
+#pragma unroll
+      for (int w = 0; w < L / 32; ++w) sm[w] = 0u;
+      if (flip)
+        for (int c = 0; c < L; ++c) sm[c >> 5] |= neg_bit(sg.s, hi * L + c) << (c & 31);
       // With HALF, sub-groups sub < SPLIT/2 own rows of the first half tile.
       const bool second_half = C::HALF && 2 * sub >= C::SPLIT;
       uint32_t it = 0;
@@ -401,7 +413,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           const int r = sub + C::SPLIT * j;
           if (r < R) {
             const int64_t row = t * R + r;
-            tc_emit_row<LO, MODE>(z[j], hi, row, row < rows, n, norm, group, out0, out1);
+            tc_emit_row<LO, MODE>(z[j], hi, row, row < rows, n, norm, group, out0, out1, flip, sm);
           }
         }
       }

@@ -53,7 +53,7 @@ template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
              const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
-             void* __restrict__ out0, void* __restrict__ out1) {
+             void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
   constexpr bool PER_TOKEN = MODE < 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -166,6 +166,12 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
       const int quarter = warp & 3;
       const int group_id = (warp - 2) >> 2;
       const int m = quarter * 32 + lane;        // block within the tile = TMEM lane
+      // Signs after the rotation (the launcher never passes SIGNS_BEFORE
+      // here): register k holds block column k.
+      const bool flip = sg.side == SIGNS_AFTER;
+      uint32_t sm[4] = {0u, 0u, 0u, 0u};
+      if (flip)
+        for (int k = 0; k < 128; ++k) sm[k >> 5] |= neg_bit(sg.s, k) << (k & 31);
       uint32_t it = 0;
       bool failed = false;   // a wait ran out: skip the work, keep joining the group's barriers
       float* gred = red + 4 * group_id;
@@ -194,6 +200,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
+        if (flip) apply_signs<128>(z, sm);
         const int64_t blk = t * blocks_per_tile + m;
         const bool ok = m < blocks_per_tile && blk < blocks;
         const int64_t e0 = blk * 128;

@@ -24,10 +24,12 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhadq.so"
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_F32, HADQ_BF16 = 0, 1
 FMTS = {"int4": 0, "int8": 1, "mxfp4": 2}
+HADQ_SIGNS_AFTER, HADQ_SIGNS_BEFORE = 0, 1
+SIDES = {"after": HADQ_SIGNS_AFTER, "before": HADQ_SIGNS_BEFORE}
 EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
-    "hadq_device_faults", "hadq_rotate_quant_host_static",
+    "hadq_device_faults", "hadq_rotate_quant_host_static", "hadq_rotate_signed", "hadq_rotate_quant_signed",
 )
 
 _lock = threading.Lock()
@@ -70,6 +72,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_device_faults.restype = i32
         lib.hadq_rotate_quant_host_static.argtypes = [vp, i32, i64, i64, i64, i32, i64, vp, vp, vp]
         lib.hadq_rotate_quant_host_static.restype = i32
+        lib.hadq_rotate_signed.argtypes = [vp, i32, i64, i64, i64, vp, i32, vp, i32, vp]
+        lib.hadq_rotate_signed.restype = i32
+        lib.hadq_rotate_quant_signed.argtypes = [vp, i32, i64, i64, i64, vp, i32, i32, i64, vp, vp, vp]
+        lib.hadq_rotate_quant_signed.restype = i32
         _lib = lib
         return lib
 
@@ -186,3 +192,43 @@ def hadq_rotate_quant_host_static(x_host: torch.Tensor, block: int, fmt: str, gr
     _check(lib.hadq_rotate_quant_host_static(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt],
                                              group, codes_host.data_ptr(), scales_host.data_ptr(),
                                              _stream_handle(stream)))
+
+
+def _signs_ptr(signs: torch.Tensor | None) -> int | None:
+    if signs is None:
+        return None
+    if signs.dtype != torch.int8 or not signs.is_contiguous():
+        raise HadqError(HADQ_ERR_INVALID_ARG, "signs must be a contiguous int8 tensor")
+    return signs.data_ptr()
+
+
+def hadq_rotate_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "after", block: int = 0,
+                       out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None,
+                       stream=None) -> torch.Tensor:
+    """Random Hadamard rotation: every block times H_b diag(s) / sqrt(b)
+    (side "after") or diag(s) H_b / sqrt(b) (side "before"); ``signs`` holds
+    the b int8 signs on the device (see include/hadq.h)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _check(lib.hadq_rotate_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, _signs_ptr(signs),
+                                  SIDES[side], out.data_ptr(), _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+def hadq_rotate_quant_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "after", block: int = 0,
+                             fmt: str = "int4", group: int = 128, codes: torch.Tensor | None = None,
+                             scales: torch.Tensor | None = None, stream=None):
+    """Random Hadamard rotation and quantization in one pass; returns (codes, scales)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    cs, cd, ss, sd = output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=x.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=x.device)
+    _check(lib.hadq_rotate_quant_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, _signs_ptr(signs),
+                                        SIDES[side], FMTS[fmt], group, codes.data_ptr(), scales.data_ptr(),
+                                        _stream_handle(stream)))
+    return codes, scales

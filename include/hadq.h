@@ -68,6 +68,11 @@ typedef enum hadq_fmt {
   HADQ_MXFP4 = 2              /* E2M1 codes, E8M0 shared exponent per 32 */
 } hadq_fmt;
 
+typedef enum hadq_sign_side {
+  HADQ_SIGNS_AFTER = 0,       /* R = H_b diag(s) / sqrt(b): the random Hadamard matrix */
+  HADQ_SIGNS_BEFORE = 1       /* R = diag(s) H_b / sqrt(b): its transpose and inverse */
+} hadq_sign_side;
+
 /*
  * hadq_rotate: out = x . diag(H_b) / sqrt(b), rotation only.
  *   x        [rows x n] of x_dtype (read only)
@@ -117,6 +122,36 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  */
 HADQ_API hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
                               hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream);
+
+/*
+ * Random Hadamard ("Rotation Transform", AutoRound docs, section 1.5:
+ * random_hadamard_matrix(size) = H @ diag(+/-1) / sqrt(N); section 1.2:
+ * random_r1..random_r4 use it in place of the deterministic matrix; section
+ * 1.7: the +/-1 signs are persisted as int8).  Every b-element block of a row
+ * is multiplied by the same R:
+ *   side HADQ_SIGNS_AFTER   R = H_b diag(s) / sqrt(b): output column j of the
+ *                           block times s_j (the random Hadamard matrix);
+ *   side HADQ_SIGNS_BEFORE  R = diag(s) H_b / sqrt(b): input column j times
+ *                           s_j, then the transform -- the transpose, so
+ *                           applying AFTER then BEFORE with the same signs
+ *                           gives x back; it is also the order of the
+ *                           Rademacher signs ahead of the block FWHT in
+ *                           orbitquant's RPBH rotation ("orbitquant 0.2.0").
+ *   signs   device pointer to b int8 values (b = the block, n when block is
+ *           0 / -1 / n); entry j < 0 means s_j = -1, any other value +1.  Read
+ *           only; it must not overlap an output.  May be null when rows == 0.
+ * Everything else (shapes, formats, alignment, errors, asynchrony) is as for
+ * hadq_rotate / hadq_rotate_quant.  The quantizer sees the signed rotation,
+ * so for AFTER the scales equal the unsigned ones and the codes of negated
+ * columns are negated (MXFP4: sign bit flipped unless the value is exactly 0).
+ */
+HADQ_API hadq_status hadq_rotate_signed(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                        const int8_t* signs, hadq_sign_side side, void* out, hadq_dtype out_dtype,
+                                        void* stream);
+
+HADQ_API hadq_status hadq_rotate_quant_signed(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n,
+                                              int64_t block, const int8_t* signs, hadq_sign_side side,
+                                              hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream);
 
 /*
  * hadq_rotate_quant_host: the same operation on HOST buffers.  Enqueues on

@@ -38,8 +38,8 @@ def unpack_nibbles(packed: np.ndarray, signed: bool) -> np.ndarray:
     return out
 
 
-def check_rotation_f32(x64: np.ndarray, y_gpu: np.ndarray, block: int) -> dict:
-    y = oracle.rotate(x64, block)
+def check_rotation_f32(x64: np.ndarray, y_gpu: np.ndarray, block: int, y=None) -> dict:
+    y = oracle.rotate(x64, block) if y is None else y
     err = np.abs(np.asarray(y_gpu, dtype=np.float64) - y).max(axis=1)
     norm = np.linalg.norm(x64, axis=1)
     rel = err / np.where(norm > 0, norm, 1.0)
@@ -52,7 +52,7 @@ def _bf16_value(bits):
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def check_rotation_bf16(x64: np.ndarray, y_bits: np.ndarray, block: int) -> dict:
+def check_rotation_bf16(x64: np.ndarray, y_bits: np.ndarray, block: int, y=None) -> dict:
     """bf16 output = round-to-nearest-even of a value within the fp32 tolerance.
 
     With d = 1e-5 * ||x_row||, the output must lie between bf16(y - d) and
@@ -60,7 +60,7 @@ def check_rotation_bf16(x64: np.ndarray, y_bits: np.ndarray, block: int) -> dict
     bf16 ulp of bf16(y); near zero the fp32 error bound (relative to the row
     norm) dominates the ulp of the element.
     """
-    y = oracle.rotate(x64, block)
+    y = oracle.rotate(x64, block) if y is None else y
     d = 1e-5 * np.linalg.norm(x64, axis=1, keepdims=True)
     lo = _bf16_value(oracle.to_bf16_bits(y - d))
     hi = _bf16_value(oracle.to_bf16_bits(y + d))
@@ -82,8 +82,8 @@ def _check_codes(got, v, w, encode):
     return ok, boundary
 
 
-def check_int4(x64, codes_packed, scales_fp16, block: int, group: int) -> dict:
-    y = oracle.rotate(x64, block)
+def check_int4(x64, codes_packed, scales_fp16, block: int, group: int, y=None) -> dict:
+    y = oracle.rotate(x64, block) if y is None else y
     rows, n = y.shape
     g = y.reshape(rows, n // group, group)
     m = np.abs(g).max(axis=-1)
@@ -111,8 +111,8 @@ def check_int4(x64, codes_packed, scales_fp16, block: int, group: int) -> dict:
             "code_differs_in_window": int((q_gpu != enc(v)).sum())}
 
 
-def check_int8(x64, codes, scales_fp32, block: int) -> dict:
-    y = oracle.rotate(x64, block)
+def check_int8(x64, codes, scales_fp32, block: int, y=None) -> dict:
+    y = oracle.rotate(x64, block) if y is None else y
     q_o, s_o = oracle.quantize_int8_per_token(y)
     s_o = s_o.astype(np.float64)
     s_gpu = np.asarray(scales_fp32, dtype=np.float32).astype(np.float64)
@@ -133,8 +133,8 @@ def check_int8(x64, codes, scales_fp32, block: int) -> dict:
             "code_boundary_cases": int(boundary.sum()), "code_differs_in_window": int((got != q_o).sum())}
 
 
-def check_mxfp4(x64, codes_packed, scales_e8m0, block: int) -> dict:
-    y = oracle.rotate(x64, block)
+def check_mxfp4(x64, codes_packed, scales_e8m0, block: int, y=None) -> dict:
+    y = oracle.rotate(x64, block) if y is None else y
     rows, n = y.shape
     g = y.reshape(rows, n // 32, 32)
     m = np.abs(g).max(axis=-1)
@@ -156,11 +156,13 @@ def check_mxfp4(x64, codes_packed, scales_e8m0, block: int) -> dict:
             "code_differs_in_window": int((got != oracle.e2m1_encode(v)).sum())}
 
 
-def check(fmt, x64, out0, out1, block, group):
+def check(fmt, x64, out0, out1, block, group, y=None):
+    """``y``: the oracle's rotation when it is not ``oracle.rotate(x64, block)``
+    (e.g. a random Hadamard rotation)."""
     if fmt == "int4":
-        return check_int4(x64, out0, out1, block, group)
+        return check_int4(x64, out0, out1, block, group, y=y)
     if fmt == "int8":
-        return check_int8(x64, out0, out1, block)
+        return check_int8(x64, out0, out1, block, y=y)
     if fmt == "mxfp4":
-        return check_mxfp4(x64, out0, out1, block)
+        return check_mxfp4(x64, out0, out1, block, y=y)
     raise ValueError(fmt)

@@ -127,3 +127,44 @@ def test_binding_raises_without_cuda_tensor(lib):
     import torch
     with pytest.raises(H.HadqError):
         H.hadq_rotate_quant(torch.zeros(4, 96, dtype=torch.float64), 0, "int4", 32)
+
+
+# ------------------------------------------------- random Hadamard entry points
+
+S = 0x60000000       # a fake device address for the signs (never dereferenced)
+
+
+def _qs(lib, x=A, rows=4, n=1024, block=0, signs=S, side=0, fmt=0, group=128, codes=B, scales=C):
+    return lib.hadq_rotate_quant_signed(x, 1, rows, n, block, signs, side, fmt, group, codes, scales, None)
+
+
+def _rs(lib, x=A, rows=4, n=1024, block=0, signs=S, side=0, out=B, od=0):
+    return lib.hadq_rotate_signed(x, 1, rows, n, block, signs, side, out, od, None)
+
+
+def test_signed_empty_calls_are_noops(lib):
+    assert _qs(lib, rows=0, x=None, signs=None, codes=None, scales=None) == H.HADQ_OK
+    assert _rs(lib, rows=0, x=None, signs=None, out=None) == H.HADQ_OK
+    assert _rs(lib, rows=0, x=None, signs=None, out=None, side=H.HADQ_SIGNS_BEFORE) == H.HADQ_OK
+
+
+@pytest.mark.parametrize("call", [_qs, _rs])
+def test_signed_validation(lib, call):
+    assert call(lib, side=2) == H.HADQ_ERR_INVALID_ARG
+    assert "side" in lib.hadq_last_error().decode()
+    assert call(lib, side=-1) == H.HADQ_ERR_INVALID_ARG
+    assert call(lib, rows=0, side=5) == H.HADQ_ERR_INVALID_ARG      # a bad side is rejected even when empty
+    assert call(lib, signs=None) == H.HADQ_ERR_INVALID_ARG
+    assert call(lib, signs=None, side=H.HADQ_SIGNS_BEFORE) == H.HADQ_ERR_INVALID_ARG
+    assert call(lib, n=1000) == H.HADQ_ERR_INVALID_ARG               # shape checks still apply
+    assert call(lib, x=A + 8) == H.HADQ_ERR_MISALIGNED
+
+
+def test_signed_rejects_signs_overlapping_an_output(lib):
+    # codes at B cover rows * n / 2 bytes; signs inside that range
+    assert _qs(lib, signs=B + 16) == H.HADQ_ERR_INVALID_ARG
+    assert "signs" in lib.hadq_last_error().decode()
+    assert _qs(lib, signs=C + 2) == H.HADQ_ERR_INVALID_ARG            # inside the scales
+    assert _rs(lib, signs=B + 100) == H.HADQ_ERR_INVALID_ARG          # inside out (fp32, 16 KB)
+    # block 128: the signs span only 128 bytes, so B - 128 just touches nothing
+    assert _rs(lib, block=128, signs=B - 128, x=None) == H.HADQ_ERR_INVALID_ARG   # null x still caught first

@@ -404,6 +404,9 @@ def test_random_hadamard_matrix_definition(b):
     np.testing.assert_array_equal(before, closed * s[:, None])
     np.testing.assert_array_equal(after[0], s)          # first row of the persisted +/-1 matrix
     np.testing.assert_array_equal(before, after.T)
+    if b <= 128:                                         # the literal products with diag(s)
+        np.testing.assert_array_equal(after, oracle.sylvester_hadamard(b) @ np.diag(s.astype(np.float64)))
+        np.testing.assert_array_equal(before, np.diag(s.astype(np.float64)) @ oracle.sylvester_hadamard(b))
 
 
 @pytest.mark.parametrize("b", [2, 8, 256, 2048])
