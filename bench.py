@@ -52,7 +52,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # A step is one pass of the fused path over one batch of a workload: the
 # launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
-STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"]}
+STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"],
+              "c2r": ["c2r"], "c2rb": ["c2rb"]}
 WORKLOAD = W.WORKLOADS["c2"]
 
 
@@ -289,14 +290,20 @@ def run_hadq(args):
     nbuf = n_buffers(cfg, args.rows)
     workers = max(1, min(16, (os.cpu_count() or 2) // 2))
 
-    host, bufs = {}, []
+    host, bufs, signs = {}, [], {}
     for k in keys:
         host[k], x0 = _device_input(k, W.rank_seed(rank), dev, workers, args.rows)
         bufs.append([x0] + [x0.clone() for _ in range(nbuf - 1)])
+        if W.WORKLOADS[k].signs is not None:
+            signs[k] = torch.from_numpy(W.generate_signs(k, W.rank_seed(rank))).to(dev)
 
     def launch(j, i, stream=None, outs=None):
         w = W.WORKLOADS[keys[j]]
         x = bufs[j][i % nbuf]
+        if w.signs is not None:
+            c, sc = (None, None) if outs is None else outs[j][i % nbuf]
+            return H.hadq_rotate_quant_signed(x, signs[w.key], w.signs, w.block, w.fmt, w.group, codes=c, scales=sc,
+                                              stream=stream)
         if w.fmt is None:
             o = None if outs is None else outs[j][i % nbuf]
             return H.hadq_rotate(x, w.block, out=o, stream=stream,
@@ -356,7 +363,7 @@ def run_hadq(args):
 
     # End to end through the host-buffer entry point (quantizing parts only).
     e2e = None
-    qkeys = [k for k in keys if W.WORKLOADS[k].fmt is not None]
+    qkeys = [k for k in keys if W.WORKLOADS[k].fmt is not None and W.WORKLOADS[k].signs is None]
     if len(qkeys) == len(keys):
         e2e_steps = max(3, min(steps, 20))
         pinned = []

@@ -20,6 +20,10 @@ permutation drawn from a ``seed + 1`` stream):
   (rotate-half pairing (i, i + 64), theta_i = 10000^(-i/64), position = s);
   per-head 128-point rotation; Q -> bf16, K -> int4 group 128.
 * ``c5``  65536 x 8192 bf16 Student-t(3); full 8192-point rotation; MXFP4.
+* ``c2r`` / ``c2rb``  the ``c2`` input and quantizer with a random Hadamard
+  rotation ("Rotation Transform", section 1.5): signs after (the random
+  Hadamard matrix) or before (its transpose); the b signs are Rademacher
+  draws (``generate_signs``), int8 +/-1.
 
 Values are drawn in float64, rounded to float32 (nearest even) and, for
 bf16 tensors, to bfloat16 (nearest even).
@@ -46,6 +50,8 @@ class Workload:
     fmt: str | None     # "int4" | "int8" | "mxfp4" | None (rotation only)
     group: int          # quant group (0 = per token for int8)
     out_dtype: str | None = None   # rotation-only output dtype
+    signs: str | None = None       # random Hadamard: "after" | "before" | None (deterministic)
+    base: str | None = None        # input recipe of another workload (same bits)
 
     @property
     def in_bytes(self) -> int:
@@ -83,9 +89,24 @@ WORKLOADS = {
                     16 * 32 * 4096, 128, 128, "bf16", "int4", 128),
     "c5": Workload("c5", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point Hadamard, MXFP4",
                    65536, 8192, 8192, "bf16", "mxfp4", 32),
+    "c2r": Workload("c2r", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard (signs after), "
+                    "int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128, signs="after", base="c2"),
+    "c2rb": Workload("c2rb", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard transpose "
+                     "(signs before), int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128,
+                     signs="before", base="c2"),
 }
 
 _STREAM = {"c1": 1, "c2": 2, "c3": 3, "c4q": 4, "c4k": 5, "c5": 6}
+_SIGN_STREAM = 100
+
+
+def generate_signs(key: str, seed: int = SEED) -> np.ndarray:
+    """The b int8 Rademacher signs (+/-1) of a random Hadamard workload."""
+    w = WORKLOADS[key]
+    if w.signs is None:
+        raise ValueError(f"{key} has no random Hadamard signs")
+    g = _rng(seed, _SIGN_STREAM, _STREAM[w.base or key])
+    return np.where(g.random(w.block) < 0.5, -1, 1).astype(np.int8)
 
 
 def _rng(seed: int, stream: int, chunk: int) -> np.random.Generator:
@@ -113,6 +134,7 @@ def bits_to_float64(x: np.ndarray, x_dtype: str) -> np.ndarray:
 
 
 def _chunk_values(key: str, chunk: int, seed: int) -> np.ndarray:
+    key = WORKLOADS[key].base or key
     w = WORKLOADS[key]
     r0 = chunk * CHUNK_ROWS
     nr = min(CHUNK_ROWS, w.rows - r0)

@@ -28,6 +28,11 @@ What it computes, and where the pages define it:
   define the format's internals; the reading used is the OCP MX v1.0 rule
   (E2M1 elements, E8M0 shared scale, floor-based exponent).
 
+* ``quantize_nvfp4`` -- the NVFP4 scheme (same page, introduction and section
+  2.1: block 16); the pages give no encoding, the reading used is NVIDIA's
+  public NVFP4 definition (E2M1 elements, an FP8 E4M3 scale per 16 elements,
+  an optional per-tensor fp32 scale).
+
 Readings of points the pages leave open (rounding half to even, the fp16 scale
 used for the codes, the symmetric +/-7 / +/-127 range, zero groups, nibble
 order, non-finite scales) are stated on each function.
@@ -43,8 +48,11 @@ from .hadq_oracle import (  # noqa: F401
     INT4_QMAX,
     INT8_QMAX,
     MX_GROUP,
+    NV_GROUP,
+    E4M3_MAX,
     codes_with_scale,
     e2m1_encode,
+    e4m3_encode,
     e8m0_exponent,
     fp16_scale_midpoint_distance,
     pack_nibbles,
@@ -52,6 +60,7 @@ from .hadq_oracle import (  # noqa: F401
     quantize_int4_sym,
     quantize_int8_per_token,
     quantize_mxfp4,
+    quantize_nvfp4,
     random_hadamard_matrix,
     resolve_block,
     rotate,
@@ -63,5 +72,6 @@ from .hadq_oracle import (  # noqa: F401
     sylvester_hadamard,
     to_bf16_bits,
     to_fp16,
+    to_e4m3,
     to_fp32,
 )

@@ -15,6 +15,8 @@ import numpy as np
 INT4_QMAX = 7      # symmetric int4 range +/-7 (scale = absmax / 7)
 INT8_QMAX = 127    # symmetric int8 range +/-127 (scale = absmax / 127)
 MX_GROUP = 32      # MX block size ("Rotation Transform", section 2.1: 32 for MXFP)
+NV_GROUP = 16      # NVFP4 block size (same section: 16 for NVFP)
+E4M3_MAX = 448.0   # largest finite FP8 E4M3 magnitude
 
 # E2M1 magnitudes indexed by the 3-bit code (exponent 2 bits, mantissa 1 bit).
 E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
@@ -311,6 +313,53 @@ def quantize_mxfp4(y):
     return codes, (e + 127).astype(np.uint8)
 
 
+def to_e4m3(v) -> np.ndarray:
+    """float64 -> FP8 E4M3 value (returns float64 values).
+
+    Round half to even onto 3 stored mantissa bits, smallest normal 2**-6
+    (subnormal spacing 2**-9); magnitudes above the largest finite value 448
+    take 448 (a saturating conversion: E4M3 has no infinity).
+    """
+    r = round_to_binary(v, 3, -6, np.inf)
+    return np.clip(r, -E4M3_MAX, E4M3_MAX)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """E4M3 byte of ``to_e4m3(v)``: sign << 7 | biased exponent (bias 7) << 3 |
+    mantissa; subnormals (below 2**-6) have exponent field 0."""
+    q = to_e4m3(v)
+    a = np.abs(q)
+    normal = a >= 2.0 ** -6
+    e = np.where(normal, _floor_log2(np.where(normal, a, 1.0)), -6)
+    mant = np.where(normal, a / np.ldexp(1.0, e) - 1.0, a / 2.0 ** -6)   # in [0, 1)
+    field = np.where(normal, (e + 7) << 3, 0).astype(np.int64) | np.rint(mant * 8).astype(np.int64)
+    return (field | (np.signbit(q) & (a > 0)).astype(np.int64) << 7).astype(np.uint8)
+
+
+def quantize_nvfp4(y, tensor_scale: float = 1.0):
+    """NVFP4: per 16 elements an E4M3 scale and E2M1 codes.
+
+    The pages name the scheme and its block of 16 ("Rotation Transform",
+    introduction and section 2.1) but not its encoding; reading: NVIDIA's
+    public NVFP4 definition.  With v = y / tensor_scale (the per-tensor
+    second-level scale, 1 for the single-level form): per block
+    s = E4M3(max|v| / 6) and code = E2M1 rne(v / s) (saturating at +/-6, sign
+    bit 3); s == 0 gives codes 0.  Dequantization is code * s * tensor_scale.
+    Returns ``(codes uint8 (rows, n) in [0, 15], scale bytes uint8 (rows, n // 16))``.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    rows, n = y.shape
+    if n % NV_GROUP:
+        raise ValueError(f"n={n} is not a multiple of {NV_GROUP}")
+    if not (np.isfinite(tensor_scale) and tensor_scale > 0):
+        raise ValueError("tensor_scale must be finite and > 0")
+    g = (y / tensor_scale).reshape(rows, n // NV_GROUP, NV_GROUP)
+    s = to_e4m3(np.abs(g).max(axis=-1) / 6.0)
+    safe = np.where(s > 0, s, 1.0)[..., None]
+    codes = np.where(s[..., None] > 0, e2m1_encode(g / safe), 0).astype(np.uint8).reshape(rows, n)
+    return codes, e4m3_encode(s)
+
+
 def pack_nibbles(codes) -> np.ndarray:
     """Two 4-bit codes per byte, the even-indexed element in the low nibble.
 
@@ -322,25 +371,32 @@ def pack_nibbles(codes) -> np.ndarray:
     return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
 
 
-def rotate_quant(x, block, fmt: str, group: int = 0):
+def rotate_quant(x, block, fmt: str, group: int = 0, tensor_scale: float = 1.0):
     """Rotate then quantize, as the fused path does in one pass.
 
     ``fmt`` is ``"int4"`` (codes packed two per byte, fp16 scales per
-    ``group``), ``"int8"`` (per-token; int8 codes, fp32 scale per row) or
-    ``"mxfp4"`` (codes packed two per byte, E8M0 bytes per 32).
-    Returns ``(y, codes_stored, scales)`` where ``y`` is the float64 rotation.
+    ``group``), ``"int8"`` (per-token; int8 codes, fp32 scale per row),
+    ``"mxfp4"`` (codes packed two per byte, E8M0 bytes per 32) or ``"nvfp4"``
+    (codes packed two per byte, E4M3 bytes per 16; ``tensor_scale`` is its
+    per-tensor scale).  Returns ``(y, codes_stored, scales)`` where ``y`` is
+    the float64 rotation.
     """
-    return quantize(rotate(x, block), fmt, group)
+    return quantize(rotate(x, block), fmt, group, tensor_scale)
 
 
-def rotate_quant_signed(x, block, signs, side: str, fmt: str, group: int = 0):
+def rotate_quant_signed(x, block, signs, side: str, fmt: str, group: int = 0, tensor_scale: float = 1.0):
     """``rotate_signed`` then the quantizer of ``rotate_quant`` (same returns)."""
-    return quantize(rotate_signed(x, block, signs, side), fmt, group)
+    return quantize(rotate_signed(x, block, signs, side), fmt, group, tensor_scale)
 
 
-def quantize(y, fmt: str, group: int = 0):
+def quantize(y, fmt: str, group: int = 0, tensor_scale: float = 1.0):
     """The quantizer step of ``rotate_quant`` applied to a rotated ``y``."""
     y = np.asarray(y, dtype=np.float64)
+    if fmt == "nvfp4":
+        if group not in (0, NV_GROUP):
+            raise ValueError("NVFP4 groups are 16 elements")
+        q, s = quantize_nvfp4(y, tensor_scale)
+        return y, pack_nibbles(q), s
     if fmt == "int4":
         q, s = quantize_int4_sym(y, group)
         return y, pack_nibbles(q), s

@@ -163,3 +163,23 @@ def test_signed_exact_zero_rows_code_as_plus_zero(path):
     codes, scales = run_signed_quant(stored, "bf16", 0, s, "after", "mxfp4", 32)
     assert (codes[::2] == 0).all() and (scales[::2] == 0).all()
     pc.check_mxfp4(x64, codes, scales, 0, y=y)
+
+
+@pytest.mark.parametrize("key", ["c2r", "c2rb"])
+def test_signed_config_full_size(key):
+    """The bench's random Hadamard workloads at full size (4096 x 4096 bf16,
+    int4 g128) in the default kernel choice: c2r on the tensor cores, c2rb
+    (signs before) on the butterfly kernels."""
+    from hadamard_rotation_bit_b200 import workloads as W
+    from tests.test_gpu_parity import NPROC
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    H.load_library()
+    w = W.WORKLOADS[key]
+    stored = W.generate(key, workers=NPROC)
+    s = W.generate_signs(key)
+    x64 = W.bits_to_float64(stored, "bf16")
+    y = oracle.rotate_signed(x64, w.block, s, w.signs)
+    H.hadq_device_faults(clear=True)
+    codes, scales = run_signed_quant(stored, "bf16", w.block, s, w.signs, "int4", 128)
+    assert H.hadq_device_faults(clear=True) == 0
+    _log(f"signed-{key}", pc.check_int4(x64, codes, scales, w.block, 128, y=y))

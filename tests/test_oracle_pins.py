@@ -480,3 +480,69 @@ def test_random_hadamard_quantized_codes_follow_the_signs():
         oracle.rotate_signed(x, 0, s[:128], "after")
     with pytest.raises(ValueError):
         oracle.rotate_signed(x, 0, s, "sideways")
+
+
+# ------------------------------------------------------------------ NVFP4
+
+def test_nvfp4_hand_cases():
+    gold = load_golden("nvfp4_cases.json")
+    assert "section 2.1" in gold["citation"]
+    for c in gold["cases"]:
+        q, s = oracle.quantize_nvfp4(np.array([c["y"]], dtype=np.float64), c["tensor_scale"])
+        np.testing.assert_array_equal(q[0], c["codes"])
+        assert int(s[0, 0]) == c["scale_byte"]
+        assert float(oracle.to_e4m3(np.max(np.abs(c["y"])) / c["tensor_scale"] / 6.0)) == c["scale"]
+    e = gold["e4m3"]
+    np.testing.assert_array_equal(oracle.e4m3_encode(np.array(e["values"])), e["bytes"])
+
+
+def test_e4m3_matches_torch_float8_in_range():
+    """Inside the finite range the rounding and the byte layout are torch's
+    float8_e4m3fn conversion (round half to even); every grid point and every
+    midpoint between neighbours is included."""
+    grid = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).float().double().numpy()
+    mids = (grid[1:] + grid[:-1]) / 2
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([grid, mids, rng.uniform(0, 448, 4000), np.exp(rng.uniform(-12, 6, 4000))])
+    vals = vals[vals <= 448]
+    vals = np.concatenate([vals, -vals])
+    want = torch.tensor(vals).to(torch.float8_e4m3fn)
+    np.testing.assert_array_equal(oracle.to_e4m3(vals), want.double().numpy())
+    got = oracle.e4m3_encode(vals)
+    nz = oracle.to_e4m3(vals) != 0
+    np.testing.assert_array_equal(got[nz], want.view(torch.uint8).numpy()[nz])
+    assert (got[~nz] == 0).all()                      # a zero scale is byte 0 (no negative zero)
+
+
+def test_e4m3_saturates_at_448():
+    v = np.array([448.0, 449.0, 464.0, 465.0, 1e6, -1e6])
+    np.testing.assert_array_equal(oracle.to_e4m3(v), [448, 448, 448, 448, 448, -448])
+    np.testing.assert_array_equal(oracle.e4m3_encode(v), [126, 126, 126, 126, 126, 254])
+
+
+def test_nvfp4_properties():
+    rng = np.random.default_rng(12)
+    y = rng.standard_t(3, (32, 256)) * np.exp(rng.uniform(-4, 4, (32, 1)))
+    q, sb = oracle.quantize_nvfp4(y)
+    g = y.reshape(32, 16, 16)
+    s = oracle.to_e4m3(np.abs(g).max(axis=-1) / 6.0)
+    np.testing.assert_array_equal(sb, oracle.e4m3_encode(s))
+    qv = oracle.E2M1_GRID[q.reshape(32, 16, 16) & 7] * np.where(q.reshape(32, 16, 16) & 8, -1.0, 1.0)
+    v = g / s[..., None]
+    # nearest grid value (or 6 when saturated)
+    err = np.abs(v - qv)
+    step = np.select([np.abs(v) < 2, np.abs(v) < 4], [0.5, 1.0], 2.0)
+    unsat = np.abs(v) <= 6
+    assert np.all(err[unsat] <= step[unsat] / 2 + 1e-12)
+    assert np.all(np.abs(qv[~unsat]) == 6)
+    # the per-tensor scale only rescales: quantize(y * t, t) == quantize(y, 1)
+    for t in (0.5, 3.0, 2.0 ** -7):
+        q2, s2 = oracle.quantize_nvfp4(y * t, t)
+        np.testing.assert_array_equal(q2, q)
+        np.testing.assert_array_equal(s2, sb)
+    with pytest.raises(ValueError):
+        oracle.quantize_nvfp4(y, 0.0)
+    y0, c, sc = oracle.rotate_quant(rng.standard_normal((3, 64)), 0, "nvfp4", 16)
+    assert c.shape == (3, 32) and sc.shape == (3, 4) and sc.dtype == np.uint8
+    with pytest.raises(ValueError):
+        oracle.rotate_quant(rng.standard_normal((3, 64)), 0, "nvfp4", 32)

@@ -73,3 +73,18 @@ def test_c5_heavy_tails():
     x = W.bits_to_float64(W.generate("c5", slice(0, 64)), "bf16")
     assert np.abs(x).max() > 30      # Student-t(3) tails
     assert 1.0 < x.std() < 3.0
+
+
+def test_random_hadamard_workloads_share_the_c2_input():
+    for key in ("c2r", "c2rb"):
+        w = W.WORKLOADS[key]
+        assert w.algorithmic_bytes == W.WORKLOADS["c2"].algorithmic_bytes
+        np.testing.assert_array_equal(W.generate(key, slice(1020, 1030)), W.generate("c2", slice(1020, 1030)))
+        s = W.generate_signs(key)
+        assert s.dtype == np.int8 and s.shape == (w.block,) and set(np.unique(s)) == {-1, 1}
+        assert abs(int(s.astype(np.int64).sum())) < 4 * np.sqrt(w.block)       # Rademacher draws
+        np.testing.assert_array_equal(s, W.generate_signs(key))
+        assert not np.array_equal(s, W.generate_signs(key, seed=W.rank_seed(1)))
+    assert W.WORKLOADS["c2r"].signs == "after" and W.WORKLOADS["c2rb"].signs == "before"
+    with pytest.raises(ValueError):
+        W.generate_signs("c2")
