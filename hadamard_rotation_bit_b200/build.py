@@ -13,6 +13,7 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -21,11 +22,15 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhadq.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ARCH_FLAGS + [
+COMPILE_FLAGS = ARCH_FLAGS + [
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-    "--shared", "-cudart", "static",
 ]
+LINK_FLAGS = ARCH_FLAGS + ["--shared", "-cudart", "static", "-Xcompiler", "-fvisibility=hidden"]
+
+# Translation units: the host side (validation, launch planning, C ABI) and
+# one unit per kernel family, compiled in parallel.
+UNITS = ["hadq_api.cu", "kernels_segment.cu", "kernels_team.cu", "kernels_team_bf16.cu", "kernels_tc.cu"]
 
 
 def _nvcc() -> str:
@@ -36,7 +41,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh"))] + [
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh", ".h"))] + [
         os.path.join(INCLUDE, "hadq.h")]
 
 
@@ -47,21 +52,36 @@ def needs_build() -> bool:
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile libhadq.so if it is missing or older than its sources; return its path."""
-    if not force and not needs_build():
-        return LIB
-    cmd = [_nvcc()] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC]
-    if ptxas_info:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, "hadq_api.cu"), "-o", LIB + ".tmp"]
+def _run(cmd, verbose):
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr[-8000:]}")
-    if verbose or ptxas_info:
-        print(res.stderr, file=sys.stderr)
+        raise RuntimeError(f"nvcc failed ({res.returncode}): {' '.join(cmd[-3:])}\n{res.stderr[-8000:]}")
+    return res.stderr
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+    """Compile libhadq.so if it is missing or older than its sources; return its path."""
+    if not force and not needs_build():
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    nvcc = _nvcc()
+    with tempfile.TemporaryDirectory(prefix="hadq_build_") as tmp:
+        objs, cmds = [], []
+        for unit in UNITS:
+            obj = os.path.join(tmp, unit.replace(".cu", ".o"))
+            cmd = [nvcc] + COMPILE_FLAGS + ["-I", INCLUDE, "-I", CSRC]
+            if ptxas_info:
+                cmd += ["-Xptxas", "-v"]
+            cmds.append(cmd + ["-c", os.path.join(CSRC, unit), "-o", obj])
+            objs.append(obj)
+        with ThreadPoolExecutor(max_workers=len(cmds)) as ex:
+            logs = list(ex.map(lambda c: _run(c, verbose), cmds))
+        if verbose or ptxas_info:
+            for log in logs:
+                print(log, file=sys.stderr)
+        _run([nvcc] + LINK_FLAGS + objs + ["-o", LIB + ".tmp"], verbose)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -5,9 +5,8 @@
 // rule the apply_spinquant docstring states for its rotation passes).  There
 // is no CPU path: a missing device or kernel image surfaces as HADQ_ERR_CUDA.
 #include "hadq.h"
-#include "hadq_kernels.cuh"
-#include "hadq_tc.cuh"
-#include "hadq_tc128.cuh"
+#include "hadq_kernels.cuh"   // launch constants only; the kernels are instantiated elsewhere
+#include "hadq_launch.h"
 
 #include <cudaTypedefs.h>
 
@@ -104,8 +103,13 @@ hadq_status check_quant(hadq_fmt fmt, int64_t group, const Shape& sh, int* eff_g
       if (sh.n % 32 != 0) return fail(HADQ_ERR_INVALID_ARG, "MXFP4 needs n to be a multiple of 32");
       *eff_group = 32;
       return HADQ_OK;
+    case HADQ_NVFP4:
+      if (group != 0 && group != 16) return fail(HADQ_ERR_INVALID_ARG, "NVFP4 group must be 0 or 16");
+      if (sh.n % 16 != 0) return fail(HADQ_ERR_INVALID_ARG, "NVFP4 needs n to be a multiple of 16");
+      *eff_group = 16;
+      return HADQ_OK;
     default:
-      return fail(HADQ_ERR_INVALID_ARG, "fmt must be HADQ_INT4_SYM, HADQ_INT8_SYM or HADQ_MXFP4");
+      return fail(HADQ_ERR_INVALID_ARG, "fmt must be HADQ_INT4_SYM, HADQ_INT8_SYM, HADQ_MXFP4 or HADQ_NVFP4");
   }
 }
 
@@ -117,97 +121,15 @@ int64_t scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int group) {
   switch (fmt) {
     case HADQ_INT4_SYM: return rows * (n / group) * 2;
     case HADQ_INT8_SYM: return rows * 4;
+    case HADQ_NVFP4: return rows * (n / 16);
     default: return rows * (n / 32);
   }
 }
 
-// ------------------------------------------------------------ kernel tables
+// ------------------------------------------------------------ kernel lookups
 
 using hadq::Signs;
-using SegFn = void (*)(const void*, int64_t, int, float, int, void*, void*, Signs);
-using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, float*, Signs);
-using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*, Signs);
-using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*, Signs);
-
-template <int LOGS, bool BF, bool FULL>
-SegFn seg_fn(int mode) {
-  switch (mode) {
-    case hadq::OUT_F32: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_F32, FULL>;
-    case hadq::OUT_BF16: return &hadq::segment_kernel<LOGS, BF, hadq::OUT_BF16, FULL>;
-    case hadq::OUT_INT4:
-      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_INT4, FULL>;
-      return nullptr;
-    default:
-      if constexpr (LOGS >= 5) return &hadq::segment_kernel<LOGS, BF, hadq::OUT_MXFP4, FULL>;
-      return nullptr;
-  }
-}
-
-template <bool BF, bool FULL>
-SegFn seg_fn_logs(int logs, int mode) {
-  switch (logs) {
-    case 3: return seg_fn<3, BF, FULL>(mode);
-    case 4: return seg_fn<4, BF, FULL>(mode);
-    case 5: return seg_fn<5, BF, FULL>(mode);
-    case 6: return seg_fn<6, BF, FULL>(mode);
-    default: return seg_fn<7, BF, FULL>(mode);
-  }
-}
-
-SegFn seg_fn_any(bool bf, bool full, int logs, int mode) {
-  if (bf) return full ? seg_fn_logs<true, true>(logs, mode) : seg_fn_logs<true, false>(logs, mode);
-  return full ? seg_fn_logs<false, true>(logs, mode) : seg_fn_logs<false, false>(logs, mode);
-}
-
-template <bool BF, bool FULL>
-SegRowFn seg_row_fn(int logs) {
-  switch (logs) {
-    case 3: return &hadq::segment_row_int8_kernel<3, BF, FULL>;
-    case 4: return &hadq::segment_row_int8_kernel<4, BF, FULL>;
-    case 5: return &hadq::segment_row_int8_kernel<5, BF, FULL>;
-    case 6: return &hadq::segment_row_int8_kernel<6, BF, FULL>;
-    default: return &hadq::segment_row_int8_kernel<7, BF, FULL>;
-  }
-}
-
-SegRowFn seg_row_fn_any(bool bf, bool full, int logs) {
-  if (bf) return full ? seg_row_fn<true, true>(logs) : seg_row_fn<true, false>(logs);
-  return full ? seg_row_fn<false, true>(logs) : seg_row_fn<false, false>(logs);
-}
-
-template <int LOGB, bool BF>
-TeamFn team_fn(int mode) {
-  switch (mode) {
-    case hadq::OUT_F32: return &hadq::team_kernel<LOGB, BF, hadq::OUT_F32>;
-    case hadq::OUT_BF16: return &hadq::team_kernel<LOGB, BF, hadq::OUT_BF16>;
-    case hadq::OUT_INT4: return &hadq::team_kernel<LOGB, BF, hadq::OUT_INT4>;
-    default: return &hadq::team_kernel<LOGB, BF, hadq::OUT_MXFP4>;
-  }
-}
-
-template <bool BF>
-TeamFn team_fn_logb(int logb, int mode) {
-  switch (logb) {
-    case 8: return team_fn<8, BF>(mode);
-    case 9: return team_fn<9, BF>(mode);
-    case 10: return team_fn<10, BF>(mode);
-    case 11: return team_fn<11, BF>(mode);
-    case 12: return team_fn<12, BF>(mode);
-    default: return team_fn<13, BF>(mode);
-  }
-}
-
-template <bool BF>
-TeamRowFn team_row_fn(int logb) {
-  switch (logb) {
-    case 8: return &hadq::team_row_int8_kernel<8, BF>;
-    case 9: return &hadq::team_row_int8_kernel<9, BF>;
-    case 10: return &hadq::team_row_int8_kernel<10, BF>;
-    case 11: return &hadq::team_row_int8_kernel<11, BF>;
-    case 12: return &hadq::team_row_int8_kernel<12, BF>;
-    default: return &hadq::team_row_int8_kernel<13, BF>;
-  }
-}
+namespace hl = hadq::launch;
 
 // ------------------------------------------------- per-device launch caches
 
@@ -318,44 +240,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, Signs);
-
-
-// Tensor-core kernel configuration: 128-column tiles, 5 operand stages, and
-// 4 (n = 4096) or 2 (n = 8192) epilogue warps per tensor-memory lane quarter
-// -- the fastest of the measured variants for each size.
-struct TcVariant {
-  TcFn fn;
-  int threads, smem, tile_n;
-};
-
-template <class C, int MODE>
-TcVariant tc_variant() {
-  return TcVariant{&hadq::tc::tc_rotate_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::TILE_N};
-}
-
-// n = 4096: 4 rows per tile, one row per epilogue warp, 3 stages.  n = 8192:
-// 2 rows per tile, 4 stages; for int4 (whose epilogue is the heaviest) the
-// MMAs are committed per row so the first row's epilogue starts early.
-TcVariant tc_pick(int lo, int mode) {
-  using hadq::tc::TcCfg;
-  using C5 = TcCfg<5, 128, 3, 4, false>;
-  using C6 = TcCfg<6, 128, 4, 2, false>;
-  using C6H = TcCfg<6, 128, 4, 2, true>;
-  switch (mode) {
-    case hadq::OUT_F32: return lo == 5 ? tc_variant<C5, hadq::OUT_F32>() : tc_variant<C6, hadq::OUT_F32>();
-    case hadq::OUT_BF16: return lo == 5 ? tc_variant<C5, hadq::OUT_BF16>() : tc_variant<C6, hadq::OUT_BF16>();
-    case hadq::OUT_INT4: return lo == 5 ? tc_variant<C5, hadq::OUT_INT4>() : tc_variant<C6H, hadq::OUT_INT4>();
-    default: return lo == 5 ? tc_variant<C5, hadq::OUT_MXFP4>() : tc_variant<C6, hadq::OUT_MXFP4>();
-  }
-}
-
 // Blocks of b = 2^(7 + LO) bf16 elements, each rotated in full: the blocks are
 // the rows of a (rows * n / b) x b matrix.
 hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
                       cudaStream_t stream, int sms, int dev, Signs sg) {
   const int lo = sh.logb - 7;
-  const TcVariant v = tc_pick(lo, mode);
+  const hl::TcVariant v = hl::tc_kernel_for(lo, mode, sg.side != hadq::SIGNS_NONE);
+  if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no tensor-core kernel for this size and format");
   const int L = 1 << lo, R = v.tile_n / L;
   const int64_t rows = sh.rows * (sh.n >> sh.logb);
   if (rows > (int64_t(1) << 31) - R) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many rows");
@@ -384,20 +275,6 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
 // Block-128 rotations of bf16 rows on the tensor cores: every 128-element
 // block is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
-using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*,
-                         Signs);
-using Tc128C = hadq::tc::Tc128Cfg<4, 2>;
-
-Tc128Fn tc128_fn(int mode) {
-  switch (mode) {
-    case hadq::OUT_F32: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_F32>;
-    case hadq::OUT_BF16: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_BF16>;
-    case hadq::OUT_INT4: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_INT4>;
-    case hadq::OUT_MXFP4: return &hadq::tc::tc128_kernel<Tc128C, hadq::OUT_MXFP4>;
-    default: return &hadq::tc::tc128_kernel<Tc128C, -1>;
-  }
-}
-
 bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
   if (x_dtype != HADQ_BF16 || sh.b != 128) return false;
   if (mode >= 0) return true;
@@ -424,14 +301,14 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   }
-  Tc128Fn fn = tc128_fn(mode);
-  const int smem = Tc128C::SMEM_BYTES;
+  const hl::Tc128Variant v = hl::tc128_kernel_for(mode, sg.side != hadq::SIGNS_NONE);
+  if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no block-128 tensor-core kernel for this format");
   int occ = 0;
-  hadq_status st = occupancy(reinterpret_cast<const void*>(fn), dev, Tc128C::THREADS, smem, &occ);
+  hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
   if (st != HADQ_OK) return st;
   const int64_t tiles = (blocks + bpt - 1) / bpt;
   const int64_t grid = std::min<int64_t>(tiles, sms);
-  return launch_result(launch_pdl(fn, grid, Tc128C::THREADS, smem, stream, maps[0], maps[1],
+  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, maps[0], maps[1],
                                   static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1, sg),
                        "tensor-core block-128 kernel launch");
 }
@@ -446,6 +323,16 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   if (st != HADQ_OK) return st;
   const bool bf = x_dtype == HADQ_BF16;
   const bool full_seg = sh.logb == sh.logs;
+  const bool sgd = sg.side != hadq::SIGNS_NONE;
+  // Segment kernels: a thread owns S = max(b, the quantizer's group span, 32)
+  // consecutive elements (at most 128 and at most the largest power of 2
+  // dividing n), so a block of b >= 32 is a whole segment (fixed butterfly,
+  // no run-time stage count) and smaller blocks keep short register arrays.
+  int seg_logs = sh.logs;
+  if (mode >= 0 && sh.b <= 128) {
+    const int need = mode == hadq::OUT_INT4 ? group : mode == hadq::OUT_MXFP4 ? 32 : 16;
+    seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 5));
+  }
   (void)cudaGetLastError();   // launch errors below must be ours
   if (kernel_choice() != KernelChoice::Butterfly && sg.side != hadq::SIGNS_BEFORE) {
     if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
@@ -453,9 +340,9 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   }
   if (mode >= 0) {
     if (sh.b <= 128) {
-      SegFn fn = seg_fn_any(bf, full_seg, sh.logs, mode);
+      const hl::SegFn fn = hl::segment_kernel_for(bf, sh.logb == seg_logs, seg_logs, mode, sgd);
       if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no kernel for this segment size and format");
-      const int64_t segs = sh.rows * (sh.n >> sh.logs);
+      const int64_t segs = sh.rows * (sh.n >> seg_logs);
       int occ = 0;
       st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, 0, &occ);
       if (st != HADQ_OK) return st;
@@ -464,7 +351,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
                                       sg),
                            "segment kernel launch");
     }
-    TeamFn fn = bf ? team_fn_logb<true>(sh.logb, mode) : team_fn_logb<false>(sh.logb, mode);
+    const hl::TeamFn fn = hl::team_kernel_for(bf, sh.logb, mode, sgd);
+    if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no kernel for this block size and format");
     const int smem = hadq::kThreads * hadq::kRowFloats * 4;
     int occ = 0;
     st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, smem, &occ);
@@ -479,7 +367,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   int8_t* codes = static_cast<int8_t*>(out0);
   float* scales = static_cast<float*>(out1);
   if (sh.b <= 128) {
-    SegRowFn fn = seg_row_fn_any(bf, full_seg, sh.logs);
+    const hl::SegRowFn fn = hl::segment_row_kernel_for(bf, full_seg, sh.logs, sgd);
+    if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no per-token kernel for this segment size");
     const int block = static_cast<int>(ceil_div(sh.n >> sh.logs, 32) * 32);
     int occ = 0;
     st = occupancy(reinterpret_cast<const void*>(fn), dev, block, 0, &occ);
@@ -488,7 +377,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     return launch_result(launch_pdl(fn, grid, block, 0, stream, x, sh.rows, sh.n, sh.logb, sh.norm, codes, scales, sg),
                          "per-token int8 kernel launch");
   }
-  TeamRowFn fn = bf ? team_row_fn<true>(sh.logb) : team_row_fn<false>(sh.logb);
+  const hl::TeamRowFn fn = hl::team_row_kernel_for(bf, sh.logb, sgd);
+  if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no per-token kernel for this block size");
   const int block = static_cast<int>(ceil_div(sh.n >> 7, 32) * 32);
   const int smem = static_cast<int>((sh.n >> 7) * hadq::kRowFloats * 4);
   int occ = 0;
@@ -521,6 +411,7 @@ hadq_status make_signs(const int8_t* signs, SideArg a, const Shape& sh, const Sp
   *sg = Signs{nullptr, hadq::SIGNS_NONE};
   if (!a.is_signed) return HADQ_OK;
   if (signs == nullptr) return fail(HADQ_ERR_INVALID_ARG, "null signs");
+  if (!aligned16(signs)) return fail(HADQ_ERR_MISALIGNED, "signs must be 16-byte aligned");
   const Span ss = span(signs, sh.b);
   for (int i = 0; i < nouts; ++i)
     if (overlaps(ss, outs[i])) return fail(HADQ_ERR_INVALID_ARG, "signs must not overlap an output");
@@ -572,19 +463,30 @@ hadq_status quant_checks(const void* x, hadq_dtype x_dtype, int64_t rows, int64_
 }
 
 int quant_mode(hadq_fmt fmt) {
-  return fmt == HADQ_INT4_SYM ? hadq::OUT_INT4 : fmt == HADQ_MXFP4 ? hadq::OUT_MXFP4 : -1;
+  switch (fmt) {
+    case HADQ_INT4_SYM: return hadq::OUT_INT4;
+    case HADQ_MXFP4: return hadq::OUT_MXFP4;
+    case HADQ_NVFP4: return hadq::OUT_NVFP4;
+    default: return -1;
+  }
 }
 
 hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
                               hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream,
-                              const int8_t* signs = nullptr, SideArg side = SideArg{false, kUnsigned}) {
+                              const int8_t* signs = nullptr, SideArg side = SideArg{false, kUnsigned},
+                              double tensor_scale = 1.0) {
   g_last_error.clear();
   Shape sh;
   int g = 0;
   hadq_status st = check_side(side);
   if (st != HADQ_OK) return st;
+  if (!(std::isfinite(tensor_scale) && tensor_scale > 0))
+    return fail(HADQ_ERR_INVALID_ARG, "tensor_scale must be finite and > 0");
   st = quant_checks(x, x_dtype, rows, n, block, fmt, group, codes, scales, &sh, &g);
   if (st != HADQ_OK || rows == 0) return st;
+  // NVFP4 quantizes y / tensor_scale: fold the division into the rotation's
+  // normalisation (one rounding, on the host, in double).
+  if (fmt == HADQ_NVFP4) sh.norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.b)) / tensor_scale);
   const Span outs[2] = {span(codes, codes_bytes(rows, n, fmt)), span(scales, scales_bytes(rows, n, fmt, g))};
   Signs sg;
   st = make_signs(signs, side, sh, outs, 2, &sg);
@@ -638,6 +540,12 @@ hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int64_t rows,
 hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, hadq_fmt fmt,
                               int64_t group, void* codes, void* scales, void* stream) {
   return rotate_quant_impl(x, x_dtype, rows, n, block, fmt, group, codes, scales, stream);
+}
+
+hadq_status hadq_rotate_quant_nvfp4(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                    float tensor_scale, void* codes, void* scales, void* stream) {
+  return rotate_quant_impl(x, x_dtype, rows, n, block, HADQ_NVFP4, 16, codes, scales, stream, nullptr,
+                           SideArg{false, kUnsigned}, static_cast<double>(tensor_scale));
 }
 
 hadq_status hadq_rotate_signed(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
@@ -726,7 +634,7 @@ hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtype x_dtype
 
 int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt) {
   if (rows < 0 || n <= 0 || n % 2 != 0) return 0;
-  if (fmt != HADQ_INT4_SYM && fmt != HADQ_INT8_SYM && fmt != HADQ_MXFP4) return 0;
+  if (fmt != HADQ_INT4_SYM && fmt != HADQ_INT8_SYM && fmt != HADQ_MXFP4 && fmt != HADQ_NVFP4) return 0;
   return codes_bytes(rows, n, fmt);
 }
 
@@ -740,6 +648,8 @@ int64_t hadq_scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int64_t group) 
       return (group == 0 || group == n) ? rows * 4 : 0;
     case HADQ_MXFP4:
       return ((group == 0 || group == 32) && n % 32 == 0) ? rows * (n / 32) : 0;
+    case HADQ_NVFP4:
+      return ((group == 0 || group == 16) && n % 16 == 0) ? rows * (n / 16) : 0;
     default:
       return 0;
   }
@@ -760,14 +670,6 @@ const char* hadq_last_error(void) { return g_last_error.c_str(); }
 
 int hadq_version(void) { return 100; }
 
-int hadq_device_faults(int clear) {
-  unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, hadq::tc::hadq_tc_fault, sizeof(v)) != cudaSuccess) return -1;
-  if (clear && v != 0) {
-    const unsigned int z = 0;
-    if (cudaMemcpyToSymbol(hadq::tc::hadq_tc_fault, &z, sizeof(z)) != cudaSuccess) return -1;
-  }
-  return static_cast<int>(v);
-}
+int hadq_device_faults(int clear) { return hadq::launch::tc_fault_bits(clear); }
 
 }  // extern "C"

@@ -15,7 +15,7 @@
 
 namespace hadq {
 
-enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3 };
+enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3, OUT_NVFP4 = 4 };
 
 // Random Hadamard signs ("Rotation Transform", section 1.5: H @ diag(+/-1) /
 // sqrt(N), the signs persisted as int8).  AFTER: output column j of every
@@ -25,13 +25,50 @@ enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3 };
 enum SignSide : int { SIGNS_NONE = 0, SIGNS_BEFORE = 1, SIGNS_AFTER = 2 };
 
 struct Signs {
-  const int8_t* s;   // b entries, device memory; unused for SIGNS_NONE
+  const int8_t* s;   // b entries, device memory, 16-byte aligned; unused for SIGNS_NONE
   int side;
 };
 
 // 1 if block column `col` is negated.
 __device__ __forceinline__ uint32_t neg_bit(const int8_t* __restrict__ s, int col) {
   return s[col] < 0 ? 1u : 0u;
+}
+
+// The sign bits (bit 7) of the four int8 in w, as bits 0..3: after masking,
+// one multiply moves bits 7, 15, 23, 31 to 21, 22, 23, 24 without carries.
+__device__ __forceinline__ uint32_t sign_nibble(uint32_t w) {
+  return (((w >> 7) & 0x01010101u) * 0x00204081u >> 21) & 0xFu;
+}
+
+// Bit k set when s[c0 + k] < 0, for k < 32 (c0 a multiple of 16).
+__device__ __forceinline__ uint32_t sign_bits32(const int8_t* __restrict__ s, int c0) {
+  const uint4 a = *reinterpret_cast<const uint4*>(s + c0);
+  const uint4 b = *reinterpret_cast<const uint4*>(s + c0 + 16);
+  return sign_nibble(a.x) | sign_nibble(a.y) << 4 | sign_nibble(a.z) << 8 | sign_nibble(a.w) << 12 |
+         sign_nibble(b.x) << 16 | sign_nibble(b.y) << 20 | sign_nibble(b.z) << 24 | sign_nibble(b.w) << 28;
+}
+
+// Bit k set when s[c0 + k] < 0, for k < W, W in {2, 4, 8, 16} (c0 a multiple of W).
+template <int W>
+__device__ __forceinline__ uint32_t sign_bits_small(const int8_t* __restrict__ s, int c0) {
+  if constexpr (W == 16) {
+    const uint4 a = *reinterpret_cast<const uint4*>(s + c0);
+    return sign_nibble(a.x) | sign_nibble(a.y) << 4 | sign_nibble(a.z) << 8 | sign_nibble(a.w) << 12;
+  } else if constexpr (W == 8) {
+    const uint2 a = *reinterpret_cast<const uint2*>(s + c0);
+    return sign_nibble(a.x) | sign_nibble(a.y) << 4;
+  } else if constexpr (W == 4) {
+    return sign_nibble(*reinterpret_cast<const uint32_t*>(s + c0));
+  } else {
+    static_assert(W == 2, "2, 4, 8 or 16 signs");
+    return sign_nibble(*reinterpret_cast<const uint16_t*>(s + c0)) & 3u;
+  }
+}
+
+// Register bit order of a mask under the quad permutation reg<true>: bits 1
+// and 2 of every nibble swap places.
+__device__ __forceinline__ uint32_t perm_quad_bits(uint32_t m) {
+  return (m & 0x99999999u) | ((m & 0x22222222u) << 1) | ((m & 0x44444444u) >> 1);
 }
 
 // 1.5 * 2^23: adding it to |v| < 2^22 leaves round-half-even(v) in the low
@@ -205,9 +242,14 @@ __host__ __device__ constexpr int reg(int e) {
 
 // Flip the sign of register i where bit i of the mask (word i / 32) is set.
 // Each thread's mask is fixed for a whole launch: a thread always holds the
-// same block columns in the same registers.
+// same block columns in the same registers.  The mask words pass through an
+// opaque move first, so the per-element sign words are formed here, at each
+// use, instead of being hoisted out of the caller's loop (N live registers).
 template <int N>
-__device__ __forceinline__ void apply_signs(float (&v)[N], const uint32_t (&m)[(N + 31) / 32]) {
+__device__ __forceinline__ void apply_signs(float (&v)[N], const uint32_t (&m_in)[(N + 31) / 32]) {
+  uint32_t m[(N + 31) / 32];
+#pragma unroll
+  for (int w = 0; w < (N + 31) / 32; ++w) asm volatile("mov.b32 %0, %1;" : "=r"(m[w]) : "r"(m_in[w]));
 #pragma unroll
   for (int i = 0; i < N; ++i)
     v[i] = __uint_as_float(__float_as_uint(v[i]) ^ ((m[i >> 5] << (31 - (i & 31))) & 0x80000000u));
@@ -311,6 +353,7 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, flo
 // the codes and scales equal the exactly rounded ones everywhere else.
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kInv127 = 1.0f / 127.0f;
+constexpr float kInv6 = 1.0f / 6.0f;
 
 __device__ __forceinline__ float fast_recip(float s) { return __fdividef(1.0f, s); }
 
@@ -406,6 +449,55 @@ __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uin
     w.w = pack_e2m1x8<PERM>(v, 32 * j + 24, f);
     reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
     scales[(e0 >> 5) + j] = static_cast<uint8_t>(byte);
+  }
+}
+
+// FP8 E4M3 bytes of two non-negative values (round half to even, saturating
+// at 448): `hi` in bits 8..15, `lo` in bits 0..7.
+__device__ __forceinline__ uint16_t e4m3x2(float hi, float lo) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The values of two E4M3 bytes (exact in fp16): .x from bits 0..7, .y from 8..15.
+__device__ __forceinline__ float2 e4m3x2_values(uint16_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(b));
+  return make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu))),
+                     __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16))));
+}
+
+// NVFP4: per 16 elements an E4M3 scale s = e4m3(m / 6) of the block absmax m
+// of v = z * nq (nq = the rotation's 1/sqrt(b) divided by the per-tensor
+// scale) and E2M1 codes of v / s; s == 0 gives codes 0.  Pairs of blocks
+// store 16 code bytes and 2 scale bytes at once.
+template <bool PERM, int N>
+__device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8_t* __restrict__ codes,
+                                            uint8_t* __restrict__ scales, int64_t e0) {
+  static_assert(N % 16 == 0, "NVFP4 blocks are 16 elements");
+  if constexpr (N == 16) {
+    const float m = absmax_regs(v, 0, 16) * nq;
+    const uint16_t b = e4m3x2(0.f, m * kInv6);
+    const float s = e4m3x2_values(b).x;
+    const float f = s > 0.f ? nq * fast_recip(s) : 0.f;
+    reinterpret_cast<uint2*>(codes + (e0 >> 1))[0] = make_uint2(pack_e2m1x8<PERM>(v, 0, f), pack_e2m1x8<PERM>(v, 8, f));
+    scales[e0 >> 4] = static_cast<uint8_t>(b & 0xFFu);
+  } else {
+    static_assert(N % 32 == 0, "NVFP4 chunks above 16 elements come in pairs of blocks");
+#pragma unroll
+    for (int j = 0; j < N / 32; ++j) {
+      const float m0 = absmax_regs(v, 32 * j, 16) * nq;
+      const float m1 = absmax_regs(v, 32 * j + 16, 16) * nq;
+      const uint16_t b = e4m3x2(m1 * kInv6, m0 * kInv6);
+      const float2 s = e4m3x2_values(b);
+      const float f0 = s.x > 0.f ? nq * fast_recip(s.x) : 0.f;
+      const float f1 = s.y > 0.f ? nq * fast_recip(s.y) : 0.f;
+      reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] =
+          make_uint4(pack_e2m1x8<PERM>(v, 32 * j, f0), pack_e2m1x8<PERM>(v, 32 * j + 8, f0),
+                     pack_e2m1x8<PERM>(v, 32 * j + 16, f1), pack_e2m1x8<PERM>(v, 32 * j + 24, f1));
+      reinterpret_cast<uint16_t*>(scales + ((e0 + 32 * j) >> 4))[0] = b;
+    }
   }
 }
 

@@ -35,10 +35,11 @@
 // grid_dependency_sync) and prefetches its next unit of input into L2 while it
 // computes the current one.
 //
-// Random Hadamard signs (Signs, SIGNS_BEFORE / SIGNS_AFTER): a thread always
-// owns the same block columns in the same registers, so it reads its signs
-// once into a bit mask and flips the loaded values (before) or the rotated
-// values (after) with one XOR of the sign bit each.
+// Random Hadamard signs (Signs, SIGNS_BEFORE / SIGNS_AFTER) are compiled in
+// only for SG = true (the deterministic kernels carry no trace of them): a
+// thread always owns the same block columns in the same registers, so it
+// reads its signs once into a bit mask and flips the loaded values (before)
+// or the rotated values (after) with one XOR of the sign bit each.
 #pragma once
 
 #include "hadq_device.cuh"
@@ -57,12 +58,21 @@ __device__ __forceinline__ void segment_sign_mask(const Signs& sg, int nbits, ui
 #pragma unroll
   for (int w = 0; w < (S + 31) / 32; ++w) sm[w] = 0u;
   if (sg.side == SIGNS_NONE) return;
-  const int bmask = (1 << nbits) - 1;
-  for (int i = 0; i < S; ++i) sm[i >> 5] |= neg_bit(sg.s, i & bmask) << (i & 31);
+  const int b = 1 << nbits;
+  if (b >= 32) {
+#pragma unroll
+    for (int w = 0; w < (S + 31) / 32; ++w) sm[w] = sign_bits32(sg.s, (32 * w) & (b - 1));
+  } else {
+    uint32_t p = 0;                      // the b signs, repeated every b bits
+    for (int i = 0; i < b; ++i) p |= neg_bit(sg.s, i) << i;
+    for (int k = b; k < 32; k <<= 1) p |= p << k;
+#pragma unroll
+    for (int w = 0; w < (S + 31) / 32; ++w) sm[w] = p;
+  }
 }
 
 // FULL: b == S, all LOGS stages unconditionally; otherwise the low nbits stages.
-template <int LOGS, bool IN_BF16, int MODE, bool FULL>
+template <int LOGS, bool IN_BF16, int MODE, bool FULL, bool SG>
 __global__ void __launch_bounds__(kThreads)
 segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, int group,
                void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
@@ -70,7 +80,7 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
   constexpr uint32_t kSegBytes = S * (IN_BF16 ? 2 : 4);
   grid_dependency_sync();
   uint32_t sm[(S + 31) / 32];
-  segment_sign_mask<S>(sg, nbits, sm);
+  if constexpr (SG) segment_sign_mask<S>(sg, nbits, sm);
   float v[S];
   const int lane = threadIdx.x & 31;
   for (int64_t s = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; s < segs;
@@ -84,19 +94,25 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
     }
     const int64_t e0 = s << LOGS;
     load_elems<IN_BF16, S>(x, e0, v);
-    if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
+    if constexpr (SG) {
+      if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
+    }
     if constexpr (FULL) {
       fwht_bits<S, 0, LOGS>(v);
     } else {
       fwht_low<S>(v, nbits);
     }
-    if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
+    if constexpr (SG) {
+      if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
+    }
     if constexpr (MODE == OUT_F32) {
       store_rotated<false, S, false>(v, norm, out0, e0);
     } else if constexpr (MODE == OUT_BF16) {
       store_rotated<false, S, true>(v, norm, out0, e0);
     } else if constexpr (MODE == OUT_INT4) {
       store_int4<false, S>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+    } else if constexpr (MODE == OUT_NVFP4) {
+      store_nvfp4<false, S>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
     } else {
       store_mxfp4<false, S>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
     }
@@ -104,14 +120,14 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
 }
 
 // Per-token int8, b <= 128: one CTA per row, blockDim = n / S rounded up to 32 (<= 256).
-template <int LOGS, bool IN_BF16, bool FULL>
+template <int LOGS, bool IN_BF16, bool FULL, bool SG>
 __global__ void __launch_bounds__(256)
 segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int nbits, float norm,
                         int8_t* __restrict__ codes, float* __restrict__ scales, Signs sg) {
   constexpr int S = 1 << LOGS;
   grid_dependency_sync();
   uint32_t sm[(S + 31) / 32];
-  segment_sign_mask<S>(sg, nbits, sm);
+  if constexpr (SG) segment_sign_mask<S>(sg, nbits, sm);
   __shared__ float red[32];
   const int segs_row = static_cast<int>(n >> LOGS);
   const bool active = static_cast<int>(threadIdx.x) < segs_row;
@@ -123,13 +139,17 @@ segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int
     const int64_t e0 = r * n + (static_cast<int64_t>(threadIdx.x) << LOGS);
     if (active) {
       load_elems<IN_BF16, S>(x, e0, v);
-      if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
+      if constexpr (SG) {
+        if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
+      }
       if constexpr (FULL) {
         fwht_bits<S, 0, LOGS>(v);
       } else {
         fwht_low<S>(v, nbits);
       }
-      if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
+      if constexpr (SG) {
+        if (sg.side == SIGNS_AFTER) apply_signs<S>(v, sm);
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < S; ++i) v[i] = 0.f;
@@ -170,20 +190,33 @@ __device__ __forceinline__ void team_sign_mask(const Signs& sg, int tau, uint32_
   using Sh = TeamShape<LOGB>;
 #pragma unroll
   for (int w = 0; w < 4; ++w) sm[w] = 0u;
-  if (sg.side == SIGNS_NONE) return;
-  for (int i = 0; i < 128; ++i) {
-    const int col = sg.side == SIGNS_BEFORE ? (i / Sh::CE) * 128 + tau * Sh::CE + (i % Sh::CE)
-                                            : tau * 128 + reg<Sh::PERM>(i);
-    sm[i >> 5] |= neg_bit(sg.s, col) << (i & 31);
+  if (sg.side == SIGNS_AFTER) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t m = sign_bits32(sg.s, tau * 128 + 32 * w);
+      sm[w] = Sh::PERM ? perm_quad_bits(m) : m;
+    }
+  } else if (sg.side == SIGNS_BEFORE) {
+    if constexpr (Sh::CE >= 32) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {   // register 32 w + k = column (32 w / CE) * 128 + tau * CE + (32 w) % CE + k
+        const int i = 32 * w;
+        sm[w] = sign_bits32(sg.s, (i / Sh::CE) * 128 + tau * Sh::CE + (i % Sh::CE));
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < Sh::T; ++h)   // registers h * CE + [0, CE) = columns h * 128 + tau * CE + [0, CE)
+        sm[(h * Sh::CE) >> 5] |= sign_bits_small<Sh::CE>(sg.s, h * 128 + tau * Sh::CE) << ((h * Sh::CE) & 31);
+    }
   }
 }
 
 // Rotate one block of 2^LOGB elements (element base `base`) by a team; on
 // return v[0..128) holds the unnormalised outputs base + tau*128 + [0, 128) in
 // register order TeamShape<LOGB>::PERM.  `rows` is this team's T x kRowFloats
-// shared buffer.  With `before`, the loaded values are first multiplied by
-// the signs in `sm` (team_sign_mask, BEFORE layout).
-template <int LOGB, bool IN_BF16>
+// shared buffer.  With SG and `before`, the loaded values are first
+// multiplied by the signs in `sm` (team_sign_mask, BEFORE layout).
+template <int LOGB, bool IN_BF16, bool SG>
 __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t base, bool valid, int tau,
                                             float* __restrict__ rows, float (&v)[128], bool before,
                                             const uint32_t (&sm)[4]) {
@@ -191,7 +224,9 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
   if (valid) {
 #pragma unroll
     for (int h = 0; h < Sh::T; ++h) load_elems<IN_BF16, Sh::CE>(x, base + h * 128 + tau * Sh::CE, &v[h * Sh::CE]);
-    if (before) apply_signs<128>(v, sm);
+    if constexpr (SG) {
+      if (before) apply_signs<128>(v, sm);
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 128; ++i) v[i] = 0.f;
@@ -235,7 +270,7 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
   fwht_bits<128, Sh::V, 7>(v);
 }
 
-template <int LOGB, bool IN_BF16, int MODE>
+template <int LOGB, bool IN_BF16, int MODE, bool SG>
 __global__ void __launch_bounds__(kThreads, 3)
 team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, void* __restrict__ out0,
             void* __restrict__ out1, Signs sg) {
@@ -249,7 +284,7 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
   const int tau = threadIdx.x & (Sh::T - 1);
   float* rows = buf + team * Sh::T * kRowFloats;
   uint32_t sm[4];
-  team_sign_mask<LOGB>(sg, tau, sm);
+  if constexpr (SG) team_sign_mask<LOGB>(sg, tau, sm);
   float v[128];
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * TEAMS; u0 < units;
        u0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
@@ -260,9 +295,11 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
     }
     const bool valid = u < units;
     const int64_t base = u << LOGB;
-    team_rotate<LOGB, IN_BF16>(x, base, valid, tau, rows, v, sg.side == SIGNS_BEFORE, sm);
+    team_rotate<LOGB, IN_BF16, SG>(x, base, valid, tau, rows, v, sg.side == SIGNS_BEFORE, sm);
     if (valid) {
-      if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
+      if constexpr (SG) {
+        if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
+      }
       const int64_t e0 = base + tau * 128;
       if constexpr (MODE == OUT_F32) {
         store_rotated<Sh::PERM, 128, false>(v, norm, out0, e0);
@@ -270,6 +307,8 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
         store_rotated<Sh::PERM, 128, true>(v, norm, out0, e0);
       } else if constexpr (MODE == OUT_INT4) {
         store_int4<Sh::PERM, 128>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+      } else if constexpr (MODE == OUT_NVFP4) {
+        store_nvfp4<Sh::PERM, 128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
       } else {
         store_mxfp4<Sh::PERM, 128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
       }
@@ -279,7 +318,7 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
 
 // Per-token int8, b >= 256: one CTA per row of n elements (n / b teams).
 // blockDim = n / 128 rounded up to 32; dynamic shared memory = n / 128 rows.
-template <int LOGB, bool IN_BF16>
+template <int LOGB, bool IN_BF16, bool SG>
 __global__ void __launch_bounds__(256)
 team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float norm, int8_t* __restrict__ codes,
                      float* __restrict__ scales, Signs sg) {
@@ -295,15 +334,17 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
   float* team_rows = buf + (active ? team * Sh::T * kRowFloats : 0);
   const int64_t row_bytes = n * (IN_BF16 ? 2 : 4);
   uint32_t sm[4];
-  team_sign_mask<LOGB>(sg, tau, sm);
+  if constexpr (SG) team_sign_mask<LOGB>(sg, tau, sm);
   float v[128];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     if (threadIdx.x == 0 && r + gridDim.x < rows)
       prefetch_l2(static_cast<const char*>(x) + (r + gridDim.x) * row_bytes, static_cast<uint32_t>(row_bytes));
     const int64_t base = r * n + (static_cast<int64_t>(team) << LOGB);
     if (active) {
-      team_rotate<LOGB, IN_BF16>(x, base, true, tau, team_rows, v, sg.side == SIGNS_BEFORE, sm);
-      if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
+      team_rotate<LOGB, IN_BF16, SG>(x, base, true, tau, team_rows, v, sg.side == SIGNS_BEFORE, sm);
+      if constexpr (SG) {
+        if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
+      }
     } else {
       // Idle threads still take part in every barrier of team_rotate.
 #pragma unroll

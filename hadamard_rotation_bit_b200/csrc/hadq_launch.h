@@ -1,0 +1,59 @@
+// Kernel entry points as the host launcher sees them.
+//
+// The kernels are instantiated in their own translation units
+// (kernels_segment.cu, kernels_team.cu, kernels_tc.cu), which nvcc compiles in
+// parallel; each exports a lookup that returns the instantiation for a call's
+// shape, output mode and sign variant.  SG selects the random Hadamard
+// (signed) instantiation; the deterministic ones are compiled without any
+// sign code.  A nullptr / fn == nullptr result means "no such instantiation".
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "hadq_device.cuh"
+
+namespace hadq {
+namespace launch {
+
+using SegFn = void (*)(const void*, int64_t, int, float, int, void*, void*, Signs);
+using SegRowFn = void (*)(const void*, int64_t, int64_t, int, float, int8_t*, float*, Signs);
+using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*, Signs);
+using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*, Signs);
+using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, Signs);
+using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*,
+                         Signs);
+
+struct TcVariant {
+  TcFn fn;
+  int threads, smem, tile_n;
+};
+
+struct Tc128Variant {
+  Tc128Fn fn;
+  int threads, smem;
+};
+
+// Segment kernels (b <= 128): log2 of the per-thread segment `logs`, FULL when
+// b equals the segment.  mode: OutMode.
+SegFn segment_kernel_for(bool bf16, bool full, int logs, int mode, bool sg);
+SegRowFn segment_row_kernel_for(bool bf16, bool full, int logs, bool sg);
+
+// Team kernels (256 <= b <= 8192); one unit per input dtype
+// (kernels_team.cu: fp32 and the dispatch, kernels_team_bf16.cu: bf16).
+TeamFn team_kernel_for(bool bf16, int logb, int mode, bool sg);
+TeamRowFn team_row_kernel_for(bool bf16, int logb, bool sg);
+TeamFn team_kernel_bf16(int logb, int mode, bool sg);
+TeamRowFn team_row_kernel_bf16(int logb, bool sg);
+
+// Tensor-core kernels: full size 2^(7 + lo), lo = 5 or 6; block 128 (mode -1 =
+// per-token int8).
+TcVariant tc_kernel_for(int lo, int mode, bool sg);
+Tc128Variant tc128_kernel_for(int mode, bool sg);
+
+// The tensor-core kernels' sticky fault word (bounded waits that ran out);
+// cleared when `clear` is non-zero.  -1 on a CUDA error.
+int tc_fault_bits(int clear);
+
+}  // namespace launch
+}  // namespace hadq

@@ -194,15 +194,15 @@ __device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits tha
 
 // Epilogue for one row of one tile: z holds the 2^LO values of TMEM lane hi'
 // (after the tensor-core stage over hi); finish the butterfly over lo and emit.
-// With `flip`, output column hi * 2^LO + c is negated where bit c of `sm` is
-// set (random Hadamard, signs after the rotation).
-template <int LO, int MODE>
+// With SG, output column hi * 2^LO + c is negated where bit c of `sm` is set
+// (random Hadamard, signs after the rotation).
+template <int LO, int MODE, bool SG>
 __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t row, bool row_ok, int n, float norm,
-                                            int group, void* __restrict__ out0, void* __restrict__ out1, bool flip,
+                                            int group, void* __restrict__ out0, void* __restrict__ out1,
                                             const uint32_t (&sm)[(1 << LO) / 32]) {
   constexpr int L = 1 << LO;
   fwht_bits<L, 0, LO>(z);
-  if (flip) apply_signs<L>(z, sm);
+  if constexpr (SG) apply_signs<L>(z, sm);
   const int64_t e0 = row * n + static_cast<int64_t>(hi) * L;   // first output element of this thread
   if constexpr (MODE == OUT_INT4) {
     // Groups of `group` outputs = L values x (group / L) consecutive lanes.
@@ -243,6 +243,8 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
     }
   } else if constexpr (MODE == OUT_MXFP4) {
     if (row_ok) store_mxfp4<false, L>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+  } else if constexpr (MODE == OUT_NVFP4) {
+    if (row_ok) store_nvfp4<false, L>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
   } else if constexpr (MODE == OUT_BF16) {
     if (row_ok) store_rotated<false, L, true>(z, norm, out0, e0);
   } else {
@@ -250,7 +252,7 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
   }
 }
 
-template <class C, int MODE>
+template <class C, int MODE, bool SG>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
                  float norm, int group, void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
@@ -374,14 +376,13 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
       const int quarter = warp & 3;            // TMEM lanes this warp may access
       const int sub = (warp - 2) >> 2;         // rows r = sub (mod SPLIT) of every tile
       const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
-      // Signs after the rotation (the launcher never passes SIGNS_BEFORE here):
-      // this thread's outputs are block columns hi * L + [0, L).
-      const bool flip = sg.side == SIGNS_AFTER;
+      // SG: signs after the rotation (the only side this kernel takes); this
+      // thread's outputs are block columns hi * L + [0, L).
       uint32_t sm[L / 32];
+      if constexpr (SG) {
 #pragma unroll
-      for (int w = 0; w < L / 32; ++w) sm[w] = 0u;
-      if (flip)
-        for (int c = 0; c < L; ++c) sm[c >> 5] |= neg_bit(sg.s, hi * L + c) << (c & 31);
+        for (int w = 0; w < L / 32; ++w) sm[w] = sign_bits32(sg.s, hi * L + 32 * w);
+      }
       // With HALF, sub-groups sub < SPLIT/2 own rows of the first half tile.
       const bool second_half = C::HALF && 2 * sub >= C::SPLIT;
       uint32_t it = 0;
@@ -413,7 +414,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           const int r = sub + C::SPLIT * j;
           if (r < R) {
             const int64_t row = t * R + r;
-            tc_emit_row<LO, MODE>(z[j], hi, row, row < rows, n, norm, group, out0, out1, flip, sm);
+            tc_emit_row<LO, MODE, SG>(z[j], hi, row, row < rows, n, norm, group, out0, out1, sm);
           }
         }
       }

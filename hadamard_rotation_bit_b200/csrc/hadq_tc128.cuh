@@ -49,7 +49,7 @@ struct Tc128Cfg {
 };
 
 // MODE: OUT_F32 / OUT_BF16 / OUT_INT4 / OUT_MXFP4, or -1 for per-token int8.
-template <class C, int MODE>
+template <class C, int MODE, bool SG>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
              const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
@@ -166,12 +166,13 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
       const int quarter = warp & 3;
       const int group_id = (warp - 2) >> 2;
       const int m = quarter * 32 + lane;        // block within the tile = TMEM lane
-      // Signs after the rotation (the launcher never passes SIGNS_BEFORE
-      // here): register k holds block column k.
-      const bool flip = sg.side == SIGNS_AFTER;
-      uint32_t sm[4] = {0u, 0u, 0u, 0u};
-      if (flip)
-        for (int k = 0; k < 128; ++k) sm[k >> 5] |= neg_bit(sg.s, k) << (k & 31);
+      // SG: signs after the rotation (the only side this kernel takes);
+      // register k holds block column k.
+      uint32_t sm[4];
+      if constexpr (SG) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) sm[w] = sign_bits32(sg.s, 32 * w);
+      }
       uint32_t it = 0;
       bool failed = false;   // a wait ran out: skip the work, keep joining the group's barriers
       float* gred = red + 4 * group_id;
@@ -200,7 +201,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        if (flip) apply_signs<128>(z, sm);
+        if constexpr (SG) apply_signs<128>(z, sm);
         const int64_t blk = t * blocks_per_tile + m;
         const bool ok = m < blocks_per_tile && blk < blocks;
         const int64_t e0 = blk * 128;
@@ -219,6 +220,8 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
           if (ok) store_int4<false, 128>(z, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
         } else if constexpr (MODE == OUT_MXFP4) {
           if (ok) store_mxfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+        } else if constexpr (MODE == OUT_NVFP4) {
+          if (ok) store_nvfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
         } else if constexpr (MODE == OUT_BF16) {
           if (ok) store_rotated<false, 128, true>(z, norm, out0, e0);
         } else {

@@ -23,13 +23,14 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhadq.so"
 
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_F32, HADQ_BF16 = 0, 1
-FMTS = {"int4": 0, "int8": 1, "mxfp4": 2}
+FMTS = {"int4": 0, "int8": 1, "mxfp4": 2, "nvfp4": 3}
 HADQ_SIGNS_AFTER, HADQ_SIGNS_BEFORE = 0, 1
 SIDES = {"after": HADQ_SIGNS_AFTER, "before": HADQ_SIGNS_BEFORE}
 EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
     "hadq_device_faults", "hadq_rotate_quant_host_static", "hadq_rotate_signed", "hadq_rotate_quant_signed",
+    "hadq_rotate_quant_nvfp4",
 )
 
 _lock = threading.Lock()
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_rotate_signed.restype = i32
         lib.hadq_rotate_quant_signed.argtypes = [vp, i32, i64, i64, i64, vp, i32, i32, i64, vp, vp, vp]
         lib.hadq_rotate_quant_signed.restype = i32
+        lib.hadq_rotate_quant_nvfp4.argtypes = [vp, i32, i64, i64, i64, ctypes.c_float, vp, vp, vp]
+        lib.hadq_rotate_quant_nvfp4.restype = i32
         _lib = lib
         return lib
 
@@ -129,6 +132,8 @@ def output_shapes(rows: int, n: int, fmt: str, group: int):
         return (rows, n), torch.int8, (rows,), torch.float32
     if fmt == "mxfp4":
         return (rows, n // 2), torch.uint8, (rows, n // 32), torch.uint8
+    if fmt == "nvfp4":
+        return (rows, n // 2), torch.uint8, (rows, n // 16), torch.uint8
     raise HadqError(HADQ_ERR_INVALID_ARG, f"unknown fmt {fmt!r}")
 
 
@@ -231,4 +236,19 @@ def hadq_rotate_quant_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "
     _check(lib.hadq_rotate_quant_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, _signs_ptr(signs),
                                         SIDES[side], FMTS[fmt], group, codes.data_ptr(), scales.data_ptr(),
                                         _stream_handle(stream)))
+    return codes, scales
+
+
+def hadq_rotate_quant_nvfp4(x: torch.Tensor, tensor_scale: float = 1.0, block: int = 0,
+                            codes: torch.Tensor | None = None, scales: torch.Tensor | None = None, stream=None):
+    """Rotate and quantize to NVFP4 with a per-tensor scale; returns (codes, E4M3 scales)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    cs, cd, ss, sd = output_shapes(rows, n, "nvfp4", 16)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=x.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=x.device)
+    _check(lib.hadq_rotate_quant_nvfp4(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, float(tensor_scale),
+                                       codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
     return codes, scales

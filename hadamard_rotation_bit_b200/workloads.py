@@ -20,6 +20,8 @@ permutation drawn from a ``seed + 1`` stream):
   (rotate-half pairing (i, i + 64), theta_i = 10000^(-i/64), position = s);
   per-head 128-point rotation; Q -> bf16, K -> int4 group 128.
 * ``c5``  65536 x 8192 bf16 Student-t(3); full 8192-point rotation; MXFP4.
+* ``c2n`` / ``c5n``  the ``c2`` / ``c5`` input quantized to NVFP4 (E4M3 scale
+  per 16 elements, per-tensor scale 1) instead.
 * ``c2r`` / ``c2rb``  the ``c2`` input and quantizer with a random Hadamard
   rotation ("Rotation Transform", section 1.5): signs after (the random
   Hadamard matrix) or before (its transpose); the b signs are Rademacher
@@ -68,6 +70,8 @@ class Workload:
             return r * n + r * 4
         if self.fmt == "mxfp4":
             return r * n // 2 + r * (n // 32)
+        if self.fmt == "nvfp4":
+            return r * n // 2 + r * (n // 16)
         raise ValueError(self.fmt)
 
     @property
@@ -89,6 +93,10 @@ WORKLOADS = {
                     16 * 32 * 4096, 128, 128, "bf16", "int4", 128),
     "c5": Workload("c5", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point Hadamard, MXFP4",
                    65536, 8192, 8192, "bf16", "mxfp4", 32),
+    "c2n": Workload("c2n", "R1 4096 tokens x hidden 4096 bf16, full 4096-point Hadamard, NVFP4 (E4M3 scale per 16)",
+                    4096, 4096, 4096, "bf16", "nvfp4", 16, base="c2"),
+    "c5n": Workload("c5n", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point Hadamard, NVFP4 "
+                    "(E4M3 scale per 16)", 65536, 8192, 8192, "bf16", "nvfp4", 16, base="c5"),
     "c2r": Workload("c2r", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard (signs after), "
                     "int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128, signs="after", base="c2"),
     "c2rb": Workload("c2rb", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard transpose "

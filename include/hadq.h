@@ -65,7 +65,8 @@ typedef enum hadq_dtype {
 typedef enum hadq_fmt {
   HADQ_INT4_SYM = 0,          /* symmetric int4 RTN per group, fp16 scales */
   HADQ_INT8_SYM = 1,          /* symmetric int8 RTN per token (row), fp32 scale */
-  HADQ_MXFP4 = 2              /* E2M1 codes, E8M0 shared exponent per 32 */
+  HADQ_MXFP4 = 2,             /* E2M1 codes, E8M0 shared exponent per 32 */
+  HADQ_NVFP4 = 3              /* E2M1 codes, FP8 E4M3 scale per 16 */
 } hadq_fmt;
 
 typedef enum hadq_sign_side {
@@ -115,6 +116,16 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  *                  code = E2M1 rne(y / 2^e), saturating at +/-6, sign bit 3.
  *                  codes:  [rows x n/2] bytes, element 2i in the low nibble.
  *                  scales: [rows x n/32] bytes = e + 127 (E8M0).
+ *   HADQ_NVFP4     group must be 0 or 16; n a multiple of 16.  The pages name
+ *                  the scheme and its block of 16 ("Rotation Transform",
+ *                  introduction and section 2.1) but not its encoding;
+ *                  reading: NVIDIA's public NVFP4 definition, single-level here
+ *                  (per-tensor scale 1; see hadq_rotate_quant_nvfp4):
+ *                  s = E4M3(m / 6), round half to even, saturating at 448;
+ *                  code = E2M1 rne(y / s), saturating at +/-6, sign bit 3;
+ *                  s == 0 -> codes 0.
+ *                  codes:  [rows x n/2] bytes, element 2i in the low nibble.
+ *                  scales: [rows x n/16] E4M3 bytes.
  *
  * Codes are computed from the fp32 rotation with the stored scale; the
  * product y * (1/s) is rounded once (fused multiply-add onto the integer grid).
@@ -122,6 +133,18 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  */
 HADQ_API hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
                               hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream);
+
+/*
+ * hadq_rotate_quant_nvfp4: HADQ_NVFP4 with its per-tensor (second-level)
+ * scale t: the block scales and codes are those of y / t, so dequantization
+ * is code * s * t.  t must be finite and > 0 (HADQ_ERR_INVALID_ARG
+ * otherwise); t = 1 is hadq_rotate_quant with HADQ_NVFP4.  A caller that
+ * uses the full E4M3 range sets t = amax(y) / (6 * 448) from a calibrated or
+ * previously measured amax.  Buffers, checks and errors as hadq_rotate_quant.
+ */
+HADQ_API hadq_status hadq_rotate_quant_nvfp4(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n,
+                                             int64_t block, float tensor_scale, void* codes, void* scales,
+                                             void* stream);
 
 /*
  * Random Hadamard ("Rotation Transform", AutoRound docs, section 1.5:
@@ -138,8 +161,9 @@ HADQ_API hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_
  *                           Rademacher signs ahead of the block FWHT in
  *                           orbitquant's RPBH rotation ("orbitquant 0.2.0").
  *   signs   device pointer to b int8 values (b = the block, n when block is
- *           0 / -1 / n); entry j < 0 means s_j = -1, any other value +1.  Read
- *           only; it must not overlap an output.  May be null when rows == 0.
+ *           0 / -1 / n), 16-byte aligned; entry j < 0 means s_j = -1, any
+ *           other value +1.  Read only; it must not overlap an output.  May be
+ *           null when rows == 0.
  * Everything else (shapes, formats, alignment, errors, asynchrony) is as for
  * hadq_rotate / hadq_rotate_quant.  The quantizer sees the signed rotation,
  * so for AFTER the scales equal the unsigned ones and the codes of negated

@@ -9,7 +9,7 @@ in DESIGN.md):
 * codes: bit-exact, except where the oracle's pre-round value lies within a
   window W = 1e-6 * (group absmax) of a rounding boundary; there either
   adjacent code is accepted and the case is counted;
-* scales: fp16 / E8M0 scales exact, except where the oracle's pre-rounding
+* scales: fp16 / E8M0 / E4M3 scales exact, except where the oracle's pre-rounding
   value lies within 1e-6 (relative) of a rounding boundary of the scale
   format, where the other neighbour is accepted (and the group's codes are
   then checked against the oracle's codes for that neighbour); fp32 int8
@@ -156,6 +156,46 @@ def check_mxfp4(x64, codes_packed, scales_e8m0, block: int, y=None) -> dict:
             "code_differs_in_window": int((got != oracle.e2m1_encode(v)).sum())}
 
 
+def _e4m3_value(byte):
+    """Value of E4M3 bytes (sign, exponent bias 7, 3 mantissa bits; 0x7F/0xFF unused)."""
+    b = np.asarray(byte, dtype=np.uint8).astype(np.int64)
+    e, m = (b >> 3) & 15, b & 7
+    mag = np.where(e > 0, np.ldexp(1.0 + m / 8.0, e - 7), np.ldexp(m / 8.0, -6))
+    return np.where(b & 0x80, -mag, mag)
+
+
+def check_nvfp4(x64, codes_packed, scales_e4m3, block: int, y=None, tensor_scale: float = 1.0) -> dict:
+    """NVFP4: E4M3 scale of max|v| / 6 per 16 elements (v = y / tensor_scale),
+    E2M1 codes of v / s.  The scale may take the other rounding neighbour only
+    when max|v| / 6 lies within 1e-6 (relative) of an E4M3 rounding boundary;
+    the codes are then checked against the oracle's codes for the GPU's scale."""
+    y = oracle.rotate(x64, block) if y is None else y
+    rows, n = y.shape
+    g = y.reshape(rows, n // 16, 16) / tensor_scale
+    m = np.abs(g).max(axis=-1)
+    s_gpu = _e4m3_value(np.asarray(scales_e4m3, dtype=np.uint8).reshape(rows, n // 16))
+    cand_lo = oracle.to_e4m3(m / 6 * (1 - WINDOW))
+    cand_mid = oracle.to_e4m3(m / 6)
+    cand_hi = oracle.to_e4m3(m / 6 * (1 + WINDOW))
+    scale_ok = (s_gpu == cand_mid) | (s_gpu == cand_lo) | (s_gpu == cand_hi)
+    assert scale_ok.all(), f"{(~scale_ok).sum()} E4M3 scales outside the oracle's candidates"
+    got = unpack_nibbles(codes_packed, signed=False).reshape(rows, n // 16, 16)
+    usable = s_gpu > 0
+    safe = np.where(usable, s_gpu, 1.0)[..., None]
+    v = g / safe
+    w = WINDOW * m[..., None] / safe
+
+    def enc(t):
+        return np.where(usable[..., None], oracle.e2m1_encode(t), 0)
+    ok, boundary = _check_codes(got, v, w, enc)
+    assert ok.all(), f"{(~ok).sum()} NVFP4 codes differ outside the boundary window"
+    return {"elements": int(y.size), "groups": int(m.size),
+            "scale_boundary_groups": int((cand_lo != cand_hi).sum()),
+            "scale_took_neighbour": int((s_gpu != cand_mid).sum()),
+            "code_boundary_cases": int(boundary.sum()),
+            "code_differs_in_window": int((got != enc(v)).sum())}
+
+
 def check(fmt, x64, out0, out1, block, group, y=None):
     """``y``: the oracle's rotation when it is not ``oracle.rotate(x64, block)``
     (e.g. a random Hadamard rotation)."""
@@ -165,4 +205,6 @@ def check(fmt, x64, out0, out1, block, group, y=None):
         return check_int8(x64, out0, out1, block, y=y)
     if fmt == "mxfp4":
         return check_mxfp4(x64, out0, out1, block, y=y)
+    if fmt == "nvfp4":
+        return check_nvfp4(x64, out0, out1, block, y=y)
     raise ValueError(fmt)

@@ -164,7 +164,25 @@ def test_signed_rejects_signs_overlapping_an_output(lib):
     # codes at B cover rows * n / 2 bytes; signs inside that range
     assert _qs(lib, signs=B + 16) == H.HADQ_ERR_INVALID_ARG
     assert "signs" in lib.hadq_last_error().decode()
-    assert _qs(lib, signs=C + 2) == H.HADQ_ERR_INVALID_ARG            # inside the scales
-    assert _rs(lib, signs=B + 100) == H.HADQ_ERR_INVALID_ARG          # inside out (fp32, 16 KB)
+    assert _qs(lib, signs=C + 16) == H.HADQ_ERR_INVALID_ARG           # inside the scales
+    assert _rs(lib, signs=B + 96) == H.HADQ_ERR_INVALID_ARG           # inside out (fp32, 16 KB)
+    assert _qs(lib, signs=S + 8) == H.HADQ_ERR_MISALIGNED             # signs must be 16-byte aligned
+    assert _rs(lib, signs=S + 1, side=H.HADQ_SIGNS_BEFORE) == H.HADQ_ERR_MISALIGNED
     # block 128: the signs span only 128 bytes, so B - 128 just touches nothing
     assert _rs(lib, block=128, signs=B - 128, x=None) == H.HADQ_ERR_INVALID_ARG   # null x still caught first
+
+
+
+def test_nvfp4_validation(lib):
+    f = lib.hadq_rotate_quant_nvfp4
+    assert f(None, 1, 0, 1024, 0, 1.0, None, None, None) == H.HADQ_OK
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert f(A, 1, 4, 1024, 0, bad, B, C, None) == H.HADQ_ERR_INVALID_ARG
+        assert "tensor_scale" in lib.hadq_last_error().decode()
+    assert f(A, 1, 4, 1000, 0, 1.0, B, C, None) == H.HADQ_ERR_INVALID_ARG           # full non-power-of-2
+    assert f(A, 1, 4, 1032, 8, 1.0, B, C, None) == H.HADQ_ERR_INVALID_ARG           # 16 does not divide n
+    assert _q(lib, fmt=3, group=32) == H.HADQ_ERR_INVALID_ARG                        # NVFP4 blocks are 16
+    assert lib.hadq_scales_bytes(4, 1024, 3, 16) == 4 * 64
+    assert lib.hadq_scales_bytes(4, 1024, 3, 0) == 4 * 64
+    assert lib.hadq_scales_bytes(4, 1024, 3, 32) == 0
+    assert lib.hadq_codes_bytes(4, 1024, 3) == 2048

@@ -101,6 +101,8 @@ def _fmt_ok(n, fmt, group):
         return n % group == 0
     if fmt == "mxfp4":
         return n % 32 == 0
+    if fmt == "nvfp4":
+        return n % 16 == 0
     return True
 
 
@@ -113,14 +115,15 @@ def test_rotate_sweep(rows, n, block, x_dtype):
 
 
 @pytest.mark.parametrize("rows,n,block", SIZES)
-@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("int8", 0), ("mxfp4", 32)])
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("int8", 0), ("mxfp4", 32),
+                                       ("nvfp4", 16)])
 def test_quant_sweep(rows, n, block, fmt, group):
     if not _fmt_ok(n, fmt, group):
         pytest.skip("group does not divide n")
     if fmt == "int8" and n > 32768:
         pytest.skip("per-token int8 limit")
     x_dtype = "bf16" if (n + rows) % 2 else "f32"
-    stored, x64 = synth(rows, n, x_dtype, seed=7 * n + block + rows, dist="t" if fmt == "mxfp4" else "normal")
+    stored, x64 = synth(rows, n, x_dtype, seed=7 * n + block + rows, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
     codes, scales = run_quant(stored, x_dtype, block, fmt, group)
     _log(f"sweep-{fmt}{group}-{rows}x{n}-b{block}-{x_dtype}", pc.check(fmt, x64, codes, scales, block, group))
 
@@ -132,6 +135,8 @@ def test_quant_sweep(rows, n, block, fmt, group):
     (3001, 8192, 0, "mxfp4", 32),      # two-warp teams, several iterations
     (1023, 14336, 128, "int8", 0),     # per-token rows, grid loops
     (517, 16384, 2048, "int8", 0),     # per-token team-row kernel
+    (3001, 8192, 0, "nvfp4", 16),      # two-warp teams, NVFP4
+    (40007, 80, 16, "nvfp4", 16),      # 16-element segments (n = 80), grid-stride tail
 ])
 def test_multi_iteration_grids(rows, n, block, fmt, group):
     stored, x64 = synth(rows, n, "bf16", seed=rows)
@@ -207,7 +212,7 @@ def test_zero_rows_is_a_noop():
     assert codes.numel() == 0 and scales.numel() == 0
 
 
-@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int8", 0), ("mxfp4", 32)])
+@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int8", 0), ("mxfp4", 32), ("nvfp4", 16)])
 @pytest.mark.parametrize("n,block", [(4096, 0), (1024, 128)])
 def test_all_zero_rows(fmt, group, n, block):
     stored = np.zeros((5, n), dtype=np.uint16)
@@ -231,6 +236,8 @@ def test_scale_overflow_and_subnormal_scales():
         _log(f"edge-int4-b{block}", rep)
         codes, scales = run_quant(v, "f32", block, "mxfp4", 32)
         _log(f"edge-mxfp4-b{block}", pc.check_mxfp4(x64, codes, scales, block))
+        codes, scales = run_quant(v, "f32", block, "nvfp4", 16)       # saturating and zero E4M3 scales
+        _log(f"edge-nvfp4-b{block}", pc.check_nvfp4(x64, codes, scales, block))
         codes, scales = run_quant(v, "f32", block, "int8", 0)
         _log(f"edge-int8-b{block}", pc.check_int8(x64, codes, scales, block))
 
@@ -245,7 +252,7 @@ def test_exact_ties_and_sign_of_zero():
     y[3, :] = -0.01
     y[3, 0] = 4.0
     x = oracle.rotate(y, 0).astype(np.float32)   # not exact: ties become near-ties (boundary window)
-    for fmt, group in (("int4", 32), ("mxfp4", 32), ("int8", 0)):
+    for fmt, group in (("int4", 32), ("mxfp4", 32), ("int8", 0), ("nvfp4", 16)):
         codes, scales = run_quant(x, "f32", 0, fmt, group)
         _log(f"ties-{fmt}", pc.check(fmt, x.astype(np.float64), codes, scales, 0, group))
 
@@ -339,3 +346,19 @@ def test_offsets_beyond_2_31_elements():
     pc.check_int4(x64, codes[-64:].cpu().numpy(), scales[-64:].cpu().numpy(), 128, 128)
     del x, codes, scales
     torch.cuda.empty_cache()
+
+
+
+@pytest.mark.parametrize("rows,n,block,x_dtype", [(37, 1024, 0, "f32"), (29, 1024, 32, "bf16"), (9, 2048, 256, "bf16"),
+                                                  (13, 48, 16, "f32")])
+@pytest.mark.parametrize("t", [1.0, 0.25, 3.0, "amax"])
+def test_nvfp4_tensor_scale(rows, n, block, x_dtype, t):
+    """hadq_rotate_quant_nvfp4: blocks and codes of y / t (t = 1, a power of
+    2, a non-power of 2, and the full-range choice amax(y) / (6 * 448))."""
+    stored, x64 = synth(rows, n, x_dtype, seed=n + rows, dist="t")
+    if t == "amax":
+        t = float(np.abs(oracle.rotate(x64, block)).max() / (6 * 448))
+    codes, scales = H.hadq_rotate_quant_nvfp4(to_dev(stored, x_dtype), t, block)
+    torch.cuda.synchronize()
+    _log(f"nvfp4-t{t:.4g}-{rows}x{n}-b{block}",
+         pc.check_nvfp4(x64, codes.cpu().numpy(), scales.cpu().numpy(), block, tensor_scale=t))

@@ -84,7 +84,7 @@ CASES = [  # (rows, n, block, x_dtype): which kernel serves it under "auto"
 
 
 def _fmt_ok(n, fmt, group):
-    return (fmt != "int4" or n % group == 0) and (fmt != "mxfp4" or n % 32 == 0)
+    return (fmt != "int4" or n % group == 0) and (fmt != "mxfp4" or n % 32 == 0) and (fmt != "nvfp4" or n % 16 == 0)
 
 
 @pytest.mark.parametrize("rows,n,block,x_dtype", CASES)
@@ -102,12 +102,12 @@ def test_signed_rotate(path, rows, n, block, x_dtype, side):
 
 @pytest.mark.parametrize("rows,n,block,x_dtype", CASES)
 @pytest.mark.parametrize("side", ["after", "before"])
-@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int4", 32), ("int8", 0), ("mxfp4", 32)])
+@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int4", 32), ("int8", 0), ("mxfp4", 32), ("nvfp4", 16)])
 def test_signed_quant(path, rows, n, block, x_dtype, side, fmt, group):
     if not _fmt_ok(n, fmt, group):
         pytest.skip("group does not divide n")
     b = oracle.resolve_block(n, block)
-    stored, x64 = synth(rows, n, x_dtype, seed=2 * n + rows + group, dist="t" if fmt == "mxfp4" else "normal")
+    stored, x64 = synth(rows, n, x_dtype, seed=2 * n + rows + group, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
     s = signs_for(b, 3 * n + block + group)
     y = oracle.rotate_signed(x64, block, s, side)
     codes, scales = run_signed_quant(stored, x_dtype, block, s, side, fmt, group)

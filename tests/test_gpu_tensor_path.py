@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from hadamard_rotation_bit_b200 import hadq as H
 from hadamard_rotation_bit_b200 import workloads as W
 from tests import parity_check as pc
@@ -49,15 +50,16 @@ def test_tc_rotate(rows, n, block):
 
 
 @pytest.mark.parametrize("rows,n,block", SIZES)
-@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32), ("nvfp4", 16)])
 def test_tc_quant(rows, n, block, fmt, group):
-    stored, x64 = synth(rows, n, "bf16", seed=3 * n + rows + group, dist="t" if fmt == "mxfp4" else "normal")
+    stored, x64 = synth(rows, n, "bf16", seed=3 * n + rows + group, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
     codes, scales = run_quant(stored, "bf16", block, fmt, group)
     _log(f"tc-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, codes, scales, block, group))
 
 
 @pytest.mark.parametrize("rows,n,fmt,group", [(2501, 4096, "int4", 128), (3001, 8192, "mxfp4", 32),
-                                              (1037, 4096, "mxfp4", 32), (999, 8192, "int4", 64)])
+                                              (1037, 4096, "mxfp4", 32), (999, 8192, "int4", 64),
+                                              (1501, 4096, "nvfp4", 16), (777, 8192, "nvfp4", 16)])
 def test_tc_many_tiles_ragged(rows, n, fmt, group):
     stored, x64 = synth(rows, n, "bf16", seed=rows + 7)
     codes, scales = run_quant(stored, "bf16", 0, fmt, group)
@@ -151,9 +153,9 @@ def test_tc128_rotate(rows, n):
 
 
 @pytest.mark.parametrize("rows,n", B128)
-@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32)])
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32), ("nvfp4", 16)])
 def test_tc128_quant(rows, n, fmt, group):
-    stored, x64 = synth(rows, n, "bf16", seed=5 * n + rows + group, dist="t" if fmt == "mxfp4" else "normal")
+    stored, x64 = synth(rows, n, "bf16", seed=5 * n + rows + group, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
     codes, scales = run_quant(stored, "bf16", 128, fmt, group)
     _log(f"tc128-{fmt}{group}-{rows}x{n}", pc.check(fmt, x64, codes, scales, 128, group))
 
@@ -201,3 +203,27 @@ def test_tc128_guard_bytes_ragged_blocks():
     assert (cb[:pad] == 0xA5).all() and (cb[pad + cbytes:] == 0xA5).all()
     assert (sb[:pad] == 0x5A).all() and (sb[pad + sbytes:] == 0x5A).all()
     pc.check_int4(x64, codes.cpu().numpy(), scales.cpu().numpy(), 128, 128)
+
+
+
+@pytest.mark.parametrize("rows,n,block", [(19, 4096, 0), (7, 8192, 0), (33, 1024, 128)])
+@pytest.mark.parametrize("t", [0.25, 3.0, "amax"])
+def test_tc_nvfp4_tensor_scale(rows, n, block, t):
+    stored, x64 = synth(rows, n, "bf16", seed=n + rows, dist="t")
+    if t == "amax":
+        t = float(np.abs(oracle.rotate(x64, block)).max() / (6 * 448))
+    codes, scales = H.hadq_rotate_quant_nvfp4(to_dev(stored, "bf16"), t, block)
+    torch.cuda.synchronize()
+    _log(f"tc-nvfp4-t{t:.4g}-{rows}x{n}-b{block}",
+         pc.check_nvfp4(x64, codes.cpu().numpy(), scales.cpu().numpy(), block, tensor_scale=t))
+
+
+@pytest.mark.parametrize("key", ["c2n", "c5n"])
+def test_tc_nvfp4_configs(key):
+    w = W.WORKLOADS[key]
+    rows = w.rows if key == "c2n" else 8192
+    stored = W.generate(key, slice(0, rows), workers=NPROC)
+    codes, scales = run_quant(stored, "bf16", w.block, "nvfp4", 16)
+    rng = np.random.default_rng(6)
+    ids = np.unique(np.concatenate([np.arange(128), np.arange(rows - 128, rows), rng.choice(rows, 1024, replace=False)]))
+    _log(f"tc-{key}", pc.check_nvfp4(W.bits_to_float64(stored[ids], "bf16"), codes[ids], scales[ids], w.block))

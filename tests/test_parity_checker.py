@@ -90,3 +90,26 @@ def test_mxfp4_checker():
     s2[0, 0] += 1
     with pytest.raises(AssertionError):
         pc.check_mxfp4(x, codes, s2, 0)
+
+
+def test_nvfp4_checker():
+    x = _x(8, 512, 4)
+    y, codes, scales = oracle.rotate_quant(x, 0, "nvfp4", 16)
+    rep = pc.check_nvfp4(x, codes, scales, 0)
+    assert rep["code_differs_in_window"] == 0 and rep["groups"] == 8 * 32
+    flipped = codes.copy()
+    flipped[1, 3] ^= 0x01                 # one code one grid step off
+    with pytest.raises(AssertionError):
+        pc.check_nvfp4(x, flipped, scales, 0)
+    s2 = scales.copy()
+    s2[0, 0] += 1                         # next E4M3 value: 6-12 % off
+    with pytest.raises(AssertionError):
+        pc.check_nvfp4(x, codes, s2, 0)
+    # the E4M3 byte decoder used by the checker agrees with the oracle's encoder
+    vals = np.exp(np.random.default_rng(1).uniform(-12, 6, 500))
+    np.testing.assert_array_equal(pc._e4m3_value(oracle.e4m3_encode(vals)), oracle.to_e4m3(vals))
+    # per-tensor scale: outputs of quantize(y, t) pass with tensor_scale=t
+    _, c3, s3 = oracle.rotate_quant(x, 0, "nvfp4", 16, tensor_scale=0.25)
+    pc.check_nvfp4(x, c3, s3, 0, tensor_scale=0.25)
+    with pytest.raises(AssertionError):
+        pc.check_nvfp4(x, c3, s3, 0, tensor_scale=1.0)

@@ -88,3 +88,10 @@ def test_random_hadamard_workloads_share_the_c2_input():
     assert W.WORKLOADS["c2r"].signs == "after" and W.WORKLOADS["c2rb"].signs == "before"
     with pytest.raises(ValueError):
         W.generate_signs("c2")
+
+
+def test_nvfp4_workloads_share_their_inputs():
+    assert W.WORKLOADS["c2n"].algorithmic_bytes == 33_554_432 + 8_388_608 + 4096 * 256
+    assert W.WORKLOADS["c5n"].algorithmic_bytes == 1_073_741_824 + 268_435_456 + 65536 * 512
+    np.testing.assert_array_equal(W.generate("c2n", slice(5, 9)), W.generate("c2", slice(5, 9)))
+    np.testing.assert_array_equal(W.generate("c5n", slice(2047, 2050)), W.generate("c5", slice(2047, 2050)))
