@@ -257,16 +257,26 @@ __device__ __forceinline__ void apply_signs(float (&v)[N], const uint32_t (&m_in
 
 // ------------------------------------------------------------------ quantizers
 
-// Absmax of registers [lo, lo + cnt) (cnt a multiple of 4; order does not matter).
+// max(|a|, |b|, |c|) in one instruction (the three-input max with absolute
+// inputs of sm_100).
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Absmax of registers [lo, lo + cnt) (cnt a multiple of 4; order does not
+// matter): two independent chains that each take two new registers per
+// three-input max, then one max of the two.
 template <int N>
 __device__ __forceinline__ float absmax_regs(const float (&v)[N], int lo, int cnt) {
-  float m0 = 0.f, m1 = 0.f;
+  float ma = v[lo], mb = v[lo + 1];     // raw: every max below takes absolute values
 #pragma unroll
-  for (int i = 0; i < cnt; i += 4) {
-    m0 = fmaxf(m0, fmaxf(fabsf(v[lo + i]), fabsf(v[lo + i + 1])));
-    m1 = fmaxf(m1, fmaxf(fabsf(v[lo + i + 2]), fabsf(v[lo + i + 3])));
+  for (int i = 2; i < cnt; i += 4) {
+    ma = max3abs(ma, v[lo + i], v[lo + i + 1]);
+    if (i + 2 < cnt) mb = max3abs(mb, v[lo + i + 2], v[lo + i + 3]);
   }
-  return fmaxf(m0, m1);
+  return max3abs(ma, mb, mb);
 }
 
 // Eight int4 codes rne(v * rn) of elements e0..e0+7 (register order PERM), as
