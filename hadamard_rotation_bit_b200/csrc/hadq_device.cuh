@@ -367,6 +367,21 @@ constexpr float kInv6 = 1.0f / 6.0f;
 
 __device__ __forceinline__ float fast_recip(float s) { return __fdividef(1.0f, s); }
 
+// 32 output bytes at p: one 256-bit store (full 32-byte sectors) when p is
+// 32-byte aligned, else two 128-bit stores.  A thread's run of outputs is
+// contiguous while the runs of the lanes of a warp are not, so 16-byte stores
+// would fill every sector in two halves.
+__device__ __forceinline__ void store32(void* p, const uint4& a, const uint4& b) {
+  if ((reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+  } else {
+    reinterpret_cast<uint4*>(p)[0] = a;
+    reinterpret_cast<uint4*>(p)[1] = b;
+  }
+}
+
 // --------------------------------------------------------------- epilogues
 // Each epilogue owns N consecutive rotated-but-unnormalised values z of one
 // row (register order PERM), starting at flattened element index e0;
@@ -378,22 +393,35 @@ __device__ __forceinline__ void store_rotated(const float (&v)[N], float norm, v
   if constexpr (OUT_IS_BF16) {
     uint16_t* o = static_cast<uint16_t*>(out) + e0;
     static_assert(N % 8 == 0, "bf16 chunk must hold whole 16-byte stores");
-#pragma unroll
-    for (int i = 0; i < N / 8; ++i) {
+    auto chunk = [&](int i) {
       uint4 w;
       w.x = pack_bf16x2(v[reg<PERM>(8 * i + 0)] * norm, v[reg<PERM>(8 * i + 1)] * norm);
       w.y = pack_bf16x2(v[reg<PERM>(8 * i + 2)] * norm, v[reg<PERM>(8 * i + 3)] * norm);
       w.z = pack_bf16x2(v[reg<PERM>(8 * i + 4)] * norm, v[reg<PERM>(8 * i + 5)] * norm);
       w.w = pack_bf16x2(v[reg<PERM>(8 * i + 6)] * norm, v[reg<PERM>(8 * i + 7)] * norm);
-      reinterpret_cast<uint4*>(o)[i] = w;
+      return w;
+    };
+    if constexpr (N % 16 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 8; i += 2) store32(o + 8 * i, chunk(i), chunk(i + 1));
+    } else {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) reinterpret_cast<uint4*>(o)[i] = chunk(i);
     }
   } else {
     float* o = static_cast<float*>(out) + e0;
     static_assert(N % 4 == 0, "fp32 chunk must hold whole float4s");
+    auto chunk = [&](int i) {
+      return make_uint4(__float_as_uint(v[reg<PERM>(4 * i)] * norm), __float_as_uint(v[reg<PERM>(4 * i + 1)] * norm),
+                        __float_as_uint(v[reg<PERM>(4 * i + 2)] * norm), __float_as_uint(v[reg<PERM>(4 * i + 3)] * norm));
+    };
+    if constexpr (N % 8 == 0) {
 #pragma unroll
-    for (int i = 0; i < N / 4; ++i)
-      reinterpret_cast<float4*>(o)[i] = make_float4(v[reg<PERM>(4 * i)] * norm, v[reg<PERM>(4 * i + 1)] * norm,
-                                                    v[reg<PERM>(4 * i + 2)] * norm, v[reg<PERM>(4 * i + 3)] * norm);
+      for (int i = 0; i < N / 4; i += 2) store32(o + 4 * i, chunk(i), chunk(i + 1));
+    } else {
+#pragma unroll
+      for (int i = 0; i < N / 4; ++i) reinterpret_cast<uint4*>(o)[i] = chunk(i);
+    }
   }
 }
 
@@ -407,6 +435,7 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
 #pragma unroll
   for (int j = 0; j < NS; ++j) m32[j] = absmax_regs(v, 32 * j, 32);   // a 32-block is closed under reg<>
   const int spg = group >> 5;  // 32-element sub-blocks per group: 1, 2 or 4
+  uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of sub-block j - 1, stored with those of j
 #pragma unroll
   for (int j = 0; j < NS; ++j) {
     float mz = m32[j];
@@ -433,7 +462,13 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
       w.z = pack_int4x8_clamped<PERM>(v, 32 * j + 16, rn);
       w.w = pack_int4x8_clamped<PERM>(v, 32 * j + 24, rn);
     }
-    reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
+    if constexpr (NS == 1) {
+      reinterpret_cast<uint4*>(codes + (e0 >> 1))[0] = w;
+    } else if (j & 1) {
+      store32(codes + ((e0 + 32 * (j - 1)) >> 1), prev, w);
+    } else {
+      prev = w;
+    }
     if ((j & (spg - 1)) == 0) scales[(e0 + 32 * j) >> (__ffs(group) - 1)] = s16;   // group is a power of 2
   }
 }
@@ -443,6 +478,7 @@ template <bool PERM, int N>
 __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales, int64_t e0) {
   static_assert(N % 32 == 0, "MX groups are 32 elements");
+  uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of sub-block j - 1, stored with those of j
 #pragma unroll
   for (int j = 0; j < N / 32; ++j) {
     const float m = absmax_regs(v, 32 * j, 32) * norm;
@@ -457,7 +493,13 @@ __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uin
     w.y = pack_e2m1x8<PERM>(v, 32 * j + 8, f);
     w.z = pack_e2m1x8<PERM>(v, 32 * j + 16, f);
     w.w = pack_e2m1x8<PERM>(v, 32 * j + 24, f);
-    reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] = w;
+    if constexpr (N == 32) {
+      reinterpret_cast<uint4*>(codes + (e0 >> 1))[0] = w;
+    } else if (j & 1) {
+      store32(codes + ((e0 + 32 * (j - 1)) >> 1), prev, w);
+    } else {
+      prev = w;
+    }
     scales[(e0 >> 5) + j] = static_cast<uint8_t>(byte);
   }
 }
@@ -495,6 +537,7 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
     scales[e0 >> 4] = static_cast<uint8_t>(b & 0xFFu);
   } else {
     static_assert(N % 32 == 0, "NVFP4 chunks above 16 elements come in pairs of blocks");
+    uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of blocks 2j - 2, 2j - 1, stored with those of 2j, 2j + 1
 #pragma unroll
     for (int j = 0; j < N / 32; ++j) {
       const float m0 = absmax_regs(v, 32 * j, 16) * nq;
@@ -503,9 +546,15 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
       const float2 s = e4m3x2_values(b);
       const float f0 = s.x > 0.f ? nq * fast_recip(s.x) : 0.f;
       const float f1 = s.y > 0.f ? nq * fast_recip(s.y) : 0.f;
-      reinterpret_cast<uint4*>(codes + ((e0 + 32 * j) >> 1))[0] =
-          make_uint4(pack_e2m1x8<PERM>(v, 32 * j, f0), pack_e2m1x8<PERM>(v, 32 * j + 8, f0),
-                     pack_e2m1x8<PERM>(v, 32 * j + 16, f1), pack_e2m1x8<PERM>(v, 32 * j + 24, f1));
+      const uint4 w = make_uint4(pack_e2m1x8<PERM>(v, 32 * j, f0), pack_e2m1x8<PERM>(v, 32 * j + 8, f0),
+                                 pack_e2m1x8<PERM>(v, 32 * j + 16, f1), pack_e2m1x8<PERM>(v, 32 * j + 24, f1));
+      if constexpr (N == 32) {
+        reinterpret_cast<uint4*>(codes + (e0 >> 1))[0] = w;
+      } else if (j & 1) {
+        store32(codes + ((e0 + 32 * (j - 1)) >> 1), prev, w);
+      } else {
+        prev = w;
+      }
       reinterpret_cast<uint16_t*>(scales + ((e0 + 32 * j) >> 4))[0] = b;
     }
   }
@@ -520,7 +569,14 @@ __device__ __forceinline__ void store_int8(const float (&v)[N], float norm, floa
   const float r = (s >= 1.0e-36f && s <= 3.0e38f) ? fast_recip(s) : (s > 0.f ? __frcp_rn(s) : 0.f);
   const float rn = r * norm;
   if (m * r < 127.25f) {         // normal scale: every |v * rn| < 127.5, no clamp
-    if constexpr (N % 16 == 0) {
+    if constexpr (N % 32 == 0) {
+      auto chunk = [&](int i) {
+        return make_uint4(pack_int8x4<PERM>(v, 16 * i, rn), pack_int8x4<PERM>(v, 16 * i + 4, rn),
+                          pack_int8x4<PERM>(v, 16 * i + 8, rn), pack_int8x4<PERM>(v, 16 * i + 12, rn));
+      };
+#pragma unroll
+      for (int i = 0; i < N / 16; i += 2) store32(codes + e0 + 16 * i, chunk(i), chunk(i + 1));
+    } else if constexpr (N % 16 == 0) {
       uint4* o = reinterpret_cast<uint4*>(codes + e0);
 #pragma unroll
       for (int i = 0; i < N / 16; ++i)
