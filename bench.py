@@ -53,7 +53,7 @@ FALLBACK_HBM_GBS = 6650.0
 # A step is one pass of the fused path over one batch of a workload: the
 # launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
 STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"],
-              "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"]}
+              "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"], "c3rb": ["c3rb"], "c5rb": ["c5rb"]}
 WORKLOAD = W.WORKLOADS["c2"]
 
 

@@ -245,7 +245,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
                       cudaStream_t stream, int sms, int dev, Signs sg) {
   const int lo = sh.logb - 7;
-  const hl::TcVariant v = hl::tc_kernel_for(lo, mode, sg.side != hadq::SIGNS_NONE);
+  const hl::TcVariant v = hl::tc_kernel_for(lo, mode, sg.side);
   if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no tensor-core kernel for this size and format");
   const int L = 1 << lo, R = v.tile_n / L;
   const int64_t rows = sh.rows * (sh.n >> sh.logb);
@@ -301,7 +301,7 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   }
-  const hl::Tc128Variant v = hl::tc128_kernel_for(mode, sg.side != hadq::SIGNS_NONE);
+  const hl::Tc128Variant v = hl::tc128_kernel_for(mode);
   if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no block-128 tensor-core kernel for this format");
   int occ = 0;
   hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
@@ -314,8 +314,7 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
 }
 
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
-// -1 for per-token int8.  Signs on the input side (SIGNS_BEFORE) are applied
-// by the butterfly kernels only; the tensor-core kernels take the others.
+// -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
                    cudaStream_t stream, Signs sg = Signs{nullptr, hadq::SIGNS_NONE}) {
   int sms = 0, dev = 0;
@@ -335,7 +334,7 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours
-  if (kernel_choice() != KernelChoice::Butterfly && sg.side != hadq::SIGNS_BEFORE) {
+  if (kernel_choice() != KernelChoice::Butterfly) {
     if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
     if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
   }

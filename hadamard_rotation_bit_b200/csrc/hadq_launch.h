@@ -48,8 +48,8 @@ TeamRowFn team_row_kernel_bf16(int logb, bool sg);
 
 // Tensor-core kernels: full size 2^(7 + lo), lo = 5 or 6; block 128 (mode -1 =
 // per-token int8).
-TcVariant tc_kernel_for(int lo, int mode, bool sg);
-Tc128Variant tc128_kernel_for(int mode, bool sg);
+TcVariant tc_kernel_for(int lo, int mode, int side);   // side: hadq::SignSide
+Tc128Variant tc128_kernel_for(int mode);   // signs of either side folded into B
 
 // The tensor-core kernels' sticky fault word (bounded waits that ran out);
 // cleared when `clear` is non-zero.  -1 on a CUDA error.

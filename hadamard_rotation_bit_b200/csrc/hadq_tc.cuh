@@ -26,12 +26,21 @@
 // The producer starts streaming as soon as the barriers exist; the other
 // warps build H_128 in shared memory and allocate tensor memory meanwhile.
 // Before anything else, thread 0 asks L2 to prefetch the CTA's first
-// kPrefetchTiles tiles.  A prefetch is only a hint (no data reaches the CTA
+// PREFETCH tiles.  A prefetch is only a hint (no data reaches the CTA
 // and nothing is observed), so it may precede the wait for the previous
 // kernel in the stream; it lets the first TMA loads after that wait hit L2
-// instead of starting cold from HBM.  With HALF, the MMAs of a tile are issued
+// instead of starting cold from HBM.  Two tiles is the measured optimum for
+// 4096 x 4096 (9.46 us per launch; 10.1 us with 4, 11.1 us with 8, where the
+// prefetches of later tiles delay the first tile's loads).  With HALF, the MMAs of a tile are issued
 // as two N/2 halves with their own commit, so the epilogue warps of the first
 // half start while the tensor core still works on the second.
+// Random Hadamard signs (section 1.5) after the rotation are applied in the
+// epilogue to the finished outputs.  Signs before it must reach the operand
+// ahead of the MMA, since every output mixes inputs with different signs:
+// with SIDE == SIGNS_BEFORE extra warps (SIGN_THREADS) flip the bf16 sign bits of each
+// landed tile in shared memory (one XOR per 32-bit word; each thread always
+// owns the same 16 chunks of the swizzled tile, so its sign masks are loaded
+// once) and release the stage to the MMA through a second mbarrier.
 // Every mbarrier wait gives up after one second (globaltimer); on timeout the
 // kernel records a fault in hadq_tc_fault, stops issuing work and still
 // releases its tensor memory.
@@ -46,10 +55,14 @@ namespace tc {
 constexpr int kABytes = 128 * 128 * 2;     // A operand: H_128 in bf16
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after 1 s
 
-constexpr int kPrefetchTiles = 2;          // tiles per CTA prefetched into L2 at kernel entry
 
-template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_>
+template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_, int PREFETCH_ = 2>
 struct TcCfg {
+  static constexpr int PREFETCH = PREFETCH_;             // tiles per CTA prefetched into L2 at entry
+  // Sign-flipping threads (signs before the rotation only): as many as the
+  // register budget allows, since they sit between a tile's arrival and its
+  // MMA (n = 4096: 60-register epilogue; n = 8192: up to 137 registers).
+  static constexpr int SIGN_THREADS = LO_ == 5 ? 256 : 128;
   static constexpr int LO = LO_, L = 1 << LO;
   static constexpr int TILE_N = TILE_N_;                  // MMA N: columns per tile
   static constexpr int R = TILE_N / L;                    // rows per tile
@@ -73,12 +86,12 @@ struct TcCfg {
   static constexpr int SM_A = 0;                          // H_128, 2 K-panels x 16 KB
   static constexpr int SM_B = SM_A + kABytes;             // STAGES x TILE_BYTES
   static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
-  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * STAGES + 3 * ACC_BUFS);
+  static constexpr int SM_SLOT = SM_BARS + 8 * (3 * STAGES + 3 * ACC_BUFS);
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;  // + alignment slack
 };
 
 // Fault codes written to hadq_tc_fault.
-constexpr unsigned kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u;
+constexpr unsigned kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u, kFaultSign = 8u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -194,15 +207,21 @@ __device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits tha
 
 // Epilogue for one row of one tile: z holds the 2^LO values of TMEM lane hi'
 // (after the tensor-core stage over hi); finish the butterfly over lo and emit.
-// With SG, output column hi * 2^LO + c is negated where bit c of `sm` is set
-// (random Hadamard, signs after the rotation).
-template <int LO, int MODE, bool SG>
+// Signs after the rotation (random Hadamard): SGK = 1, output column
+// hi * 2^LO + c is negated where bit c of the mask words sm[c / 32] is set;
+// SGK = 2, sm holds one XOR word (0 or the fp32 sign bit) per column c.
+template <int LO, int MODE, int SGK>
 __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t row, bool row_ok, int n, float norm,
                                             int group, void* __restrict__ out0, void* __restrict__ out1,
-                                            const uint32_t (&sm)[(1 << LO) / 32]) {
+                                            const uint32_t* sm) {
   constexpr int L = 1 << LO;
   fwht_bits<L, 0, LO>(z);
-  if constexpr (SG) apply_signs<L>(z, sm);
+  if constexpr (SGK == 1) {
+    apply_signs<L>(z, *reinterpret_cast<const uint32_t(*)[L / 32]>(sm));
+  } else if constexpr (SGK == 2) {
+#pragma unroll
+    for (int c = 0; c < L; ++c) z[c] = __uint_as_float(__float_as_uint(z[c]) ^ sm[c]);
+  }
   const int64_t e0 = row * n + static_cast<int64_t>(hi) * L;   // first output element of this thread
   if constexpr (MODE == OUT_INT4) {
     // Groups of `group` outputs = L values x (group / L) consecutive lanes.
@@ -252,11 +271,20 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
   }
 }
 
-template <class C, int MODE, bool SG>
-__global__ void __launch_bounds__(C::THREADS, 1)
+// Threads of tc_rotate_kernel<C, MODE, SIDE>.
+template <class C, int SIDE>
+__host__ __device__ constexpr int tc_threads() {
+  return C::THREADS + (SIDE == SIGNS_BEFORE ? C::SIGN_THREADS : 0);
+}
+
+template <class C, int MODE, int SIDE>
+__global__ void __launch_bounds__(tc_threads<C, SIDE>(), 1)
 tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
                  float norm, int group, void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
   constexpr int LO = C::LO, L = C::L, R = C::R;
+  constexpr bool SG = SIDE == SIGNS_AFTER, SB = SIDE == SIGNS_BEFORE;
+  constexpr int T = tc_threads<C, SIDE>();
+  constexpr int kFirstSignWarp = 2 + 4 * C::SPLIT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
@@ -264,6 +292,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::ACC_BUFS;
   uint64_t* acc_full2 = acc_empty + C::ACC_BUFS;   // second half of a tile (HALF)
+  uint64_t* flipped = acc_full2 + C::ACC_BUFS;     // stage signed (SB): the MMA may read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -271,15 +300,17 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
 
   if (threadIdx.x == 0) {
     int64_t t = blockIdx.x;
-    for (int i = 0; i < kPrefetchTiles && t < tiles; ++i, t += gridDim.x) {
+    for (int i = 0; i < C::PREFETCH && t < tiles; ++i, t += gridDim.x) {
       const int64_t r1 = (t + 1) * R < rows ? (t + 1) * R : rows;   // a tile is rows [t R, r1), contiguous
       prefetch_l2(x + t * R * n, static_cast<uint32_t>((r1 - t * R) * n * 2));
     }
+    if constexpr (SIDE != SIGNS_NONE) prefetch_l2(sg.s, 128 * L);   // the b signs (int8)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&flipped[s], C::SIGN_THREADS / 32);   // one arrival per sign warp
     }
     for (int b = 0; b < C::ACC_BUFS; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -310,7 +341,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
     // A = H_128 (K-major, 128-byte swizzle, two K-panels of 64): element (m, k)
     // at panel (k / 64) + m * 128 + (k % 64) * 2 bytes, 16-byte chunk index
     // XOR-ed with (m % 8).  Entry (m, k) = (-1)^popcount(m & k) as bf16.
-    for (int i = threadIdx.x - 32; i < 128 * 16; i += C::THREADS - 32) {
+    for (int i = threadIdx.x - 32; i < 128 * 16; i += T - 32) {
       const int m = i >> 4, kc = i & 15;              // 8 consecutive k per 16-byte chunk
       uint32_t w[4];
 #pragma unroll
@@ -329,7 +360,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
     }
     tc_fence_before();
-    asm volatile("bar.sync 1, %0;" ::"r"(C::THREADS - 32) : "memory");   // warps 1.. only
+    asm volatile("bar.sync 1, %0;" ::"r"(T - 32) : "memory");   // warps 1.. only
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -343,7 +374,8 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           const uint32_t ph = (it / C::STAGES) & 1;
           const int b = it % C::ACC_BUFS;
           const uint32_t aph = (it / C::ACC_BUFS) & 1;
-          if (!mbar_wait(&full[s], ph) || (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
+          if (!mbar_wait(SB ? &flipped[s] : &full[s], ph) ||
+              (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
             atomicOr(&hadq_tc_fault, kFaultMma);
             break;
           }
@@ -370,18 +402,75 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           }
         }
       }
+    } else if (SB && warp >= kFirstSignWarp) {
+      // ------------------------------------------- signs before the rotation
+      // The stage holds the box (lo, hi, r) of the rows with lo innermost:
+      // 2L-byte lines (hi, r), 16-byte chunks permuted by the 64-byte
+      // (L = 32: chunk bits 4..5 ^= address bits 7..8) or 128-byte (L = 64:
+      // bits 4..6 ^= bits 7..9) swizzle.  A chunk holds the 8 columns
+      // hi * L + 8 * (logical chunk) + [0, 8) of one row; a negative int8
+      // sign has bit 7 set, which byte_perm moves onto the bf16 sign bits.
+      grid_dependency_sync();                  // the signs are caller memory
+      constexpr int kChunks = C::TILE_BYTES / 16 / C::SIGN_THREADS;
+      constexpr uint32_t kSwz = LO == 5 ? 3u : 7u;
+      const int j = threadIdx.x - 32 * kFirstSignWarp;
+      uint32_t q[kChunks][2];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const uint32_t p = 16u * static_cast<uint32_t>(j + C::SIGN_THREADS * i);
+        const uint32_t hi = (p / (2 * L)) & 127u;
+        const uint32_t c = ((p % (2 * L)) >> 4) ^ ((p >> 7) & kSwz);
+        const uint2 v = *reinterpret_cast<const uint2*>(sg.s + hi * L + 8 * c);
+        q[i][0] = v.x & 0x80808080u;
+        q[i][1] = v.y & 0x80808080u;
+      }
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (!mbar_wait(&full[s], ph)) {
+          atomicOr(&hadq_tc_fault, kFaultSign);
+          break;
+        }
+        uint4* stage = reinterpret_cast<uint4*>(smem + C::SM_B + s * C::TILE_BYTES) + j;
+        constexpr int kBatch = 8;              // loads in flight before the first store
+#pragma unroll
+        for (int i0 = 0; i0 < kChunks; i0 += kBatch) {
+          uint4 v[kBatch];
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) v[i] = stage[C::SIGN_THREADS * (i0 + i)];
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) {
+            v[i].x ^= __byte_perm(q[i0 + i][0], 0u, 0x1404);
+            v[i].y ^= __byte_perm(q[i0 + i][0], 0u, 0x3424);
+            v[i].z ^= __byte_perm(q[i0 + i][1], 0u, 0x1404);
+            v[i].w ^= __byte_perm(q[i0 + i][1], 0u, 0x3424);
+            stage[C::SIGN_THREADS * (i0 + i)] = v[i];
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&flipped[s]);
+      }
     } else {
       // --------------------------------------------------------- epilogue
       grid_dependency_sync();                  // outputs may still be read by the previous kernel
       const int quarter = warp & 3;            // TMEM lanes this warp may access
       const int sub = (warp - 2) >> 2;         // rows r = sub (mod SPLIT) of every tile
       const int hi = quarter * 32 + lane;      // the H_128 output index this thread owns
-      // SG: signs after the rotation (the only side this kernel takes); this
-      // thread's outputs are block columns hi * L + [0, L).
-      uint32_t sm[L / 32];
-      if constexpr (SG) {
+      // SG: signs after the rotation; this thread's outputs are block columns
+      // hi * L + [0, L).
+      // n = 4096 keeps one XOR word per column (32 registers; the epilogue
+      // has room), n = 8192 the 2 bit-mask words.
+      constexpr int SGK = !SG ? 0 : (LO == 5 ? 2 : 1);
+      uint32_t sm[SGK == 2 ? L : L / 32];
+      if constexpr (SGK == 1) {
 #pragma unroll
         for (int w = 0; w < L / 32; ++w) sm[w] = sign_bits32(sg.s, hi * L + 32 * w);
+      } else if constexpr (SGK == 2) {
+        const uint32_t m = sign_bits32(sg.s, hi * L);
+#pragma unroll
+        for (int c = 0; c < L; ++c) sm[c] = (m << (31 - c)) & 0x80000000u;
       }
       // With HALF, sub-groups sub < SPLIT/2 own rows of the first half tile.
       const bool second_half = C::HALF && 2 * sub >= C::SPLIT;
@@ -414,7 +503,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           const int r = sub + C::SPLIT * j;
           if (r < R) {
             const int64_t row = t * R + r;
-            tc_emit_row<LO, MODE, SG>(z[j], hi, row, row < rows, n, norm, group, out0, out1, sm);
+            tc_emit_row<LO, MODE, SGK>(z[j], hi, row, row < rows, n, norm, group, out0, out1, sm);
           }
         }
       }

@@ -17,12 +17,18 @@
 // A = X_blk is K-major with the 128-byte swizzle, loaded by TMA (no
 // multicast) as two 64-element K-panels per tile from two 2-D tensor maps
 // whose bases differ by 128 bytes; B = H_128 (symmetric) is built in shared
-// memory in the same layout.  Roles as in hadq_tc.cuh: warp 0 TMA producer,
+// memory in the same layout.  Random Hadamard signs cost nothing per tile:
+// they are folded into B when it is built, as diag(s) H_128 for signs before
+// the rotation and H_128 diag(s) for signs after it (section 1.5), so the
+// MMA applies the signed rotation and the epilogue is the unsigned one.  Roles as in hadq_tc.cuh: warp 0 TMA producer,
 // warp 1 TMEM allocator + single-thread MMA issuer, warps 2.. EPI_GROUPS
 // groups of 4 epilogue warps taking whole tiles round-robin.  Waits are
 // bounded (hadq_tc_fault).  As there, thread 0 first asks L2 to prefetch the
-// CTA's first kPrefetchTiles tiles (a hint, so it may precede the wait for
-// the previous kernel).
+// CTA's first PREFETCH tiles (a hint, so it may precede the wait for the
+// previous kernel).  These kernels run for tens of microseconds or more, so a
+// deep prefetch (8 tiles = 256 KB per CTA) pays: it keeps HBM busy through the
+// previous kernel's drain and the dependency release, which a short prefetch
+// leaves idle (8192 x 14336 int8: 54.5 us with 2 tiles, 51.5 us with 8).
 #pragma once
 
 #include "hadq_tc.cuh"
@@ -30,10 +36,11 @@
 namespace hadq {
 namespace tc {
 
-template <int STAGES_, int EPI_GROUPS_>
+template <int STAGES_, int EPI_GROUPS_, int PREFETCH_>
 struct Tc128Cfg {
   static constexpr int STAGES = STAGES_;
   static constexpr int EPI_GROUPS = EPI_GROUPS_;
+  static constexpr int PREFETCH = PREFETCH_;                    // tiles per CTA prefetched into L2 at entry
   static constexpr int PANEL_BYTES = 128 * 128;                 // 128 blocks x 64 bf16
   static constexpr int TILE_BYTES = 2 * PANEL_BYTES;            // A operand per tile (<= 128 blocks)
   static constexpr int ACC_BUFS = 4;                            // 4 x 128 TMEM columns
@@ -48,8 +55,9 @@ struct Tc128Cfg {
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
 };
 
-// MODE: OUT_F32 / OUT_BF16 / OUT_INT4 / OUT_MXFP4, or -1 for per-token int8.
-template <class C, int MODE, bool SG>
+// MODE: OUT_F32 / OUT_BF16 / OUT_INT4 / OUT_MXFP4 / OUT_NVFP4, or -1 for
+// per-token int8.  sg: none, or signs on either side (folded into B).
+template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
              const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
@@ -70,7 +78,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
 
   if (threadIdx.x == 0) {
     int64_t t = blockIdx.x;
-    for (int i = 0; i < kPrefetchTiles && t < tiles; ++i, t += gridDim.x) {
+    for (int i = 0; i < C::PREFETCH && t < tiles; ++i, t += gridDim.x) {
       const int64_t b0 = t * blocks_per_tile;   // a tile is blocks [b0, b1), contiguous
       const int64_t b1 = b0 + blocks_per_tile < blocks ? b0 + blocks_per_tile : blocks;
       prefetch_l2(x + b0 * 128, static_cast<uint32_t>((b1 - b0) * 256));
@@ -109,7 +117,12 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
       }
     }
   } else {
-    // B = H_128, K-major with the 128-byte swizzle (row n holds H[n][k] over k).
+    // B = H_128, K-major with the 128-byte swizzle (row n holds B[n][k] over
+    // k; D = A B^T).  With signs, B[n][k] = H[n][k] s[k] (before) or s[n]
+    // H[n][k] (after): one XOR of the bf16 sign bit.  The signs are caller
+    // memory, so they are read only after the previous kernel has completed.
+    const bool signed_b = sg.side != SIGNS_NONE;
+    if (signed_b) grid_dependency_sync();
     for (int i = threadIdx.x - 32; i < 128 * 16; i += C::THREADS - 32) {
       const int m = i >> 4, kc = i & 15;
       uint32_t w[4];
@@ -117,6 +130,21 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
       for (int p = 0; p < 4; ++p) {
         const int k = kc * 8 + 2 * p;
         w[p] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+      }
+      if (signed_b) {
+        if (sg.side == SIGNS_BEFORE) {
+          // s[kc*8 .. kc*8+7]: 8-byte aligned (s is 16-byte aligned); a negative
+          // entry has bit 7 set, which lands on the bf16 sign bit.
+          const uint2 q = *reinterpret_cast<const uint2*>(sg.s + kc * 8);
+          const uint32_t q0 = q.x & 0x80808080u, q1 = q.y & 0x80808080u;
+          w[0] ^= __byte_perm(q0, 0u, 0x1404);
+          w[1] ^= __byte_perm(q0, 0u, 0x3424);
+          w[2] ^= __byte_perm(q1, 0u, 0x1404);
+          w[3] ^= __byte_perm(q1, 0u, 0x3424);
+        } else if (neg_bit(sg.s, m)) {
+#pragma unroll
+          for (int p = 0; p < 4; ++p) w[p] ^= 0x80008000u;
+        }
       }
       const int panel = kc >> 3, chunk = kc & 7;
       const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
@@ -166,13 +194,6 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
       const int quarter = warp & 3;
       const int group_id = (warp - 2) >> 2;
       const int m = quarter * 32 + lane;        // block within the tile = TMEM lane
-      // SG: signs after the rotation (the only side this kernel takes);
-      // register k holds block column k.
-      uint32_t sm[4];
-      if constexpr (SG) {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) sm[w] = sign_bits32(sg.s, 32 * w);
-      }
       uint32_t it = 0;
       bool failed = false;   // a wait ran out: skip the work, keep joining the group's barriers
       float* gred = red + 4 * group_id;
@@ -201,7 +222,6 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        if constexpr (SG) apply_signs<128>(z, sm);
         const int64_t blk = t * blocks_per_tile + m;
         const bool ok = m < blocks_per_tile && blk < blocks;
         const int64_t e0 = blk * 128;

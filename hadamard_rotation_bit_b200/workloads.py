@@ -26,6 +26,8 @@ permutation drawn from a ``seed + 1`` stream):
   rotation ("Rotation Transform", section 1.5): signs after (the random
   Hadamard matrix) or before (its transpose); the b signs are Rademacher
   draws (``generate_signs``), int8 +/-1.
+* ``c3rb`` / ``c5rb``  the ``c3`` / ``c5`` input and quantizer with signs
+  before the rotation (block 128 / full 8192).
 
 Values are drawn in float64, rounded to float32 (nearest even) and, for
 bf16 tensors, to bfloat16 (nearest even).
@@ -102,6 +104,11 @@ WORKLOADS = {
     "c2rb": Workload("c2rb", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard transpose "
                      "(signs before), int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128,
                      signs="before", base="c2"),
+    "c3rb": Workload("c3rb", "R4 8192 tokens x intermediate 14336 bf16, block 128 random Hadamard transpose "
+                     "(signs before), int8 per token", 8192, 14336, 128, "bf16", "int8", 0, signs="before", base="c3"),
+    "c5rb": Workload("c5rb", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point random Hadamard "
+                     "transpose (signs before), MXFP4", 65536, 8192, 8192, "bf16", "mxfp4", 32, signs="before",
+                     base="c5"),
 }
 
 _STREAM = {"c1": 1, "c2": 2, "c3": 3, "c4q": 4, "c4k": 5, "c5": 6}

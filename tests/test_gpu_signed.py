@@ -6,9 +6,10 @@ R = H_b diag(s) / sqrt(b) (side "after", the random_hadamard_matrix of
 (side "before").  Each case runs through the C ABI on seeded inputs and is
 compared element by element with oracle.rotate_signed under the same
 tolerances as the deterministic rotation.  Both implementations are covered:
-the tensor-core kernels (default for bf16 at b = 4096, 8192 and 128, side
-after) and the CUDA-core butterfly kernels (everything else, and every side
-"before").
+the tensor-core kernels (default for bf16 at b = 4096, 8192 and 128, either
+side: signs after in the epilogue, signs before flipped in the staged tile
+ahead of the MMA, and at b = 128 both folded into the H_128 operand) and the
+CUDA-core butterfly kernels (everything else).
 """
 
 import os
@@ -114,15 +115,16 @@ def test_signed_quant(path, rows, n, block, x_dtype, side, fmt, group):
     _log(f"signed-{path}-{side}-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, codes, scales, block, group, y=y))
 
 
-@pytest.mark.parametrize("rows,n,block,x_dtype", [(19, 4096, 0, "bf16"), (33, 1024, 128, "bf16"),
+@pytest.mark.parametrize("rows,n,block,x_dtype", [(19, 4096, 0, "bf16"), (7, 8192, 0, "bf16"), (33, 1024, 128, "bf16"),
                                                   (37, 1024, 0, "f32"), (29, 1024, 32, "f32")])
-def test_signed_any_negative_int8_is_minus_one(path, rows, n, block, x_dtype):
+@pytest.mark.parametrize("side", ["after", "before"])
+def test_signed_any_negative_int8_is_minus_one(path, rows, n, block, x_dtype, side):
     b = oracle.resolve_block(n, block)
     stored, x64 = synth(rows, n, x_dtype, seed=rows)
     s = signs_for(b, 99, odd_values=True)
     assert set(np.unique(s)) - {-1, 1}
-    y = oracle.rotate_signed(x64, block, s, "after")
-    codes, scales = run_signed_quant(stored, x_dtype, block, s, "after", "int4", 128)
+    y = oracle.rotate_signed(x64, block, s, side)
+    codes, scales = run_signed_quant(stored, x_dtype, block, s, side, "int4", 128)
     pc.check_int4(x64, codes, scales, block, 128, y=y)
 
 
@@ -165,11 +167,14 @@ def test_signed_exact_zero_rows_code_as_plus_zero(path):
     pc.check_mxfp4(x64, codes, scales, 0, y=y)
 
 
-@pytest.mark.parametrize("key", ["c2r", "c2rb"])
+@pytest.mark.parametrize("key", ["c2r", "c2rb", "c3rb", "c5rb"])
 def test_signed_config_full_size(key):
-    """The bench's random Hadamard workloads at full size (4096 x 4096 bf16,
-    int4 g128) in the default kernel choice: c2r on the tensor cores, c2rb
-    (signs before) on the butterfly kernels."""
+    """The bench's random Hadamard workloads at full size in the default
+    kernel choice, all on the tensor cores: c2r (4096 x 4096 bf16 -> int4
+    g128, signs after, applied in the epilogue), c2rb (the same, signs before,
+    flipped in each staged tile ahead of the MMA), c3rb (8192 x 14336, block
+    128, int8 per token, signs folded into the H_128 operand) and c5rb
+    (65536 x 8192 -> MXFP4, signs before; oracle on a seeded row sample)."""
     from hadamard_rotation_bit_b200 import workloads as W
     from tests.test_gpu_parity import NPROC
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
@@ -177,9 +182,14 @@ def test_signed_config_full_size(key):
     w = W.WORKLOADS[key]
     stored = W.generate(key, workers=NPROC)
     s = W.generate_signs(key)
-    x64 = W.bits_to_float64(stored, "bf16")
+    ids = slice(None)
+    if key == "c5rb":
+        rng = np.random.default_rng(7)
+        ids = np.unique(np.concatenate([np.arange(256), np.arange(w.rows - 256, w.rows),
+                                        rng.choice(w.rows, 2048, replace=False)]))
+    x64 = W.bits_to_float64(stored[ids], "bf16")
     y = oracle.rotate_signed(x64, w.block, s, w.signs)
     H.hadq_device_faults(clear=True)
-    codes, scales = run_signed_quant(stored, "bf16", w.block, s, w.signs, "int4", 128)
+    codes, scales = run_signed_quant(stored, "bf16", w.block, s, w.signs, w.fmt, w.group)
     assert H.hadq_device_faults(clear=True) == 0
-    _log(f"signed-{key}", pc.check_int4(x64, codes, scales, w.block, 128, y=y))
+    _log(f"signed-{key}", pc.check(w.fmt, x64, codes[ids], scales[ids], w.block, w.group, y=y))

@@ -86,6 +86,11 @@ def test_random_hadamard_workloads_share_the_c2_input():
         np.testing.assert_array_equal(s, W.generate_signs(key))
         assert not np.array_equal(s, W.generate_signs(key, seed=W.rank_seed(1)))
     assert W.WORKLOADS["c2r"].signs == "after" and W.WORKLOADS["c2rb"].signs == "before"
+    for key, base in (("c3rb", "c3"), ("c5rb", "c5")):
+        w, wb = W.WORKLOADS[key], W.WORKLOADS[base]
+        assert w.signs == "before" and w.algorithmic_bytes == wb.algorithmic_bytes and w.block == wb.block
+        np.testing.assert_array_equal(W.generate(key, slice(0, 3)), W.generate(base, slice(0, 3)))
+        assert W.generate_signs(key).shape == (w.block,)
     with pytest.raises(ValueError):
         W.generate_signs("c2")
 
