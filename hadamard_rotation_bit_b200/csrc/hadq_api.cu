@@ -353,11 +353,11 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     }
     const hl::TeamFn fn = hl::team_kernel_for(bf, sh.logb, mode, sgd);
     if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no kernel for this block size and format");
-    const int smem = hadq::kThreads * hadq::kRowFloats * 4;
+    const int smem = hadq::team_smem_bytes(sh.logb);
     int occ = 0;
     st = occupancy(reinterpret_cast<const void*>(fn), dev, hadq::kThreads, smem, &occ);
     if (st != HADQ_OK) return st;
-    const int teams = hadq::kThreads >> (sh.logb - 7);
+    const int teams = hadq::kThreads >> (sh.logb - hadq::team_logp(sh.logb));
     const int64_t units = sh.rows * (sh.n >> sh.logb);
     const int64_t grid = std::min<int64_t>(ceil_div(units, teams), int64_t(sms) * occ);
     return launch_result(launch_pdl(fn, grid, hadq::kThreads, smem, stream, x, units, sh.norm, group, out0, out1, sg),

@@ -179,11 +179,41 @@ __device__ __forceinline__ uint32_t ldg_stream(const uint32_t* p) {
   return r;
 }
 
+// 32 bytes (one whole sector) in one 256-bit load; p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_stream32(const void* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
 // NE contiguous input elements starting at element index e -> dst[0..NE).
+// A thread's run is far from its neighbours' (a segment or a team chunk), so
+// a 16-byte load uses half of each 32-byte sector it fetches and the next
+// load fetches the sector again (L1 is bypassed); runs of 32 bytes or more
+// therefore load whole sectors with 256-bit loads when the run is 32-byte
+// aligned (the API promises 16), and 16-byte loads otherwise.
 template <bool IN_BF16, int NE>
 __device__ __forceinline__ void load_elems(const void* __restrict__ x, int64_t e, float* dst) {
   if constexpr (IN_BF16) {
     const uint16_t* p = static_cast<const uint16_t*>(x) + e;
+    if constexpr (NE % 16 == 0) {
+      if ((reinterpret_cast<uintptr_t>(p) & 31) == 0) {
+#pragma unroll
+        for (int i = 0; i < NE / 16; ++i) {
+          uint4 w, u;
+          ldg_stream32(p + 16 * i, w, u);
+          unpack_bf16x2(w.x, dst[16 * i + 0], dst[16 * i + 1]);
+          unpack_bf16x2(w.y, dst[16 * i + 2], dst[16 * i + 3]);
+          unpack_bf16x2(w.z, dst[16 * i + 4], dst[16 * i + 5]);
+          unpack_bf16x2(w.w, dst[16 * i + 6], dst[16 * i + 7]);
+          unpack_bf16x2(u.x, dst[16 * i + 8], dst[16 * i + 9]);
+          unpack_bf16x2(u.y, dst[16 * i + 10], dst[16 * i + 11]);
+          unpack_bf16x2(u.z, dst[16 * i + 12], dst[16 * i + 13]);
+          unpack_bf16x2(u.w, dst[16 * i + 14], dst[16 * i + 15]);
+        }
+        return;
+      }
+    }
     if constexpr (NE % 8 == 0) {
 #pragma unroll
       for (int i = 0; i < NE / 8; ++i) {
@@ -204,6 +234,24 @@ __device__ __forceinline__ void load_elems(const void* __restrict__ x, int64_t e
     }
   } else {
     const float* p = static_cast<const float*>(x) + e;
+    if constexpr (NE % 8 == 0) {
+      if ((reinterpret_cast<uintptr_t>(p) & 31) == 0) {
+#pragma unroll
+        for (int i = 0; i < NE / 8; ++i) {
+          uint4 w, u;
+          ldg_stream32(p + 8 * i, w, u);
+          dst[8 * i + 0] = __uint_as_float(w.x);
+          dst[8 * i + 1] = __uint_as_float(w.y);
+          dst[8 * i + 2] = __uint_as_float(w.z);
+          dst[8 * i + 3] = __uint_as_float(w.w);
+          dst[8 * i + 4] = __uint_as_float(u.x);
+          dst[8 * i + 5] = __uint_as_float(u.y);
+          dst[8 * i + 6] = __uint_as_float(u.z);
+          dst[8 * i + 7] = __uint_as_float(u.w);
+        }
+        return;
+      }
+    }
     if constexpr (NE % 4 == 0) {
 #pragma unroll
       for (int i = 0; i < NE / 4; ++i) {
@@ -470,6 +518,38 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
       prev = w;
     }
     if ((j & (spg - 1)) == 0) scales[(e0 + 32 * j) >> (__ffs(group) - 1)] = s16;   // group is a power of 2
+  }
+}
+
+// Symmetric int4 with group 128 for a thread holding 64 consecutive outputs
+// (a group-aligned half when e0 % 128 == 0, the other half in lane ^ 1): the
+// group absmax is exchanged with that lane.  Every lane of the warp must call
+// it; ok = false computes and stores nothing.
+template <bool PERM>
+__device__ __forceinline__ void store_int4_pair(const float (&v)[64], float norm, uint8_t* __restrict__ codes,
+                                                __half* __restrict__ scales, int64_t e0, bool ok) {
+  float mz = fmaxf(absmax_regs(v, 0, 32), absmax_regs(v, 32, 32));
+  mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 1));
+  const float m = mz * norm;
+  const __half s16 = __float2half_rn(m * kInv7);
+  const float s = __half2float(s16);
+  const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
+  const float rn = r * norm;
+  uint4 w0, w1;
+  if (mz * rn < 7.25f) {
+    w0 = make_uint4(pack_int4x8<PERM>(v, 0, rn), pack_int4x8<PERM>(v, 8, rn), pack_int4x8<PERM>(v, 16, rn),
+                    pack_int4x8<PERM>(v, 24, rn));
+    w1 = make_uint4(pack_int4x8<PERM>(v, 32, rn), pack_int4x8<PERM>(v, 40, rn), pack_int4x8<PERM>(v, 48, rn),
+                    pack_int4x8<PERM>(v, 56, rn));
+  } else {
+    w0 = make_uint4(pack_int4x8_clamped<PERM>(v, 0, rn), pack_int4x8_clamped<PERM>(v, 8, rn),
+                    pack_int4x8_clamped<PERM>(v, 16, rn), pack_int4x8_clamped<PERM>(v, 24, rn));
+    w1 = make_uint4(pack_int4x8_clamped<PERM>(v, 32, rn), pack_int4x8_clamped<PERM>(v, 40, rn),
+                    pack_int4x8_clamped<PERM>(v, 48, rn), pack_int4x8_clamped<PERM>(v, 56, rn));
+  }
+  if (ok) {
+    store32(codes + (e0 >> 1), w0, w1);
+    if ((e0 & 127) == 0) scales[e0 >> 7] = s16;
   }
 }
 

@@ -8,19 +8,22 @@
 //    consecutive elements of a row (S >= b, b | S), runs the log2(b) butterfly
 //    stages on the low index bits in registers, and writes its S outputs.
 //    One thread per segment, no cross-thread traffic.
-//  * team kernels (256 <= b <= 8192): a team of T = b / 128 threads owns one
-//    block.  Index bits: e = [hi: t bits | mid: t bits | vec: 7 - t bits],
-//    t = log2 T.  Phase 1: each thread loads, for every hi value, one
-//    contiguous chunk of 2^(7-t) elements (the team reads 128 contiguous
-//    elements per hi value) and runs the stages of its register bits (vec +
-//    hi).  A transpose through shared memory (fp32 rows of 128 + 4 pad floats:
-//    conflict-free on both sides for t >= 5, immediate offsets) hands every
-//    thread the 128 consecutive elements with hi = its team index.  Phase 2
-//    runs the remaining stages (mid bits); the thread then holds a whole run of
-//    128 consecutive outputs for the quantizer.  When the chunk holds at least
-//    4 elements, the transpose stores every quad as (e0, e2, e1, e3), so the
-//    element-bit-0 stage runs in phase 2 on packed f32x2 pairs instead of as
-//    scalar adds in phase 1.
+//  * team kernels (256 <= b <= 8192): a team of T = b / P threads owns one
+//    block, P = 2^p values per thread (P = 64 for b <= 2048, 128 above).
+//    Index bits: e = [hi: t bits | mid: t bits | vec: p - t bits], t = log2 T.
+//    Phase 1: each thread loads, for every hi value, one contiguous chunk of
+//    2^(p-t) elements (the team reads P contiguous elements per hi value) and
+//    runs the stages of its register bits (vec + hi).  A transpose through
+//    shared memory (fp32 rows of P + 4 pad floats: conflict-free on both
+//    sides for P = 128 and t >= 5, immediate offsets) hands every thread the P
+//    consecutive elements with hi = its team index.  Phase 2 runs the
+//    remaining stages (mid bits); the thread then holds a whole run of P
+//    consecutive outputs for the quantizer (an int4 group of 128 at P = 64
+//    spans a thread and its neighbour lane: one shuffle of the absmax).  When
+//    the chunk holds at least 4 elements, the transpose stores every quad as
+//    (e0, e2, e1, e3), so the element-bit-0 stage runs in phase 2 on packed
+//    f32x2 pairs instead of as scalar adds in phase 1.  P = 64 halves the
+//    registers of the short blocks, so more warps per SM hide the loads.
 //
 // The per-token int8 format needs the whole row before any code is written,
 // so it has row kernels: one CTA per row, the same two layouts inside, and a
@@ -47,7 +50,12 @@
 namespace hadq {
 
 constexpr int kThreads = 128;
-constexpr int kRowFloats = 132;   // transpose row: 128 floats + one quad of padding
+constexpr int kRowFloats = 132;   // per-token team rows: 128 floats + one quad of padding
+
+// log2 of the values per team thread for block 2^logb, and the team kernel's
+// dynamic shared memory (one transpose row of P + 4 floats per thread).
+__host__ __device__ constexpr int team_logp(int logb) { return logb <= 11 ? 6 : 7; }
+__host__ __device__ constexpr int team_smem_bytes(int logb) { return kThreads * ((1 << team_logp(logb)) + 4) * 4; }
 
 // ----------------------------------------------------------- segment kernels
 
@@ -162,15 +170,18 @@ segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int
 
 // --------------------------------------------------------------- team kernels
 
-template <int LOGB>
+template <int LOGB, int LOGP = team_logp(LOGB)>
 struct TeamShape {
-  static constexpr int t = LOGB - 7;          // log2(threads per team)
+  static constexpr int P = 1 << LOGP;         // values per thread
+  static constexpr int t = LOGB - LOGP;       // log2(threads per team)
   static constexpr int T = 1 << t;            // threads per team
-  static constexpr int V = 7 - t;             // vec bits per phase-1 chunk
+  static constexpr int V = LOGP - t;          // vec bits per phase-1 chunk
   static constexpr int CE = 1 << V;           // elements per phase-1 chunk
   static constexpr int B = 1 << LOGB;
+  static constexpr int ROW = P + 4;           // transpose row (floats), one quad of padding
+  static constexpr int W = P / 32;            // sign-mask words
   static constexpr bool PERM = V >= 2;        // quads transposed as (e0, e2, e1, e3)
-  static_assert(LOGB >= 8 && LOGB <= 13, "team kernels cover 256..8192");
+  static_assert(LOGB >= 8 && LOGB <= 13 && t >= 1 && V >= 1, "team kernels cover 256..8192");
 };
 
 template <int T>
@@ -183,64 +194,65 @@ __device__ __forceinline__ void team_sync() {
 }
 
 // Sign mask of team thread tau.  BEFORE: phase-1 register h * CE + j holds
-// block column h * 128 + tau * CE + j.  AFTER: register i holds output column
-// tau * 128 + reg<PERM>(i).
-template <int LOGB>
-__device__ __forceinline__ void team_sign_mask(const Signs& sg, int tau, uint32_t (&sm)[4]) {
-  using Sh = TeamShape<LOGB>;
+// block column h * P + tau * CE + j.  AFTER: register i holds output column
+// tau * P + reg<PERM>(i).
+template <int LOGB, int LOGP>
+__device__ __forceinline__ void team_sign_mask(const Signs& sg, int tau, uint32_t (&sm)[TeamShape<LOGB, LOGP>::W]) {
+  using Sh = TeamShape<LOGB, LOGP>;
 #pragma unroll
-  for (int w = 0; w < 4; ++w) sm[w] = 0u;
+  for (int w = 0; w < Sh::W; ++w) sm[w] = 0u;
   if (sg.side == SIGNS_AFTER) {
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const uint32_t m = sign_bits32(sg.s, tau * 128 + 32 * w);
+    for (int w = 0; w < Sh::W; ++w) {
+      const uint32_t m = sign_bits32(sg.s, tau * Sh::P + 32 * w);
       sm[w] = Sh::PERM ? perm_quad_bits(m) : m;
     }
   } else if (sg.side == SIGNS_BEFORE) {
     if constexpr (Sh::CE >= 32) {
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {   // register 32 w + k = column (32 w / CE) * 128 + tau * CE + (32 w) % CE + k
+      for (int w = 0; w < Sh::W; ++w) {   // register 32 w + k = column (32 w / CE) * P + tau * CE + (32 w) % CE + k
         const int i = 32 * w;
-        sm[w] = sign_bits32(sg.s, (i / Sh::CE) * 128 + tau * Sh::CE + (i % Sh::CE));
+        sm[w] = sign_bits32(sg.s, (i / Sh::CE) * Sh::P + tau * Sh::CE + (i % Sh::CE));
       }
     } else {
 #pragma unroll
-      for (int h = 0; h < Sh::T; ++h)   // registers h * CE + [0, CE) = columns h * 128 + tau * CE + [0, CE)
-        sm[(h * Sh::CE) >> 5] |= sign_bits_small<Sh::CE>(sg.s, h * 128 + tau * Sh::CE) << ((h * Sh::CE) & 31);
+      for (int h = 0; h < Sh::T; ++h)   // registers h * CE + [0, CE) = columns h * P + tau * CE + [0, CE)
+        sm[(h * Sh::CE) >> 5] |= sign_bits_small<Sh::CE>(sg.s, h * Sh::P + tau * Sh::CE) << ((h * Sh::CE) & 31);
     }
   }
 }
 
 // Rotate one block of 2^LOGB elements (element base `base`) by a team; on
-// return v[0..128) holds the unnormalised outputs base + tau*128 + [0, 128) in
-// register order TeamShape<LOGB>::PERM.  `rows` is this team's T x kRowFloats
+// return v[0..P) holds the unnormalised outputs base + tau*P + [0, P) in
+// register order TeamShape<LOGB, LOGP>::PERM.  `rows` is this team's T x ROW
 // shared buffer.  With SG and `before`, the loaded values are first
 // multiplied by the signs in `sm` (team_sign_mask, BEFORE layout).
-template <int LOGB, bool IN_BF16, bool SG>
+template <int LOGB, int LOGP, bool IN_BF16, bool SG>
 __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t base, bool valid, int tau,
-                                            float* __restrict__ rows, float (&v)[128], bool before,
-                                            const uint32_t (&sm)[4]) {
-  using Sh = TeamShape<LOGB>;
+                                            float* __restrict__ rows, float (&v)[1 << LOGP], bool before,
+                                            const uint32_t (&sm)[TeamShape<LOGB, LOGP>::W]) {
+  using Sh = TeamShape<LOGB, LOGP>;
+  constexpr int P = Sh::P;
   if (valid) {
 #pragma unroll
-    for (int h = 0; h < Sh::T; ++h) load_elems<IN_BF16, Sh::CE>(x, base + h * 128 + tau * Sh::CE, &v[h * Sh::CE]);
+    for (int h = 0; h < Sh::T; ++h) load_elems<IN_BF16, Sh::CE>(x, base + h * P + tau * Sh::CE, &v[h * Sh::CE]);
     if constexpr (SG) {
-      if (before) apply_signs<128>(v, sm);
+      if (before) apply_signs<P>(v, sm);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 128; ++i) v[i] = 0.f;
+    for (int i = 0; i < P; ++i) v[i] = 0.f;
   }
-  // Phase 1: register index h * CE + j (j = element bits 0..V-1, h = element bits 7..).
+  // Phase 1: register index h * CE + j (j = element bits 0..V-1, h = element bits LOGB-t..).
   if constexpr (Sh::PERM) {
-    fwht_bits<128, 1, 7>(v);          // element bit 0 waits for phase 2
+    fwht_bits<P, 1, LOGP>(v);          // element bit 0 waits for phase 2
   } else {
-    fwht_bits<128, 0, 7>(v);
+    fwht_bits<P, 0, LOGP>(v);
   }
-  // Transpose: buffer row h holds elements h*128 + [0, 128).
+  // Transpose: buffer row h holds elements h*P + [0, P).
 #pragma unroll
   for (int h = 0; h < Sh::T; ++h) {
-    float* rowp = rows + h * kRowFloats;
+    float* rowp = rows + h * Sh::ROW;
     if constexpr (Sh::CE >= 4) {
 #pragma unroll
       for (int k = 0; k < Sh::CE / 4; ++k) {
@@ -254,9 +266,9 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
   }
   team_sync<Sh::T>();
   {
-    const float4* rowp = reinterpret_cast<const float4*>(rows + tau * kRowFloats);
+    const float4* rowp = reinterpret_cast<const float4*>(rows + tau * Sh::ROW);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
+    for (int q = 0; q < P / 4; ++q) {
       const float4 f = rowp[q];
       v[4 * q] = f.x;
       v[4 * q + 1] = f.y;
@@ -265,16 +277,18 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
     }
   }
   team_sync<Sh::T>();
-  // Phase 2: the mid bits (element bits V..6), and element bit 0 (register bit 1 under PERM).
-  if constexpr (Sh::PERM) fwht_stage<128, 1>(v);
-  fwht_bits<128, Sh::V, 7>(v);
+  // Phase 2: the mid bits (element bits V..LOGP-1), and element bit 0 (register bit 1 under PERM).
+  if constexpr (Sh::PERM) fwht_stage<P, 1>(v);
+  fwht_bits<P, Sh::V, LOGP>(v);
 }
 
 template <int LOGB, bool IN_BF16, int MODE, bool SG>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, team_logp(LOGB) == 6 ? 4 : 3)
 team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, void* __restrict__ out0,
             void* __restrict__ out1, Signs sg) {
-  using Sh = TeamShape<LOGB>;
+  constexpr int LOGP = team_logp(LOGB);
+  using Sh = TeamShape<LOGB, LOGP>;
+  constexpr int P = Sh::P;
   constexpr int TEAMS = kThreads / Sh::T;
   constexpr uint32_t kUnitBytes = Sh::B * (IN_BF16 ? 2 : 4);
   grid_dependency_sync();
@@ -282,10 +296,10 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
   float* buf = reinterpret_cast<float*>(smem_f4);
   const int team = threadIdx.x >> Sh::t;
   const int tau = threadIdx.x & (Sh::T - 1);
-  float* rows = buf + team * Sh::T * kRowFloats;
-  uint32_t sm[4];
-  if constexpr (SG) team_sign_mask<LOGB>(sg, tau, sm);
-  float v[128];
+  float* rows = buf + team * Sh::T * Sh::ROW;
+  uint32_t sm[Sh::W];
+  if constexpr (SG) team_sign_mask<LOGB, LOGP>(sg, tau, sm);
+  float v[P];
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * TEAMS; u0 < units;
        u0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
     const int64_t u = u0 + team;
@@ -295,22 +309,30 @@ team_kernel(const void* __restrict__ x, int64_t units, float norm, int group, vo
     }
     const bool valid = u < units;
     const int64_t base = u << LOGB;
-    team_rotate<LOGB, IN_BF16, SG>(x, base, valid, tau, rows, v, sg.side == SIGNS_BEFORE, sm);
-    if (valid) {
-      if constexpr (SG) {
-        if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
+    team_rotate<LOGB, LOGP, IN_BF16, SG>(x, base, valid, tau, rows, v, sg.side == SIGNS_BEFORE, sm);
+    if constexpr (SG) {
+      if (sg.side == SIGNS_AFTER) apply_signs<P>(v, sm);
+    }
+    const int64_t e0 = base + tau * P;
+    if constexpr (MODE == OUT_INT4 && P < 128) {
+      // A group of 128 spans this thread and lane ^ 1: every lane joins the
+      // shuffle (invalid teams hold zeros and store nothing).
+      if (group > P) {
+        store_int4_pair<Sh::PERM>(v, norm, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0, valid);
+      } else if (valid) {
+        store_int4<Sh::PERM, P>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
       }
-      const int64_t e0 = base + tau * 128;
+    } else if (valid) {
       if constexpr (MODE == OUT_F32) {
-        store_rotated<Sh::PERM, 128, false>(v, norm, out0, e0);
+        store_rotated<Sh::PERM, P, false>(v, norm, out0, e0);
       } else if constexpr (MODE == OUT_BF16) {
-        store_rotated<Sh::PERM, 128, true>(v, norm, out0, e0);
+        store_rotated<Sh::PERM, P, true>(v, norm, out0, e0);
       } else if constexpr (MODE == OUT_INT4) {
-        store_int4<Sh::PERM, 128>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+        store_int4<Sh::PERM, P>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
       } else if constexpr (MODE == OUT_NVFP4) {
-        store_nvfp4<Sh::PERM, 128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+        store_nvfp4<Sh::PERM, P>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
       } else {
-        store_mxfp4<Sh::PERM, 128>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+        store_mxfp4<Sh::PERM, P>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
       }
     }
   }
@@ -322,7 +344,7 @@ template <int LOGB, bool IN_BF16, bool SG>
 __global__ void __launch_bounds__(256)
 team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float norm, int8_t* __restrict__ codes,
                      float* __restrict__ scales, Signs sg) {
-  using Sh = TeamShape<LOGB>;
+  using Sh = TeamShape<LOGB, 7>;   // 128 values per thread (blockDim = n / 128)
   grid_dependency_sync();
   extern __shared__ float4 smem_f4[];
   float* buf = reinterpret_cast<float*>(smem_f4);
@@ -331,17 +353,17 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
   const bool active = static_cast<int>(threadIdx.x) < nthreads;
   const int team = threadIdx.x >> Sh::t;
   const int tau = threadIdx.x & (Sh::T - 1);
-  float* team_rows = buf + (active ? team * Sh::T * kRowFloats : 0);
+  float* team_rows = buf + (active ? team * Sh::T * Sh::ROW : 0);
   const int64_t row_bytes = n * (IN_BF16 ? 2 : 4);
-  uint32_t sm[4];
-  if constexpr (SG) team_sign_mask<LOGB>(sg, tau, sm);
+  uint32_t sm[Sh::W];
+  if constexpr (SG) team_sign_mask<LOGB, 7>(sg, tau, sm);
   float v[128];
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     if (threadIdx.x == 0 && r + gridDim.x < rows)
       prefetch_l2(static_cast<const char*>(x) + (r + gridDim.x) * row_bytes, static_cast<uint32_t>(row_bytes));
     const int64_t base = r * n + (static_cast<int64_t>(team) << LOGB);
     if (active) {
-      team_rotate<LOGB, IN_BF16, SG>(x, base, true, tau, team_rows, v, sg.side == SIGNS_BEFORE, sm);
+      team_rotate<LOGB, 7, IN_BF16, SG>(x, base, true, tau, team_rows, v, sg.side == SIGNS_BEFORE, sm);
       if constexpr (SG) {
         if (sg.side == SIGNS_AFTER) apply_signs<128>(v, sm);
       }
