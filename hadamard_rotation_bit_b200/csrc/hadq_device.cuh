@@ -189,14 +189,14 @@ __device__ __forceinline__ void ldg_stream32(const void* p, uint4& a, uint4& b) 
 // NE contiguous input elements starting at element index e -> dst[0..NE).
 // A thread's run is far from its neighbours' (a segment or a team chunk), so
 // a 16-byte load uses half of each 32-byte sector it fetches and the next
-// load fetches the sector again (L1 is bypassed); runs of 32 bytes or more
-// therefore load whole sectors with 256-bit loads when the run is 32-byte
-// aligned (the API promises 16), and 16-byte loads otherwise.
-template <bool IN_BF16, int NE>
+// load fetches the sector again (L1 is bypassed); with WIDE, runs of 32 bytes
+// or more therefore load whole sectors with 256-bit loads when the run is
+// 32-byte aligned (the API promises 16), and 16-byte loads otherwise.
+template <bool IN_BF16, int NE, bool WIDE = true>
 __device__ __forceinline__ void load_elems(const void* __restrict__ x, int64_t e, float* dst) {
   if constexpr (IN_BF16) {
     const uint16_t* p = static_cast<const uint16_t*>(x) + e;
-    if constexpr (NE % 16 == 0) {
+    if constexpr (WIDE && NE % 16 == 0) {
       if ((reinterpret_cast<uintptr_t>(p) & 31) == 0) {
 #pragma unroll
         for (int i = 0; i < NE / 16; ++i) {
@@ -234,7 +234,7 @@ __device__ __forceinline__ void load_elems(const void* __restrict__ x, int64_t e
     }
   } else {
     const float* p = static_cast<const float*>(x) + e;
-    if constexpr (NE % 8 == 0) {
+    if constexpr (WIDE && NE % 8 == 0) {
       if ((reinterpret_cast<uintptr_t>(p) & 31) == 0) {
 #pragma unroll
         for (int i = 0; i < NE / 8; ++i) {
