@@ -323,14 +323,15 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   const bool bf = x_dtype == HADQ_BF16;
   const bool full_seg = sh.logb == sh.logs;
   const bool sgd = sg.side != hadq::SIGNS_NONE;
-  // Segment kernels: a thread owns S = max(b, the quantizer's group span, 16)
+  // Segment kernels: a thread owns S = max(b, the quantizer's span, 16)
   // consecutive elements (at most 128 and at most the largest power of 2
-  // dividing n), so a block of b >= 16 whose groups fit in it is a whole
-  // segment (fixed butterfly, no run-time stage count) and smaller blocks
-  // keep short register arrays.
+  // dividing n), so a block of b >= 16 is a whole segment (fixed butterfly,
+  // no run-time stage count) and smaller blocks keep short register arrays.
+  // The span is 32 for int4 (larger groups span 2 or 4 neighbouring
+  // segments, joined by shuffles) and MXFP4, 16 for NVFP4 and rotations.
   int seg_logs = sh.logs;
   if (mode >= 0 && sh.b <= 128) {
-    const int need = mode == hadq::OUT_INT4 ? group : mode == hadq::OUT_MXFP4 ? 32 : 16;
+    const int need = mode == hadq::OUT_INT4 || mode == hadq::OUT_MXFP4 ? 32 : 16;
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours

@@ -553,6 +553,52 @@ __device__ __forceinline__ void store_int4_pair(const float (&v)[64], float norm
   }
 }
 
+// Symmetric int4 for a thread holding N consecutive outputs (register order
+// natural), group in {32, 64, 128}.  A group larger than N spans group / N
+// (2 or 4) consecutive lanes, group-aligned: its absmax is exchanged with
+// shuffles, so every lane of the warp must call this; ok = false computes and
+// stores nothing.
+template <int N>
+__device__ __forceinline__ void store_int4_lanes(const float (&v)[N], float norm, int group,
+                                                 uint8_t* __restrict__ codes, __half* __restrict__ scales,
+                                                 int64_t e0, bool ok) {
+  static_assert(N % 32 == 0 && N <= 128, "32..128 outputs per thread");
+  if (group <= N) {
+    if (ok) store_int4<false, N>(v, norm, group, codes, scales, e0);
+    return;
+  }
+  float mz = absmax_regs(v, 0, N);
+  mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 1));
+  if (group >= 4 * N) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 2));
+  const float m = mz * norm;
+  const __half s16 = __float2half_rn(m * kInv7);
+  const float s = __half2float(s16);
+  const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
+  const float rn = r * norm;
+  const bool plain = mz * rn < 7.25f;
+  uint4 prev = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int j = 0; j < N / 32; ++j) {
+    uint4 w;
+    if (plain) {
+      w = make_uint4(pack_int4x8<false>(v, 32 * j, rn), pack_int4x8<false>(v, 32 * j + 8, rn),
+                     pack_int4x8<false>(v, 32 * j + 16, rn), pack_int4x8<false>(v, 32 * j + 24, rn));
+    } else {
+      w = make_uint4(pack_int4x8_clamped<false>(v, 32 * j, rn), pack_int4x8_clamped<false>(v, 32 * j + 8, rn),
+                     pack_int4x8_clamped<false>(v, 32 * j + 16, rn), pack_int4x8_clamped<false>(v, 32 * j + 24, rn));
+    }
+    if (ok) {
+      if constexpr (N == 32) {
+        reinterpret_cast<uint4*>(codes + (e0 >> 1))[0] = w;
+      } else if (j & 1) {
+        store32(codes + ((e0 + 32 * (j - 1)) >> 1), prev, w);
+      }
+    }
+    prev = w;
+  }
+  if (ok && (e0 & (group - 1)) == 0) scales[e0 >> (__ffs(group) - 1)] = s16;   // the group's first lane
+}
+
 // MXFP4: per 32 elements an E8M0 exponent e = clamp(floor(log2 m) - 2, -127, 127).
 template <bool PERM, int N>
 __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uint8_t* __restrict__ codes,

@@ -87,6 +87,11 @@ __device__ __forceinline__ void segment_sign_mask(const Signs& sg, int nbits, ui
 }
 
 // FULL: b == S, all LOGS stages unconditionally; otherwise the low nbits stages.
+// An int4 group may span 2 or 4 consecutive segments (S >= 32, group <= 128):
+// their threads are consecutive lanes, so the group absmax is one or two
+// shuffles.  The grid loop is therefore warp-uniform: every lane runs every
+// iteration (past the last segment with zeros, storing nothing), so that all
+// lanes take part in the shuffles.
 template <int LOGS, bool IN_BF16, int MODE, bool FULL, bool SG>
 __global__ void __launch_bounds__(kThreads)
 segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, int group,
@@ -98,9 +103,14 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
   if constexpr (SG) segment_sign_mask<S>(sg, nbits, sm);
   float v[S];
   const int lane = threadIdx.x & 31;
-  for (int64_t s = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; s < segs;
-       s += static_cast<int64_t>(gridDim.x) * kThreads) {
-    if (lane == 0) {   // the warp's next 32 segments are contiguous
+  for (int64_t s0 = static_cast<int64_t>(blockIdx.x) * kThreads; s0 < segs;
+       s0 += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t s = s0 + threadIdx.x;
+    const bool valid = s < segs;
+    if constexpr (MODE != OUT_INT4) {
+      if (!valid) break;   // no cross-lane work: the lanes past the end may leave
+    }
+    if (lane == 0 && valid) {   // the warp's next 32 segments are contiguous
       const int64_t nxt = s + static_cast<int64_t>(gridDim.x) * kThreads;
       if (nxt < segs) {
         const int64_t cnt = segs - nxt < 32 ? segs - nxt : 32;
@@ -108,7 +118,12 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
       }
     }
     const int64_t e0 = s << LOGS;
-    load_elems<IN_BF16, S, kWideRun<IN_BF16, S>>(x, e0, v);
+    if (valid) {
+      load_elems<IN_BF16, S, kWideRun<IN_BF16, S>>(x, e0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < S; ++i) v[i] = 0.f;
+    }
     if constexpr (SG) {
       if (sg.side == SIGNS_BEFORE) apply_signs<S>(v, sm);
     }
@@ -125,7 +140,7 @@ segment_kernel(const void* __restrict__ x, int64_t segs, int nbits, float norm, 
     } else if constexpr (MODE == OUT_BF16) {
       store_rotated<false, S, true>(v, norm, out0, e0);
     } else if constexpr (MODE == OUT_INT4) {
-      store_int4<false, S>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+      store_int4_lanes<S>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0, valid);
     } else if constexpr (MODE == OUT_NVFP4) {
       store_nvfp4<false, S>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
     } else {
