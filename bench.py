@@ -32,6 +32,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -112,12 +113,19 @@ def measured_peak():
 C2_KERNEL_SOURCES = ("hadq_api.cu", "hadq_device.cuh", "hadq_launch.h", "hadq_tc.cuh", "kernels_tc.cu")
 
 
+def _strip_comments(src):
+    """C++ source without // and /* */ comments (they do not change the binary)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.sub(r"//[^\n]*", "", src)
+
+
 def kernel_source_hash():
+    """Hash of the C2 kernel's sources with their comments removed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_rotation_bit_b200", "csrc")
     for f in C2_KERNEL_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,7 +17,7 @@
 // Roles (one CTA per SM, persistent over tiles; tile = TILE_N columns =
 // TILE_N / 2^LO rows, contiguous in global memory):
 //   warp 0      TMA producer: X tiles (box 2^LO x 128 x R, 64B/128B swizzle,
-//               no multicast) into a ring of STAGES shared-memory stages;
+//               each CTA loading its own) into a ring of STAGES stages;
 //   warp 1      TMEM allocator and MMA issuer (one thread); accumulators in
 //               512 / TILE_N tensor-memory buffers;
 //   warps 2..   4 * SPLIT epilogue warps; warp w reads TMEM lanes

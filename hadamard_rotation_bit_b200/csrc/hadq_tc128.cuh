@@ -14,8 +14,8 @@
 // (n / 128 <= 128 blocks) and reduces the row absmax across the 4 warps of
 // the epilogue group that owns the tile.
 //
-// A = X_blk is K-major with the 128-byte swizzle, loaded by TMA (no
-// multicast) as two 64-element K-panels per tile from two 2-D tensor maps
+// A = X_blk is K-major with the 128-byte swizzle, loaded by TMA (each CTA
+// its own tiles) as two 64-element K-panels per tile from two 2-D tensor maps
 // whose bases differ by 128 bytes; B = H_128 (symmetric) is built in shared
 // memory in the same layout.  Random Hadamard signs cost nothing per tile:
 // they are folded into B when it is built, as diag(s) H_128 for signs before
