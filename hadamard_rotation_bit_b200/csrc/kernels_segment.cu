@@ -25,14 +25,21 @@ SegFn seg_fn(int mode) {
   }
 }
 
+// The launcher makes a segment max(b, 16) or max(b, 32) elements (at most the
+// largest power of 2 dividing n), so a segment longer than its block (!FULL)
+// is at most 32 elements; 64- and 128-element segments are whole blocks.
 template <bool BF, bool FULL, bool SG>
 SegFn seg_fn_logs(int logs, int mode) {
   switch (logs) {
     case 3: return seg_fn<3, BF, FULL, SG>(mode);
     case 4: return seg_fn<4, BF, FULL, SG>(mode);
     case 5: return seg_fn<5, BF, FULL, SG>(mode);
-    case 6: return seg_fn<6, BF, FULL, SG>(mode);
-    case 7: return seg_fn<7, BF, FULL, SG>(mode);
+    case 6:
+      if constexpr (FULL) return seg_fn<6, BF, FULL, SG>(mode);
+      return nullptr;
+    case 7:
+      if constexpr (FULL) return seg_fn<7, BF, FULL, SG>(mode);
+      return nullptr;
     default: return nullptr;
   }
 }
