@@ -104,6 +104,42 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _on_device(name: str, t: torch.Tensor, dev: torch.device) -> None:
+    """The C ABI takes device pointers: a host tensor here would be read or
+    written by the kernel through a host address."""
+    if not t.is_cuda:
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"{name} must be a CUDA tensor (got {t.device})")
+    if t.device != dev:
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"{name} is on {t.device}, x on {dev}")
+
+
+def _on_host(name: str, t: torch.Tensor) -> None:
+    if t.is_cuda:
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"{name} must be a host tensor (got {t.device})")
+
+
+def _holds(name: str, t: torch.Tensor, nbytes: int) -> None:
+    """A caller-supplied buffer must be contiguous and at least nbytes long:
+    the C ABI receives only its address."""
+    if not t.is_contiguous():
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if t.numel() * t.element_size() < nbytes:
+        raise HadqError(HADQ_ERR_INVALID_ARG,
+                        f"{name} holds {t.numel() * t.element_size()} bytes, the call writes {nbytes}")
+
+
+def _quant_outputs(lib, rows: int, n: int, fmt: str, group: int, codes, scales, dev) -> None:
+    if fmt not in FMTS:
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"unknown fmt {fmt!r}")
+    for name, t, nbytes in (("codes", codes, int(lib.hadq_codes_bytes(rows, n, FMTS[fmt]))),
+                            ("scales", scales, int(lib.hadq_scales_bytes(rows, n, FMTS[fmt], group)))):
+        if dev is None:
+            _on_host(name, t)
+        else:
+            _on_device(name, t, dev)
+        _holds(name, t, nbytes)
+
+
 def _rows_n(x: torch.Tensor):
     if not x.is_contiguous():
         raise HadqError(HADQ_ERR_INVALID_ARG, "tensors must be contiguous")
@@ -142,8 +178,11 @@ def hadq_rotate(x: torch.Tensor, block: int = 0, out: torch.Tensor | None = None
     """out = x . diag(H_b) / sqrt(b) along the last dimension (see include/hadq.h)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
     if out is None:
         out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _on_device("out", out, x.device)
+    _holds("out", out, rows * n * out.element_size())
     _check(lib.hadq_rotate(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, out.data_ptr(),
                            _dtype_code(out.dtype), _stream_handle(stream)))
     return out
@@ -154,8 +193,11 @@ def hadq_rotate_inverse(x: torch.Tensor, block: int = 0, out: torch.Tensor | Non
     """Inverse rotation (the same symmetric, involutory operation)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
     if out is None:
         out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _on_device("out", out, x.device)
+    _holds("out", out, rows * n * out.element_size())
     _check(lib.hadq_rotate_inverse(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, out.data_ptr(),
                                    _dtype_code(out.dtype), _stream_handle(stream)))
     return out
@@ -166,11 +208,13 @@ def hadq_rotate_quant(x: torch.Tensor, block: int = 0, fmt: str = "int4", group:
     """Rotate and quantize in one pass; returns (codes, scales) (see include/hadq.h)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
     cs, cd, ss, sd = output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
     if codes is None:
         codes = torch.empty(cs, dtype=cd, device=x.device)
     if scales is None:
         scales = torch.empty(ss, dtype=sd, device=x.device)
+    _quant_outputs(lib, rows, n, fmt, group, codes, scales, x.device)
     _check(lib.hadq_rotate_quant(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, FMTS[fmt], group,
                                  codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
     return codes, scales
@@ -183,6 +227,11 @@ def hadq_rotate_quant_host(x_host: torch.Tensor, block: int, fmt: str, group: in
     """Host-buffer form: copy in, rotate+quantize, copy out, all enqueued on `stream`."""
     lib = load_library()
     rows, n = _rows_n(x_host)
+    _on_host("x_host", x_host)
+    _quant_outputs(lib, rows, n, fmt, group, codes_host, scales_host, None)
+    _on_device("x_dev", x_dev, x_dev.device)
+    _holds("x_dev", x_dev, rows * n * x_host.element_size())
+    _quant_outputs(lib, rows, n, fmt, group, codes_dev, scales_dev, x_dev.device)
     _check(lib.hadq_rotate_quant_host(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt], group,
                                       codes_host.data_ptr(), scales_host.data_ptr(), x_dev.data_ptr(),
                                       codes_dev.data_ptr(), scales_dev.data_ptr(), _stream_handle(stream)))
@@ -194,17 +243,26 @@ def hadq_rotate_quant_host_static(x_host: torch.Tensor, block: int, fmt: str, gr
     array (32 MiB per GPU), so this call allocates no device memory."""
     lib = load_library()
     rows, n = _rows_n(x_host)
+    _on_host("x_host", x_host)
+    _quant_outputs(lib, rows, n, fmt, group, codes_host, scales_host, None)
     _check(lib.hadq_rotate_quant_host_static(x_host.data_ptr(), _dtype_code(x_host.dtype), rows, n, block, FMTS[fmt],
                                              group, codes_host.data_ptr(), scales_host.data_ptr(),
                                              _stream_handle(stream)))
 
 
-def _signs_ptr(signs: torch.Tensor | None) -> int | None:
+def _signs_ptr(signs: torch.Tensor | None, dev: torch.device, b: int) -> int | None:
     if signs is None:
         return None
     if signs.dtype != torch.int8 or not signs.is_contiguous():
         raise HadqError(HADQ_ERR_INVALID_ARG, "signs must be a contiguous int8 tensor")
+    _on_device("signs", signs, dev)
+    _holds("signs", signs, b)
     return signs.data_ptr()
+
+
+def _block_len(n: int, block: int) -> int:
+    """b of the call (block 0 or -1: the whole row)."""
+    return n if block in (0, -1) or block >= n else block
 
 
 def hadq_rotate_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "after", block: int = 0,
@@ -215,9 +273,13 @@ def hadq_rotate_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "after"
     the b int8 signs on the device (see include/hadq.h)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
+    sp = _signs_ptr(signs, x.device, _block_len(n, block))
     if out is None:
         out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
-    _check(lib.hadq_rotate_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, _signs_ptr(signs),
+    _on_device("out", out, x.device)
+    _holds("out", out, rows * n * out.element_size())
+    _check(lib.hadq_rotate_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, sp,
                                   SIDES[side], out.data_ptr(), _dtype_code(out.dtype), _stream_handle(stream)))
     return out
 
@@ -228,12 +290,15 @@ def hadq_rotate_quant_signed(x: torch.Tensor, signs: torch.Tensor, side: str = "
     """Random Hadamard rotation and quantization in one pass; returns (codes, scales)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
+    sp = _signs_ptr(signs, x.device, _block_len(n, block))
     cs, cd, ss, sd = output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
     if codes is None:
         codes = torch.empty(cs, dtype=cd, device=x.device)
     if scales is None:
         scales = torch.empty(ss, dtype=sd, device=x.device)
-    _check(lib.hadq_rotate_quant_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, _signs_ptr(signs),
+    _quant_outputs(lib, rows, n, fmt, group, codes, scales, x.device)
+    _check(lib.hadq_rotate_quant_signed(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, sp,
                                         SIDES[side], FMTS[fmt], group, codes.data_ptr(), scales.data_ptr(),
                                         _stream_handle(stream)))
     return codes, scales
@@ -244,11 +309,13 @@ def hadq_rotate_quant_nvfp4(x: torch.Tensor, tensor_scale: float = 1.0, block: i
     """Rotate and quantize to NVFP4 with a per-tensor scale; returns (codes, E4M3 scales)."""
     lib = load_library()
     rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
     cs, cd, ss, sd = output_shapes(rows, n, "nvfp4", 16)
     if codes is None:
         codes = torch.empty(cs, dtype=cd, device=x.device)
     if scales is None:
         scales = torch.empty(ss, dtype=sd, device=x.device)
+    _quant_outputs(lib, rows, n, "nvfp4", 16, codes, scales, x.device)
     _check(lib.hadq_rotate_quant_nvfp4(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, float(tensor_scale),
                                        codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
     return codes, scales

@@ -186,3 +186,38 @@ def test_nvfp4_validation(lib):
     assert lib.hadq_scales_bytes(4, 1024, 3, 0) == 4 * 64
     assert lib.hadq_scales_bytes(4, 1024, 3, 32) == 0
     assert lib.hadq_codes_bytes(4, 1024, 3) == 2048
+
+
+# ------------------------------------------------- binding-level buffer checks
+
+def test_binding_rejects_host_tensors_for_device_arguments(lib):
+    """The C ABI takes device pointers; the binding refuses host tensors
+    before any call (a host address would reach the kernel otherwise)."""
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    for call in (lambda: H.hadq_rotate(x, 0), lambda: H.hadq_rotate_quant(x, 0, "int4", 128),
+                 lambda: H.hadq_rotate_quant_nvfp4(x, 1.0, 0),
+                 lambda: H.hadq_rotate_signed(x, torch.ones(128, dtype=torch.int8), "after", 0),
+                 lambda: H.hadq_rotate_quant_signed(x, torch.ones(128, dtype=torch.int8), "before", 0, "mxfp4", 32)):
+        with pytest.raises(H.HadqError) as e:
+            call()
+        assert e.value.status == H.HADQ_ERR_INVALID_ARG and "CUDA tensor" in str(e.value)
+
+
+def test_binding_checks_host_output_sizes(lib):
+    """Caller-supplied outputs must hold what the call writes; the sizes the
+    binding allocates itself (output_shapes) are exactly the library's."""
+    import torch
+    for rows, n, fmt, group in [(5, 4096, "int4", 128), (5, 4096, "int4", 32), (3, 14336, "int8", 0),
+                                (7, 8192, "mxfp4", 32), (9, 48, "nvfp4", 16)]:
+        cs, cd, ss, sd = H.output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
+        codes, scales = torch.empty(cs, dtype=cd), torch.empty(ss, dtype=sd)
+        assert codes.numel() * codes.element_size() == lib.hadq_codes_bytes(rows, n, H.FMTS[fmt])
+        assert scales.numel() * scales.element_size() == lib.hadq_scales_bytes(rows, n, H.FMTS[fmt], group)
+        H._quant_outputs(lib, rows, n, fmt, group, codes, scales, None)          # host side: accepted
+        with pytest.raises(H.HadqError) as e:
+            H._quant_outputs(lib, rows, n, fmt, group, codes[:-1], scales, None)
+        assert "holds" in str(e.value)
+    with pytest.raises(H.HadqError):
+        H._holds("out", torch.empty(8, 4)[:, :2], 16)                             # not contiguous
+    assert H._block_len(4096, 0) == 4096 and H._block_len(4096, -1) == 4096 and H._block_len(4096, 128) == 128
