@@ -4,6 +4,12 @@ Every function follows a passage of the pages (cited in its docstring) or,
 where the pages are silent, a reading stated in the docstring.  The code is
 deliberately plain: explicit matrices, dense products, whole-array numpy
 expressions, no blocking or fusion beyond what the definitions state.
+
+Every function is pinned, in tests/test_oracle_pins.py, to something other
+than itself (hand-worked cases, closed forms, invariants, library routines).
+End-to-end rotated-and-quantized values of a whole workload are parity
+unpinned by the pages: none prints a worked example, so they are pinned only
+through the pinned parts.
 """
 
 from __future__ import annotations
