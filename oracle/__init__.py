@@ -15,6 +15,11 @@ What it computes, and where the pages define it:
   ``block_size`` blocks (same page, sections 1.2 and 2.1).  The orthogonality
   the page states in its introduction (R @ R^T = I) is what lets the rotated
   activations meet pre-rotated weights.
+* ``paley_hadamard`` / ``hadamard_matrix`` -- the non-power-of-2 sizes of
+  the same section 1.5: n = K * 2^m combines a base Hadamard matrix of order
+  K with a Sylvester block.  The pages print no base matrix; the reading is
+  Paley's second construction (a published method, cited on the function)
+  and the Kronecker product H_K (x) H_(2^m).
 * ``random_hadamard_matrix`` / ``rotate_signed`` -- the random Hadamard
   matrix H @ diag(+/-1) / sqrt(N) of the same section 1.5 (signs persisted as
   int8, section 1.7), and its transpose diag(+/-1) @ H / sqrt(N), which is its
@@ -55,6 +60,12 @@ from .hadq_oracle import (  # noqa: F401
     e4m3_encode,
     e8m0_exponent,
     fp16_scale_midpoint_distance,
+    hadamard_matrix,
+    jacobsthal,
+    paley_hadamard,
+    PALEY_FIELDS,
+    quadratic_character,
+    split_size,
     pack_nibbles,
     quantize,
     quantize_int4_sym,

@@ -59,22 +59,136 @@ def sylvester_hadamard(size: int) -> np.ndarray:
     return _sylvester(size)
 
 
+# ---------------------------------------------------------------------------
+# Non-power-of-2 sizes: n = K * 2^m
+# ---------------------------------------------------------------------------
+# "Rotation Transform", section 1.5: for non-power-of-2 dimensions
+# get_hadamard_K(n) factors n = K * 2^m and combines a known base Hadamard
+# matrix of order K with a Sylvester block.  The pages name the orders (12,
+# 20, 28, 36, 40, 52, 60, 108, 140, 156, 172) but print no base matrix.
+# Reading: the base matrix of order K = 2 (q + 1) is Paley's second
+# construction over the field of q elements (q = 1 mod 4 a prime power;
+# R. E. A. C. Paley, "On orthogonal matrices", J. Math. Phys. 12, 1933), and
+# the combination is the Kronecker product H_n = H_K (x) H_(2^m), the base
+# factor outermost as the Sylvester doubling H_2k = H_2 (x) H_k puts its own.
+# These K are covered: 12, 20, 28, 36, 52, 60, 108 (40 = 2 * 20 is the K = 20
+# matrix with one more Sylvester factor).  The matrices are symmetric, so
+# H_n / sqrt(n) stays its own inverse.
+
+# K -> (p, k): the field GF(p^k), q = p^k = K / 2 - 1.
+PALEY_FIELDS = {12: (5, 1), 20: (3, 2), 28: (13, 1), 36: (17, 1), 52: (5, 2), 60: (29, 1), 108: (53, 1)}
+# GF(p^2) = GF(p)[i] / (i^2 - nu), nu a quadratic non-residue mod p.
+GF2_NONRESIDUE = {3: 2, 5: 2}
+
+
+def _gf_elements(p: int, k: int):
+    """Field elements as coefficient pairs (a, b) meaning a + b*i; element
+    index t = a + p * b (k = 1: b = 0, index = the residue)."""
+    return [(t % p, t // p) for t in range(p ** k)]
+
+
+def _gf_index(e, p: int) -> int:
+    return e[0] + p * e[1]
+
+
+def _gf_sub(e1, e2, p: int):
+    return ((e1[0] - e2[0]) % p, (e1[1] - e2[1]) % p)
+
+
+def _gf_mul(e1, e2, p: int, nu: int):
+    a, b = e1
+    c, d = e2
+    return ((a * c + nu * b * d) % p, (a * d + b * c) % p)
+
+
+def quadratic_character(p: int, k: int) -> np.ndarray:
+    """chi over GF(p^k) by element index: 0 at 0, +1 on the nonzero squares,
+    -1 on the non-squares (the squares found by squaring every element)."""
+    nu = GF2_NONRESIDUE.get(p, 0) if k == 2 else 0
+    els = _gf_elements(p, k)
+    chi = -np.ones(len(els), dtype=np.int64)
+    chi[0] = 0
+    for e in els[1:]:
+        chi[_gf_index(_gf_mul(e, e, p, nu), p)] = 1
+    return chi
+
+
+def jacobsthal(p: int, k: int) -> np.ndarray:
+    """Q[a, b] = chi(a - b) over the field elements in index order."""
+    els = _gf_elements(p, k)
+    chi = quadratic_character(p, k)
+    return np.array([[chi[_gf_index(_gf_sub(a, b, p), p)] for b in els] for a in els], dtype=np.int64)
+
+
+def paley_hadamard(order: int) -> np.ndarray:
+    """Paley II Hadamard matrix of order K = 2 (q + 1) (entries +/-1).
+
+    C = [[0, 1^T], [1, Q]] is the symmetric conference matrix of order q + 1
+    (index 0 the point at infinity, then the field elements in index order);
+    H = C (x) [[1, 1], [1, -1]] + I (x) [[1, -1], [-1, -1]].
+    """
+    if order not in PALEY_FIELDS:
+        raise ValueError(f"no base Hadamard matrix of order {order}; covered: {sorted(PALEY_FIELDS)}")
+    p, k = PALEY_FIELDS[order]
+    q = p ** k
+    c = np.zeros((q + 1, q + 1), dtype=np.int64)
+    c[0, 1:] = 1
+    c[1:, 0] = 1
+    c[1:, 1:] = jacobsthal(p, k)
+    a = np.array([[1, 1], [1, -1]])
+    b = np.array([[1, -1], [-1, -1]])
+    return (np.kron(c, a) + np.kron(np.eye(q + 1, dtype=np.int64), b)).astype(np.float64)
+
+
+def split_size(size: int):
+    """(K, 2^m) with size = K * 2^m: K = 1 for a power of 2, else the covered
+    base order K = 4 * (odd part of size) (a Hadamard order above 2 is a
+    multiple of 4).  Raises for a size with no covered base matrix."""
+    size = int(size)
+    if _is_pow2(size):
+        return 1, size
+    odd = size
+    while odd % 2 == 0:
+        odd //= 2
+    k = 4 * odd
+    if k not in PALEY_FIELDS or size % k != 0:
+        raise ValueError(f"size {size} = K * 2^m needs a base Hadamard matrix of order {k}, "
+                         f"not covered ({sorted(PALEY_FIELDS)})")
+    return k, size // k
+
+
+@functools.lru_cache(maxsize=2)
+def _kron_hadamard(size: int) -> np.ndarray:
+    k, s = split_size(size)
+    h = np.kron(paley_hadamard(k), sylvester_hadamard(s))
+    h.setflags(write=False)
+    return h
+
+
+def hadamard_matrix(size: int) -> np.ndarray:
+    """Unnormalised Hadamard matrix of order ``size`` used by the rotation:
+    Sylvester for a power of 2, H_K (x) H_(2^m) otherwise (read-only, cached)."""
+    k, _ = split_size(size)
+    return sylvester_hadamard(size) if k == 1 else _kron_hadamard(int(size))
+
+
 def resolve_block(n: int, block) -> int:
     """Block size actually applied to a row of length ``n``.
 
     ``None``, ``-1``, ``0`` and ``n`` all mean the full dimension ("Rotation
     Transform", section 2.1: block_size None/-1 means full-dimension
-    Hadamard).  Otherwise the block must be a positive power of 2 dividing
-    ``n`` (section 1.2: rotation_size must be a positive power of 2).  A full
-    rotation needs ``n`` itself to be a power of 2 (section 1.5).
+    Hadamard).  Otherwise the block must divide ``n`` and be a size with a
+    Hadamard matrix: a power of 2 (sections 1.2 and 1.5) or K * 2^m with a
+    covered base order K (section 1.5, non-power-of-2 dimensions).
     """
     n = int(n)
     if block is None or int(block) in (-1, 0, n):
         b = n
     else:
         b = int(block)
-    if not _is_pow2(b) or n % b != 0:
-        raise ValueError(f"block {block!r} is not a power of 2 dividing n={n}")
+    if b < 1 or n % b != 0:
+        raise ValueError(f"block {block!r} does not divide n={n}")
+    split_size(b)
     return b
 
 
@@ -85,7 +199,8 @@ def rotate(x, block=0) -> np.ndarray:
     residual stream, R3 per head on Q/K, R4 on the down_proj input) and the
     per-Linear block-diagonal mode of section 2: each row is cut into
     consecutive blocks of ``b`` elements and each block is multiplied by the
-    normalised Sylvester matrix (section 1.5).  The product is a dense
+    normalised Hadamard matrix of section 1.5 (Sylvester for a power of 2,
+    H_K (x) H_(2^m) for b = K * 2^m, see ``hadamard_matrix``).  The product is a dense
     O(b^2)-per-block float64 matmul of the exact upcast input.  H is
     symmetric, so x . H and H . x agree, and H/sqrt(b) is its own inverse.
     """
@@ -94,7 +209,7 @@ def rotate(x, block=0) -> np.ndarray:
         raise ValueError("rotate expects a 2-D (rows, n) array")
     rows, n = x.shape
     b = resolve_block(n, block)
-    h = sylvester_hadamard(b)
+    h = hadamard_matrix(b)
     y = (x.reshape(rows * (n // b), b) @ h) / np.sqrt(float(b))
     return y.reshape(rows, n)
 
@@ -120,7 +235,7 @@ def random_hadamard_matrix(signs, side: str = "after") -> np.ndarray:
     of orbitquant's RPBH rotation ("orbitquant 0.2.0", how it works).
     """
     s = sign_vector(signs)
-    h = sylvester_hadamard(s.size)
+    h = hadamard_matrix(s.size)
     # A product with a diagonal matrix scales columns (on the right) or rows
     # (on the left); written out that way it costs O(b^2) instead of O(b^3).
     if side == "after":

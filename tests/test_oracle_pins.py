@@ -168,8 +168,88 @@ def test_block_argument_forms():
     for bad in (3, 12, 32):
         with pytest.raises(ValueError):
             oracle.rotate(x, bad)
-    with pytest.raises(ValueError):
-        oracle.rotate(np.zeros((1, 12)), 0)   # full size must be a power of 2
+    for n in (10, 44, 6):                     # full sizes with no Hadamard matrix here
+        with pytest.raises(ValueError):
+            oracle.rotate(np.zeros((1, n)), 0)
+    assert oracle.rotate(np.zeros((1, 12)), 0).shape == (1, 12)   # K = 12 is covered
+
+
+# -------------------------------------------- non-power-of-2 sizes K * 2^m
+
+def test_paley_k12_matches_hand_worked_fixture(golden):
+    g = golden("paley_k12.json")
+    chi = oracle.quadratic_character(5, 1)
+    assert sorted(np.nonzero(chi == 1)[0].tolist()) == g["squares_mod_5"]
+    np.testing.assert_array_equal(oracle.jacobsthal(5, 1), np.array(g["Q5"]))
+    h = oracle.paley_hadamard(12)
+    np.testing.assert_array_equal(h[:4], np.array(g["H12_rows_0_to_3"], dtype=np.float64))
+    # every entry from the conference matrix written out by hand
+    c, a, b = np.array(g["C6"]), np.array([[1, 1], [1, -1]]), np.array([[1, -1], [-1, -1]])
+    for i in range(6):
+        for j in range(6):
+            for u in range(2):
+                for v in range(2):
+                    want = c[i, j] * a[u, v] + (b[u, v] if i == j else 0)
+                    assert h[2 * i + u, 2 * j + v] == want
+
+
+def test_field_squares_match_hand_worked_sets(golden):
+    g = golden("paley_k12.json")
+    assert sorted(np.nonzero(oracle.quadratic_character(3, 2) == 1)[0].tolist()) == g["squares_GF9"]
+    assert sorted(np.nonzero(oracle.quadratic_character(13, 1) == 1)[0].tolist()) == g["squares_mod_13"]
+    for k, (p, e) in oracle.PALEY_FIELDS.items():
+        chi = oracle.quadratic_character(p, e)
+        q = p ** e
+        assert chi[0] == 0 and (chi == 1).sum() == (q - 1) // 2 and (chi == -1).sum() == (q - 1) // 2
+        # the squares of a prime field are exactly {t^2 mod p}
+        if e == 1:
+            assert set(np.nonzero(chi == 1)[0].tolist()) == {t * t % p for t in range(1, p)}
+
+
+@pytest.mark.parametrize("k", sorted(oracle.PALEY_FIELDS))
+def test_paley_base_matrices_are_symmetric_hadamard(k):
+    h = oracle.paley_hadamard(k)
+    assert h.shape == (k, k) and set(np.unique(h).tolist()) == {-1.0, 1.0}
+    np.testing.assert_array_equal(h @ h.T, k * np.eye(k))
+    np.testing.assert_array_equal(h, h.T)
+    # the Jacobsthal matrix of q = 1 (mod 4) is symmetric with zero diagonal and Q Q^T = q I - J
+    p, e = oracle.PALEY_FIELDS[k]
+    q = p ** e
+    jq = oracle.jacobsthal(p, e)
+    np.testing.assert_array_equal(jq, jq.T)
+    np.testing.assert_array_equal(jq @ jq.T, q * np.eye(q) - np.ones((q, q)))
+
+
+@pytest.mark.parametrize("n", [12, 24, 48 * 8, 20 * 16, 28 * 32, 36 * 8, 52 * 4, 60 * 4, 108 * 2, 28 * 64])
+def test_k_size_rotation_is_orthogonal_and_involutory(n):
+    k, s = oracle.split_size(n)
+    assert k * s == n and k in oracle.PALEY_FIELDS
+    h = oracle.hadamard_matrix(n)
+    np.testing.assert_array_equal(h @ h.T, n * np.eye(n))
+    x = np.random.default_rng(n).standard_normal((5, n))
+    y = oracle.rotate(x, 0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(oracle.rotate(y, 0), x, rtol=0, atol=1e-12 * np.abs(x).max())
+
+
+@pytest.mark.parametrize("n", [12 * 16, 28 * 64, 20 * 8])
+def test_k_size_rotation_equals_two_stage_product(n):
+    """Kronecker index convention: element e = k * 2^m + j; the dense product
+    equals mixing the K sub-blocks by H_K after (or before) a 2^m-point
+    butterfly inside each sub-block, computed here with an independent FWHT."""
+    k, s = oracle.split_size(n)
+    x = np.random.default_rng(n + 1).standard_normal((3, n))
+    z = _fwht_butterflies(x.reshape(3 * k, s)).reshape(3, k, s)
+    want = np.einsum("rkj,kl->rlj", z, oracle.paley_hadamard(k)).reshape(3, n) / np.sqrt(n)
+    np.testing.assert_allclose(oracle.rotate(x, 0), want, rtol=0, atol=1e-12 * np.sqrt(n) * np.abs(x).max())
+
+
+def test_k_size_blocks_are_per_block_full_transforms():
+    x = np.random.default_rng(5).standard_normal((4, 28 * 32 * 3))
+    y = oracle.rotate(x, 28 * 32)
+    for j in range(3):
+        sl = slice(j * 896, (j + 1) * 896)
+        np.testing.assert_allclose(y[:, sl], oracle.rotate(x[:, sl], 0), rtol=0, atol=1e-12)
 
 
 # ----------------------------------------------------------- float formats
