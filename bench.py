@@ -11,16 +11,24 @@ written once) and its fraction of the measured HBM copy bandwidth.
 Timing: inputs resident in HBM; for C2, 8 buffer sets (input + outputs) are
 rotated so each step touches data last used 7 steps earlier (338 MB > L2).  The K steps
 are captured back to back in one CUDA graph; the graph is replayed once
-untimed and once timed (CUDA events on the launching stream) between barriers
-and device synchronisations.  `value` = bytes of all ranks / max-over-ranks
-elapsed time; `roofline.achieved` = bytes per launch / mean launch interval
-(kernel plus inter-kernel gap).  A median over per-launch event pairs (queued
-behind a sleep kernel) is reported beside it.
+untimed and once timed between barriers and device synchronisations.  The
+timed replay and the CUDA events around it are queued on the launching
+stream behind a sleep kernel, so the host's submission of the graph falls
+before the start event and the window holds exactly the K steps, run back
+to back.  `value` = bytes of all ranks / max-over-ranks elapsed time;
+`roofline.achieved` = bytes per launch / mean launch interval (kernel plus
+inter-kernel gap).  Beside it the line reports the same replay with the
+events recorded while the host submits the graph (the window then also holds
+the submission latency) and a median over per-launch event pairs.
 `e2e` repeats the metric through hadq_rotate_quant_host (pinned host input,
 copies in and out inside the timed region).
 
-Under torchrun every rank processes its own batch (weak scaling, no
-collective on the data path); rank 0 prints one JSON line.
+Ranks: under torchrun (WORLD_SIZE set) every rank processes its own batch
+(weak scaling, no collective on the data path); rank 0 prints one JSON line.
+Without WORLD_SIZE, `--gpus N` with N > 1 starts the N ranks itself (one
+process per local GPU, 127.0.0.1 rendezvous) and returns the worst exit code.
+`--dry-run` runs the rank plumbing alone on CPU (gloo, each rank timing the
+oracle on a few rows of its own batch) for tests of the launcher.
 `--impl reference` times the float64 CPU oracle on the host cores instead.
 `--rows R` keeps only the first R rows of every workload part (a smaller case
 of the same kernel, for profiler captures); the default is the full workload.
@@ -50,11 +58,13 @@ METRIC = "fused Hadamard+quant GB/s and % of B200 HBM peak (4096x4096 bf16->int4
 UNIT = "GB/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+SLEEP_CYCLES = 20_000_000      # ~10 ms of GPU sleep ahead of a timed region
 
 # A step is one pass of the fused path over one batch of a workload: the
 # launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
 STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"],
-              "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"], "c3rb": ["c3rb"], "c5rb": ["c5rb"]}
+              "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"], "c3rb": ["c3rb"], "c5rb": ["c5rb"],
+              "c3k": ["c3k"]}
 WORKLOAD = W.WORKLOADS["c2"]
 
 
@@ -194,17 +204,53 @@ class ClockSampler:
                 "samples": len(self.samples), "reasons": sorted(self.reasons - {"gpu_idle"})}
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
     world = _env_int("WORLD_SIZE", 1)
     if world > 1:
         import datetime
         import torch.distributed as dist
         rank, local = _env_int("RANK", 0), _env_int("LOCAL_RANK", 0)
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return dist, rank, world, local
     return None, 0, 1, 0
+
+
+def check_world(gpus):
+    """--gpus must agree with the world size a launcher gave us."""
+    world = _env_int("WORLD_SIZE", 1)
+    if "WORLD_SIZE" in os.environ and world != gpus:
+        raise SystemExit(f"bench.py: --gpus {gpus} but WORLD_SIZE={world}")
+    return world
+
+
+def _free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(n, argv):
+    """Start this script once per rank (RANK = LOCAL_RANK = i, WORLD_SIZE = n,
+    rendezvous on 127.0.0.1) and wait for all of them; the worst exit code is
+    returned.  Each rank takes the GPU of its local rank."""
+    import subprocess
+    port = str(_free_port())
+    procs = []
+    for i in range(n):
+        env = dict(os.environ, RANK=str(i), LOCAL_RANK=str(i), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=port)
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__)] + argv, env=env))
+    rc = 0
+    for p in procs:
+        r = p.wait()
+        rc = r if rc == 0 else rc
+    return rc
 
 
 def barrier(dist):
@@ -248,11 +294,9 @@ def cpu_baseline(seconds=12.0):
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step a row slice of the workload."""
-    dist, rank, world, _ = dist_setup()
-    if rank != 0:
-        if dist is not None:
-            dist.destroy_process_group()
+    """The oracle as the reference arm: each step a row slice of the workload.
+    Rank 0 alone runs it; the other ranks of a multi-rank launch exit at once."""
+    if _env_int("RANK", 0) != 0:
         return
     import oracle
     w = WORKLOAD
@@ -274,6 +318,33 @@ def run_reference(args):
                              "sample": f"{rows} rows of the 4096x4096 batch per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_dry(args):
+    """Rank plumbing without a GPU: gloo process group, every rank times the
+    oracle on a few rows of its own batch (per-rank seed), max over ranks,
+    whole-job aggregate; rank 0 prints the line (impl "dry-run")."""
+    import oracle
+    dist, rank, world, _ = dist_setup("gloo")
+    rows = 4
+    x = W.bits_to_float64(W.generate("c2", slice(0, rows), seed=W.rank_seed(rank)), "bf16")
+    if dist is not None:
+        dist.barrier()
+    t0 = time.perf_counter()
+    _, codes, _ = oracle.rotate_quant(x, 0, "int4", 128)
+    elapsed = max_over_ranks(dist, time.perf_counter() - t0)
+    digest = int(codes.astype(np.int64).sum())
+    digests = [digest]
+    if dist is not None:
+        t = torch.tensor([digest], dtype=torch.int64)
+        gathered = [torch.zeros_like(t) for _ in range(world)]
+        dist.all_gather(gathered, t)
+        digests = [int(g.item()) for g in gathered]
+    if rank == 0:
+        b = WORKLOAD.algorithmic_bytes * rows // WORKLOAD.rows
+        print(json.dumps({"metric": METRIC, "value": aggregate_gbs(b, 1, world, elapsed), "unit": UNIT,
+                          "n_gpus": world, "impl": "dry-run", "rank_digests": digests,
+                          "elapsed_max_s": elapsed}), flush=True)
     if dist is not None:
         dist.destroy_process_group()
 
@@ -342,11 +413,16 @@ def run_hadq(args):
         g.replay()                       # untimed replay (warm-up of the graph itself)
     stream.synchronize()
 
+    # Timed region: the K steps of one graph replay, between CUDA events on
+    # `stream`.  Events and replay are queued behind a sleep kernel, so the
+    # host's submission of the graph is done before the start event fires and
+    # the window holds the K steps alone, back to back.
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(dist)
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
+            torch.cuda._sleep(SLEEP_CYCLES)
             t_start.record(stream)
             g.replay()
             t_end.record(stream)
@@ -356,12 +432,25 @@ def run_hadq(args):
     elapsed_max = max_over_ranks(dist, elapsed)
     interval_max = elapsed_max / steps
 
+    # The same replay with the events recorded while the host submits the
+    # graph: the window also holds the submission latency (reported beside).
+    h_start = torch.cuda.Event(enable_timing=True)
+    h_end = torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    with torch.cuda.stream(stream):
+        h_start.record(stream)
+        g.replay()
+        h_end.record(stream)
+    stream.synchronize()
+    barrier(dist)
+    host_submit_max = max_over_ranks(dist, h_start.elapsed_time(h_end) / 1e3)
+
     # Diagnostic: an event pair around each step, all queued behind a sleep
     # kernel so the steps run back to back without host gaps.
     n_ev = min(steps, 200)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
     with torch.cuda.stream(stream):
-        torch.cuda._sleep(50_000_000)
+        torch.cuda._sleep(SLEEP_CYCLES)
         for i in range(n_ev):
             ev[i][0].record(stream)
             step(i)
@@ -449,8 +538,10 @@ def run_hadq(args):
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                          "traffic": recorded_traffic() if cfg == "c2" and args.rows is None else None,
                          "duration": "mean launch interval of K back-to-back steps in one CUDA graph "
-                                     "(CUDA events on the launching stream around the graph replay)",
+                                     "(CUDA events on the launching stream around the graph replay, "
+                                     "queued behind a sleep kernel)",
                          "step_interval_us": interval_max * 1e6,
+                         "step_interval_us_host_submit": host_submit_max / steps * 1e6,
                          "step_us_event_pairs_median": step_ev * 1e6},
             "e2e": e2e,
             "gpu_launches": steps * len(keys),
@@ -475,8 +566,17 @@ def main():
                     help="workload (default c2, the metric's configuration; others for reference)")
     ap.add_argument("--rows", type=int, default=None,
                     help="only the first ROWS rows of each workload part (smaller case for profiler captures)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="rank plumbing only, on CPU (gloo): launcher, per-rank seeds, max-over-ranks")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.gpus < 1:
+        raise SystemExit("bench.py: --gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
+    check_world(args.gpus)
+    if args.dry_run:
+        run_dry(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_hadq(args)

@@ -6,9 +6,12 @@
 // is no CPU path: a missing device or kernel image surfaces as HADQ_ERR_CUDA.
 #include "hadq.h"
 #include "hadq_kernels.cuh"   // launch constants only; the kernels are instantiated elsewhere
+#include "hadq_ksize.cuh"
 #include "hadq_launch.h"
 
 #include <cudaTypedefs.h>
+
+#include <atomic>
 
 #include <cmath>
 #include <cstdint>
@@ -57,31 +60,65 @@ constexpr int64_t kMaxInt8N = 32768;
 // What the kernels need to know about one call.
 struct Shape {
   int64_t rows = 0, n = 0, b = 0;
-  int logb = 0;
+  int kbase = 1;  // b = kbase * 2^logk: 1 for a power of 2, else a covered Paley order
+  int logk = 0;
+  int logb = 0;   // log2(b) when kbase == 1
   int logs = 0;   // segment kernels: log2 of the per-thread segment
   float norm = 1.f;
 };
+
+// Base orders K of the non-power-of-2 sizes b = K * 2^m (Paley II matrices;
+// the kernels build the same ones at compile time).
+constexpr int kPaleyOrders[] = {12, 20, 28, 36, 52, 60, 108};
+
+// b = K * 2^m with a covered K: K (or 0 if none), and m.
+int split_size(int64_t b, int* logk) {
+  int64_t odd = b;
+  int m = 0;
+  while (odd % 2 == 0) {
+    odd /= 2;
+    ++m;
+  }
+  for (int k : kPaleyOrders)
+    if (k == 4 * odd && m >= 2) {
+      *logk = m - 2;
+      return k;
+    }
+  return 0;
+}
 
 hadq_status check_shape(hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, Shape* sh) {
   if (x_dtype != HADQ_F32 && x_dtype != HADQ_BF16) return fail(HADQ_ERR_INVALID_ARG, "x_dtype must be HADQ_F32 or HADQ_BF16");
   if (rows < 0) return fail(HADQ_ERR_INVALID_ARG, "rows must be >= 0");
   if (n <= 0) return fail(HADQ_ERR_INVALID_ARG, "n must be > 0");
-  if (block < -1) return fail(HADQ_ERR_INVALID_ARG, "block must be -1, 0 (full) or a power of 2 dividing n");
+  if (block < -1) return fail(HADQ_ERR_INVALID_ARG, "block must be -1, 0 (full) or a block size dividing n");
   const bool full = block == -1 || block == 0 || block == n;
   const int64_t b = full ? n : block;
-  if (!is_pow2(b))
-    return fail(HADQ_ERR_INVALID_ARG, full ? "a full rotation needs n to be a power of 2" : "block must be a power of 2");
   if (n % b != 0) return fail(HADQ_ERR_INVALID_ARG, "block must divide n");
-  if (b > kMaxBlock) return fail(HADQ_ERR_UNSUPPORTED, "rotation blocks above 8192 are not supported");
   if (n % 8 != 0) return fail(HADQ_ERR_UNSUPPORTED, "n must be a multiple of 8");
   if (rows > (INT64_MAX / 8) / n) return fail(HADQ_ERR_INVALID_ARG, "rows * n overflows");
   sh->rows = rows;
   sh->n = n;
   sh->b = b;
-  sh->logb = ilog2(b);
+  sh->norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
   const int64_t low = n & (-n);                 // largest power of 2 dividing n
   sh->logs = ilog2(low < 128 ? low : 128);
-  sh->norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(b)));
+  if (is_pow2(b)) {
+    if (b > kMaxBlock) return fail(HADQ_ERR_UNSUPPORTED, "rotation blocks above 8192 are not supported");
+    sh->kbase = 1;
+    sh->logb = ilog2(b);
+    return HADQ_OK;
+  }
+  int logk = 0;
+  const int k = split_size(b, &logk);
+  if (k == 0)
+    return fail(HADQ_ERR_INVALID_ARG, full ? "a full rotation needs n = 2^m or K * 2^m with K in {12, 20, 28, 36, 52, 60, 108}"
+                                           : "block must be 2^m or K * 2^m with K in {12, 20, 28, 36, 52, 60, 108}");
+  if (logk < 6 || b / 64 > hadq::ksize::kMaxThreads)
+    return fail(HADQ_ERR_UNSUPPORTED, "K * 2^m rotations need 2^m >= 64 and K * 2^m <= 32768");
+  sh->kbase = k;
+  sh->logk = logk;
+  sh->logb = -1;
   return HADQ_OK;
 }
 
@@ -95,7 +132,9 @@ hadq_status check_quant(hadq_fmt fmt, int64_t group, const Shape& sh, int* eff_g
     case HADQ_INT8_SYM:
       if (group != 0 && group != sh.n) return fail(HADQ_ERR_INVALID_ARG, "int8 is per token: group must be 0 or n");
       if (sh.n > kMaxInt8N) return fail(HADQ_ERR_UNSUPPORTED, "per-token int8 supports n <= 32768");
-      if (sh.b <= 128 && (sh.n >> sh.logs) > 256) return fail(HADQ_ERR_UNSUPPORTED, "per-token int8: n / segment exceeds 256 threads");
+      if (sh.kbase > 1 && sh.b != sh.n) return fail(HADQ_ERR_UNSUPPORTED, "per-token int8 with a K * 2^m block needs the full row");
+      if (sh.kbase == 1 && sh.b <= 128 && (sh.n >> sh.logs) > 256)
+        return fail(HADQ_ERR_UNSUPPORTED, "per-token int8: n / segment exceeds 256 threads");
       *eff_group = static_cast<int>(sh.n);
       return HADQ_OK;
     case HADQ_MXFP4:
@@ -209,22 +248,13 @@ hadq_status launch_result(cudaError_t e, const char* what) {
 
 // ------------------------------------------------------- tensor-core path
 
-// Which implementation serves bf16 rotations the tensor-core kernels cover
-// (full size 4096 / 8192, and block 128): HADQ_KERNEL = "auto" or unset (the
-// tcgen05 + TMA kernels), "tensor" (the same), or "butterfly" (the CUDA-core
-// kernels, kept for comparison).
-enum class KernelChoice { Auto, Butterfly, Tensor };
-
-KernelChoice kernel_choice() {
-  const char* v = std::getenv("HADQ_KERNEL");
-  if (v == nullptr || std::strcmp(v, "auto") == 0) return KernelChoice::Auto;
-  if (std::strcmp(v, "butterfly") == 0) return KernelChoice::Butterfly;
-  if (std::strcmp(v, "tensor") == 0) return KernelChoice::Tensor;
-  return KernelChoice::Auto;
-}
+// Which implementation serves the calls both implementations cover (bf16
+// input at full size 4096 / 8192 and at block 128): set process-wide through
+// hadq_set_impl, HADQ_IMPL_AUTO (the tcgen05 + TMA kernels) by default.
+std::atomic<int> g_impl{HADQ_IMPL_AUTO};
 
 bool tc_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
-  return x_dtype == HADQ_BF16 && (sh.logb == 12 || sh.logb == 13) && mode >= 0;
+  return x_dtype == HADQ_BF16 && sh.kbase == 1 && (sh.logb == 12 || sh.logb == 13) && mode >= 0;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -276,7 +306,7 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
 // block is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
 bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
-  if (x_dtype != HADQ_BF16 || sh.b != 128) return false;
+  if (x_dtype != HADQ_BF16 || sh.kbase != 1 || sh.b != 128) return false;
   if (mode >= 0) return true;
   const int64_t bpr = sh.n >> 7;            // whole 8-row swizzle atoms per tile
   return bpr >= 32 && bpr <= 128 && bpr % 8 == 0;
@@ -313,6 +343,26 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                        "tensor-core block-128 kernel launch");
 }
 
+// Blocks of b = K * 2^m elements (one CTA per block, persistent over blocks).
+hadq_status launch_ksize(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0,
+                         void* out1, cudaStream_t stream, int sms, int dev, Signs sg) {
+  const bool bf = x_dtype == HADQ_BF16;
+  const bool sgd = sg.side != hadq::SIGNS_NONE;
+  const hl::KsFn fn = hl::ksize_kernel_for(sh.kbase, bf, mode, sgd);
+  if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no K * 2^m kernel for this base order and format");
+  const int64_t smem = hadq::ksize::smem_bytes(sh.b, bf ? 2 : 4, sgd);
+  if (smem > 227 * 1024) return fail(HADQ_ERR_UNSUPPORTED, "K * 2^m block too large for shared memory");
+  const int threads = static_cast<int>(ceil_div(sh.b / 64, 32) * 32);
+  int occ = 0;
+  hadq_status st = occupancy(reinterpret_cast<const void*>(fn), dev, threads, static_cast<int>(smem), &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t units = sh.rows * (sh.n / sh.b);
+  const int64_t grid = std::min<int64_t>(units, int64_t(sms) * occ);
+  return launch_result(launch_pdl(fn, grid, threads, static_cast<int>(smem), stream, x, units, sh.logk, sh.norm, group,
+                                  out0, out1, sg),
+                       "K * 2^m kernel launch");
+}
+
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
 // -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
@@ -335,7 +385,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours
-  if (kernel_choice() != KernelChoice::Butterfly) {
+  if (sh.kbase > 1) return launch_ksize(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg);
+  if (g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY) {
     if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
     if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
   }
@@ -669,7 +720,17 @@ const char* hadq_status_string(hadq_status status) {
 
 const char* hadq_last_error(void) { return g_last_error.c_str(); }
 
-int hadq_version(void) { return 100; }
+int hadq_version(void) { return 200; }
+
+hadq_status hadq_set_impl(hadq_impl impl) {
+  g_last_error.clear();
+  if (impl != HADQ_IMPL_AUTO && impl != HADQ_IMPL_BUTTERFLY && impl != HADQ_IMPL_TENSOR)
+    return fail(HADQ_ERR_INVALID_ARG, "impl must be HADQ_IMPL_AUTO, HADQ_IMPL_BUTTERFLY or HADQ_IMPL_TENSOR");
+  g_impl.store(static_cast<int>(impl), std::memory_order_relaxed);
+  return HADQ_OK;
+}
+
+hadq_impl hadq_get_impl(void) { return static_cast<hadq_impl>(g_impl.load(std::memory_order_relaxed)); }
 
 int hadq_device_faults(int clear) { return hadq::launch::tc_fault_bits(clear); }
 

@@ -404,16 +404,18 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, flo
   return w;
 }
 
-// Scale arithmetic.  The scales are m / 7 (int4, then rounded to fp16) and
-// m / 127 (int8, fp32); they are formed as m * fp32(1/q) and inverted with the
-// fast reciprocal.  Each step is within 2 ulp (relative error < 3e-7), far
-// inside the 1e-6 window in which a rounding decision may go either way, so
-// the codes and scales equal the exactly rounded ones everywhere else.
-constexpr float kInv7 = 1.0f / 7.0f;
-constexpr float kInv127 = 1.0f / 127.0f;
-constexpr float kInv6 = 1.0f / 6.0f;
-
-__device__ __forceinline__ float fast_recip(float s) { return __fdividef(1.0f, s); }
+// Scale arithmetic.  Every scale is a correctly rounded fp32 quotient of
+// the group absmax m: m / 7 (int4, then rounded to fp16), m / 127 (int8) and
+// m / 6 (NVFP4, then rounded to E4M3).  The factor that takes an unnormalised
+// rotated value z to code units is the correctly rounded quotient norm / s, so
+// an int code is the single rounding of the exact product z * (norm / s) onto
+// the integer grid: it can differ from the exactly rounded y / s only through
+// the fp32 rotation's own error and the factor's half-ulp (about 4.5e-7 of a
+// code unit at |y / s| = 7.5).
+__device__ __forceinline__ float int4_scale_f32(float m) { return __fdiv_rn(m, 7.0f); }
+__device__ __forceinline__ float int8_scale(float m) { return __fdiv_rn(m, 127.0f); }
+__device__ __forceinline__ float nvfp4_scale_f32(float m) { return __fdiv_rn(m, 6.0f); }
+__device__ __forceinline__ float code_factor(float norm, float s) { return __fdiv_rn(norm, s); }
 
 // 32 output bytes at p: one 256-bit store (full 32-byte sectors) when p is
 // 32-byte aligned, else two 128-bit stores.  A thread's run of outputs is
@@ -494,10 +496,9 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
       if (spg >= 4) mz = fmaxf(mz, fmaxf(m32[j ^ 2], m32[j ^ 3]));
     }
     const float m = mz * norm;                         // absmax of y (rounding is monotone)
-    const __half s16 = __float2half_rn(m * kInv7);
+    const __half s16 = __float2half_rn(int4_scale_f32(m));
     const float s = __half2float(s16);
-    const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;   // zero / inf scale -> zero codes
-    const float rn = r * norm;
+    const float rn = (s > 0.f && s <= 65504.f) ? code_factor(norm, s) : 0.f;   // zero / inf scale -> zero codes
     uint4 w;
     if (mz * rn < 7.25f) {        // normal scale: every |v * rn| <= 7.0035, no clamp
       w.x = pack_int4x8<PERM>(v, 32 * j + 0, rn);
@@ -531,10 +532,9 @@ __device__ __forceinline__ void store_int4_pair(const float (&v)[64], float norm
   float mz = fmaxf(absmax_regs(v, 0, 32), absmax_regs(v, 32, 32));
   mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 1));
   const float m = mz * norm;
-  const __half s16 = __float2half_rn(m * kInv7);
+  const __half s16 = __float2half_rn(int4_scale_f32(m));
   const float s = __half2float(s16);
-  const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
-  const float rn = r * norm;
+  const float rn = (s > 0.f && s <= 65504.f) ? code_factor(norm, s) : 0.f;
   uint4 w0, w1;
   if (mz * rn < 7.25f) {
     w0 = make_uint4(pack_int4x8<PERM>(v, 0, rn), pack_int4x8<PERM>(v, 8, rn), pack_int4x8<PERM>(v, 16, rn),
@@ -571,10 +571,9 @@ __device__ __forceinline__ void store_int4_lanes(const float (&v)[N], float norm
   mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 1));
   if (group >= 4 * N) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, 2));
   const float m = mz * norm;
-  const __half s16 = __float2half_rn(m * kInv7);
+  const __half s16 = __float2half_rn(int4_scale_f32(m));
   const float s = __half2float(s16);
-  const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
-  const float rn = r * norm;
+  const float rn = (s > 0.f && s <= 65504.f) ? code_factor(norm, s) : 0.f;
   const bool plain = mz * rn < 7.25f;
   uint4 prev = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
@@ -656,9 +655,9 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
   static_assert(N % 16 == 0, "NVFP4 blocks are 16 elements");
   if constexpr (N == 16) {
     const float m = absmax_regs(v, 0, 16) * nq;
-    const uint16_t b = e4m3x2(0.f, m * kInv6);
+    const uint16_t b = e4m3x2(0.f, nvfp4_scale_f32(m));
     const float s = e4m3x2_values(b).x;
-    const float f = s > 0.f ? nq * fast_recip(s) : 0.f;
+    const float f = s > 0.f ? code_factor(nq, s) : 0.f;
     reinterpret_cast<uint2*>(codes + (e0 >> 1))[0] = make_uint2(pack_e2m1x8<PERM>(v, 0, f), pack_e2m1x8<PERM>(v, 8, f));
     scales[e0 >> 4] = static_cast<uint8_t>(b & 0xFFu);
   } else {
@@ -668,10 +667,10 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
     for (int j = 0; j < N / 32; ++j) {
       const float m0 = absmax_regs(v, 32 * j, 16) * nq;
       const float m1 = absmax_regs(v, 32 * j + 16, 16) * nq;
-      const uint16_t b = e4m3x2(m1 * kInv6, m0 * kInv6);
+      const uint16_t b = e4m3x2(nvfp4_scale_f32(m1), nvfp4_scale_f32(m0));
       const float2 s = e4m3x2_values(b);
-      const float f0 = s.x > 0.f ? nq * fast_recip(s.x) : 0.f;
-      const float f1 = s.y > 0.f ? nq * fast_recip(s.y) : 0.f;
+      const float f0 = s.x > 0.f ? code_factor(nq, s.x) : 0.f;
+      const float f1 = s.y > 0.f ? code_factor(nq, s.y) : 0.f;
       const uint4 w = make_uint4(pack_e2m1x8<PERM>(v, 32 * j, f0), pack_e2m1x8<PERM>(v, 32 * j + 8, f0),
                                  pack_e2m1x8<PERM>(v, 32 * j + 16, f1), pack_e2m1x8<PERM>(v, 32 * j + 24, f1));
       if constexpr (N == 32) {
@@ -691,10 +690,10 @@ template <bool PERM, int N>
 __device__ __forceinline__ void store_int8(const float (&v)[N], float norm, float m, int8_t* __restrict__ codes,
                                            int64_t e0) {
   static_assert(N % 8 == 0, "int8 chunk must hold whole 8-byte stores");
-  const float s = m * kInv127;
-  const float r = (s >= 1.0e-36f && s <= 3.0e38f) ? fast_recip(s) : (s > 0.f ? __frcp_rn(s) : 0.f);
-  const float rn = r * norm;
-  if (m * r < 127.25f) {         // normal scale: every |v * rn| < 127.5, no clamp
+  const float s = int8_scale(m);
+  const bool tiny = s > 0.f && s < 1.0e-36f;   // norm / s may be inexact or overflow: divide per element
+  const float rn = (s >= 1.0e-36f && s <= 3.0e38f) ? code_factor(norm, s) : 0.f;
+  if (!tiny) {                   // normal scale: every |v * rn| < 127.5, no clamp; zero scale: zero codes
     if constexpr (N % 32 == 0) {
       auto chunk = [&](int i) {
         return make_uint4(pack_int8x4<PERM>(v, 16 * i, rn), pack_int8x4<PERM>(v, 16 * i + 4, rn),
@@ -715,7 +714,7 @@ __device__ __forceinline__ void store_int8(const float (&v)[N], float norm, floa
         o[i] = make_uint2(pack_int8x4<PERM>(v, 8 * i, rn), pack_int8x4<PERM>(v, 8 * i + 4, rn));
     }
   } else {
-    // Subnormal scale: the reciprocal is inexact or overflows -- divide, clamp.
+    // Tiny scale: norm / s may be inexact or overflow -- divide per element, clamp.
 #pragma unroll
     for (int i = 0; i < N / 4; ++i) {
       uint32_t w = 0;

@@ -186,7 +186,7 @@ segment_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, int
     }
     const float m = cta_max(absmax_regs(v, 0, S), red) * norm;
     if (active) store_int8<false, S>(v, norm, m, codes, e0);
-    if (threadIdx.x == 0) scales[r] = m * kInv127;
+    if (threadIdx.x == 0) scales[r] = int8_scale(m);
   }
 }
 
@@ -398,7 +398,7 @@ team_row_int8_kernel(const void* __restrict__ x, int64_t rows, int64_t n, float 
     }
     const float m = cta_max(absmax_regs(v, 0, 128), red) * norm;
     if (active) store_int8<Sh::PERM, 128>(v, norm, m, codes, base + tau * 128);
-    if (threadIdx.x == 0) scales[r] = m * kInv127;
+    if (threadIdx.x == 0) scales[r] = int8_scale(m);
   }
 }
 

@@ -242,10 +242,9 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
 #pragma unroll
     for (int j = 0; j < L / 32; ++j) {
       const float m = (j == 0 ? mz_lo : mz_hi) * norm;
-      const __half s16 = __float2half_rn(m * kInv7);
+      const __half s16 = __float2half_rn(int4_scale_f32(m));
       const float s = __half2float(s16);
-      const float r = (s > 0.f && s <= 65504.f) ? fast_recip(s) : 0.f;
-      const float rn = r * norm;
+      const float rn = (s > 0.f && s <= 65504.f) ? code_factor(norm, s) : 0.f;
       uint4 w;
       if ((j == 0 ? mz_lo : mz_hi) * rn < 7.25f) {
         w = make_uint4(pack_int4x8<false>(z, 32 * j, rn), pack_int4x8<false>(z, 32 * j + 8, rn),

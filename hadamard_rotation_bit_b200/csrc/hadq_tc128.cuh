@@ -235,7 +235,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
           const float mrow = fmaxf(fmaxf(gred[0], gred[1]), fmaxf(gred[2], gred[3])) * norm;
           asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");   // gred may be rewritten next tile
           if (ok) store_int8<false, 128>(z, norm, mrow, static_cast<int8_t*>(out0), e0);
-          if (m == 0) static_cast<float*>(out1)[t] = mrow * kInv127;
+          if (m == 0) static_cast<float*>(out1)[t] = int8_scale(mrow);
         } else if constexpr (MODE == OUT_INT4) {
           if (ok) store_int4<false, 128>(z, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
         } else if constexpr (MODE == OUT_MXFP4) {

@@ -30,8 +30,9 @@ EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
     "hadq_device_faults", "hadq_rotate_quant_host_static", "hadq_rotate_signed", "hadq_rotate_quant_signed",
-    "hadq_rotate_quant_nvfp4",
+    "hadq_rotate_quant_nvfp4", "hadq_set_impl", "hadq_get_impl",
 )
+IMPLS = {"auto": 0, "butterfly": 1, "tensor": 2}
 
 _lock = threading.Lock()
 _lib = None
@@ -79,6 +80,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_rotate_quant_signed.restype = i32
         lib.hadq_rotate_quant_nvfp4.argtypes = [vp, i32, i64, i64, i64, ctypes.c_float, vp, vp, vp]
         lib.hadq_rotate_quant_nvfp4.restype = i32
+        lib.hadq_set_impl.argtypes = [i32]
+        lib.hadq_set_impl.restype = i32
+        lib.hadq_get_impl.argtypes = []
+        lib.hadq_get_impl.restype = i32
         _lib = lib
         return lib
 
@@ -150,6 +155,22 @@ def _rows_n(x: torch.Tensor):
 def hadq_device_faults(clear: bool = True) -> int:
     """Fault bits of kernels whose bounded waits ran out (0 = none)."""
     return int(load_library().hadq_device_faults(1 if clear else 0))
+
+
+def hadq_set_impl(impl: str) -> str:
+    """Choose the implementation for the shapes both cover ("auto", "tensor"
+    or "butterfly", see include/hadq.h); returns the previous choice."""
+    lib = load_library()
+    if impl not in IMPLS:
+        raise HadqError(HADQ_ERR_INVALID_ARG, f"unknown impl {impl!r}")
+    prev = hadq_get_impl()
+    _check(lib.hadq_set_impl(IMPLS[impl]))
+    return prev
+
+
+def hadq_get_impl() -> str:
+    code = int(load_library().hadq_get_impl())
+    return {v: k for k, v in IMPLS.items()}[code]
 
 
 def codes_nbytes(rows: int, n: int, fmt: str) -> int:

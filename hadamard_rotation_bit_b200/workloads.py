@@ -28,6 +28,10 @@ permutation drawn from a ``seed + 1`` stream):
   draws (``generate_signs``), int8 +/-1.
 * ``c3rb`` / ``c5rb``  the ``c3`` / ``c5`` input and quantizer with signs
   before the rotation (block 128 / full 8192).
+* ``c3k``  the ``c3`` input rotated in full instead of by blocks of 128: the
+  14336-point rotation of a non-power-of-2 size ("Rotation Transform",
+  section 1.5: 14336 = 28 * 2^9, a base matrix of order 28 with a Sylvester
+  block); int8 per token.
 
 Values are drawn in float64, rounded to float32 (nearest even) and, for
 bf16 tensors, to bfloat16 (nearest even).
@@ -104,6 +108,8 @@ WORKLOADS = {
     "c2rb": Workload("c2rb", "R1 4096 tokens x hidden 4096 bf16, full 4096-point random Hadamard transpose "
                      "(signs before), int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128,
                      signs="before", base="c2"),
+    "c3k": Workload("c3k", "R4 8192 tokens x intermediate 14336 bf16, full 14336-point Hadamard (K = 28 base "
+                    "(x) 512-point Sylvester), int8 per token", 8192, 14336, 14336, "bf16", "int8", 0, base="c3"),
     "c3rb": Workload("c3rb", "R4 8192 tokens x intermediate 14336 bf16, block 128 random Hadamard transpose "
                      "(signs before), int8 per token", 8192, 14336, 128, "bf16", "int8", 0, signs="before", base="c3"),
     "c5rb": Workload("c5rb", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point random Hadamard "

@@ -242,6 +242,30 @@ HADQ_API int hadq_device_faults(int clear);
 /* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
 HADQ_API int hadq_version(void);
 
+/*
+ * Implementation choice.  Two implementations compute the same operation:
+ * the tensor-core kernels (tcgen05 MMA with H_128 for the high index bits,
+ * operands staged by TMA) and the CUDA-core butterfly kernels.  The tensor-core
+ * kernels cover bf16 input at full size 4096 / 8192 and at block 128; every
+ * other call runs the butterfly kernels whatever the choice.
+ *   HADQ_IMPL_AUTO       the default: the tensor-core kernels wherever they apply
+ *   HADQ_IMPL_TENSOR     the same (named for callers that want to say so)
+ *   HADQ_IMPL_BUTTERFLY  the butterfly kernels everywhere
+ * Results agree within the parity tolerances, not bit for bit (the two sum in
+ * different orders).  hadq_set_impl is process-wide and takes effect for calls
+ * made after it returns; it returns HADQ_ERR_INVALID_ARG for any other value.
+ * No paper counterpart: it exists so that both implementations can be tested
+ * and measured on the same shapes.
+ */
+typedef enum hadq_impl {
+  HADQ_IMPL_AUTO = 0,
+  HADQ_IMPL_BUTTERFLY = 1,
+  HADQ_IMPL_TENSOR = 2
+} hadq_impl;
+
+HADQ_API hadq_status hadq_set_impl(hadq_impl impl);
+HADQ_API hadq_impl hadq_get_impl(void);
+
 #ifdef __cplusplus
 }
 #endif

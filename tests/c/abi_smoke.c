@@ -34,7 +34,9 @@ static int fails = 0;
   } while (0)
 
 static int host_checks(void) {
-  CHECK(hadq_version() == 100, "version %d", hadq_version());
+  CHECK(hadq_version() == 200, "version %d", hadq_version());
+  CHECK(hadq_get_impl() == HADQ_IMPL_AUTO, "impl %d", (int)hadq_get_impl());
+  CHECK(hadq_set_impl((hadq_impl)9) == HADQ_ERR_INVALID_ARG, "bad impl accepted");
   CHECK(strcmp(hadq_status_string(HADQ_OK), "ok") == 0, "status string");
   CHECK(hadq_codes_bytes(4, 1024, HADQ_INT4_SYM) == 2048, "int4 code bytes");
   CHECK(hadq_scales_bytes(4, 1024, HADQ_INT4_SYM, 128) == 64, "int4 scale bytes");

@@ -45,7 +45,7 @@ def test_exports_every_declared_symbol(lib):
 def test_status_strings_and_version(lib):
     for st in range(5):
         assert lib.hadq_status_string(st)
-    assert lib.hadq_version() == 100
+    assert lib.hadq_version() == 200
 
 
 def _q(lib, x=A, xd=1, rows=4, n=1024, block=0, fmt=0, group=128, codes=B, scales=C):
@@ -221,3 +221,31 @@ def test_binding_checks_host_output_sizes(lib):
     with pytest.raises(H.HadqError):
         H._holds("out", torch.empty(8, 4)[:, :2], 16)                             # not contiguous
     assert H._block_len(4096, 0) == 4096 and H._block_len(4096, -1) == 4096 and H._block_len(4096, 128) == 128
+
+
+def test_impl_choice_is_explicit_and_checked(lib):
+    """hadq_set_impl selects the implementation for the shapes both cover; it
+    touches no device and rejects values outside the enum."""
+    assert H.hadq_get_impl() == "auto"
+    assert H.hadq_set_impl("butterfly") == "auto"
+    assert H.hadq_get_impl() == "butterfly"
+    assert H.hadq_set_impl("auto") == "butterfly"
+    assert lib.hadq_set_impl(7) == H.HADQ_ERR_INVALID_ARG
+    assert "HADQ_IMPL" in lib.hadq_last_error().decode()
+    assert H.hadq_get_impl() == "auto"
+
+
+def test_k_size_shape_rules(lib):
+    """Non-power-of-2 sizes b = K * 2^m: covered K run, others are refused on
+    the host before any CUDA call (fake aligned addresses, never touched)."""
+    a, c, sc = 0x100000, 0x20000000, 0x40000000
+    f = lib.hadq_rotate_quant
+    bf, i4, i8 = H.HADQ_BF16, H.FMTS["int4"], H.FMTS["int8"]
+    assert f(a, bf, 0, 28 * 512, 0, i4, 128, c, sc, None) == H.HADQ_OK            # empty call, covered size
+    assert f(a, bf, 0, 44 * 64, 0, i4, 128, c, sc, None) == H.HADQ_ERR_INVALID_ARG   # K = 44 not covered
+    assert "K * 2^m" in lib.hadq_last_error().decode()
+    assert f(a, bf, 0, 28 * 32, 0, i4, 32, c, sc, None) == H.HADQ_ERR_UNSUPPORTED    # 2^m < 64
+    assert f(a, bf, 0, 28 * 2048, 0, i4, 128, c, sc, None) == H.HADQ_ERR_UNSUPPORTED  # above 32768
+    assert f(a, bf, 0, 3 * 28 * 64, 28 * 64, i8, 0, c, sc, None) == H.HADQ_ERR_UNSUPPORTED  # int8 needs full rows
+    assert f(a, bf, 0, 3 * 28 * 64, 28 * 64, i4, 64, c, sc, None) == H.HADQ_OK       # block-diagonal K-size
+    assert f(a, bf, 0, 28 * 64 + 8, 28 * 64, i4, 32, c, sc, None) == H.HADQ_ERR_INVALID_ARG  # block must divide n

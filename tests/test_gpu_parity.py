@@ -36,13 +36,9 @@ def _cuda():
     # This module covers the CUDA-core kernels everywhere (the full-size bf16
     # 4096 / 8192 rotations would otherwise take the tensor-core path, which
     # tests/test_gpu_tensor_path.py covers).
-    old = os.environ.get("HADQ_KERNEL")
-    os.environ["HADQ_KERNEL"] = "butterfly"
+    old = H.hadq_set_impl("butterfly")
     yield
-    if old is None:
-        os.environ.pop("HADQ_KERNEL", None)
-    else:
-        os.environ["HADQ_KERNEL"] = old
+    H.hadq_set_impl(old)
 
 
 def _log(name, rep):

@@ -12,7 +12,6 @@ ahead of the MMA, and at b = 128 both folded into the H_128 operand) and the
 CUDA-core butterfly kernels (everything else).
 """
 
-import os
 
 import numpy as np
 import pytest
@@ -30,16 +29,12 @@ pytestmark = pytest.mark.gpu
 def path(request):
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     H.load_library()
-    old = os.environ.get("HADQ_KERNEL")
-    os.environ["HADQ_KERNEL"] = request.param
+    old = H.hadq_set_impl(request.param)
     H.hadq_device_faults(clear=True)
     yield request.param
     torch.cuda.synchronize()
     faults = H.hadq_device_faults(clear=True)
-    if old is None:
-        os.environ.pop("HADQ_KERNEL", None)
-    else:
-        os.environ["HADQ_KERNEL"] = old
+    H.hadq_set_impl(old)
     assert faults == 0, f"tensor-core kernel reported fault bits {faults}"
 
 

@@ -2,12 +2,11 @@
 
 The path serves full-size rotations of b = 4096 and 8192 and block-128
 rotations (R3 heads, R4 rotation_size 128) with bf16 input and is the
-default there.  Every test runs it (HADQ_KERNEL=tensor), compares with
+default there.  Every test runs it (hadq_set_impl(tensor)), compares with
 the oracle exactly as the butterfly tests do, and checks that no bounded wait
 inside the kernel ran out (hadq_device_faults() == 0).
 """
 
-import os
 
 import numpy as np
 import pytest
@@ -25,16 +24,12 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(autouse=True)
 def tensor_path():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    old = os.environ.get("HADQ_KERNEL")
-    os.environ["HADQ_KERNEL"] = "tensor"
+    old = H.hadq_set_impl("tensor")
     H.hadq_device_faults(clear=True)
     yield
     torch.cuda.synchronize()
     faults = H.hadq_device_faults(clear=True)
-    if old is None:
-        os.environ.pop("HADQ_KERNEL", None)
-    else:
-        os.environ["HADQ_KERNEL"] = old
+    H.hadq_set_impl(old)
     assert faults == 0, f"tensor-core kernel reported fault bits {faults}"
 
 
@@ -67,13 +62,13 @@ def test_tc_many_tiles_ragged(rows, n, fmt, group):
 
 
 def test_default_path_is_the_tensor_core_kernel():
-    """With HADQ_KERNEL unset the full-size bf16 rotation takes the tensor-core
+    """With the default choice (auto) the full-size bf16 rotation takes the tensor-core
     kernel: same codes as the forced tensor path, bit for bit."""
     stored, x64 = synth(64, 4096, "bf16", seed=5)
     c_t, s_t = run_quant(stored, "bf16", 0, "int4", 128)
-    os.environ.pop("HADQ_KERNEL", None)
+    H.hadq_set_impl("auto")
     c_d, s_d = run_quant(stored, "bf16", 0, "int4", 128)
-    os.environ["HADQ_KERNEL"] = "tensor"
+    H.hadq_set_impl("tensor")
     np.testing.assert_array_equal(c_d, c_t)
     np.testing.assert_array_equal(s_d, s_t)
 
@@ -100,9 +95,9 @@ def test_tc_matches_butterfly_codes():
     outside the oracle's boundary window (same C2 slice, same format)."""
     stored, x64 = synth(512, 4096, "bf16", seed=77)
     c_tc, s_tc = run_quant(stored, "bf16", 0, "int4", 128)
-    os.environ["HADQ_KERNEL"] = "butterfly"
+    H.hadq_set_impl("butterfly")
     c_bf, s_bf = run_quant(stored, "bf16", 0, "int4", 128)
-    os.environ["HADQ_KERNEL"] = "tensor"
+    H.hadq_set_impl("tensor")
     pc.check_int4(x64, c_tc, s_tc, 0, 128)
     pc.check_int4(x64, c_bf, s_bf, 0, 128)
     differ = (pc.unpack_nibbles(c_tc, True) != pc.unpack_nibbles(c_bf, True)).sum()
