@@ -25,6 +25,11 @@ What it computes, and where the pages define it:
   int8, section 1.7), and its transpose diag(+/-1) @ H / sqrt(N), which is its
   inverse and puts the signs ahead of the transform as in orbitquant's RPBH
   ("orbitquant 0.2.0", how it works).
+* ``rpbh_rotate`` / ``sphere_lloyd_max`` / ``quantize_codebook`` -- the
+  orbitquant method ("orbitquant 0.2.0", Method Conformance): RPBH rotation
+  (permutation, Rademacher signs, block FWHT, orthonormal scaling) and the
+  online quantizer (per-token norm, normalized rotation, nearest centroid of
+  the unit-sphere Lloyd-Max codebook, rescaling).  Readings on each function.
 * ``quantize_int4_sym`` / ``quantize_int8_per_token`` -- round-to-nearest
   with symmetric range (the RTN proxy with wbits / groupsize / sym of
   "Pre-Process (Rotation Preprocessing)", OneCompression docs, Workflow note).
@@ -66,7 +71,14 @@ from .hadq_oracle import (  # noqa: F401
     PALEY_FIELDS,
     quadratic_character,
     split_size,
+    pack_codes,
     pack_nibbles,
+    quantize_codebook,
+    rpbh_inverse,
+    rpbh_rotate,
+    sphere_lloyd_max,
+    sphere_marginal_cdf,
+    sphere_partial_first_moment,
     quantize,
     quantize_int4_sym,
     quantize_int8_per_token,

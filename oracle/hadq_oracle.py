@@ -532,3 +532,136 @@ def quantize(y, fmt: str, group: int = 0, tensor_scale: float = 1.0):
         q, s = quantize_mxfp4(y)
         return y, pack_nibbles(q), s
     raise ValueError(f"unknown fmt {fmt!r}")
+
+
+# ---------------------------------------------------------------------------
+# orbitquant: RPBH rotation and the unit-sphere Lloyd-Max codebook quantizer
+# ---------------------------------------------------------------------------
+# "orbitquant 0.2.0" (PyPI page), Method Conformance: the rotation is RPBH --
+# a permutation, Rademacher signs, a block FWHT and orthonormal scaling -- and
+# activations are quantized online by a per-token norm, rotation of the
+# normalized activation, nearest-centroid quantization and rescaling, with one
+# fixed codebook per (input dimension, bit width) from "exact unit-sphere
+# Lloyd-Max codebooks" (Features).  The page gives no formula; readings:
+#   * RPBH(x) = (x[pi] * s) . diag(H_B, ..., H_B) / sqrt(B): v_e = x_pi(e) s_e
+#     for every column e of the row (pi a permutation of the n columns, s n
+#     signs), then the block rotation of ``rotate``;
+#   * the codebook is the Lloyd-Max (minimum mean-square error) quantizer of
+#     one coordinate T of a uniformly random unit vector in R^d, whose density
+#     is f_d(t) = (1 - t^2)^((d - 3) / 2) / B(1/2, (d - 1) / 2) on [-1, 1]: a
+#     rotated, normalized activation is such a vector when the rotation is
+#     random, which is why the codebook needs no data;
+#   * code = index of the nearest centroid of y / ||y|| (a value exactly on a
+#     threshold takes the lower index); the per-token scale is ||y|| = ||x||.
+
+
+def rpbh_rotate(x, block, perm, signs) -> np.ndarray:
+    """RPBH rotation of every row: permute the columns by ``perm``
+    (v_e = x[pi(e)]), multiply by the signs (negative int8 = -1), then the
+    block-diagonal normalised Hadamard rotation of ``rotate``."""
+    x = np.asarray(x, dtype=np.float64)
+    rows, n = x.shape
+    perm = np.asarray(perm, dtype=np.int64).reshape(-1)
+    if perm.size != n or not np.array_equal(np.sort(perm), np.arange(n)):
+        raise ValueError("perm must be a permutation of the n columns")
+    s = sign_vector(signs)
+    if s.size != n:
+        raise ValueError("RPBH takes one sign per column (n signs)")
+    return rotate(x[:, perm] * s[None, :], block)
+
+
+def rpbh_inverse(y, block, perm, signs) -> np.ndarray:
+    """Inverse of ``rpbh_rotate``: rotate back (H / sqrt(B) is its own
+    inverse), undo the signs, scatter the columns back to their places."""
+    y = np.asarray(y, dtype=np.float64)
+    v = rotate(y, block) * sign_vector(signs)[None, :]
+    x = np.empty_like(v)
+    x[:, np.asarray(perm, dtype=np.int64)] = v
+    return x
+
+
+def sphere_marginal_cdf(t, d: int) -> np.ndarray:
+    """P(T <= t) for one coordinate T of a uniform unit vector in R^d (d >= 2):
+    1/2 + sign(t) / 2 * I_(t^2)(1/2, (d - 1) / 2), I the regularized
+    incomplete beta function (the integral of (1 - t^2)^((d-3)/2) from 0 to x
+    is B(x^2; 1/2, (d - 1)/2) / 2 after t^2 = w)."""
+    from scipy.special import betainc
+    t = np.clip(np.asarray(t, dtype=np.float64), -1.0, 1.0)
+    return 0.5 + 0.5 * np.sign(t) * betainc(0.5, (d - 1) / 2.0, t * t)
+
+
+def sphere_partial_first_moment(a, b, d: int) -> np.ndarray:
+    """The integral of t f_d(t) over [a, b]: with k = (d - 3) / 2 the
+    antiderivative of t (1 - t^2)^k is -(1 - t^2)^(k + 1) / (2 (k + 1))."""
+    from scipy.special import betaln
+    a = np.clip(np.asarray(a, dtype=np.float64), -1.0, 1.0)
+    b = np.clip(np.asarray(b, dtype=np.float64), -1.0, 1.0)
+    e = (d - 1) / 2.0
+    norm = np.exp(betaln(0.5, e))
+
+    def g(t):                      # (1 - t^2)^e, 0 at t = +/-1
+        if e == 0:
+            return np.ones_like(t)
+        with np.errstate(divide="ignore"):
+            return np.exp(e * np.log1p(-np.minimum(t * t, 1.0)))
+    return (g(a) - g(b)) / ((d - 1) * norm)
+
+
+@functools.lru_cache(maxsize=16)
+def sphere_lloyd_max(d: int, bits: int, tol: float = 1e-13, max_iter: int = 200000):
+    """Lloyd-Max codebook of the unit-sphere marginal f_d: ``(centroids,
+    thresholds)`` with 2^bits centroids (ascending) and 2^bits - 1 thresholds.
+
+    Lloyd's iteration, in the order of its definition: thresholds are the
+    midpoints of adjacent centroids; each centroid is the conditional mean of
+    T over its cell, from the exact CDF and first moment above.  Starts from
+    the quantiles of the cell mid-probabilities; stops when no centroid moves
+    by more than ``tol`` times the largest centroid.
+    """
+    from scipy.special import betaincinv
+    d, bits = int(d), int(bits)
+    if d < 2 or bits < 1:
+        raise ValueError("need d >= 2 and bits >= 1")
+    levels = 1 << bits
+    p = (np.arange(levels) + 0.5) / levels
+    q = betaincinv(0.5, (d - 1) / 2.0, np.abs(2 * p - 1))
+    c = np.sign(p - 0.5) * np.sqrt(q)
+    for _ in range(max_iter):
+        t = 0.5 * (c[:-1] + c[1:])
+        lo = np.concatenate([[-1.0], t])
+        hi = np.concatenate([t, [1.0]])
+        mass = sphere_marginal_cdf(hi, d) - sphere_marginal_cdf(lo, d)
+        c_new = sphere_partial_first_moment(lo, hi, d) / mass
+        moved = np.abs(c_new - c).max()
+        c = c_new
+        if moved <= tol * np.abs(c).max():
+            break
+    t = 0.5 * (c[:-1] + c[1:])
+    c.setflags(write=False)
+    t.setflags(write=False)
+    return c, t
+
+
+def quantize_codebook(y, centroids, thresholds):
+    """Per-token norm, normalized values, nearest centroid.
+
+    For every row: r = ||y||_2; u = y / r; code = number of thresholds
+    strictly below u (the index of the nearest centroid; thresholds are the
+    midpoints); r = 0 gives codes of u = 0.  Returns ``(codes uint8 (rows, n),
+    norms float64 (rows,))``; dequantization is r * centroids[code].
+    """
+    y = np.asarray(y, dtype=np.float64)
+    r = np.sqrt((y * y).sum(axis=1))
+    u = y / np.where(r > 0, r, 1.0)[:, None]
+    codes = np.searchsorted(np.asarray(thresholds, dtype=np.float64), u, side="left")
+    return codes.astype(np.uint8), r
+
+
+def pack_codes(codes, bits: int) -> np.ndarray:
+    """8 // bits codes per byte, code i of a byte in bits [i * bits, (i + 1) * bits)."""
+    c = np.asarray(codes).astype(np.int64)
+    per = 8 // bits
+    if c.shape[-1] % per:
+        raise ValueError(f"row length must be a multiple of {per}")
+    c = c.reshape(*c.shape[:-1], c.shape[-1] // per, per)
+    return (c << (bits * np.arange(per))).sum(axis=-1).astype(np.uint8)

@@ -626,3 +626,121 @@ def test_nvfp4_properties():
     assert c.shape == (3, 32) and sc.shape == (3, 4) and sc.dtype == np.uint8
     with pytest.raises(ValueError):
         oracle.rotate_quant(rng.standard_normal((3, 64)), 0, "nvfp4", 32)
+
+
+# ------------------------------------------- orbitquant: RPBH and codebooks
+
+def test_rpbh_equals_explicit_permutation_sign_and_hadamard_matrices():
+    """RPBH(x) = x P D H_blk / sqrt(B) with P the permutation matrix of pi
+    (column e of x P is column pi(e) of x) and D = diag(s)."""
+    rng = np.random.default_rng(11)
+    n, block = 64, 16
+    x = rng.standard_normal((5, n))
+    perm = rng.permutation(n)
+    signs = np.where(rng.random(n) < 0.5, -1, 1).astype(np.int8)
+    p = np.zeros((n, n))
+    p[perm, np.arange(n)] = 1.0
+    hb = np.kron(np.eye(n // block), oracle.sylvester_hadamard(block)) / np.sqrt(block)
+    want = x @ p @ np.diag(signs.astype(np.float64)) @ hb
+    np.testing.assert_allclose(oracle.rpbh_rotate(x, block, perm, signs), want, rtol=0, atol=1e-12)
+    # identity permutation and all-plus signs: the plain block rotation
+    np.testing.assert_allclose(oracle.rpbh_rotate(x, block, np.arange(n), np.ones(n, np.int8)),
+                               oracle.rotate(x, block), rtol=0, atol=1e-13)
+    y = oracle.rpbh_rotate(x, block, perm, signs)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(oracle.rpbh_inverse(y, block, perm, signs), x, rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.rpbh_rotate(x, block, np.zeros(n, np.int64), signs)
+
+
+def test_sphere_cdf_matches_sampled_unit_vectors():
+    """Coordinates of normalized Gaussian vectors (uniform on the sphere)."""
+    rng = np.random.default_rng(3)
+    for d in (3, 16, 256):
+        v = rng.standard_normal((200000, d))
+        t = v[:, 0] / np.linalg.norm(v, axis=1)
+        for q in (-0.5, -0.1, 0.0, 0.05, 0.3):
+            q = q * 3 / np.sqrt(d)
+            assert abs((t <= q).mean() - oracle.sphere_marginal_cdf(q, d)) < 4e-3
+
+
+def test_sphere_first_moment_matches_quadrature():
+    from scipy.integrate import quad
+    from scipy.special import beta
+    for d in (4, 17, 1024):
+        f = lambda t, d=d: (1 - t * t) ** ((d - 3) / 2) / beta(0.5, (d - 1) / 2)   # noqa: E731
+        for a, b in ((-1.0, -0.2), (-0.05, 0.02), (0.01, 1.0)):
+            want, _ = quad(lambda t: t * f(t), a, b, epsabs=1e-14, points=[0.0] if a < 0 < b else None)
+            assert abs(oracle.sphere_partial_first_moment(a, b, d) - want) < 1e-10
+            mass, _ = quad(f, a, b, epsabs=1e-14)
+            got = oracle.sphere_marginal_cdf(b, d) - oracle.sphere_marginal_cdf(a, d)
+            assert abs(got - mass) < 1e-10
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_lloyd_max_of_d3_is_the_uniform_quantizer(bits):
+    """d = 3: one coordinate of a uniform point on the 2-sphere is uniform on
+    [-1, 1] (Archimedes), and the Lloyd-Max quantizer of a uniform density is
+    the uniform one: centroids -1 + (2i + 1) / L, thresholds -1 + 2i / L."""
+    c, t = oracle.sphere_lloyd_max(3, bits)
+    levels = 1 << bits
+    np.testing.assert_allclose(c, -1 + (2 * np.arange(levels) + 1) / levels, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(t, -1 + 2 * np.arange(1, levels) / levels, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("d", [2, 5, 64, 4096])
+def test_one_bit_codebook_is_plus_minus_mean_abs(d):
+    """Two levels: threshold 0 by symmetry, centroids +/- E|T| with
+    E|T| = Gamma(d / 2) / (sqrt(pi) Gamma((d + 1) / 2))."""
+    from scipy.special import gammaln
+    c, t = oracle.sphere_lloyd_max(d, 1)
+    m = np.exp(gammaln(d / 2) - gammaln((d + 1) / 2)) / np.sqrt(np.pi)
+    np.testing.assert_allclose(c, [-m, m], rtol=1e-10)
+    assert abs(t[0]) < 1e-15
+
+
+@pytest.mark.parametrize("d,bits", [(8, 2), (128, 3), (4096, 4), (14336, 4), (4096, 2)])
+def test_lloyd_max_optimality_conditions(d, bits):
+    """Thresholds are the midpoints of adjacent centroids and every centroid
+    is the conditional mean of its cell (cell integrals by quadrature)."""
+    from scipy.integrate import quad
+    from scipy.special import betaln
+    c, t = oracle.sphere_lloyd_max(d, bits)
+    np.testing.assert_allclose(t, 0.5 * (c[:-1] + c[1:]), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(c, -c[::-1], rtol=0, atol=1e-14)
+    logb = betaln(0.5, (d - 1) / 2)
+    f = lambda v: np.exp(((d - 3) / 2) * np.log1p(-v * v) - logb)   # noqa: E731
+    edges = np.concatenate([[-1.0], t, [1.0]])
+    s = 12.0 / np.sqrt(d)          # the density is negligible beyond 12 standard deviations
+    for i in range(len(c)):
+        a, b = max(edges[i], -min(1.0, s)), min(edges[i + 1], min(1.0, s))
+        num, _ = quad(lambda v: v * f(v), a, b, epsabs=1e-16, epsrel=1e-12, limit=200)
+        den, _ = quad(f, a, b, epsabs=1e-16, epsrel=1e-12, limit=200)
+        assert abs(num / den - c[i]) <= 1e-9 * abs(c).max()
+
+
+def test_lloyd_max_large_d_approaches_the_gaussian_quantizer():
+    """sqrt(d) T tends to N(0, 1): the 4-bit codebook times sqrt(d) at
+    d = 10^6 matches a Lloyd-Max quantizer of the standard normal computed
+    here from the normal's own conditional means."""
+    from scipy.stats import norm
+    c, _ = oracle.sphere_lloyd_max(10 ** 6, 4)
+    g = norm.ppf((np.arange(16) + 0.5) / 16)
+    for _ in range(20000):
+        t = np.concatenate([[-np.inf], 0.5 * (g[:-1] + g[1:]), [np.inf]])
+        g = (norm.pdf(t[:-1]) - norm.pdf(t[1:])) / (norm.cdf(t[1:]) - norm.cdf(t[:-1]))
+    np.testing.assert_allclose(c * np.sqrt(10 ** 6), g, rtol=2e-5, atol=2e-5)
+
+
+def test_codebook_quantizer_hand_case_and_packing():
+    """d = 3, 2 bits: centroids -0.75, -0.25, 0.25, 0.75; thresholds -0.5, 0,
+    0.5.  Row (3, 0, 4, -4.5) has norm sqrt(45.25); u = (0.446, 0, 0.595,
+    -0.669): codes 2 (0.446 in (0, 0.5]), 1 (0 takes the lower side), 3, 0."""
+    c, t = oracle.sphere_lloyd_max(3, 2)
+    codes, r = oracle.quantize_codebook(np.array([[3.0, 0.0, 4.0, -4.5]]), c, t)
+    np.testing.assert_array_equal(codes, [[2, 1, 3, 0]])
+    assert r[0] == np.sqrt(45.25)
+    assert oracle.pack_codes(codes, 2).tolist() == [[2 | (1 << 2) | (3 << 4) | (0 << 6)]]
+    assert oracle.pack_codes(np.array([[5, 12]]), 4).tolist() == [[5 | (12 << 4)]]
+    z, rz = oracle.quantize_codebook(np.zeros((1, 4)), c, t)
+    assert rz[0] == 0 and (z == 1).all()       # u = 0 sits on the middle threshold
