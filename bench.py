@@ -12,14 +12,17 @@ Timing: inputs resident in HBM; for C2, 8 buffer sets (input + outputs) are
 rotated so each step touches data last used 7 steps earlier (338 MB > L2).  The K steps
 are captured back to back in one CUDA graph; the graph is replayed once
 untimed and once timed between barriers and device synchronisations.  The
-timed replay and the CUDA events around it are queued on the launching
-stream behind a sleep kernel, so the host's submission of the graph falls
-before the start event and the window holds exactly the K steps, run back
-to back.  `value` = bytes of all ranks / max-over-ranks elapsed time;
+timed graph holds the W untimed warm-up steps, then the K timed steps, with
+CUDA event record nodes inside it: the start event marks the last warm-up
+step's completion (recorded on a side stream, so the first timed step keeps
+its programmatic launch on the warm-up step), the end event follows the K-th
+step.  The window holds exactly the K steps, back to back, and none of the
+host's submission or the graph's launch latency.  `value` = bytes of all ranks / max-over-ranks elapsed time;
 `roofline.achieved` = bytes per launch / mean launch interval (kernel plus
-inter-kernel gap).  Beside it the line reports the same replay with the
+inter-kernel gap).  Beside it the line reports a K-step replay with host-side
 events recorded while the host submits the graph (the window then also holds
-the submission latency) and a median over per-launch event pairs.
+the submission and graph-launch latency) and a median over per-launch event
+pairs.
 `e2e` repeats the metric through hadq_rotate_quant_host (pinned host input,
 copies in and out inside the timed region).
 
@@ -64,7 +67,7 @@ SLEEP_CYCLES = 20_000_000      # ~10 ms of GPU sleep ahead of a timed region
 # launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
 STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"],
               "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"], "c3rb": ["c3rb"], "c5rb": ["c5rb"],
-              "c3k": ["c3k"]}
+              "c3k": ["c3k"], "c2p": ["c2p"], "c2q": ["c2q"]}
 WORKLOAD = W.WORKLOADS["c2"]
 
 
@@ -369,16 +372,30 @@ def run_hadq(args):
     nbuf = n_buffers(cfg, args.rows)
     workers = max(1, min(16, (os.cpu_count() or 2) // 2))
 
-    host, bufs, signs = {}, [], {}
+    host, bufs, signs, rpbh, thr = {}, [], {}, {}, {}
     for k in keys:
+        w = W.WORKLOADS[k]
         host[k], x0 = _device_input(k, W.rank_seed(rank), dev, workers, args.rows)
         bufs.append([x0] + [x0.clone() for _ in range(nbuf - 1)])
-        if W.WORKLOADS[k].signs is not None:
+        if w.signs is not None:
             signs[k] = torch.from_numpy(W.generate_signs(k, W.rank_seed(rank))).to(dev)
+        if w.rpbh:
+            rpbh[k] = tuple(torch.from_numpy(a).to(dev) for a in W.generate_rpbh(k, W.rank_seed(rank)))
+        if w.fmt == "codebook":
+            thr[k] = torch.from_numpy(H.hadq_codebook(w.n, w.group)[1].copy()).to(dev)
 
     def launch(j, i, stream=None, outs=None):
         w = W.WORKLOADS[keys[j]]
         x = bufs[j][i % nbuf]
+        if w.fmt == "codebook":
+            c, nr = (None, None) if outs is None else outs[j][i % nbuf]
+            p, sg = rpbh.get(w.key, (None, None))
+            return H.hadq_rotate_quant_codebook(x, w.group, thr[w.key], w.block, perm=p, signs=sg, codes=c, norms=nr,
+                                                stream=stream)
+        if w.rpbh:
+            c, sc = (None, None) if outs is None else outs[j][i % nbuf]
+            return H.hadq_rotate_quant_rpbh(x, rpbh[w.key][0], rpbh[w.key][1], w.block, w.fmt, w.group, codes=c,
+                                            scales=sc, stream=stream)
         if w.signs is not None:
             c, sc = (None, None) if outs is None else outs[j][i % nbuf]
             return H.hadq_rotate_quant_signed(x, signs[w.key], w.signs, w.block, w.fmt, w.group, codes=c, scales=sc,
@@ -413,19 +430,38 @@ def run_hadq(args):
         g.replay()                       # untimed replay (warm-up of the graph itself)
     stream.synchronize()
 
-    # Timed region: the K steps of one graph replay, between CUDA events on
-    # `stream`.  Events and replay are queued behind a sleep kernel, so the
-    # host's submission of the graph is done before the start event fires and
-    # the window holds the K steps alone, back to back.
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    # Timed region: one graph holds the W untimed warm-up steps, then the K
+    # timed steps, with CUDA events recorded inside the graph (event record
+    # nodes on the launching stream's work).  The start event is recorded on
+    # a side stream forked after the last warm-up step, so it marks that
+    # step's completion while the first timed step keeps its programmatic
+    # launch on the warm-up step, as every later step has on its predecessor;
+    # the end event follows the K-th step.  The window holds exactly the K
+    # steps, each measured from its predecessor's completion to its own, and
+    # none of the host's submission or of the graph's launch latency.
+    t_start = torch.cuda.Event(enable_timing=True, external=True)
+    t_end = torch.cuda.Event(enable_timing=True, external=True)
+    ev_fork = torch.cuda.Event()
+    side = torch.cuda.Stream(device=dev)
+    gt = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gt, stream=stream):
+        for i in range(warm):
+            step(steps + i)
+        ev_fork.record(stream)
+        side.wait_event(ev_fork)
+        t_start.record(side)
+        for i in range(steps):
+            step(i)
+        stream.wait_stream(side)
+        t_end.record(stream)
+    with torch.cuda.stream(stream):
+        gt.replay()                      # untimed replay (warm-up of the graph itself)
+    stream.synchronize()
     barrier(dist)
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
-            torch.cuda._sleep(SLEEP_CYCLES)
-            t_start.record(stream)
-            g.replay()
-            t_end.record(stream)
+            torch.cuda._sleep(SLEEP_CYCLES)   # the host submits the graph while the GPU is held busy
+            gt.replay()
         stream.synchronize()
     barrier(dist)
     elapsed = t_start.elapsed_time(t_end) / 1e3
@@ -463,7 +499,8 @@ def run_hadq(args):
     # device staging and host output buffers, so the copy in of one step runs
     # while the copy out of the previous one drains (PCIe is full duplex).
     e2e = None
-    qkeys = [k for k in keys if W.WORKLOADS[k].fmt is not None and W.WORKLOADS[k].signs is None]
+    qkeys = [k for k in keys if W.WORKLOADS[k].fmt not in (None, "codebook") and W.WORKLOADS[k].signs is None
+             and not W.WORKLOADS[k].rpbh]
     if len(qkeys) == len(keys):
         e2e_steps = max(4, min(steps, 20))
         streams = [stream, torch.cuda.Stream(device=dev)]
@@ -537,9 +574,9 @@ def run_hadq(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                          "traffic": recorded_traffic() if cfg == "c2" and args.rows is None else None,
-                         "duration": "mean launch interval of K back-to-back steps in one CUDA graph "
-                                     "(CUDA events on the launching stream around the graph replay, "
-                                     "queued behind a sleep kernel)",
+                         "duration": "mean interval of K back-to-back steps in one CUDA graph after W untimed "
+                                     "warm-up steps (CUDA event record nodes in the graph: start at the last "
+                                     "warm-up step's completion, end at the K-th step's)",
                          "step_interval_us": interval_max * 1e6,
                          "step_interval_us_host_submit": host_submit_max / steps * 1e6,
                          "step_us_event_pairs_median": step_ev * 1e6},
@@ -550,7 +587,7 @@ def run_hadq(args):
         if world == 1 and cfg == "c2" and args.rows is None and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)
-    del g
+    del g, gt
     if dist is not None:
         dist.destroy_process_group()
 

@@ -18,6 +18,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <utility>
 #include <mutex>
 #include <string>
 #include <tuple>
@@ -193,17 +194,23 @@ hadq_status device_sms(int* sms, int* dev_out) {
   return HADQ_OK;
 }
 
-// Resident CTAs per SM for `fn` at this block/smem size; also raises the
-// dynamic shared memory limit of `fn` on this device when it needs > 48 KB.
+// Resident CTAs per SM for `fn` at this block/smem size.  Also raises the
+// dynamic shared memory limit of `fn` on this device when it needs more than
+// 48 KB; the limit only ever grows (a kernel whose shared memory depends on
+// the call must keep the largest size any earlier call of it needed).
+std::map<std::pair<int, const void*>, int> g_smem_limit;   // (device, fn) -> dynamic smem limit set
+
 hadq_status occupancy(const void* fn, int dev, int block, int smem, int* occ) {
   std::lock_guard<std::mutex> lk(g_mu);
   const auto key = std::make_tuple(dev, fn, block, smem);
   auto it = g_occ.find(key);
   if (it == g_occ.end()) {
     cudaError_t e = cudaSuccess;
-    if (smem > 0) {   // dynamic + static shared memory above 48 KB needs the opt-in
+    int& limit = g_smem_limit[std::make_pair(dev, fn)];
+    if (smem > limit) {
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      limit = smem;
     }
     int v = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, block, smem);
@@ -344,29 +351,64 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
 }
 
 // Blocks of b = K * 2^m elements (one CTA per block, persistent over blocks).
-hadq_status launch_ksize(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0,
-                         void* out1, cudaStream_t stream, int sms, int dev, Signs sg) {
+// What the shared-memory staged kernels need beyond the shape: the RPBH
+// permutation (with n signs) and the codebook thresholds.
+struct Extra {
+  const int32_t* perm = nullptr;
+  const int8_t* rpbh_signs = nullptr;
+  const double* thr = nullptr;
+  int bits = 0;
+};
+
+// Shared-memory staged kernels (hadq_ksize.cuh): blocks of K * 2^m elements,
+// and any power-of-2 block with the RPBH permutation or the codebook
+// quantizer.  A unit is a block, or the whole row when the quantizer needs
+// row statistics (per-token int8, codebook) or the permutation spans the row.
+hadq_status launch_staged(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0,
+                          void* out1, cudaStream_t stream, int sms, int dev, Signs sg, const Extra& ex) {
+  namespace ks = hadq::ksize;
   const bool bf = x_dtype == HADQ_BF16;
-  const bool sgd = sg.side != hadq::SIGNS_NONE;
-  const hl::KsFn fn = hl::ksize_kernel_for(sh.kbase, bf, mode, sgd);
-  if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no K * 2^m kernel for this base order and format");
-  const int64_t smem = hadq::ksize::smem_bytes(sh.b, bf ? 2 : 4, sgd);
-  if (smem > 227 * 1024) return fail(HADQ_ERR_UNSUPPORTED, "K * 2^m block too large for shared memory");
-  const int threads = static_cast<int>(ceil_div(sh.b / 64, 32) * 32);
+  const int sgk = ex.perm != nullptr ? ks::SGK_RPBH : (sg.side != hadq::SIGNS_NONE ? ks::SGK_BLOCK : ks::SGK_NONE);
+  const bool per_row = mode < 0 || mode == hadq::OUT_CODEBOOK || sgk == ks::SGK_RPBH;
+  const int64_t unit = per_row ? sh.n : sh.b;
+  if (unit % 64 != 0 || unit / 64 > ks::kMaxThreads)
+    return fail(HADQ_ERR_UNSUPPORTED, per_row ? "this quantizer / permutation needs n a multiple of 64 and n <= 32768"
+                                              : "K * 2^m blocks need 2^m >= 64 and K * 2^m <= 32768");
+  int shi = 1, logs_lo = sh.logk;
+  if (sh.kbase == 1) {
+    logs_lo = std::min(sh.logb, 11);               // the butterfly stage runs at most 2048 points per column
+    shi = 1 << (sh.logb - logs_lo);
+  }
+  const hl::KsFn fn = hl::staged_kernel_for(sh.kbase, shi, bf, mode, sgk);
+  if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no staged kernel for this size, format and sign variant");
+  const int64_t smem = ks::smem_bytes(unit, bf ? 2 : 4, sgk, sh.b);
+  if (smem > 227 * 1024) return fail(HADQ_ERR_UNSUPPORTED, "row or block too large for the staged kernel's shared memory");
+  const int threads = static_cast<int>(ceil_div(unit / 64, 32) * 32);
   int occ = 0;
   hadq_status st = occupancy(reinterpret_cast<const void*>(fn), dev, threads, static_cast<int>(smem), &occ);
   if (st != HADQ_OK) return st;
-  const int64_t units = sh.rows * (sh.n / sh.b);
-  const int64_t grid = std::min<int64_t>(units, int64_t(sms) * occ);
-  return launch_result(launch_pdl(fn, grid, threads, static_cast<int>(smem), stream, x, units, sh.logk, sh.norm, group,
-                                  out0, out1, sg),
-                       "K * 2^m kernel launch");
+  ks::StageArgs a;
+  a.x = x;
+  a.units = sh.rows * (sh.n / unit);
+  a.unit_len = static_cast<int>(unit);
+  a.b = static_cast<int>(sh.b);
+  a.logs_lo = logs_lo;
+  a.norm = sh.norm;
+  a.group = group;
+  a.bits = ex.bits;
+  a.out0 = out0;
+  a.out1 = out1;
+  a.sg = sgk == ks::SGK_RPBH ? Signs{ex.rpbh_signs, hadq::SIGNS_BEFORE} : sg;
+  a.perm = ex.perm;
+  a.thr = ex.thr;
+  const int64_t grid = std::min<int64_t>(a.units, int64_t(sms) * occ);
+  return launch_result(launch_pdl(fn, grid, threads, static_cast<int>(smem), stream, a), "staged kernel launch");
 }
 
 // Launch the kernel for an already validated call.  mode: hadq::OutMode, or
 // -1 for per-token int8.
 hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode, int group, void* out0, void* out1,
-                   cudaStream_t stream, Signs sg = Signs{nullptr, hadq::SIGNS_NONE}) {
+                   cudaStream_t stream, Signs sg = Signs{nullptr, hadq::SIGNS_NONE}, const Extra& ex = Extra{}) {
   int sms = 0, dev = 0;
   hadq_status st = device_sms(&sms, &dev);
   if (st != HADQ_OK) return st;
@@ -385,7 +427,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours
-  if (sh.kbase > 1) return launch_ksize(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg);
+  if (sh.kbase > 1 || ex.perm != nullptr || mode == hadq::OUT_CODEBOOK)
+    return launch_staged(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg, ex);
   if (g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY) {
     if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
     if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
@@ -471,9 +514,24 @@ hadq_status make_signs(const int8_t* signs, SideArg a, const Shape& sh, const Sp
   return HADQ_OK;
 }
 
+// RPBH: n int32 permutation entries and n int8 signs on the device; they
+// are read while outputs are written, so they must not overlap an output.
+hadq_status make_rpbh(const int32_t* perm, const int8_t* signs, const Shape& sh, const Span* outs, int nouts,
+                      Extra* ex) {
+  if (perm == nullptr || signs == nullptr) return fail(HADQ_ERR_INVALID_ARG, "RPBH needs both perm and signs");
+  if (!aligned16(perm) || !aligned16(signs)) return fail(HADQ_ERR_MISALIGNED, "perm and signs must be 16-byte aligned");
+  const Span sp = span(perm, sh.n * 4), ss = span(signs, sh.n);
+  for (int i = 0; i < nouts; ++i)
+    if (overlaps(sp, outs[i]) || overlaps(ss, outs[i]))
+      return fail(HADQ_ERR_INVALID_ARG, "perm and signs must not overlap an output");
+  ex->perm = perm;
+  ex->rpbh_signs = signs;
+  return HADQ_OK;
+}
+
 hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block, void* out,
                         hadq_dtype out_dtype, void* stream, const int8_t* signs = nullptr,
-                        SideArg side = SideArg{false, kUnsigned}) {
+                        SideArg side = SideArg{false, kUnsigned}, const int32_t* perm = nullptr) {
   g_last_error.clear();
   Shape sh;
   hadq_status st = check_shape(x_dtype, rows, n, block, &sh);
@@ -488,11 +546,12 @@ hadq_status rotate_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t
   const Span so = span(out, rows * n * esize(out_dtype));
   if (overlaps(sx, so) && !(x == out && x_dtype == out_dtype))
     return fail(HADQ_ERR_INVALID_ARG, "out overlaps x (only exact in-place with equal dtypes is allowed)");
-  Signs sg;
-  st = make_signs(signs, side, sh, &so, 1, &sg);
+  Signs sg{nullptr, hadq::SIGNS_NONE};
+  Extra ex;
+  st = perm != nullptr ? make_rpbh(perm, signs, sh, &so, 1, &ex) : make_signs(signs, side, sh, &so, 1, &sg);
   if (st != HADQ_OK) return st;
   return launch(x, x_dtype, sh, out_dtype == HADQ_F32 ? hadq::OUT_F32 : hadq::OUT_BF16, 0, out, nullptr,
-                static_cast<cudaStream_t>(stream), sg);
+                static_cast<cudaStream_t>(stream), sg, ex);
 }
 
 
@@ -526,7 +585,7 @@ int quant_mode(hadq_fmt fmt) {
 hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
                               hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream,
                               const int8_t* signs = nullptr, SideArg side = SideArg{false, kUnsigned},
-                              double tensor_scale = 1.0) {
+                              double tensor_scale = 1.0, const int32_t* perm = nullptr) {
   g_last_error.clear();
   Shape sh;
   int g = 0;
@@ -540,10 +599,44 @@ hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, i
   // normalisation (one rounding, on the host, in double).
   if (fmt == HADQ_NVFP4) sh.norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.b)) / tensor_scale);
   const Span outs[2] = {span(codes, codes_bytes(rows, n, fmt)), span(scales, scales_bytes(rows, n, fmt, g))};
-  Signs sg;
-  st = make_signs(signs, side, sh, outs, 2, &sg);
+  Signs sg{nullptr, hadq::SIGNS_NONE};
+  Extra ex;
+  st = perm != nullptr ? make_rpbh(perm, signs, sh, outs, 2, &ex) : make_signs(signs, side, sh, outs, 2, &sg);
   if (st != HADQ_OK) return st;
-  return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream), sg);
+  return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream), sg, ex);
+}
+
+// The codebook quantizer: per-token norm, nearest centroid of the normalized
+// rotated row; codes bits / 8 bytes per element, one fp32 norm per row.
+hadq_status codebook_impl(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                          const int32_t* perm, const int8_t* signs, int bits, const double* thresholds, void* codes,
+                          float* norms, void* stream) {
+  g_last_error.clear();
+  Shape sh;
+  hadq_status st = check_shape(x_dtype, rows, n, block, &sh);
+  if (st != HADQ_OK) return st;
+  if (bits != 2 && bits != 4) return fail(HADQ_ERR_UNSUPPORTED, "codebook bits must be 2 or 4");
+  if ((perm == nullptr) != (signs == nullptr)) return fail(HADQ_ERR_INVALID_ARG, "give both perm and signs, or neither");
+  if (rows == 0) return HADQ_OK;
+  if (x == nullptr || codes == nullptr || norms == nullptr || thresholds == nullptr)
+    return fail(HADQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(norms) || !aligned16(thresholds))
+    return fail(HADQ_ERR_MISALIGNED, "x, codes, norms and thresholds must be 16-byte aligned");
+  const int64_t cb = rows * n * bits / 8;
+  const Span sx = span(x, rows * n * esize(x_dtype)), sc = span(codes, cb), sn = span(norms, rows * 4);
+  const Span st_thr = span(thresholds, ((int64_t(1) << bits) - 1) * 8);
+  if (overlaps(sx, sc) || overlaps(sx, sn) || overlaps(sc, sn) || overlaps(st_thr, sc) || overlaps(st_thr, sn))
+    return fail(HADQ_ERR_INVALID_ARG, "x, codes, norms and thresholds must not overlap");
+  const Span outs[2] = {sc, sn};
+  Extra ex;
+  if (perm != nullptr) {
+    st = make_rpbh(perm, signs, sh, outs, 2, &ex);
+    if (st != HADQ_OK) return st;
+  }
+  ex.thr = thresholds;
+  ex.bits = bits;
+  return launch(x, x_dtype, sh, hadq::OUT_CODEBOOK, 0, codes, norms, static_cast<cudaStream_t>(stream),
+                Signs{nullptr, hadq::SIGNS_NONE}, ex);
 }
 
 // ----------------------------------------------- allocation-free host path
@@ -611,6 +704,32 @@ hadq_status hadq_rotate_quant_signed(const void* x, hadq_dtype x_dtype, int64_t 
                                      void* codes, void* scales, void* stream) {
   return rotate_quant_impl(x, x_dtype, rows, n, block, fmt, group, codes, scales, stream, signs,
                            SideArg{true, static_cast<int>(side)});
+}
+
+hadq_status hadq_rotate_rpbh(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                             const int32_t* perm, const int8_t* signs, void* out, hadq_dtype out_dtype, void* stream) {
+  if (perm == nullptr && rows > 0) {
+    g_last_error.clear();
+    return fail(HADQ_ERR_INVALID_ARG, "null perm");
+  }
+  return rotate_impl(x, x_dtype, rows, n, block, out, out_dtype, stream, signs, SideArg{false, kUnsigned}, perm);
+}
+
+hadq_status hadq_rotate_quant_rpbh(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                   const int32_t* perm, const int8_t* signs, hadq_fmt fmt, int64_t group, void* codes,
+                                   void* scales, void* stream) {
+  if (perm == nullptr && rows > 0) {
+    g_last_error.clear();
+    return fail(HADQ_ERR_INVALID_ARG, "null perm");
+  }
+  return rotate_quant_impl(x, x_dtype, rows, n, block, fmt, group, codes, scales, stream, signs,
+                           SideArg{false, kUnsigned}, 1.0, perm);
+}
+
+hadq_status hadq_rotate_quant_codebook(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                       const int32_t* perm, const int8_t* signs, int bits, const double* thresholds,
+                                       void* codes, float* norms, void* stream) {
+  return codebook_impl(x, x_dtype, rows, n, block, perm, signs, bits, thresholds, codes, norms, stream);
 }
 
 hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,

@@ -15,7 +15,7 @@
 
 namespace hadq {
 
-enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3, OUT_NVFP4 = 4 };
+enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3, OUT_NVFP4 = 4, OUT_CODEBOOK = 5 };
 
 // Random Hadamard signs ("Rotation Transform", section 1.5: H @ diag(+/-1) /
 // sqrt(N), the signs persisted as int8).  AFTER: output column j of every
@@ -404,17 +404,23 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[N], int e0, flo
   return w;
 }
 
-// Scale arithmetic.  Every scale is a correctly rounded fp32 quotient of
-// the group absmax m: m / 7 (int4, then rounded to fp16), m / 127 (int8) and
-// m / 6 (NVFP4, then rounded to E4M3).  The factor that takes an unnormalised
-// rotated value z to code units is the correctly rounded quotient norm / s, so
-// an int code is the single rounding of the exact product z * (norm / s) onto
-// the integer grid: it can differ from the exactly rounded y / s only through
-// the fp32 rotation's own error and the factor's half-ulp (about 4.5e-7 of a
-// code unit at |y / s| = 7.5).
-__device__ __forceinline__ float int4_scale_f32(float m) { return __fdiv_rn(m, 7.0f); }
+// Scale arithmetic.  The int4 and NVFP4 scales are m * fp32(1/7) and
+// m * fp32(1/6) (within 1.5 ulp of m / 7, m / 6) before their rounding to
+// fp16 / E4M3: the rounded scale can differ from the rounding of the exact
+// quotient only within 2^-23 (relative) of a rounding midpoint of the scale
+// format, where either neighbour is a valid scale.  The int8 scale, stored in
+// fp32, is the correctly rounded quotient m / 127.  The factor that takes an
+// unnormalised rotated value z to code units is the correctly rounded
+// quotient norm / s of the stored scale, so an int code is the single
+// rounding of the exact product z * (norm / s) onto the integer grid: it can
+// differ from the exactly rounded y / s only through the fp32 rotation's own
+// error and the factor's half-ulp (at most 4.5e-7 of a code unit at
+// |y / s| = 7.5).
+constexpr float kInv7 = 1.0f / 7.0f;
+constexpr float kInv6 = 1.0f / 6.0f;
+__device__ __forceinline__ float int4_scale_f32(float m) { return m * kInv7; }
 __device__ __forceinline__ float int8_scale(float m) { return __fdiv_rn(m, 127.0f); }
-__device__ __forceinline__ float nvfp4_scale_f32(float m) { return __fdiv_rn(m, 6.0f); }
+__device__ __forceinline__ float nvfp4_scale_f32(float m) { return m * kInv6; }
 __device__ __forceinline__ float code_factor(float norm, float s) { return __fdiv_rn(norm, s); }
 
 // 32 output bytes at p: one 256-bit store (full 32-byte sectors) when p is

@@ -158,71 +158,150 @@ __device__ __forceinline__ void kstage_column(Get& get, Put& put) {
 
 constexpr int kMaxThreads = 512;
 constexpr int kRunPad = 68;   // words per 64-value run in the shared buffer
+constexpr int kMaxSlo = 2048; // longest butterfly the 2^m stage runs inside one warp
 
-// Bytes of dynamic shared memory for a block of b elements.
-__host__ __device__ constexpr int64_t smem_bytes(int64_t b, int esize, bool sg) {
-  return b * esize + (b / 64) * kRunPad * 4 + (sg ? b : 0) + 32 * 4;
+// Sign variants: none; one sign per block column shared by every block (the
+// random Hadamard of "Rotation Transform", section 1.5); or RPBH, a
+// permutation of the row's columns and one sign per column ("orbitquant
+// 0.2.0", Method Conformance).
+enum StageSigns : int { SGK_NONE = 0, SGK_BLOCK = 1, SGK_RPBH = 2 };
+
+// Everything a launch passes: the row (unit) layout, the rotation block
+// b = K * SHI * S_lo and the quantizer.
+struct StageArgs {
+  const void* x;
+  int64_t units;       // units of unit_len elements, back to back
+  int unit_len;        // elements per unit: a block, or a whole row (per-row quantizers, RPBH)
+  int b;               // rotation block (divides unit_len)
+  int logs_lo;         // log2 S_lo: the butterfly the 2^m stage runs per column
+  float norm;          // 1 / sqrt(b) (NVFP4: also divided by the per-tensor scale)
+  int group;           // int4 group
+  int bits;            // codebook bits (2 or 4)
+  void* out0;
+  void* out1;
+  Signs sg;            // SGK_BLOCK: b signs; SGK_RPBH: unit_len signs
+  const int32_t* perm; // SGK_RPBH: v_e = x_perm[e]
+  const double* thr;   // codebook thresholds (2^bits - 1, ascending)
+};
+
+// Bytes of dynamic shared memory for a unit of u elements.
+__host__ __device__ constexpr int64_t smem_bytes(int64_t u, int esize, int sgk, int64_t b) {
+  return u * esize + (u / 64) * kRunPad * 4 + (sgk == SGK_BLOCK ? b : 0) + 32 * 8 + 16 * 8;
 }
 
-// Blocks of b = K * 2^logs elements (64 <= 2^logs, b / 64 <= kMaxThreads),
-// `units` of them back to back; blockDim.x = b / 64 rounded up to 32.
-// MODE: OutMode, or -1 for per-token int8 (then b = n and a unit is a row).
-template <int K, bool IN_BF16, int MODE, bool SG>
+// Sum over the CTA in double (blockDim.x a multiple of 32, every thread calling).
+__device__ __forceinline__ double cta_sum(double v, double* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  v = lane < nw ? red[lane] : 0.0;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  __syncthreads();
+  return v;
+}
+
+// Codebook index of z: the number of thresholds tau_j = hi_j + lo_j below z
+// (binary search over L - 1 thresholds in shared memory; z - hi_j is exact
+// near the threshold, so the comparison is that of z with tau_j).
+template <int L>
+__device__ __forceinline__ uint32_t codebook_index(float z, const float2* tau) {
+  uint32_t idx = 0;
+#pragma unroll
+  for (int step = L / 2; step >= 1; step >>= 1) {
+    const float2 t = tau[idx + step - 1];
+    if (__fsub_rn(z, t.x) > t.y) idx += step;
+  }
+  return idx;
+}
+
+// Units of unit_len elements; blockDim.x = unit_len / 64 rounded up to 32.
+// MODE: OutMode, or -1 for per-token int8.  K: 1 (Sylvester) or a Paley
+// order; SHI: how many S_lo-long pieces the 2^m factor spans (K = 1 and
+// b > kMaxSlo), mixed in the column stage with the K sub-blocks.
+template <int K, int SHI, bool IN_BF16, int MODE, int SGK>
 __global__ void __launch_bounds__(kMaxThreads)
-ksize_kernel(const void* __restrict__ x, int64_t units, int logs, float norm, int group, void* __restrict__ out0,
-             void* __restrict__ out1, Signs sg) {
+staged_kernel(const __grid_constant__ StageArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int ES = IN_BF16 ? 2 : 4;
-  const int S = 1 << logs;
-  const int b = K * S;
-  const int rps = S >> 6;                      // 64-value runs per sub-block
-  const int runs = K * rps;
-  uint8_t* xs = smem;                          // the staged block
-  float* wbuf = reinterpret_cast<float*>(smem + static_cast<size_t>(b) * ES);
+  constexpr int KH = K * SHI;                  // values mixed per column
+  const int U = a.unit_len, b = a.b;
+  const int slo = 1 << a.logs_lo;
+  const int runs = U >> 6;
+  uint8_t* xs = smem;                          // the staged unit
+  float* wbuf = reinterpret_cast<float*>(smem + static_cast<size_t>(U) * ES);
   int8_t* ssm = reinterpret_cast<int8_t*>(wbuf + static_cast<size_t>(runs) * kRunPad);
-  float* red = reinterpret_cast<float*>(ssm + (SG ? b : 0));
+  double* red = reinterpret_cast<double*>(ssm + (SGK == SGK_BLOCK ? b : 0));
+  float2* tau = reinterpret_cast<float2*>(red + 32);
   const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31;
-  const int64_t block_bytes = static_cast<int64_t>(b) * ES;
+  const int64_t unit_bytes = static_cast<int64_t>(U) * ES;
+  const float norm = a.norm;
 
-  if (tid == 0 && blockIdx.x < units)
-    prefetch_l2(static_cast<const uint8_t*>(x) + blockIdx.x * block_bytes, static_cast<uint32_t>(block_bytes));
+  if (tid == 0 && blockIdx.x < a.units)
+    prefetch_l2(static_cast<const uint8_t*>(a.x) + blockIdx.x * unit_bytes, static_cast<uint32_t>(unit_bytes));
   grid_dependency_sync();
-  if constexpr (SG) {
-    for (int c = tid; c < b / 16; c += T)
-      reinterpret_cast<uint4*>(ssm)[c] = reinterpret_cast<const uint4*>(sg.s)[c];
+  if constexpr (SGK == SGK_BLOCK) {
+    for (int c = tid; c < b / 16; c += T) reinterpret_cast<uint4*>(ssm)[c] = reinterpret_cast<const uint4*>(a.sg.s)[c];
   }
-  const bool before = SG && sg.side == SIGNS_BEFORE;
+  const bool before = SGK == SGK_BLOCK && a.sg.side == SIGNS_BEFORE;
 
-  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
-    const uint8_t* xu = static_cast<const uint8_t*>(x) + u * block_bytes;
-    if (tid == 0 && u + gridDim.x < units)
-      prefetch_l2(xu + gridDim.x * block_bytes, static_cast<uint32_t>(block_bytes));
-    for (int c = tid; c < b * ES / 16; c += T)
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+    const uint8_t* xu = static_cast<const uint8_t*>(a.x) + u * unit_bytes;
+    if (tid == 0 && u + gridDim.x < a.units)
+      prefetch_l2(xu + gridDim.x * unit_bytes, static_cast<uint32_t>(unit_bytes));
+    for (int c = tid; c < U * ES / 16; c += T)
       reinterpret_cast<uint4*>(xs)[c] = ldg_stream(reinterpret_cast<const uint4*>(xu) + c);
-    __syncthreads();   // block staged (and the previous block's runs consumed)
+    __syncthreads();   // unit staged (and the previous unit's runs consumed)
 
-    // ------------------------------------------------------------ K stage
-    for (int j = tid; j < S; j += T) {
-      auto get = [&](int k) {
-        const int e = k * S + j;
+    // ------------------------------------------------------- column stage
+    // Column (blk, j), j < S_lo: the KH values at unit offsets
+    // blk b + (k SHI + h) S_lo + j are permuted / signed as the variant
+    // says, mixed by H_SHI over h and H_K over k, and written to the runs.
+    const int ncols = U / KH;
+    for (int col = tid; col < ncols; col += T) {
+      const int blk = col >> a.logs_lo, j = col & (slo - 1);
+      const int base = blk * b + j;
+      auto get = [&](int kh) {
+        const int e = base + kh * slo;
         float v;
-        if constexpr (IN_BF16) {
-          v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(xs)[e]) << 16);
-        } else {
-          v = reinterpret_cast<const float*>(xs)[e];
+        int src = e;
+        if constexpr (SGK == SGK_RPBH) {   // an entry outside the row is clamped (memory-safe, result unspecified)
+          src = static_cast<int>(min(static_cast<unsigned>(__ldg(a.perm + e)), static_cast<unsigned>(U - 1)));
         }
-        if constexpr (SG) {
-          if (before && ssm[e] < 0) v = -v;
+        if constexpr (IN_BF16) {
+          v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(xs)[src]) << 16);
+        } else {
+          v = reinterpret_cast<const float*>(xs)[src];
+        }
+        if constexpr (SGK == SGK_RPBH) {
+          if (__ldg(a.sg.s + e) < 0) v = -v;
+        } else if constexpr (SGK == SGK_BLOCK) {
+          if (before && ssm[e - blk * b] < 0) v = -v;
         }
         return v;
       };
-      float* wcol = wbuf + (j >> 6) * kRunPad + (j & 63);
-      auto put = [&](int k, float v) { wcol[k * rps * kRunPad] = v; };
-      kstage_column<K>(get, put);
+      auto put = [&](int kh, float v) {
+        const int e = base + kh * slo;
+        wbuf[(e >> 6) * kRunPad + (e & 63)] = v;
+      };
+      if constexpr (K == 1) {
+        float z[SHI];
+#pragma unroll
+        for (int h = 0; h < SHI; ++h) z[h] = get(h);
+        if constexpr (SHI > 1) fwht_bits<SHI, 0, (SHI == 2 ? 1 : 2)>(z);
+#pragma unroll
+        for (int h = 0; h < SHI; ++h) put(h, z[h]);
+      } else {
+        static_assert(SHI == 1, "a Paley base order is mixed with the whole 2^m factor in the butterfly stage");
+        kstage_column<K>(get, put);
+      }
     }
-    __syncthreads();   // every run of the block mixed
+    __syncthreads();   // every run of the unit mixed
 
-    // ---------------------------------------------------------- 2^m stage
+    // ---------------------------------------------------- butterfly stage
     const int r = tid;
     const bool active = r < runs;
     float v[64];
@@ -240,41 +319,95 @@ ksize_kernel(const void* __restrict__ x, int64_t units, int logs, float norm, in
 #pragma unroll
       for (int i = 0; i < 64; ++i) v[i] = 0.f;
     }
-    fwht_bits<64, 0, 6>(v);
-    for (int d = 0; d < logs - 6; ++d) {   // j bits 6 and up: the sub-block's neighbouring lanes
-      const float sgn = ((lane >> d) & 1) ? -1.f : 1.f;
+    if (a.logs_lo >= 6) {
+      fwht_bits<64, 0, 6>(v);
+      for (int d = 0; d < a.logs_lo - 6; ++d) {   // column bits 6 and up: neighbouring lanes
+        const float sgn = ((lane >> d) & 1) ? -1.f : 1.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], 1 << d);
-        v[i] = fmaf(v[i], sgn, o);   // lower lane: own + other; upper lane: other - own
+        for (int i = 0; i < 64; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, v[i], 1 << d);
+          v[i] = fmaf(v[i], sgn, o);   // lower lane: own + other; upper lane: other - own
+        }
       }
+    } else {
+      fwht_low<64>(v, a.logs_lo);      // blocks shorter than a run
     }
-    const int64_t e0 = u * b + static_cast<int64_t>(r) * 64;   // run r holds block columns 64 r ..
-    if constexpr (SG) {
+    const int64_t e0 = u * U + static_cast<int64_t>(r) * 64;   // run r holds unit columns 64 r ..
+    if constexpr (SGK == SGK_BLOCK) {
       if (!before && active) {
-        const uint32_t m[2] = {sign_bits32(ssm, r * 64), sign_bits32(ssm, r * 64 + 32)};
+        const int c0 = (r * 64) % b;
+        uint32_t m[2] = {0u, 0u};
+        if (b >= 64) {
+          m[0] = sign_bits32(ssm, c0);
+          m[1] = sign_bits32(ssm, c0 + 32);
+        } else {   // the run holds 64 / b blocks, each with the same b signs
+          for (int i = 0; i < 64; ++i)
+            if (ssm[i & (b - 1)] < 0) m[i >> 5] |= 1u << (i & 31);
+        }
         apply_signs<64>(v, m);
       }
     }
     if constexpr (MODE == OUT_INT4) {
-      if (group == 128) {
-        store_int4_pair<false>(v, norm, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0, active);
+      if (a.group == 128) {
+        store_int4_pair<false>(v, norm, static_cast<uint8_t*>(a.out0), static_cast<__half*>(a.out1), e0, active);
       } else if (active) {
-        store_int4<false, 64>(v, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
+        store_int4<false, 64>(v, norm, a.group, static_cast<uint8_t*>(a.out0), static_cast<__half*>(a.out1), e0);
       }
     } else if constexpr (MODE == OUT_MXFP4) {
-      if (active) store_mxfp4<false, 64>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+      if (active) store_mxfp4<false, 64>(v, norm, static_cast<uint8_t*>(a.out0), static_cast<uint8_t*>(a.out1), e0);
     } else if constexpr (MODE == OUT_NVFP4) {
-      if (active) store_nvfp4<false, 64>(v, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+      if (active) store_nvfp4<false, 64>(v, norm, static_cast<uint8_t*>(a.out0), static_cast<uint8_t*>(a.out1), e0);
     } else if constexpr (MODE == OUT_BF16) {
-      if (active) store_rotated<false, 64, true>(v, norm, out0, e0);
+      if (active) store_rotated<false, 64, true>(v, norm, a.out0, e0);
     } else if constexpr (MODE == OUT_F32) {
-      if (active) store_rotated<false, 64, false>(v, norm, out0, e0);
+      if (active) store_rotated<false, 64, false>(v, norm, a.out0, e0);
+    } else if constexpr (MODE == OUT_CODEBOOK) {
+      // Per-token norm (double sum of squares of the unnormalised rotation),
+      // then the thresholds in the same units, tau_j = ||z|| t_j, split as an
+      // exact float pair.
+      double ss = 0.0;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) ss = fma(static_cast<double>(v[i]), static_cast<double>(v[i]), ss);
+      const double zn = sqrt(cta_sum(ss, red));
+      const double zs = zn > 0.0 ? zn : 1.0;   // a zero row codes u = 0
+      const int levels = 1 << a.bits;
+      if (tid < levels - 1) {
+        const double t = zs * a.thr[tid];
+        const float hi = static_cast<float>(t);
+        tau[tid] = make_float2(hi, static_cast<float>(t - static_cast<double>(hi)));
+      }
+      if (tid == 0) static_cast<float*>(a.out1)[u] = static_cast<float>(zn * static_cast<double>(norm));
+      __syncthreads();
+      if (active) {
+        uint8_t* codes = static_cast<uint8_t*>(a.out0);
+        if (a.bits == 4) {
+          uint32_t w[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) word |= codebook_index<16>(v[8 * q + i], tau) << (4 * i);
+            w[q] = word;
+          }
+          store32(codes + (e0 >> 1), make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+        } else {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) word |= codebook_index<4>(v[16 * q + i], tau) << (2 * i);
+            w[q] = word;
+          }
+          reinterpret_cast<uint4*>(codes + (e0 >> 2))[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      __syncthreads();   // tau may be rewritten for the next unit
     } else {
       static_assert(MODE == -1, "per-token int8");
-      const float m = cta_max(absmax_regs(v, 0, 64), red) * norm;
-      if (active) store_int8<false, 64>(v, norm, m, static_cast<int8_t*>(out0), e0);
-      if (tid == 0) static_cast<float*>(out1)[u] = int8_scale(m);
+      const float m = cta_max(absmax_regs(v, 0, 64), reinterpret_cast<float*>(red)) * norm;
+      if (active) store_int8<false, 64>(v, norm, m, static_cast<int8_t*>(a.out0), e0);
+      if (tid == 0) static_cast<float*>(a.out1)[u] = int8_scale(m);
     }
   }
 }

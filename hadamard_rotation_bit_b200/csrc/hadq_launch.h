@@ -23,7 +23,12 @@ using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*
 using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, Signs);
 using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*,
                          Signs);
-using KsFn = void (*)(const void*, int64_t, int, float, int, void*, void*, Signs);
+}  // namespace launch
+namespace ksize {
+struct StageArgs;
+}
+namespace launch {
+using KsFn = void (*)(const ksize::StageArgs);
 
 struct TcVariant {
   TcFn fn;
@@ -52,12 +57,14 @@ TeamRowFn team_row_kernel_bf16(int logb, bool sg);
 TcVariant tc_kernel_for(int lo, int mode, int side);   // side: hadq::SignSide
 Tc128Variant tc128_kernel_for(int mode);   // signs of either side folded into B
 
-// Blocks of K * 2^m elements, K a covered Paley order (12, 20, 28, 36, 52, 60,
-// 108); mode -1 = per-token int8.  One unit per input dtype
+// Shared-memory staged kernels: blocks of K * 2^m elements (K a covered Paley
+// order 12 .. 108, or 1 with the RPBH permutation or the codebook quantizer);
+// shi = pieces of the 2^m factor mixed in the column stage; mode -1 =
+// per-token int8; sgk: ksize::StageSigns.  One unit per input dtype
 // (kernels_ksize.cu: fp32 and the dispatch, kernels_ksize_bf16.cu: bf16).
-KsFn ksize_kernel_for(int k, bool bf16, int mode, bool sg);
-KsFn ksize_kernel_f32(int k, int mode, bool sg);
-KsFn ksize_kernel_bf16(int k, int mode, bool sg);
+KsFn staged_kernel_for(int k, int shi, bool bf16, int mode, int sgk);
+KsFn staged_kernel_f32(int k, int shi, int mode, int sgk);
+KsFn staged_kernel_bf16(int k, int shi, int mode, int sgk);
 
 // The tensor-core kernels' sticky fault word (bounded waits that ran out);
 // cleared when `clear` is non-zero.  -1 on a CUDA error.

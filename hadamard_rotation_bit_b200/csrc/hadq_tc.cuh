@@ -42,8 +42,9 @@
 // owns the same 16 chunks of the swizzled tile, so its sign masks are loaded
 // once) and release the stage to the MMA through a second mbarrier.
 // Every mbarrier wait gives up after one second (globaltimer); on timeout the
-// kernel records a fault in hadq_tc_fault, stops issuing work and still
-// releases its tensor memory.
+// kernel records a fault in hadq_tc_fault, stops issuing work, waits (bounded
+// the same way) for the loads and MMAs it already issued, and still releases
+// its tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -56,9 +57,10 @@ constexpr int kABytes = 128 * 128 * 2;     // A operand: H_128 in bf16
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after 1 s
 
 
-template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_, int PREFETCH_ = 2>
+template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_, int PREFETCH_ = 2, bool AHEAD_ = false>
 struct TcCfg {
   static constexpr int PREFETCH = PREFETCH_;             // tiles per CTA prefetched into L2 at entry
+  static constexpr bool AHEAD = AHEAD_;                  // keep the prefetch PREFETCH tiles ahead of the loads
   // Sign-flipping threads (signs before the rotation only): as many as the
   // register budget allows, since they sit between a tile's arrival and its
   // MMA (n = 4096: 60-register epilogue; n = 8192: up to 137 registers).
@@ -205,6 +207,21 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 __device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits that ran out)
 
+// After a wait ran out, what this thread already issued must finish before
+// the CTA exits: a TMA write into shared memory, or an MMA reading it, must
+// not outlive the CTA.  Loads: the full phases of the last min(issued,
+// stages) tiles.  MMAs complete in order, so the stage-release commit of the
+// last issued tile covers all earlier ones.  Every wait is bounded like the
+// others; one that runs out leaves the rest in flight (already a fault).
+__device__ __forceinline__ void drain_loads(uint64_t* full, int stages, uint32_t issued) {
+  for (uint32_t i = issued > static_cast<uint32_t>(stages) ? issued - stages : 0; i < issued; ++i)
+    if (!mbar_wait(&full[i % stages], (i / stages) & 1)) return;
+}
+
+__device__ __forceinline__ void drain_mmas(uint64_t* empty, int stages, uint32_t issued) {
+  if (issued > 0) (void)mbar_wait(&empty[(issued - 1) % stages], ((issued - 1) / stages) & 1);
+}
+
 // Epilogue for one row of one tile: z holds the 2^LO values of TMEM lane hi'
 // (after the tensor-core stage over hi); finish the butterfly over lo and emit.
 // Signs after the rotation (random Hadamard): SGK = 1, output column
@@ -330,10 +347,18 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
         const uint32_t ph = (it / C::STAGES) & 1;
         if (it >= C::STAGES && !mbar_wait(&empty[s], ph ^ 1)) {
           atomicOr(&hadq_tc_fault, kFaultProducer);
+          drain_loads(full, C::STAGES, it);
           break;
         }
         mbar_arrive_expect_tx(&full[s], C::TILE_BYTES);
         tma_load_3d(smem + C::SM_B + s * C::TILE_BYTES, &xmap, 0, 0, static_cast<int>(t * R), &full[s]);
+        if constexpr (C::AHEAD) {
+          const int64_t tp = t + static_cast<int64_t>(C::PREFETCH) * gridDim.x;   // this CTA's tile it + PREFETCH
+          if (tp < tiles) {
+            const int64_t r1 = (tp + 1) * R < rows ? (tp + 1) * R : rows;
+            prefetch_l2(x + tp * R * n, static_cast<uint32_t>((r1 - tp * R) * n * 2));
+          }
+        }
       }
     }
   } else {
@@ -376,6 +401,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           if (!mbar_wait(SB ? &flipped[s] : &full[s], ph) ||
               (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
             atomicOr(&hadq_tc_fault, kFaultMma);
+            drain_mmas(empty, C::STAGES, it);
             break;
           }
           tc_fence_after();

@@ -107,6 +107,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
         const uint32_t ph = (it / C::STAGES) & 1;
         if (it >= C::STAGES && !mbar_wait(&empty[s], ph ^ 1)) {
           atomicOr(&hadq_tc_fault, kFaultProducer);
+          drain_loads(full, C::STAGES, it);
           break;
         }
         mbar_arrive_expect_tx(&full[s], tile_bytes);
@@ -173,6 +174,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
           const uint32_t aph = (it / C::ACC_BUFS) & 1;
           if (!mbar_wait(&full[s], ph) || (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
             atomicOr(&hadq_tc_fault, kFaultMma);
+            drain_mmas(empty, C::STAGES, it);
             break;
           }
           tc_fence_after();

@@ -1,7 +1,10 @@
-// Instantiations of the K * 2^m rotation kernels (non-power-of-2 blocks) for
-// one input dtype, and their lookup.  The unit is compiled twice: with
+// Instantiations of the shared-memory staged kernels (hadq_ksize.cuh) for one
+// input dtype, and their lookup.  The unit is compiled twice: with
 // HADQ_KSIZE_BF16 for bf16 input (kernels_ksize_bf16.cu) and without it for
-// fp32 input.
+// fp32 input.  Instantiated: every Paley base order K with the plain and
+// block-signed rotations, all formats and the codebook quantizer; the pure
+// Sylvester blocks (K = 1, SHI = 1, 2, 4) with the RPBH permutation and the
+// codebook quantizer, the variants no other kernel family covers.
 #include "hadq_ksize.cuh"
 #include "hadq_launch.h"
 
@@ -13,48 +16,74 @@ namespace hadq {
 namespace launch {
 namespace {
 
+using ksize::SGK_BLOCK;
+using ksize::SGK_NONE;
+using ksize::SGK_RPBH;
+using ksize::staged_kernel;
 constexpr bool kBf16 = HADQ_KSIZE_BF16 != 0;
 
-template <int K, bool SG>
-KsFn ks_mode(int mode) {
+template <int K, int SHI, int SGK>
+KsFn with_mode(int mode) {
   switch (mode) {
-    case OUT_F32: return &ksize::ksize_kernel<K, kBf16, OUT_F32, SG>;
-    case OUT_BF16: return &ksize::ksize_kernel<K, kBf16, OUT_BF16, SG>;
-    case OUT_INT4: return &ksize::ksize_kernel<K, kBf16, OUT_INT4, SG>;
-    case OUT_MXFP4: return &ksize::ksize_kernel<K, kBf16, OUT_MXFP4, SG>;
-    case OUT_NVFP4: return &ksize::ksize_kernel<K, kBf16, OUT_NVFP4, SG>;
-    case -1: return &ksize::ksize_kernel<K, kBf16, -1, SG>;
+    case OUT_F32: return &staged_kernel<K, SHI, kBf16, OUT_F32, SGK>;
+    case OUT_BF16: return &staged_kernel<K, SHI, kBf16, OUT_BF16, SGK>;
+    case OUT_INT4: return &staged_kernel<K, SHI, kBf16, OUT_INT4, SGK>;
+    case OUT_MXFP4: return &staged_kernel<K, SHI, kBf16, OUT_MXFP4, SGK>;
+    case OUT_NVFP4: return &staged_kernel<K, SHI, kBf16, OUT_NVFP4, SGK>;
+    case -1: return &staged_kernel<K, SHI, kBf16, -1, SGK>;
     default: return nullptr;
   }
 }
 
-template <int K>
-KsFn ks_sign(int mode, bool sg) {
-  return sg ? ks_mode<K, true>(mode) : ks_mode<K, false>(mode);
+template <int K, int SHI>
+KsFn pick(int mode, int sgk) {
+  if (mode == OUT_CODEBOOK) {
+    if (sgk == SGK_NONE) return &staged_kernel<K, SHI, kBf16, OUT_CODEBOOK, SGK_NONE>;
+    if constexpr (K == 1) {
+      if (sgk == SGK_RPBH) return &staged_kernel<K, SHI, kBf16, OUT_CODEBOOK, SGK_RPBH>;
+    }
+    return nullptr;
+  }
+  if constexpr (K == 1) {
+    return sgk == SGK_RPBH ? with_mode<K, SHI, SGK_RPBH>(mode) : nullptr;
+  } else {
+    if (sgk == SGK_NONE) return with_mode<K, SHI, SGK_NONE>(mode);
+    if (sgk == SGK_BLOCK) return with_mode<K, SHI, SGK_BLOCK>(mode);
+    return nullptr;
+  }
 }
 
 }  // namespace
 
 #if HADQ_KSIZE_BF16
-KsFn ksize_kernel_bf16(int k, int mode, bool sg) {
+KsFn staged_kernel_bf16(int k, int shi, int mode, int sgk) {
 #else
-KsFn ksize_kernel_f32(int k, int mode, bool sg) {
+KsFn staged_kernel_f32(int k, int shi, int mode, int sgk) {
 #endif
+  if (k == 1) {
+    switch (shi) {
+      case 1: return pick<1, 1>(mode, sgk);
+      case 2: return pick<1, 2>(mode, sgk);
+      case 4: return pick<1, 4>(mode, sgk);
+      default: return nullptr;
+    }
+  }
+  if (shi != 1) return nullptr;
   switch (k) {
-    case 12: return ks_sign<12>(mode, sg);
-    case 20: return ks_sign<20>(mode, sg);
-    case 28: return ks_sign<28>(mode, sg);
-    case 36: return ks_sign<36>(mode, sg);
-    case 52: return ks_sign<52>(mode, sg);
-    case 60: return ks_sign<60>(mode, sg);
-    case 108: return ks_sign<108>(mode, sg);
+    case 12: return pick<12, 1>(mode, sgk);
+    case 20: return pick<20, 1>(mode, sgk);
+    case 28: return pick<28, 1>(mode, sgk);
+    case 36: return pick<36, 1>(mode, sgk);
+    case 52: return pick<52, 1>(mode, sgk);
+    case 60: return pick<60, 1>(mode, sgk);
+    case 108: return pick<108, 1>(mode, sgk);
     default: return nullptr;
   }
 }
 
 #if !HADQ_KSIZE_BF16
-KsFn ksize_kernel_for(int k, bool bf16, int mode, bool sg) {
-  return bf16 ? ksize_kernel_bf16(k, mode, sg) : ksize_kernel_f32(k, mode, sg);
+KsFn staged_kernel_for(int k, int shi, bool bf16, int mode, int sgk) {
+  return bf16 ? staged_kernel_bf16(k, shi, mode, sgk) : staged_kernel_f32(k, shi, mode, sgk);
 }
 #endif
 

@@ -30,7 +30,8 @@ EXPORTS = (
     "hadq_rotate", "hadq_rotate_inverse", "hadq_rotate_quant", "hadq_rotate_quant_host",
     "hadq_codes_bytes", "hadq_scales_bytes", "hadq_status_string", "hadq_last_error", "hadq_version",
     "hadq_device_faults", "hadq_rotate_quant_host_static", "hadq_rotate_signed", "hadq_rotate_quant_signed",
-    "hadq_rotate_quant_nvfp4", "hadq_set_impl", "hadq_get_impl",
+    "hadq_rotate_quant_nvfp4", "hadq_set_impl", "hadq_get_impl", "hadq_codebook",
+    "hadq_rotate_rpbh", "hadq_rotate_quant_rpbh", "hadq_rotate_quant_codebook",
 )
 IMPLS = {"auto": 0, "butterfly": 1, "tensor": 2}
 
@@ -84,6 +85,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hadq_set_impl.restype = i32
         lib.hadq_get_impl.argtypes = []
         lib.hadq_get_impl.restype = i32
+        lib.hadq_codebook.argtypes = [i64, i32, vp, vp]
+        lib.hadq_codebook.restype = i32
+        lib.hadq_rotate_rpbh.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i32, vp]
+        lib.hadq_rotate_rpbh.restype = i32
+        lib.hadq_rotate_quant_rpbh.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, i64, vp, vp, vp]
+        lib.hadq_rotate_quant_rpbh.restype = i32
+        lib.hadq_rotate_quant_codebook.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, vp, vp, vp, vp]
+        lib.hadq_rotate_quant_codebook.restype = i32
         _lib = lib
         return lib
 
@@ -171,6 +180,17 @@ def hadq_set_impl(impl: str) -> str:
 def hadq_get_impl() -> str:
     code = int(load_library().hadq_get_impl())
     return {v: k for k, v in IMPLS.items()}[code]
+
+
+def hadq_codebook(d: int, bits: int):
+    """The library's unit-sphere Lloyd-Max codebook for rows of length d:
+    (centroids, thresholds) as float64 numpy arrays (see include/hadq.h)."""
+    import numpy as np
+    lib = load_library()
+    c = np.empty(1 << bits, dtype=np.float64)
+    t = np.empty(max(1, (1 << bits) - 1), dtype=np.float64)
+    _check(lib.hadq_codebook(int(d), int(bits), c.ctypes.data, t.ctypes.data))
+    return c, t[: (1 << bits) - 1]
 
 
 def codes_nbytes(rows: int, n: int, fmt: str) -> int:
@@ -340,3 +360,78 @@ def hadq_rotate_quant_nvfp4(x: torch.Tensor, tensor_scale: float = 1.0, block: i
     _check(lib.hadq_rotate_quant_nvfp4(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, float(tensor_scale),
                                        codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
     return codes, scales
+
+
+def _rpbh_ptrs(perm, signs, dev, n):
+    if perm is None or signs is None:
+        raise HadqError(HADQ_ERR_INVALID_ARG, "RPBH needs perm (int32) and signs (int8)")
+    if perm.dtype != torch.int32 or signs.dtype != torch.int8:
+        raise HadqError(HADQ_ERR_INVALID_ARG, "perm must be int32 and signs int8")
+    for name, t, nb in (("perm", perm, 4 * n), ("signs", signs, n)):
+        _on_device(name, t, dev)
+        _holds(name, t, nb)
+    return perm.data_ptr(), signs.data_ptr()
+
+
+def hadq_rotate_rpbh(x: torch.Tensor, perm: torch.Tensor, signs: torch.Tensor, block: int = 0,
+                     out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
+    """RPBH rotation: x[..., perm] * signs, then the block rotation (see include/hadq.h)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
+    pp, sp = _rpbh_ptrs(perm, signs, x.device, n)
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _on_device("out", out, x.device)
+    _holds("out", out, rows * n * out.element_size())
+    _check(lib.hadq_rotate_rpbh(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, pp, sp, out.data_ptr(),
+                                _dtype_code(out.dtype), _stream_handle(stream)))
+    return out
+
+
+def hadq_rotate_quant_rpbh(x: torch.Tensor, perm: torch.Tensor, signs: torch.Tensor, block: int = 0,
+                           fmt: str = "int4", group: int = 128, codes: torch.Tensor | None = None,
+                           scales: torch.Tensor | None = None, stream=None):
+    """RPBH rotation and quantization in one pass; returns (codes, scales)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
+    pp, sp = _rpbh_ptrs(perm, signs, x.device, n)
+    cs, cd, ss, sd = output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=x.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=x.device)
+    _quant_outputs(lib, rows, n, fmt, group, codes, scales, x.device)
+    _check(lib.hadq_rotate_quant_rpbh(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, pp, sp, FMTS[fmt], group,
+                                      codes.data_ptr(), scales.data_ptr(), _stream_handle(stream)))
+    return codes, scales
+
+
+def hadq_rotate_quant_codebook(x: torch.Tensor, bits: int, thresholds: torch.Tensor, block: int = 0,
+                               perm: torch.Tensor | None = None, signs: torch.Tensor | None = None,
+                               codes: torch.Tensor | None = None, norms: torch.Tensor | None = None, stream=None):
+    """Per-token norm + nearest-centroid codes of the (RPBH or plain) rotation;
+    ``thresholds``: float64 device tensor of 2^bits - 1 decision boundaries
+    (e.g. from hadq_codebook(n, bits)).  Returns (codes uint8, norms fp32)."""
+    lib = load_library()
+    rows, n = _rows_n(x)
+    _on_device("x", x, x.device)
+    pp = sp = None
+    if perm is not None or signs is not None:
+        pp, sp = _rpbh_ptrs(perm, signs, x.device, n)
+    if thresholds.dtype != torch.float64:
+        raise HadqError(HADQ_ERR_INVALID_ARG, "thresholds must be float64")
+    _on_device("thresholds", thresholds, x.device)
+    _holds("thresholds", thresholds, ((1 << bits) - 1) * 8)
+    if codes is None:
+        codes = torch.empty((rows, n * bits // 8), dtype=torch.uint8, device=x.device)
+    if norms is None:
+        norms = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    for name, t, nb in (("codes", codes, rows * n * bits // 8), ("norms", norms, rows * 4)):
+        _on_device(name, t, x.device)
+        _holds(name, t, nb)
+    _check(lib.hadq_rotate_quant_codebook(x.data_ptr(), _dtype_code(x.dtype), rows, n, block, pp, sp, int(bits),
+                                          thresholds.data_ptr(), codes.data_ptr(), norms.data_ptr(),
+                                          _stream_handle(stream)))
+    return codes, norms

@@ -28,6 +28,11 @@ permutation drawn from a ``seed + 1`` stream):
   draws (``generate_signs``), int8 +/-1.
 * ``c3rb`` / ``c5rb``  the ``c3`` / ``c5`` input and quantizer with signs
   before the rotation (block 128 / full 8192).
+* ``c2p`` / ``c2q``  the ``c2`` input through orbitquant's RPBH rotation (a
+  seeded random permutation of the 4096 columns and 4096 Rademacher signs,
+  ``generate_rpbh``, then the full 4096-point rotation), quantized to int4 g128
+  (``c2p``) or by the per-token norm and the 4-bit unit-sphere Lloyd-Max
+  codebook (``c2q``, "orbitquant 0.2.0", Method Conformance).
 * ``c3k``  the ``c3`` input rotated in full instead of by blocks of 128: the
   14336-point rotation of a non-power-of-2 size ("Rotation Transform",
   section 1.5: 14336 = 28 * 2^9, a base matrix of order 28 with a Sylvester
@@ -60,6 +65,7 @@ class Workload:
     out_dtype: str | None = None   # rotation-only output dtype
     signs: str | None = None       # random Hadamard: "after" | "before" | None (deterministic)
     base: str | None = None        # input recipe of another workload (same bits)
+    rpbh: bool = False             # RPBH: a column permutation and n signs ahead of the block rotation
 
     @property
     def in_bytes(self) -> int:
@@ -78,6 +84,8 @@ class Workload:
             return r * n // 2 + r * (n // 32)
         if self.fmt == "nvfp4":
             return r * n // 2 + r * (n // 16)
+        if self.fmt == "codebook":       # group = bits per code; one fp32 norm per row
+            return r * n * self.group // 8 + r * 4
         raise ValueError(self.fmt)
 
     @property
@@ -112,6 +120,11 @@ WORKLOADS = {
                     "(x) 512-point Sylvester), int8 per token", 8192, 14336, 14336, "bf16", "int8", 0, base="c3"),
     "c3rb": Workload("c3rb", "R4 8192 tokens x intermediate 14336 bf16, block 128 random Hadamard transpose "
                      "(signs before), int8 per token", 8192, 14336, 128, "bf16", "int8", 0, signs="before", base="c3"),
+    "c2p": Workload("c2p", "R1 4096 tokens x hidden 4096 bf16, RPBH (random column permutation, n signs, full "
+                    "4096-point Hadamard), int4 sym g128 fp16 scales", 4096, 4096, 4096, "bf16", "int4", 128,
+                    base="c2", rpbh=True),
+    "c2q": Workload("c2q", "R1 4096 tokens x hidden 4096 bf16, RPBH (full 4096-point), per-token norm + 4-bit "
+                    "unit-sphere Lloyd-Max codebook", 4096, 4096, 4096, "bf16", "codebook", 4, base="c2", rpbh=True),
     "c5rb": Workload("c5rb", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point random Hadamard "
                      "transpose (signs before), MXFP4", 65536, 8192, 8192, "bf16", "mxfp4", 32, signs="before",
                      base="c5"),
@@ -128,6 +141,21 @@ def generate_signs(key: str, seed: int = SEED) -> np.ndarray:
         raise ValueError(f"{key} has no random Hadamard signs")
     g = _rng(seed, _SIGN_STREAM, _STREAM[w.base or key])
     return np.where(g.random(w.block) < 0.5, -1, 1).astype(np.int8)
+
+
+_RPBH_STREAM = 200
+
+
+def generate_rpbh(key: str, seed: int = SEED):
+    """The RPBH permutation (int32, a shuffle of the n columns) and its n int8
+    Rademacher signs for an RPBH workload."""
+    w = WORKLOADS[key]
+    if not w.rpbh:
+        raise ValueError(f"{key} has no RPBH permutation")
+    g = _rng(seed, _RPBH_STREAM, _STREAM[w.base or key])
+    perm = g.permutation(w.n).astype(np.int32)
+    signs = np.where(g.random(w.n) < 0.5, -1, 1).astype(np.int8)
+    return perm, signs
 
 
 def _rng(seed: int, stream: int, chunk: int) -> np.random.Generator:

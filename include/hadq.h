@@ -20,9 +20,14 @@
  *     16-byte aligned (HADQ_ERR_MISALIGNED otherwise).
  *   - Rows are contiguous with stride n elements.
  *   - rows == 0 is a valid empty call: nothing is launched, HADQ_OK.
- *   - Supported sizes: 1 <= b <= 8192, b a power of 2; n a multiple of 8
- *     and of b; a full rotation needs n itself to be a power of 2 <= 8192.
- *     Larger b returns HADQ_ERR_UNSUPPORTED.
+ *   - Supported sizes: n a multiple of 8 and of b, with b either a power of
+ *     2, 1 <= b <= 8192, or b = K * 2^m, K in {12, 20, 28, 36, 52, 60, 108},
+ *     2^m >= 64, b <= 32768 (the non-power-of-2 sizes of "Rotation
+ *     Transform" section 1.5: H_b = H_K (x) H_(2^m), H_K the Paley II
+ *     Hadamard matrix of order K -- the page names these K but prints no
+ *     matrix, so this is the construction used).  Other sizes return
+ *     HADQ_ERR_UNSUPPORTED (a K * 2^m size) or HADQ_ERR_INVALID_ARG (no
+ *     Hadamard matrix of that order here).
  *   - The caller owns every buffer; the library allocates nothing.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  The caller synchronizes before reading results.
@@ -127,8 +132,12 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  *                  codes:  [rows x n/2] bytes, element 2i in the low nibble.
  *                  scales: [rows x n/16] E4M3 bytes.
  *
- * Codes are computed from the fp32 rotation with the stored scale; the
- * product y * (1/s) is rounded once (fused multiply-add onto the integer grid).
+ * Codes are computed from the fp32 rotation z (y = z / sqrt(b)) with the
+ * stored scale s: the factor f = (1/sqrt(b)) / s is a correctly rounded fp32
+ * quotient, and the exact product z * f is rounded once onto the integer grid
+ * (int4, int8; a fused multiply-add) or onto fp32 and then to E2M1 (MXFP4,
+ * NVFP4).  Scales are correctly rounded fp32 quotients m / 7, m / 127, m / 6
+ * before their rounding to fp16 / E4M3.
  * codes and scales must not overlap x or each other.
  */
 HADQ_API hadq_status hadq_rotate_quant(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
@@ -178,6 +187,59 @@ HADQ_API hadq_status hadq_rotate_quant_signed(const void* x, hadq_dtype x_dtype,
                                               hadq_fmt fmt, int64_t group, void* codes, void* scales, void* stream);
 
 /*
+ * RPBH rotation ("orbitquant 0.2.0", Method Conformance: RPBH permutation,
+ * Rademacher signs, block FWHT and orthonormal scaling).  For every row,
+ *     v_e = x[perm[e]] * s_e          (e = 0 .. n - 1),
+ *     out = v . diag(H_b, ..., H_b) / sqrt(b),
+ * i.e. the columns are gathered through the permutation, signed, and rotated
+ * block by block as hadq_rotate does.
+ *   perm    device pointer to n int32: a permutation of 0 .. n - 1 (the page
+ *           gives no rule for choosing it; the caller supplies it).  Entries
+ *           outside 0 .. n - 1 are clamped: memory-safe, result unspecified.
+ *   signs   device pointer to n int8, one per column; negative = -1.
+ *   block   0 / n = full, else a power of 2 dividing n, or K * 2^m as for
+ *           hadq_rotate; n must be a multiple of 64 and at most 32768.
+ * perm and signs are 16-byte aligned and must not overlap an output; x and
+ * out may be the same buffer (equal dtypes).  Other rules as hadq_rotate /
+ * hadq_rotate_quant.  hadq_rotate_quant_rpbh quantizes the RPBH rotation
+ * with any hadq_fmt.
+ */
+HADQ_API hadq_status hadq_rotate_rpbh(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                      const int32_t* perm, const int8_t* signs, void* out, hadq_dtype out_dtype,
+                                      void* stream);
+
+HADQ_API hadq_status hadq_rotate_quant_rpbh(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n, int64_t block,
+                                            const int32_t* perm, const int8_t* signs, hadq_fmt fmt, int64_t group,
+                                            void* codes, void* scales, void* stream);
+
+/*
+ * hadq_rotate_quant_codebook: orbitquant's online activation quantizer
+ * ("orbitquant 0.2.0", Method Conformance: online per-token norm, normalized
+ * activation rotation, nearest-centroid quantization, rescaling).  For every
+ * row, y = the rotation (RPBH when perm and signs are given, else the plain
+ * block rotation of hadq_rotate), r = ||y||_2, and element e codes the index
+ * of the nearest centroid of y_e / r: the number of thresholds strictly below
+ * it (the thresholds are the midpoints of adjacent centroids; a value exactly
+ * on one takes the lower index).  Dequantization is r * centroid[code].
+ *   bits        2 or 4
+ *   thresholds  device pointer to 2^bits - 1 ascending doubles, usually
+ *               those hadq_codebook(n, bits) returns (the codebook for rows
+ *               of length n), copied to the device by the caller
+ *   codes       [rows x n * bits / 8] bytes; code i of a byte in bits
+ *               [i * bits, (i + 1) * bits), element 0 lowest
+ *   norms       [rows] fp32: r
+ *   perm, signs both null (plain rotation) or both given (RPBH, as above)
+ * n must be a multiple of 64 and at most 32768.  The norm is accumulated in
+ * double and the comparison of y_e with r * t_j is exact for the fp32 y_e,
+ * so a code differs from the exactly computed one only through the fp32
+ * rotation's own rounding.  Buffers 16-byte aligned, no overlaps; other
+ * rules as hadq_rotate_quant.
+ */
+HADQ_API hadq_status hadq_rotate_quant_codebook(const void* x, hadq_dtype x_dtype, int64_t rows, int64_t n,
+                                                int64_t block, const int32_t* perm, const int8_t* signs, int bits,
+                                                const double* thresholds, void* codes, float* norms, void* stream);
+
+/*
  * hadq_rotate_quant_host: the same operation on HOST buffers.  Enqueues on
  * `stream`: copy x_host -> x_dev, hadq_rotate_quant on the device buffers,
  * copy codes_dev -> codes_host and scales_dev -> scales_host.  The caller
@@ -221,6 +283,24 @@ HADQ_API hadq_status hadq_rotate_quant_host(const void* x_host, hadq_dtype x_dty
 HADQ_API hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtype x_dtype, int64_t rows, int64_t n,
                                                    int64_t block, hadq_fmt fmt, int64_t group, void* codes_host,
                                                    void* scales_host, void* stream);
+
+/*
+ * hadq_codebook: the unit-sphere Lloyd-Max codebook of "orbitquant 0.2.0"
+ * (Features: exact unit-sphere Lloyd-Max codebooks; Method Conformance: one
+ * fixed codebook per input dimension and bit width).  A rotated, normalized
+ * row behaves as a uniform unit vector in R^d; one coordinate then has the
+ * density (1 - t^2)^((d - 3) / 2) on [-1, 1] (normalized), and the codebook
+ * is the minimum mean-square-error quantizer of that density with 2^bits
+ * levels (Lloyd's iteration, in double precision, on the host).
+ *   d           the row length the codebook serves (>= 2)
+ *   bits        1 .. 8
+ *   centroids   host array of 2^bits doubles, ascending (written)
+ *   thresholds  host array of 2^bits - 1 doubles: the midpoints of adjacent
+ *               centroids, the decision boundaries (written)
+ * Synchronous, no CUDA call, nothing allocated on the device.
+ * HADQ_ERR_INVALID_ARG for a bad d, bits or a null pointer.
+ */
+HADQ_API hadq_status hadq_codebook(int64_t d, int bits, double* centroids, double* thresholds);
 
 /* Bytes of the code and scale outputs of hadq_rotate_quant for these sizes
  * (0 for an invalid combination). */

@@ -206,6 +206,41 @@ def check_nvfp4(x64, codes_packed, scales_e4m3, block: int, y=None, tensor_scale
             "code_differs_in_window": int((got != enc(v)).sum())}
 
 
+def unpack_codes(packed, bits: int) -> np.ndarray:
+    """8 // bits codes per byte, code i in bits [i * bits, (i + 1) * bits)."""
+    p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    per = 8 // bits
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * per,), dtype=np.int64)
+    for i in range(per):
+        out[..., i::per] = (p >> (bits * i)) & ((1 << bits) - 1)
+    return out
+
+
+def check_codebook(x64, codes_packed, norms, block: int, bits: int, y=None) -> dict:
+    """Codebook quantizer: norms within 1e-6 relative of ||y||; codes the
+    oracle's nearest centroid of y / ||y|| (its own Lloyd-Max codebook for
+    d = n), except within 1e-6 of a decision threshold in code units -- the
+    distance between the two centroids that threshold separates."""
+    y = oracle.rotate(x64, block) if y is None else y
+    rows, n = y.shape
+    c, t = oracle.sphere_lloyd_max(n, bits)
+    q_o, r_o = oracle.quantize_codebook(y, c, t)
+    r_gpu = np.asarray(norms, dtype=np.float32).astype(np.float64).reshape(rows)
+    rel = np.abs(r_gpu - r_o) / np.where(r_o > 0, r_o, 1.0)
+    assert (rel <= 1e-6).all() and ((r_o == 0) == (r_gpu == 0)).all(), f"norm rel err {rel.max():.3e}"
+    u = y / np.where(r_o > 0, r_o, 1.0)[:, None]
+    j = np.abs(u[..., None] - t).argmin(axis=-1)          # nearest threshold
+    w = WINDOW * (c[j + 1] - c[j])
+    got = unpack_codes(codes_packed, bits).reshape(rows, n)
+
+    def enc(v):
+        return np.searchsorted(t, v, side="left")
+    ok, boundary = _check_codes(got, u, w, enc)
+    assert ok.all(), f"{(~ok).sum()} codebook codes differ outside the boundary window"
+    return {"elements": int(y.size), "rows": rows, "worst_norm_rel_err": float(rel.max()),
+            "code_boundary_cases": int(boundary.sum()), "code_differs_in_window": int((got != q_o).sum())}
+
+
 def check(fmt, x64, out0, out1, block, group, y=None):
     """``y``: the oracle's rotation when it is not ``oracle.rotate(x64, block)``
     (e.g. a random Hadamard rotation)."""

@@ -5,7 +5,8 @@
 Each configuration runs through the C ABI at full size, in the default
 implementation choice (the launches bench.py times), and is compared element
 by element with the float64 oracle by tests/parity_check.py, the only
-checker.  The oracle sees every row of c1, c2, c3, c2r, c2rb, c3rb, c2n and c3k;
+checker.  The oracle sees every row of c1, c2, c3, c2r, c2rb, c3rb, c2n, c3k,
+c2p and c2q;
 for c4, c5, c5rb and c5n it sees a seeded row sample (first and last rows,
 random rows and, for c5, the rows with the largest inputs), as the GPU tests
 do.  A failing comparison raises, so a written record means every compared
@@ -47,7 +48,7 @@ from hadamard_rotation_bit_b200 import workloads as W  # noqa: E402
 from tests import parity_check as pc  # noqa: E402
 
 NPROC = max(1, min(16, (os.cpu_count() or 2) // 2))
-CONFIGS = ["c1", "c2", "c3", "c4", "c5", "c2r", "c2rb", "c3rb", "c5rb", "c2n", "c5n", "c3k"]
+CONFIGS = ["c1", "c2", "c3", "c4", "c5", "c2r", "c2rb", "c3rb", "c5rb", "c2n", "c5n", "c3k", "c2p", "c2q"]
 
 
 def _dev(stored, x_dtype):
@@ -60,7 +61,16 @@ def _gpu(key, stored):
     """The call bench.py makes for this workload part; host copies of its outputs."""
     w = W.WORKLOADS[key]
     x = _dev(stored, w.x_dtype)
-    if w.fmt is None:
+    if w.fmt == "codebook" or w.rpbh:
+        p, sg = (torch.from_numpy(a).cuda() for a in W.generate_rpbh(key)) if w.rpbh else (None, None)
+        if w.fmt == "codebook":
+            thr = torch.from_numpy(H.hadq_codebook(w.n, w.group)[1].copy()).cuda()
+            c, sc = H.hadq_rotate_quant_codebook(x, w.group, thr, w.block, perm=p, signs=sg)
+        else:
+            c, sc = H.hadq_rotate_quant_rpbh(x, p, sg, w.block, w.fmt, w.group)
+        torch.cuda.synchronize()
+        res = (c.cpu().numpy(), sc.cpu().numpy())
+    elif w.fmt is None:
         out = H.hadq_rotate(x, w.block, out_dtype=torch.bfloat16 if w.out_dtype == "bf16" else torch.float32)
         torch.cuda.synchronize()
         res = (out.view(torch.int16).cpu().numpy().view(np.uint16) if w.out_dtype == "bf16" else out.cpu().numpy(),)
@@ -96,8 +106,15 @@ def _record_part(key, ids=None):
     if w.fmt is None:
         rep = pc.check_rotation_bf16(x64, out[0][ids], w.block)
     else:
-        y = oracle.rotate_signed(x64, w.block, W.generate_signs(key), w.signs) if w.signs else None
-        rep = pc.check(w.fmt, x64, out[0][ids], out[1][ids], w.block, w.group, y=y)
+        y = None
+        if w.signs:
+            y = oracle.rotate_signed(x64, w.block, W.generate_signs(key), w.signs)
+        if w.rpbh:
+            y = oracle.rpbh_rotate(x64, w.block, *W.generate_rpbh(key))
+        if w.fmt == "codebook":
+            rep = pc.check_codebook(x64, out[0][ids], out[1][ids], w.block, w.group, y=y)
+        else:
+            rep = pc.check(w.fmt, x64, out[0][ids], out[1][ids], w.block, w.group, y=y)
     rep["rows_checked"] = int(len(ids))
     rep["rows_total"] = int(w.rows)
     rep["workload"] = w.name

@@ -10,6 +10,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from hadamard_rotation_bit_b200 import build as hbuild
@@ -249,3 +251,27 @@ def test_k_size_shape_rules(lib):
     assert f(a, bf, 0, 3 * 28 * 64, 28 * 64, i8, 0, c, sc, None) == H.HADQ_ERR_UNSUPPORTED  # int8 needs full rows
     assert f(a, bf, 0, 3 * 28 * 64, 28 * 64, i4, 64, c, sc, None) == H.HADQ_OK       # block-diagonal K-size
     assert f(a, bf, 0, 28 * 64 + 8, 28 * 64, i4, 32, c, sc, None) == H.HADQ_ERR_INVALID_ARG  # block must divide n
+
+
+@pytest.mark.parametrize("d,bits", [(3, 2), (16, 1), (64, 3), (4096, 4), (4096, 2), (14336, 4), (256, 6)])
+def test_library_codebook_agrees_with_the_oracle(lib, d, bits):
+    """The library's own Lloyd-Max codebook (C++, host) against the oracle's
+    independent one.  Both stop Lloyd's iteration when no centroid moves by
+    more than 1e-13 of the largest; the iteration converges linearly, slowly
+    at 256 levels, so the two agree to 1e-9 of the largest centroid up to 4
+    bits (1e-8 of a centroid spacing) and to 1e-6 beyond."""
+    import oracle
+    c, t = H.hadq_codebook(d, bits)
+    oc, ot = oracle.sphere_lloyd_max(d, bits)
+    tol = (1e-9 if bits <= 4 else 1e-6) * np.abs(oc).max()
+    np.testing.assert_allclose(c, oc, rtol=0, atol=tol)
+    np.testing.assert_allclose(t, ot, rtol=0, atol=tol)
+
+
+def test_library_codebook_rejects_bad_arguments(lib):
+    c = np.zeros(256)
+    t = np.zeros(255)
+    assert lib.hadq_codebook(1, 4, c.ctypes.data, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
+    assert lib.hadq_codebook(64, 0, c.ctypes.data, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
+    assert lib.hadq_codebook(64, 9, c.ctypes.data, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
+    assert lib.hadq_codebook(64, 4, None, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG

@@ -27,7 +27,7 @@ pytestmark = pytest.mark.gpu
 # rows and block-diagonal ones
 SIZES = [(13, 12 * 64, 0), (9, 12 * 1024, 0), (11, 20 * 64, 0), (7, 20 * 256, 0), (10, 28 * 64, 0),
          (6, 28 * 512, 0), (5, 36 * 128, 0), (5, 52 * 64, 0), (5, 52 * 256, 0), (4, 60 * 128, 0),
-         (3, 108 * 64, 0), (3, 108 * 256, 0), (4, 3 * 28 * 64, 28 * 64), (3, 2 * 20 * 128, 20 * 128)]
+         (3, 108 * 64, 0), (2, 108 * 128, 0), (4, 3 * 28 * 64, 28 * 64), (3, 2 * 20 * 128, 20 * 128)]
 
 
 @pytest.fixture(autouse=True)

@@ -1,0 +1,130 @@
+"""GPU parity of the orbitquant path: RPBH rotation and the codebook quantizer.
+
+"orbitquant 0.2.0", Method Conformance: RPBH is a permutation, Rademacher
+signs, a block FWHT and orthonormal scaling; activations are quantized online
+by a per-token norm, rotation of the normalized activation, the nearest
+centroid of a fixed unit-sphere Lloyd-Max codebook per (dimension, bits), and
+rescaling.  The oracle gathers, signs and rotates with explicit matrices and
+builds its own codebook; the library's codebook (hadq_codebook, host code)
+feeds the kernel.  Random permutations at blocks 128, 4096 and 8192, every
+output format, both input dtypes, 2- and 4-bit codebooks with and without
+the permutation, a non-power-of-2 row (14336 = 28 * 512), zero rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hadamard_rotation_bit_b200 import hadq as H
+from tests import parity_check as pc
+from tests.test_gpu_parity import _log, synth, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    H.load_library()
+
+
+def rpbh_args(n, seed):
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(n).astype(np.int32)
+    signs = np.where(rng.random(n) < 0.5, -1, 1).astype(np.int8)
+    return perm, signs, torch.from_numpy(perm).cuda(), torch.from_numpy(signs).cuda()
+
+
+@pytest.mark.parametrize("rows,n,block", [(5, 4096, 128), (7, 4096, 4096), (3, 8192, 8192), (9, 1024, 32),
+                                          (4, 14336, 128), (6, 2048, 0), (3, 8192, 1024)])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_rpbh_rotate(rows, n, block, x_dtype):
+    stored, x64 = synth(rows, n, x_dtype, seed=n + block + rows)
+    perm, signs, pd, sd = rpbh_args(n, n + 1)
+    y = oracle.rpbh_rotate(x64, block, perm, signs)
+    out = H.hadq_rotate_rpbh(to_dev(stored, x_dtype), pd, sd, block, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _log(f"rpbh-rot-{x_dtype}-{rows}x{n}-b{block}", pc.check_rotation_f32(x64, out.cpu().numpy(), block, y=y))
+    ob = H.hadq_rotate_rpbh(to_dev(stored, x_dtype), pd, sd, block, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    pc.check_rotation_bf16(x64, ob.view(torch.int16).cpu().numpy().view(np.uint16), block, y=y)
+
+
+@pytest.mark.parametrize("n,block", [(4096, 128), (4096, 4096), (8192, 8192), (4096, 512)])
+@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int4", 32), ("int8", 0), ("mxfp4", 32), ("nvfp4", 16)])
+def test_rpbh_quant(n, block, fmt, group):
+    rows = 11
+    stored, x64 = synth(rows, n, "bf16", seed=3 * n + block, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
+    perm, signs, pd, sd = rpbh_args(n, block)
+    c, s = H.hadq_rotate_quant_rpbh(to_dev(stored, "bf16"), pd, sd, block, fmt, group)
+    torch.cuda.synchronize()
+    y = oracle.rpbh_rotate(x64, block, perm, signs)
+    _log(f"rpbh-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, c.cpu().numpy(), s.cpu().numpy(), block, group,
+                                                             y=y))
+
+
+def test_rpbh_identity_is_the_plain_rotation():
+    """Identity permutation and all-plus signs: the same codes as hadq_rotate_quant."""
+    stored, _ = synth(9, 4096, "bf16", seed=5)
+    x = to_dev(stored, "bf16")
+    perm = torch.arange(4096, dtype=torch.int32, device="cuda")
+    ones = torch.ones(4096, dtype=torch.int8, device="cuda")
+    H.hadq_set_impl("butterfly")
+    try:
+        c0, s0 = H.hadq_rotate_quant(x, 128, "int4", 128)
+        c1, s1 = H.hadq_rotate_quant_rpbh(x, perm, ones, 128, "int4", 128)
+        torch.cuda.synchronize()
+    finally:
+        H.hadq_set_impl("auto")
+    assert torch.equal(c0, c1) and torch.equal(s0.view(torch.int16), s1.view(torch.int16))
+
+
+def _codebook_dev(n, bits):
+    c, t = H.hadq_codebook(n, bits)
+    return torch.from_numpy(t.copy()).cuda()
+
+
+@pytest.mark.parametrize("rows,n,block", [(9, 4096, 4096), (7, 4096, 128), (5, 8192, 8192), (6, 1024, 64),
+                                          (4, 14336, 0), (5, 2048, 16)])
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("rpbh", [False, True])
+def test_codebook_quantizer(rows, n, block, bits, rpbh):
+    if rpbh and n == 14336 and block == 0:
+        pytest.skip("RPBH's block FWHT is a power-of-2 block")
+    stored, x64 = synth(rows, n, "bf16", seed=n + bits + block)
+    thr = _codebook_dev(n, bits)
+    if rpbh:
+        perm, signs, pd, sd = rpbh_args(n, n + bits)
+        y = oracle.rpbh_rotate(x64, block, perm, signs)
+        codes, norms = H.hadq_rotate_quant_codebook(to_dev(stored, "bf16"), bits, thr, block, perm=pd, signs=sd)
+    else:
+        y = oracle.rotate(x64, block)
+        codes, norms = H.hadq_rotate_quant_codebook(to_dev(stored, "bf16"), bits, thr, block)
+    torch.cuda.synchronize()
+    _log(f"codebook{bits}-{'rpbh-' if rpbh else ''}{rows}x{n}-b{block}",
+         pc.check_codebook(x64, codes.cpu().numpy(), norms.cpu().numpy(), block, bits, y=y))
+
+
+def test_codebook_fp32_input_and_zero_rows():
+    rows, n, bits = 6, 4096, 4
+    stored, x64 = synth(rows, n, "f32", seed=21)
+    stored[1] = 0
+    x64[1] = 0
+    thr = _codebook_dev(n, bits)
+    codes, norms = H.hadq_rotate_quant_codebook(to_dev(stored, "f32"), bits, thr, 256)
+    torch.cuda.synchronize()
+    assert norms[1].item() == 0.0
+    pc.check_codebook(x64, codes.cpu().numpy(), norms.cpu().numpy(), 256, bits)
+
+
+def test_codebook_many_rows_grid_loops():
+    """More rows than resident CTAs, and the full-size R1 shape (4096 x 4096)."""
+    rows, n, bits = 4096, 4096, 4
+    stored, x64 = synth(rows, n, "bf16", seed=33)
+    thr = _codebook_dev(n, bits)
+    perm, signs, pd, sd = rpbh_args(n, 34)
+    codes, norms = H.hadq_rotate_quant_codebook(to_dev(stored, "bf16"), bits, thr, 4096, perm=pd, signs=sd)
+    torch.cuda.synchronize()
+    _log("codebook4-rpbh-4096x4096", pc.check_codebook(x64, codes.cpu().numpy(), norms.cpu().numpy(), 4096, bits,
+                                                       y=oracle.rpbh_rotate(x64, 4096, perm, signs)))

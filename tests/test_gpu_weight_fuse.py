@@ -8,8 +8,10 @@ Transform", introduction and section 1.1 R1 / R4; section 2 for the
 block-diagonal per-Linear mode; section 1.5 for the random Hadamard R).
 
 Both halves go through the C ABI (hadq_rotate / hadq_rotate_signed, fp32
-output) on seeded synthetic activations and weights; the check is the
-invariant itself, in float64, against x W^T from the stored input bits.
+output) on seeded synthetic activations and weights.  The rotated W is first
+compared element by element with the oracle's W R (1e-5 of each row's norm);
+then the invariant itself is checked, in float64, against x W^T from the
+stored input bits.
 The fp32 rotation error is about 1e-7 of each row's norm, so the product
 error is bounded by a few 1e-7 x |x_row| |w_row|; the test allows 1e-5.
 """
@@ -18,7 +20,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from hadamard_rotation_bit_b200 import hadq as H
+from tests import parity_check as pc
 from tests.test_gpu_parity import synth, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -41,6 +45,7 @@ def test_weight_side_rotation_keeps_the_layer_output(n, block, x_dtype):
     xr = H.hadq_rotate(to_dev(xs, x_dtype), block, out_dtype=torch.float32)
     wr = H.hadq_rotate(to_dev(ws, x_dtype), block, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    pc.check_rotation_f32(w64, wr.cpu().numpy(), block)          # W R against the oracle
     err = _fused_error(x64, w64, xr.cpu().numpy(), wr.cpu().numpy())
     assert err < 1e-5, err
 
@@ -57,5 +62,6 @@ def test_weight_side_random_hadamard_keeps_the_layer_output(n, block):
     xr = H.hadq_rotate_signed(to_dev(xs, "bf16"), signs, "after", block, out_dtype=torch.float32)
     wr = H.hadq_rotate_signed(to_dev(ws, "bf16"), signs, "after", block, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    pc.check_rotation_f32(w64, wr.cpu().numpy(), block, y=oracle.rotate_signed(w64, block, signs.cpu().numpy(), "after"))
     err = _fused_error(x64, w64, xr.cpu().numpy(), wr.cpu().numpy())
     assert err < 1e-5, err

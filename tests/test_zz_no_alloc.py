@@ -3,11 +3,13 @@ allocate device memory (a host-only application linking libhadq, or a plugin
 inside a framework that owns every device allocation).  It stages through the
 library's own static device array, so the caller passes host buffers only.
 
-The GPU test calls it through the C ABI twice in a row (different shapes and
-formats, then the first call again, so a stale array from the previous call
-cannot go unnoticed) and compares every output with the existing host-buffer
-entry point, which uses caller-owned device buffers.  Both run the same
-kernels, so the outputs must be identical.  This file is collected last.
+The GPU test calls it through the C ABI three times in a row: two shapes and
+formats, then the first shape again with another seed, so outputs left in the
+shared array by an earlier call (a kernel that did not run) cannot match.
+Every output is compared with the existing host-buffer entry point, which
+uses caller-owned device buffers and runs the same kernels (so the two must
+be identical), and element by element with the float64 oracle under the
+parity rule of the other GPU tests.  This file is collected last.
 """
 
 import ctypes
@@ -19,6 +21,7 @@ import torch
 from hadamard_rotation_bit_b200 import build as hbuild
 from hadamard_rotation_bit_b200 import hadq as H
 from hadamard_rotation_bit_b200 import workloads as W
+from tests import parity_check as pc
 
 CASES = [(512, 4096, 0, "int4", 128, 1), (1024, 1024, 128, "mxfp4", 32, 2), (512, 4096, 0, "int4", 128, 3)]
 
@@ -27,7 +30,7 @@ def _pinned_input(rows, n, seed):
     v = np.random.default_rng(seed).standard_normal((rows, n)).astype(np.float32)
     v[:, :: max(1, n // 40)] *= 30.0
     bits = W.f32_to_bf16_bits(v)
-    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory(), W.bits_to_float64(bits, "bf16")
 
 
 @pytest.mark.gpu
@@ -37,7 +40,7 @@ def test_static_scratch_entry_point_matches_host_entry_point():
     lib = H.load_library()
     stream = torch.cuda.current_stream()
     for rows, n, block, fmt, group, seed in CASES:
-        xh = _pinned_input(rows, n, seed)
+        xh, x64 = _pinned_input(rows, n, seed)
         cs, cd, ss, sd = H.output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
         c_static = torch.full(cs, 0x5A, dtype=cd).pin_memory()
         s_static = torch.zeros(ss, dtype=sd).pin_memory()
@@ -56,6 +59,7 @@ def test_static_scratch_entry_point_matches_host_entry_point():
         torch.cuda.synchronize()
         assert torch.equal(c_static, c_ref), f"codes differ for {rows}x{n} {fmt}"
         assert torch.equal(s_static.view(torch.uint8), s_ref.view(torch.uint8)), f"scales differ for {rows}x{n} {fmt}"
+        pc.check(fmt, x64, c_static.numpy(), s_static.numpy(), block, group)
 
 
 def test_static_scratch_entry_point_rejects_oversize_and_bad_args():
