@@ -203,6 +203,19 @@ struct TeamShape {
   static constexpr int ROW = P + 4;           // transpose row (floats), one quad of padding
   static constexpr int W = P / 32;            // sign-mask words
   static constexpr bool PERM = V >= 2;        // quads transposed as (e0, e2, e1, e3)
+  static constexpr int C4 = CE / 4;           // quads per phase-1 chunk (0: float2 chunks)
+  // Quad q of a transpose row is stored at swz(q).  Team thread tau writes
+  // its chunk into quads tau * C4 + k of every row and reads back all quads of
+  // row tau; the XOR (an involution inside the row) spreads the writes of the
+  // 8 lanes a 128-byte wavefront serves over 8 distinct 16-byte bank groups
+  // where the plain layout repeats them: C4 = 4 (b = 256: the 4 threads of a
+  // team 16 quads apart, two teams 68 quads apart) and C4 = 2 (b = 512: 8
+  // threads 2 quads apart).  The reads stay conflict-free (row stride 17 quads).
+  static __device__ __forceinline__ int swz(int q) {
+    if constexpr (C4 == 4) return q ^ ((q >> 2) & 3);
+    if constexpr (C4 == 2) return q ^ ((q >> 3) & 1);
+    return q;
+  }
   static_assert(LOGB >= 8 && LOGB <= 13 && t >= 1 && V >= 1, "team kernels cover 256..8192");
 };
 
@@ -279,7 +292,7 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
 #pragma unroll
       for (int k = 0; k < Sh::CE / 4; ++k) {
         const float* s = &v[h * Sh::CE + 4 * k];
-        reinterpret_cast<float4*>(rowp)[tau * (Sh::CE / 4) + k] =
+        reinterpret_cast<float4*>(rowp)[Sh::swz(tau * (Sh::CE / 4) + k)] =
             Sh::PERM ? make_float4(s[0], s[2], s[1], s[3]) : make_float4(s[0], s[1], s[2], s[3]);
       }
     } else {
@@ -291,7 +304,7 @@ __device__ __forceinline__ void team_rotate(const void* __restrict__ x, int64_t 
     const float4* rowp = reinterpret_cast<const float4*>(rows + tau * Sh::ROW);
 #pragma unroll
     for (int q = 0; q < P / 4; ++q) {
-      const float4 f = rowp[q];
+      const float4 f = rowp[Sh::swz(q)];
       v[4 * q] = f.x;
       v[4 * q + 1] = f.y;
       v[4 * q + 2] = f.z;

@@ -33,6 +33,10 @@ permutation drawn from a ``seed + 1`` stream):
   ``generate_rpbh``, then the full 4096-point rotation), quantized to int4 g128
   (``c2p``) or by the per-token norm and the 4-bit unit-sphere Lloyd-Max
   codebook (``c2q``, "orbitquant 0.2.0", Method Conformance).
+* ``pl256`` / ``pl1024``  per-Linear shapes of "Rotation Transform" section 2
+  on the butterfly kernels: the ``c5`` input with block 256 and int4 g128;
+  131072 x 1024 bf16 ~ N(0, 1) with 1 % of the channels x50, rotated in full
+  to MXFP4.
 * ``c3k``  the ``c3`` input rotated in full instead of by blocks of 128: the
   14336-point rotation of a non-power-of-2 size ("Rotation Transform",
   section 1.5: 14336 = 28 * 2^9, a base matrix of order 28 with a Sylvester
@@ -125,12 +129,16 @@ WORKLOADS = {
                     base="c2", rpbh=True),
     "c2q": Workload("c2q", "R1 4096 tokens x hidden 4096 bf16, RPBH (full 4096-point), per-token norm + 4-bit "
                     "unit-sphere Lloyd-Max codebook", 4096, 4096, 4096, "bf16", "codebook", 4, base="c2", rpbh=True),
+    "pl256": Workload("pl256", "per-Linear block-diagonal: 65536 tokens x 8192 bf16 Student-t(3), block 256, int4 sym "
+                      "g128", 65536, 8192, 256, "bf16", "int4", 128, base="c5"),
+    "pl1024": Workload("pl1024", "per-Linear full 1024: 131072 tokens x 1024 bf16 ~ N(0,1), 1 % channels x50, full "
+                       "1024-point Hadamard, MXFP4", 131072, 1024, 1024, "bf16", "mxfp4", 32),
     "c5rb": Workload("c5rb", "large R1 65536 tokens x hidden 8192 bf16 Student-t(3), full 8192-point random Hadamard "
                      "transpose (signs before), MXFP4", 65536, 8192, 8192, "bf16", "mxfp4", 32, signs="before",
                      base="c5"),
 }
 
-_STREAM = {"c1": 1, "c2": 2, "c3": 3, "c4q": 4, "c4k": 5, "c5": 6}
+_STREAM = {"c1": 1, "c2": 2, "c3": 3, "c4q": 4, "c4k": 5, "c5": 6, "pl1024": 7}
 _SIGN_STREAM = 100
 
 
@@ -218,6 +226,10 @@ def _chunk_values(key: str, chunk: int, seed: int) -> np.ndarray:
         return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)
     if key == "c5":
         return g.standard_t(3, (nr, w.n))
+    if key == "pl1024":
+        v = g.standard_normal((nr, w.n))
+        v[:, _outlier_set(seed, _STREAM[key], w.n, round(0.01 * w.n))] *= 50.0
+        return v
     raise KeyError(key)
 
 
