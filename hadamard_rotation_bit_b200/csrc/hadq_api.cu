@@ -374,16 +374,23 @@ hadq_status launch_staged(const void* x, hadq_dtype x_dtype, const Shape& sh, in
   if (unit % 64 != 0 || unit / 64 > ks::kMaxThreads)
     return fail(HADQ_ERR_UNSUPPORTED, per_row ? "this quantizer / permutation needs n a multiple of 64 and n <= 32768"
                                               : "K * 2^m blocks need 2^m >= 64 and K * 2^m <= 32768");
-  int shi = 1, logs_lo = sh.logk;
-  if (sh.kbase == 1) {
-    logs_lo = std::min(sh.logb, 11);               // the butterfly stage runs at most 2048 points per column
-    shi = 1 << (sh.logb - logs_lo);
-  }
+  // The column stage mixes K * SHI values per column in registers (at most
+  // 64); the butterfly stage runs the S_lo = 2^m / SHI points left, 64 and
+  // more in runs of 64 with shuffles across lanes for the rest.  SHI as large
+  // as both allow, so as few shuffle stages as possible remain.
+  const int logm = sh.kbase == 1 ? sh.logb : sh.logk;
+  int logshi = 0;
+  while ((sh.kbase << (logshi + 1)) <= 64 && logm - (logshi + 1) >= 6) ++logshi;
+  const int shi = 1 << logshi, logs_lo = logm - logshi;
   const hl::KsFn fn = hl::staged_kernel_for(sh.kbase, shi, bf, mode, sgk);
   if (fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no staged kernel for this size, format and sign variant");
   const int64_t smem = ks::smem_bytes(unit, bf ? 2 : 4, sgk, sh.b);
   if (smem > 227 * 1024) return fail(HADQ_ERR_UNSUPPORTED, "row or block too large for the staged kernel's shared memory");
-  const int threads = static_cast<int>(ceil_div(unit / 64, 32) * 32);
+  // One thread per 64-value run in the butterfly stage and one per column in
+  // the column stage, whichever needs more (threads beyond either sit out).
+  const int64_t cols = unit / (int64_t(sh.kbase) * shi);
+  const int threads = static_cast<int>(
+      std::min<int64_t>(ceil_div(std::max<int64_t>(unit / 64, cols), 32) * 32, hadq::ksize::kMaxThreads));
   int occ = 0;
   hadq_status st = occupancy(reinterpret_cast<const void*>(fn), dev, threads, static_cast<int>(smem), &occ);
   if (st != HADQ_OK) return st;

@@ -29,8 +29,9 @@
 //             f32x2 adds; results go to a shared fp32 buffer whose 64-value
 //             runs are padded to 68 words (128-bit accesses without conflicts);
 //   2^m stage each thread takes one 64-value run of one sub-block: 6 butterfly
-//             stages in registers, m - 6 more with shuffles across the
-//             2^(m-6) neighbouring lanes that hold the sub-block; then the
+//             stages in registers, and those of the remaining S_lo points
+//             with shuffles across the neighbouring lanes that hold the
+//             piece (the column stage has already mixed the pieces); then the
 //             epilogue of the butterfly kernels (1/sqrt(b), quantize, store).
 #pragma once
 
@@ -220,8 +221,12 @@ __device__ __forceinline__ uint32_t codebook_index(float z, const float2* tau) {
 
 // Units of unit_len elements; blockDim.x = unit_len / 64 rounded up to 32.
 // MODE: OutMode, or -1 for per-token int8.  K: 1 (Sylvester) or a Paley
-// order; SHI: how many S_lo-long pieces the 2^m factor spans (K = 1 and
-// b > kMaxSlo), mixed in the column stage with the K sub-blocks.
+// order; SHI: how many S_lo-long pieces the 2^m factor is cut into: the
+// column stage mixes those pieces (H_SHI) along with the K sub-blocks, the
+// butterfly stage runs the S_lo points that remain.  The host takes SHI as
+// large as K * SHI <= 64 registers and S_lo >= 64 allow, which keeps the
+// lane-crossing butterfly stages (shuffles) few or none: a 4096-point block
+// is 64 x 64, both halves in registers.
 template <int K, int SHI, bool IN_BF16, int MODE, int SGK>
 __global__ void __launch_bounds__(kMaxThreads)
 staged_kernel(const __grid_constant__ StageArgs a) {
@@ -287,16 +292,35 @@ staged_kernel(const __grid_constant__ StageArgs a) {
         const int e = base + kh * slo;
         wbuf[(e >> 6) * kRunPad + (e & 63)] = v;
       };
-      if constexpr (K == 1) {
-        float z[SHI];
+      // z[k SHI + h] = the value at (k SHI + h) S_lo + j: H_SHI over h for
+      // every k (Sylvester), then H_K over k for every h.
+      float z[KH];
 #pragma unroll
-        for (int h = 0; h < SHI; ++h) z[h] = get(h);
-        if constexpr (SHI > 1) fwht_bits<SHI, 0, (SHI == 2 ? 1 : 2)>(z);
+      for (int kh = 0; kh < KH; ++kh) z[kh] = get(kh);
+#pragma unroll
+      for (int d = 1; d < SHI; d <<= 1) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+#pragma unroll
+          for (int h = 0; h < SHI; ++h) {
+            if ((h & d) == 0) {
+              const float u = z[k * SHI + h], w = z[k * SHI + h + d];
+              z[k * SHI + h] = __fadd_rn(u, w);
+              z[k * SHI + h + d] = __fsub_rn(u, w);
+            }
+          }
+        }
+      }
+      if constexpr (K == 1) {
 #pragma unroll
         for (int h = 0; h < SHI; ++h) put(h, z[h]);
       } else {
-        static_assert(SHI == 1, "a Paley base order is mixed with the whole 2^m factor in the butterfly stage");
-        kstage_column<K>(get, put);
+#pragma unroll
+        for (int h = 0; h < SHI; ++h) {
+          auto geth = [&](int k) { return z[k * SHI + h]; };
+          auto puth = [&](int k, float v) { put(k * SHI + h, v); };
+          kstage_column<K>(geth, puth);
+        }
       }
     }
     __syncthreads();   // every run of the unit mixed

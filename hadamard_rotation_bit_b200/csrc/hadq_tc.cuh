@@ -57,8 +57,13 @@ constexpr int kABytes = 128 * 128 * 2;     // A operand: H_128 in bf16
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after 1 s
 
 
-template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_, int PREFETCH_ = 2, bool AHEAD_ = false>
+template <int LO_, int TILE_N_, int STAGES_, int SPLIT_, bool HALF_, int PREFETCH_ = 2, bool AHEAD_ = false,
+          bool A_TMEM_ = false>
 struct TcCfg {
+  // A_TMEM: H_128 lives in tensor memory (64 columns after the accumulators)
+  // instead of shared memory, so the MMAs read only the B tile from shared
+  // memory; one accumulator buffer fewer.
+  static constexpr bool A_TMEM = A_TMEM_;
   static constexpr int PREFETCH = PREFETCH_;             // tiles per CTA prefetched into L2 at entry
   static constexpr bool AHEAD = AHEAD_;                  // keep the prefetch PREFETCH tiles ahead of the loads
   // Sign-flipping threads (signs before the rotation only): as many as the
@@ -71,7 +76,8 @@ struct TcCfg {
   static constexpr int STAGES = STAGES_;
   static constexpr int TILE_BYTES = 128 * TILE_N * 2;     // B operand: K = 128 x N bf16
   static constexpr int TMEM_COLS = 512;                   // the whole tensor memory of the SM
-  static constexpr int ACC_BUFS = TMEM_COLS / TILE_N;
+  static constexpr int ACC_BUFS = (TMEM_COLS - (A_TMEM ? 64 : 0)) / TILE_N;
+  static constexpr int A_COL = ACC_BUFS * TILE_N;         // A_TMEM: first column of H_128
   static constexpr int SPLIT = SPLIT_;                    // epilogue warps per TMEM lane quarter
   static constexpr int THREADS = 32 * (2 + 4 * SPLIT);
   static constexpr bool HALF = HALF_;                      // two N/2 MMA halves per tile, committed apart
@@ -85,8 +91,8 @@ struct TcCfg {
                                     (static_cast<uint32_t>(TILE_N >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
   static constexpr uint32_t IDESC_HALF = (IDESC & ~(63u << 17)) | (static_cast<uint32_t>(TILE_N >> 4) << 17);
   // Shared memory (offsets from a 1024-byte aligned base).
-  static constexpr int SM_A = 0;                          // H_128, 2 K-panels x 16 KB
-  static constexpr int SM_B = SM_A + kABytes;             // STAGES x TILE_BYTES
+  static constexpr int SM_A = 0;                          // H_128, 2 K-panels x 16 KB (not A_TMEM)
+  static constexpr int SM_B = SM_A + (A_TMEM ? 0 : kABytes);   // STAGES x TILE_BYTES
   static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
   static constexpr int SM_SLOT = SM_BARS + 8 * (3 * STAGES + 3 * ACC_BUFS);
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;  // + alignment slack
@@ -177,6 +183,27 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// The same with A in tensor memory (lane m = row m, column c = the bf16 pair
+// k = 2c, 2c + 1).
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -365,19 +392,21 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
     // A = H_128 (K-major, 128-byte swizzle, two K-panels of 64): element (m, k)
     // at panel (k / 64) + m * 128 + (k % 64) * 2 bytes, 16-byte chunk index
     // XOR-ed with (m % 8).  Entry (m, k) = (-1)^popcount(m & k) as bf16.
-    for (int i = threadIdx.x - 32; i < 128 * 16; i += T - 32) {
-      const int m = i >> 4, kc = i & 15;              // 8 consecutive k per 16-byte chunk
-      uint32_t w[4];
+    if constexpr (!C::A_TMEM) {
+      for (int i = threadIdx.x - 32; i < 128 * 16; i += T - 32) {
+        const int m = i >> 4, kc = i & 15;              // 8 consecutive k per 16-byte chunk
+        uint32_t w[4];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int k = kc * 8 + 2 * p;
-        w[p] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+        for (int p = 0; p < 4; ++p) {
+          const int k = kc * 8 + 2 * p;
+          w[p] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+        }
+        const int panel = kc >> 3, chunk = kc & 7;
+        const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
+        *reinterpret_cast<uint4*>(smem + C::SM_A + off) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      const int panel = kc >> 3, chunk = kc & 7;
-      const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
-      *reinterpret_cast<uint4*>(smem + C::SM_A + off) = make_uint4(w[0], w[1], w[2], w[3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // A visible to the tensor core
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // A visible to the tensor core
     if (warp == 1) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                    "r"(C::TMEM_COLS));
@@ -387,6 +416,27 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
     asm volatile("bar.sync 1, %0;" ::"r"(T - 32) : "memory");   // warps 1.. only
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if constexpr (C::A_TMEM) {
+      // H_128 into tensor memory by the four warps of the first epilogue
+      // group (warp w reaches lanes 32 (w % 4) ..): lane m holds row m,
+      // column A_COL + c the bf16 pair (k = 2c, 2c + 1).
+      if (warp >= 2 && warp < 6) {
+        const int m = (warp & 3) * 32 + lane;
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k = 2 * (c0 + i);
+            w[i] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+          }
+          tmem_st16(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::A_COL + c0, w);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+      tc_fence_before();
+      asm volatile("bar.sync 1, %0;" ::"r"(T - 32) : "memory");   // A written before the first MMA
+      tc_fence_after();
+    }
 
     if (warp == 1) {
       // ------------------------------------------------------- MMA issuer
@@ -416,11 +466,16 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
             const uint32_t bh = b_base + h * (C::TILE_BYTES / 2);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {   // K = 128 in steps of 16
-              const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
               const uint64_t b_desc = (LO == 5) ? smem_desc(bh + kk * 1024, 8192, 512, kSwizzle64)
                                                 : smem_desc(bh + kk * 2048, 16384, 1024, kSwizzle128);
-              mma_bf16(d + h * (C::TILE_N / 2), a_desc, b_desc, C::HALF ? C::IDESC_HALF : C::IDESC,
-                       kk > 0 ? 1u : 0u);
+              if constexpr (C::A_TMEM) {
+                mma_bf16_ta(d + h * (C::TILE_N / 2), tmem_base + C::A_COL + kk * 8, b_desc,
+                            C::HALF ? C::IDESC_HALF : C::IDESC, kk > 0 ? 1u : 0u);
+              } else {
+                const uint64_t a_desc = smem_desc(a_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
+                mma_bf16(d + h * (C::TILE_N / 2), a_desc, b_desc, C::HALF ? C::IDESC_HALF : C::IDESC,
+                         kk > 0 ? 1u : 0u);
+              }
             }
             if (h == NH - 1) mma_commit(&empty[s]);   // stage s may be refilled once these MMAs have read it
             mma_commit(h == 0 ? &acc_full[b] : &acc_full2[b]);   // (this half of) accumulator b is ready

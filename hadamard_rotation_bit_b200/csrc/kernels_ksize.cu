@@ -3,8 +3,9 @@
 // HADQ_KSIZE_BF16 for bf16 input (kernels_ksize_bf16.cu) and without it for
 // fp32 input.  Instantiated: every Paley base order K with the plain and
 // block-signed rotations, all formats and the codebook quantizer; the pure
-// Sylvester blocks (K = 1, SHI = 1, 2, 4) with the RPBH permutation and the
-// codebook quantizer, the variants no other kernel family covers.
+// Sylvester blocks (K = 1) with the RPBH permutation and the codebook
+// quantizer, the variants no other kernel family covers.  SHI: the pieces of
+// the 2^m factor mixed in the column stage (K * SHI <= 64).
 #include "hadq_ksize.cuh"
 #include "hadq_launch.h"
 
@@ -65,18 +66,22 @@ KsFn staged_kernel_f32(int k, int shi, int mode, int sgk) {
       case 1: return pick<1, 1>(mode, sgk);
       case 2: return pick<1, 2>(mode, sgk);
       case 4: return pick<1, 4>(mode, sgk);
+      case 8: return pick<1, 8>(mode, sgk);
+      case 16: return pick<1, 16>(mode, sgk);
+      case 32: return pick<1, 32>(mode, sgk);
+      case 64: return pick<1, 64>(mode, sgk);
       default: return nullptr;
     }
   }
-  if (shi != 1) return nullptr;
   switch (k) {
-    case 12: return pick<12, 1>(mode, sgk);
-    case 20: return pick<20, 1>(mode, sgk);
-    case 28: return pick<28, 1>(mode, sgk);
-    case 36: return pick<36, 1>(mode, sgk);
-    case 52: return pick<52, 1>(mode, sgk);
-    case 60: return pick<60, 1>(mode, sgk);
-    case 108: return pick<108, 1>(mode, sgk);
+    case 12: return shi == 1 ? pick<12, 1>(mode, sgk) : shi == 2 ? pick<12, 2>(mode, sgk)
+                  : shi == 4 ? pick<12, 4>(mode, sgk) : nullptr;
+    case 20: return shi == 1 ? pick<20, 1>(mode, sgk) : shi == 2 ? pick<20, 2>(mode, sgk) : nullptr;
+    case 28: return shi == 1 ? pick<28, 1>(mode, sgk) : shi == 2 ? pick<28, 2>(mode, sgk) : nullptr;
+    case 36: return shi == 1 ? pick<36, 1>(mode, sgk) : nullptr;
+    case 52: return shi == 1 ? pick<52, 1>(mode, sgk) : nullptr;
+    case 60: return shi == 1 ? pick<60, 1>(mode, sgk) : nullptr;
+    case 108: return shi == 1 ? pick<108, 1>(mode, sgk) : nullptr;
     default: return nullptr;
   }
 }

@@ -15,15 +15,16 @@ TcVariant tc_variant() {
   return TcVariant{&tc::tc_rotate_kernel<C, MODE, SIDE>, tc::tc_threads<C, SIDE>(), C::SMEM_BYTES, C::TILE_N};
 }
 
-// n = 4096: 4 rows per tile, one row per epilogue warp, 3 stages (4 with
-// signs before the rotation, whose flipping pass holds each stage longer:
-// 4096 x 4096 int4 11.09 us per launch with 4 stages, 11.3 with 3, while the
-// other sides are fastest with 3: 9.42 us unsigned, 9.65 with 4).  n = 8192:
-// 2 rows per tile, 4 stages; for int4 (whose epilogue is the heaviest) the
-// MMAs are committed per row so the first row's epilogue starts early.
+// n = 4096: 4 rows per tile, one row per epilogue warp, 3 stages, H_128 held
+// in tensor memory (the MMAs read only the B tile from shared memory):
+// 4096 x 4096 int4 9.57 us per launch against 9.62 with H_128 in shared
+// memory; signs before the rotation 11.42 against 11.54 (the best shared-
+// memory layout there, 4 stages).  n = 8192: 2 rows per tile, 4 stages; for
+// int4 (whose epilogue is the heaviest) the MMAs are committed per row so the
+// first row's epilogue starts early.
 template <int SIDE>
 TcVariant tc_pick(int lo, int mode) {
-  using C5 = std::conditional_t<SIDE == SIGNS_BEFORE, tc::TcCfg<5, 128, 4, 4, false>, tc::TcCfg<5, 128, 3, 4, false>>;
+  using C5 = tc::TcCfg<5, 128, 3, 4, false, 2, false, true>;
   using C6 = tc::TcCfg<6, 128, 4, 2, false>;
   using C6H = tc::TcCfg<6, 128, 4, 2, true>;
   switch (mode) {
