@@ -31,7 +31,7 @@ LINK_FLAGS = ARCH_FLAGS + ["--shared", "-cudart", "static", "-Xcompiler", "-fvis
 # Translation units: the host side (validation, launch planning, C ABI) and
 # one unit per kernel family, compiled in parallel.
 UNITS = ["hadq_api.cu", "kernels_segment.cu", "kernels_team.cu", "kernels_team_bf16.cu", "kernels_tc.cu",
-         "kernels_ksize.cu", "kernels_ksize_bf16.cu", "hadq_codebook.cu"]
+         "kernels_tck.cu", "kernels_ksize.cu", "kernels_ksize_bf16.cu", "hadq_codebook.cu"]
 
 
 def _nvcc() -> str:

@@ -350,6 +350,51 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                        "tensor-core block-128 kernel launch");
 }
 
+// Blocks of b = K * 128 * hi bf16 elements on the tensor cores
+// (hadq_tck.cuh): H_128 on every 128-element chunk by one MMA, the H_hi and
+// Paley H_K factors in the registers of the thread that holds one output of
+// every chunk, so K * hi <= 128.  Rotation outputs, and per-token int8 over
+// whole rows (b = n); signs, the RPBH permutation and the other quantizers
+// take the staged kernels.
+bool tck_eligible(hadq_dtype x_dtype, const Shape& sh, int mode, Signs sg) {
+  if (x_dtype != HADQ_BF16 || sh.kbase == 1 || sh.logk < 7 || sg.side != hadq::SIGNS_NONE) return false;
+  if (static_cast<int64_t>(sh.kbase) << (sh.logk - 7) > 128) return false;
+  if (mode < 0) return sh.b == sh.n;
+  return mode == hadq::OUT_F32 || mode == hadq::OUT_BF16;
+}
+
+hadq_status launch_tck(const void* x, const Shape& sh, int mode, void* out0, void* out1, cudaStream_t stream, int sms,
+                       int dev) {
+  const hl::TckVariant v = hl::tck_kernel_for(sh.kbase, 1 << (sh.logk - 7), mode);
+  if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no K * 2^m tensor-core kernel for this size and format");
+  const int64_t chunks = sh.rows * (sh.n >> 7);
+  if (chunks > (int64_t(1) << 31) - 256) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many blocks");
+  const int64_t blocks = sh.rows * (sh.n / sh.b);
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (encode == nullptr) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  // The chunks are the rows of a chunks x 128 matrix, loaded as two 64-wide
+  // K-panels of v.np chunks (the block's chunks, then padding that is never read).
+  CUtensorMap maps[2];
+  for (int p = 0; p < 2; ++p) {
+    cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(chunks)};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(v.np)};
+    cuuint32_t estr[2] = {1, 1};
+    void* base = const_cast<char*>(static_cast<const char*>(x)) + 128 * p;
+    const CUresult r = encode(&maps[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  }
+  int occ = 0;
+  hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t grid = std::min<int64_t>(blocks, sms);
+  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, maps[0], maps[1],
+                                  static_cast<const uint16_t*>(x), blocks, sh.norm, out0, out1),
+                       "K * 2^m tensor-core kernel launch");
+}
+
 // Blocks of b = K * 2^m elements (one CTA per block, persistent over blocks).
 // What the shared-memory staged kernels need beyond the shape: the RPBH
 // permutation (with n signs) and the codebook thresholds.
@@ -434,6 +479,9 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours
+  if (ex.perm == nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
+      tck_eligible(x_dtype, sh, mode, sg))
+    return launch_tck(x, sh, mode, out0, out1, stream, sms, dev);
   if (sh.kbase > 1 || ex.perm != nullptr || mode == hadq::OUT_CODEBOOK)
     return launch_staged(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg, ex);
   if (g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY) {
@@ -858,6 +906,9 @@ hadq_status hadq_set_impl(hadq_impl impl) {
 
 hadq_impl hadq_get_impl(void) { return static_cast<hadq_impl>(g_impl.load(std::memory_order_relaxed)); }
 
-int hadq_device_faults(int clear) { return hadq::launch::tc_fault_bits(clear); }
+int hadq_device_faults(int clear) {
+  const int a = hadq::launch::tc_fault_bits(clear), b = hadq::launch::tck_fault_bits(clear);
+  return a < 0 || b < 0 ? -1 : (a | b);
+}
 
 }  // extern "C"

@@ -1,7 +1,7 @@
 // Kernel entry points as the host launcher sees them.
 //
 // The kernels are instantiated in their own translation units
-// (kernels_segment.cu, kernels_team.cu, kernels_tc.cu), which nvcc compiles in
+// (kernels_segment.cu, kernels_team.cu, kernels_tc.cu, kernels_tck.cu, ...), which nvcc compiles in
 // parallel; each exports a lookup that returns the instantiation for a call's
 // shape, output mode and sign variant.  SG selects the random Hadamard
 // (signed) instantiation; the deterministic ones are compiled without any
@@ -40,6 +40,13 @@ struct Tc128Variant {
   int threads, smem;
 };
 
+using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, void*, void*);
+
+struct TckVariant {
+  TckFn fn;
+  int threads, smem, np;   // np: MMA N = chunks per block rounded up to 16
+};
+
 // Segment kernels (b <= 128): log2 of the per-thread segment `logs`, FULL when
 // b equals the segment.  mode: OutMode.
 SegFn segment_kernel_for(bool bf16, bool full, int logs, int mode, bool sg);
@@ -66,9 +73,16 @@ KsFn staged_kernel_for(int k, int shi, bool bf16, int mode, int sgk);
 KsFn staged_kernel_f32(int k, int shi, int mode, int sgk);
 KsFn staged_kernel_bf16(int k, int shi, int mode, int sgk);
 
-// The tensor-core kernels' sticky fault word (bounded waits that ran out);
-// cleared when `clear` is non-zero.  -1 on a CUDA error.
+// Tensor-core kernels for blocks of K * 128 * hi elements (K a Paley order,
+// K * hi <= 128 chunks of 128); mode OUT_F32 / OUT_BF16, or -1 = per-token
+// int8 (block = row).
+TckVariant tck_kernel_for(int k, int hi, int mode);
+
+// The tensor-core kernels' sticky fault words (bounded waits that ran out),
+// one per translation unit; cleared when `clear` is non-zero.  -1 on a CUDA
+// error.
 int tc_fault_bits(int clear);
+int tck_fault_bits(int clear);
 
 }  // namespace launch
 }  // namespace hadq

@@ -232,7 +232,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-__device__ unsigned int hadq_tc_fault;   // sticky fault bits (bounded waits that ran out)
+// Sticky fault bits (bounded waits that ran out), one word per translation
+// unit that instantiates these kernels; the host ORs them.
+static __device__ unsigned int hadq_tc_fault;
 
 // After a wait ran out, what this thread already issued must finish before
 // the CTA exits: a TMA write into shared memory, or an MMA reading it, must

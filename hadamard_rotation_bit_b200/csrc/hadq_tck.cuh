@@ -1,0 +1,341 @@
+// Tensor-core variant for blocks of b = K * 2^m elements with 2^m = 128 * HI
+// (K a Paley order, HI = 1, 2, 4, ...), bf16 input.
+//
+// "Rotation Transform" (AutoRound docs), section 1.5: a size that is not a
+// power of 2 is rotated by a base Hadamard matrix of order K combined with a
+// Sylvester block, H_b = H_K (x) H_(2^m).  With 2^m = HI * 128 the Sylvester
+// block splits once more, H_(2^m) = H_HI (x) H_128, over the index split
+//
+//     e = c * 128 + i,   c = k * HI + h   (chunk c of the block),
+//
+// so a block is C = K * HI consecutive 128-element chunks.  One tcgen05 MMA
+// per block rotates every chunk by H_128,
+//
+//     D[i', c] = sum_i H_128[i', i] * X[c * 128 + i]
+//
+// (M = 128, K = 128, N = C rounded up to a multiple of 16): A = H_128 in
+// shared memory, B = the chunks exactly as they lie in global memory,
+// K-major with the 128-byte swizzle, loaded by the block-128 kernel's pair of
+// 2-D tensor maps (columns beyond C hold whatever follows the block and are
+// never read).  Operands are exact in bf16; products accumulate in fp32 in
+// tensor memory.  TMEM lane i' then holds output index i' of every chunk of
+// the block, so the rest of the rotation runs in one thread's registers with
+// no data exchange: H_HI over h (Sylvester stages), then the Paley K-point
+// mix over k for each h (the compile-time residue table of hadq_ksize.cuh).
+// The thread's outputs y[c * 128 + i'] are one per chunk: for each chunk a
+// warp writes 32 consecutive outputs.
+//
+// Roles as in the block-128 kernel: warp 0 TMA producer, warp 1 TMEM
+// allocator and single-thread MMA issuer, then EPI_GROUPS groups of 4
+// epilogue warps (one TMEM lane quarter each) taking whole blocks round-robin.
+// Per-token int8 takes a whole row per block (b = n) and joins the row absmax
+// of the group's 4 warps in shared memory.  Every wait is bounded
+// (hadq_tc_fault), and thread 0 first asks L2 to prefetch the CTA's first
+// PREFETCH blocks.
+#pragma once
+
+#include <utility>
+
+#include "hadq_ksize.cuh"
+#include "hadq_tc.cuh"
+
+namespace hadq {
+namespace tc {
+
+template <int K_, int HI_, int STAGES_, int EPI_GROUPS_, int PREFETCH_>
+struct TckCfg {
+  static constexpr int K = K_, HI = HI_, C = K * HI;   // chunks per block
+  static constexpr int NP = (C + 15) / 16 * 16;         // MMA N
+  static_assert(C % 4 == 0 && NP <= 128, "a thread holds one output of every chunk in registers");
+  static constexpr int STAGES = STAGES_;
+  static constexpr int EPI_GROUPS = EPI_GROUPS_;
+  static constexpr int PREFETCH = PREFETCH_;            // blocks per CTA prefetched into L2 at entry
+  static constexpr int PANEL_BYTES = NP * 128;          // NP chunks x 64 bf16 (one K-panel)
+  static constexpr int TILE_BYTES = 2 * PANEL_BYTES;    // B operand per block
+  static constexpr int ACC_BUFS = 4;                    // accumulators at TMEM columns 0, 128, 256, 384
+  static constexpr int THREADS = 32 * (2 + 4 * EPI_GROUPS);
+  // kind::f16, fp32 accumulate, bf16 A and B, both K-major, N = NP, M = 128.
+  static constexpr uint32_t IDESC =
+      (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(NP >> 3) << 17) | (8u << 24);
+  static constexpr int SM_A = 0;                        // H_128
+  static constexpr int SM_B = SM_A + kABytes;           // STAGES x TILE_BYTES
+  static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
+  static constexpr int SM_RED = SM_BARS + 8 * (2 * STAGES + 2 * ACC_BUFS);   // per-token row max
+  static constexpr int SM_SLOT = SM_RED + 4 * 4 * EPI_GROUPS;
+  static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
+  static_assert(PANEL_BYTES % 1024 == 0, "swizzle atoms of 8 chunks");
+};
+
+// 16, 8 and 4 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float* v) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Columns [0, C) of this thread's lane, C a multiple of 4.
+template <int C>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&z)[C]) {
+  constexpr int C32 = C / 32 * 32;
+#pragma unroll
+  for (int c = 0; c < C32; c += 32) tmem_ld32(taddr + c, &z[c]);
+  constexpr int R = C - C32;
+  if constexpr (R & 16) tmem_ld16(taddr + C32, &z[C32]);
+  if constexpr (R & 8) tmem_ld8(taddr + C32 + (R & 16), &z[C32 + (R & 16)]);
+  if constexpr (R & 4) tmem_ld4(taddr + C32 + (R & 24), &z[C32 + (R & 24)]);
+}
+
+// H_K over k of the values z[k * HI + H] (one h = H).
+template <int K, int HI, int H, int C>
+__device__ __forceinline__ void paley_mix_h(float (&z)[C]) {
+  auto get = [&](int k) { return z[k * HI + H]; };
+  auto put = [&](int k, float v) { z[k * HI + H] = v; };
+  ksize::kstage_column<K>(get, put);   // reads every value before writing any
+}
+
+template <int K, int HI, int C, int... Hs>
+__device__ __forceinline__ void paley_mix(float (&z)[C], std::integer_sequence<int, Hs...>) {
+  (paley_mix_h<K, HI, Hs>(z), ...);
+}
+
+// The rest of the block rotation for one output index: z[c] = D[i', c] on
+// entry, the unnormalised y[c * 128 + i'] on exit.
+template <int K, int HI, int C>
+__device__ __forceinline__ void tck_finish(float (&z)[C]) {
+#pragma unroll
+  for (int d = 1; d < HI; d <<= 1) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      if (((c % HI) & d) == 0) {
+        const float u = z[c], w = z[c + d];
+        z[c] = __fadd_rn(u, w);
+        z[c + d] = __fsub_rn(u, w);
+      }
+    }
+  }
+  paley_mix<K, HI>(z, std::make_integer_sequence<int, HI>{});
+}
+
+// MODE: OUT_F32 / OUT_BF16, or -1 for per-token int8 (one block = one row).
+template <class C, int MODE>
+__global__ void __launch_bounds__(C::THREADS, 1)
+tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
+           const uint16_t* __restrict__ x, int64_t blocks, float norm, void* __restrict__ out0,
+           void* __restrict__ out1) {
+  constexpr bool PER_TOKEN = MODE < 0;
+  static_assert(PER_TOKEN || MODE == OUT_F32 || MODE == OUT_BF16, "rotation or per-token int8");
+  constexpr int NC = C::C;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  float* red = reinterpret_cast<float*>(smem + C::SM_RED);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_SLOT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int64_t kBlockElems = static_cast<int64_t>(NC) * 128;
+
+  if (threadIdx.x == 0) {
+    int64_t t = blockIdx.x;
+    for (int i = 0; i < C::PREFETCH && t < blocks; ++i, t += gridDim.x)
+      prefetch_l2(x + t * kBlockElems, static_cast<uint32_t>(kBlockElems * 2));
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);             // the 4 warps of the group that took the block
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      grid_dependency_sync();
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < blocks; t += gridDim.x, ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (it >= C::STAGES && !mbar_wait(&empty[s], ph ^ 1)) {
+          atomicOr(&hadq_tc_fault, kFaultProducer);
+          drain_loads(full, C::STAGES, it);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], C::TILE_BYTES);
+        uint8_t* dst = smem + C::SM_B + s * C::TILE_BYTES;
+        const int c0 = static_cast<int>(t * NC);   // first chunk of the block
+        tma_load_2d(dst, &map_p0, 0, c0, &full[s]);
+        tma_load_2d(dst + C::PANEL_BYTES, &map_p1, 0, c0, &full[s]);
+      }
+    }
+  } else {
+    // A = H_128, K-major with the 128-byte swizzle (row m holds H[m][k] over k).
+    for (int i = threadIdx.x - 32; i < 128 * 16; i += C::THREADS - 32) {
+      const int m = i >> 4, kc = i & 15;
+      uint32_t w[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int k = kc * 8 + 2 * p;
+        w[p] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+      }
+      const int panel = kc >> 3, chunk = kc & 7;
+      const uint32_t off = panel * 16384 + m * 128 + ((chunk ^ (m & 7)) << 4);
+      *reinterpret_cast<uint4*>(smem + C::SM_A + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(512));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(C::THREADS - 32) : "memory");
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 1) {
+      // ------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t h_base = smem_u32(smem + C::SM_A);
+        uint32_t it = 0;
+        for (int64_t t = blockIdx.x; t < blocks; t += gridDim.x, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          const int b = it % C::ACC_BUFS;
+          const uint32_t aph = (it / C::ACC_BUFS) & 1;
+          if (!mbar_wait(&full[s], ph) || (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
+            atomicOr(&hadq_tc_fault, kFaultMma);
+            drain_mmas(empty, C::STAGES, it);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t x_base = smem_u32(smem + C::SM_B + s * C::TILE_BYTES);
+          const uint32_t d = tmem_base + b * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff_h = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t koff_x = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
+            mma_bf16(d, smem_desc(h_base + koff_h, 16, 1024, kSwizzle128),
+                     smem_desc(x_base + koff_x, 16, 1024, kSwizzle128), C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&acc_full[b]);
+        }
+      }
+    } else {
+      // --------------------------------------------------------- epilogue
+      grid_dependency_sync();
+      const int quarter = warp & 3;
+      const int group_id = (warp - 2) >> 2;
+      const int ip = quarter * 32 + lane;       // output index within each chunk = TMEM lane
+      uint32_t it = 0;
+      bool failed = false;   // a wait ran out: skip the work, keep joining the group's barriers
+      float* gred = red + 4 * group_id;
+      const int bar = 2 + group_id;
+      for (int64_t t = blockIdx.x; t < blocks; t += gridDim.x, ++it) {
+        if (static_cast<int>(it % C::EPI_GROUPS) != group_id) continue;
+        const int b = it % C::ACC_BUFS;
+        const uint32_t aph = (it / C::ACC_BUFS) & 1;
+        if (!failed && !mbar_wait(&acc_full[b], aph)) {
+          atomicOr(&hadq_tc_fault, kFaultEpilogue);
+          failed = true;
+        }
+        if (failed) {
+          if constexpr (PER_TOKEN) {
+            asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+            asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+          }
+          continue;
+        }
+        tc_fence_after();
+        float z[NC];
+        tmem_ld_cols<NC>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128, z);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        tck_finish<C::K, C::HI>(z);
+        const int64_t e0 = t * kBlockElems + ip;   // output of chunk c at e0 + 128 c
+        if constexpr (PER_TOKEN) {
+          float mz = absmax_regs(z, 0, NC);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, off));
+          if (lane == 0) gred[quarter] = mz;
+          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+          const float m = fmaxf(fmaxf(gred[0], gred[1]), fmaxf(gred[2], gred[3])) * norm;
+          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");   // gred may be rewritten next block
+          // The per-token int8 arithmetic of the other kernels: s = fp32(m / 127),
+          // codes rne(z * (norm / s)); a tiny scale divides per element.
+          const float s = int8_scale(m);
+          const bool tiny = s > 0.f && s < 1.0e-36f;
+          const float rn = (s >= 1.0e-36f && s <= 3.0e38f) ? code_factor(norm, s) : 0.f;
+          uint8_t* codes = static_cast<uint8_t*>(out0) + e0;
+          if (!tiny) {
+            const float2 r2 = make_float2(rn, rn), m2 = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+            for (int c = 0; c < NC; c += 2) {
+              const float2 p = __ffma2_rn(make_float2(z[c], z[c + 1]), r2, m2);
+              codes[128 * c] = static_cast<uint8_t>(__float_as_uint(p.x) & 0xFFu);
+              codes[128 * (c + 1)] = static_cast<uint8_t>(__float_as_uint(p.y) & 0xFFu);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+              const float q = fminf(fmaxf(__fdiv_rn(z[c] * norm, s), -127.f), 127.f);
+              codes[128 * c] = static_cast<uint8_t>((__float_as_uint(__fadd_rn(q, kRoundMagic)) - kRoundMagicBits) & 0xFFu);
+            }
+          }
+          if (ip == 0) static_cast<float*>(out1)[t] = s;
+        } else if constexpr (MODE == OUT_BF16) {
+          uint16_t* o = static_cast<uint16_t*>(out0) + e0;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) o[128 * c] = __bfloat16_as_ushort(__float2bfloat16_rn(z[c] * norm));
+        } else {
+          float* o = static_cast<float*>(out0) + e0;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) o[128 * c] = z[c] * norm;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512));
+  }
+}
+
+}  // namespace tc
+}  // namespace hadq

@@ -1,0 +1,66 @@
+// Instantiations of the tensor-core kernels for blocks of K * 128 * HI
+// elements (hadq_tck.cuh) and their lookup; this unit owns their fault word.
+#include "hadq_launch.h"
+#include "hadq_tck.cuh"
+
+namespace hadq {
+namespace launch {
+namespace {
+
+// 4 stages of one block each, two epilogue groups (a thread holds up to 128
+// values plus the K-point mix's temporaries, so 10 warps of up to 204
+// registers), 8 blocks per CTA prefetched into L2 at entry.
+template <int K, int HI, int MODE>
+TckVariant tck_variant() {
+  using C = tc::TckCfg<K, HI, 4, 2, 8>;
+  return TckVariant{&tc::tck_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::NP};
+}
+
+template <int K, int HI>
+TckVariant tck_modes(int mode) {
+  switch (mode) {
+    case OUT_F32: return tck_variant<K, HI, OUT_F32>();
+    case OUT_BF16: return tck_variant<K, HI, OUT_BF16>();
+    case -1: return tck_variant<K, HI, -1>();
+    default: return TckVariant{nullptr, 0, 0, 0};
+  }
+}
+
+}  // namespace
+
+// Every Paley order with K * HI <= 128 chunks.
+TckVariant tck_kernel_for(int k, int hi, int mode) {
+  switch (k * 1000 + hi) {
+    case 12001: return tck_modes<12, 1>(mode);
+    case 12002: return tck_modes<12, 2>(mode);
+    case 12004: return tck_modes<12, 4>(mode);
+    case 12008: return tck_modes<12, 8>(mode);
+    case 20001: return tck_modes<20, 1>(mode);
+    case 20002: return tck_modes<20, 2>(mode);
+    case 20004: return tck_modes<20, 4>(mode);
+    case 28001: return tck_modes<28, 1>(mode);
+    case 28002: return tck_modes<28, 2>(mode);
+    case 28004: return tck_modes<28, 4>(mode);
+    case 36001: return tck_modes<36, 1>(mode);
+    case 36002: return tck_modes<36, 2>(mode);
+    case 52001: return tck_modes<52, 1>(mode);
+    case 52002: return tck_modes<52, 2>(mode);
+    case 60001: return tck_modes<60, 1>(mode);
+    case 60002: return tck_modes<60, 2>(mode);
+    case 108001: return tck_modes<108, 1>(mode);
+    default: return TckVariant{nullptr, 0, 0, 0};
+  }
+}
+
+int tck_fault_bits(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tc::hadq_tc_fault, sizeof(v)) != cudaSuccess) return -1;
+  if (clear && v != 0) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(tc::hadq_tc_fault, &z, sizeof(z)) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(v);
+}
+
+}  // namespace launch
+}  // namespace hadq

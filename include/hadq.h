@@ -326,8 +326,11 @@ HADQ_API int hadq_version(void);
  * Implementation choice.  Two implementations compute the same operation:
  * the tensor-core kernels (tcgen05 MMA with H_128 for the high index bits,
  * operands staged by TMA) and the CUDA-core butterfly kernels.  The tensor-core
- * kernels cover bf16 input at full size 4096 / 8192 and at block 128; every
- * other call runs the butterfly kernels whatever the choice.
+ * kernels cover bf16 input at full size 4096 / 8192 and at block 128 (every
+ * format and sign variant), and blocks of K * 2^m with 2^m >= 128 and
+ * K * 2^m / 128 <= 128 chunks (no signs or permutation; rotation outputs, and
+ * per-token int8 when the block is the whole row); every other call runs the
+ * butterfly (staged) kernels whatever the choice.
  *   HADQ_IMPL_AUTO       the default: the tensor-core kernels wherever they apply
  *   HADQ_IMPL_TENSOR     the same (named for callers that want to say so)
  *   HADQ_IMPL_BUTTERFLY  the butterfly kernels everywhere
