@@ -22,12 +22,14 @@
 //             z_2i - z_2i+1), F = sum_{i >= 1} w_i and P_i = the sum of the w_i'
 //             with chi(a_i' - a_i) = +1 (a_i = field element of row i >= 1),
 //               y_0 = F + (w_0.y, -w_0.x),
-//               y_i = w_0 + 2 P_i - F + w_i + (w_i.y, -w_i.x),
+//               y_i = w_0 + 2 P_i - F + w_i + (w_i.y, -w_i.x)
+//                   = (w_0 - F) + 2 (P_i + (z_2i, -z_2i+1)),
 //             since row i of C sums its field columns to 2 P_i - (F - w_i)
 //             and adds w_0, and B adds (w_i.y, -w_i.x).  The sign pattern is a
-//             compile-time table, so a column costs about q^2 / 2 + 5 q packed
-//             f32x2 adds; results go to a shared fp32 buffer whose 64-value
-//             runs are padded to 68 words (128-bit accesses without conflicts);
+//             compile-time table and the P_i share pair sums, so a column
+//             costs about q^2 / 3 + 4 q packed f32x2 operations; results go to
+//             a shared fp32 buffer whose 64-value runs are padded to 68 words
+//             (128-bit accesses without conflicts);
 //   2^m stage each thread takes one 64-value run of one sub-block: 6 butterfly
 //             stages in registers, and those of the remaining S_lo points
 //             with shuffles across the neighbouring lanes that hold the
@@ -107,7 +109,103 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return r;
 }
 
-// acc += w[T + 1] where chi(a_T - a_(I-1)) = +1 (row I of C, field column T).
+// The residue sums P_I share work: for every output pair the set of field
+// columns T with chi(T - a_(I-1)) = +1 is covered by neighbouring index pairs
+// {t, t + 1 (mod q)} (their sums w_t + w_(t+1) computed once for all rows)
+// and single columns.  For prime q the sets are translates of the residues,
+// so every row finds the same pairs (q = 13: 2 pairs + 2 singles, 52 packed
+// adds for all P_I instead of 65).
+template <int K>
+struct PaleyCover {
+  static constexpr int q = Paley<K>::q;
+  struct Table {
+    int cnt[q];            // terms of row r (output pair r + 1)
+    int term[q][q];        // field column index of each term
+    bool pair[q][q];       // the term is the pair sum starting at that column
+    bool pair_used[q];     // some row uses the pair sum starting at column t
+  };
+  static constexpr Table make() {
+    Table tab{};
+    for (int r = 0; r < q; ++r) {
+      bool in[q] = {}, used[q] = {};
+      for (int t = 0; t < q; ++t) in[t] = Paley<K>::tab.plus[t][r];
+      int n = 0;
+      for (int t = 0; t < q; ++t) {
+        const int u = (t + 1) % q;
+        if (in[t] && !used[t] && in[u] && !used[u]) {
+          used[t] = used[u] = true;
+          tab.term[r][n] = t;
+          tab.pair[r][n] = true;
+          tab.pair_used[t] = true;
+          ++n;
+        }
+      }
+      for (int t = 0; t < q; ++t)
+        if (in[t] && !used[t]) {
+          used[t] = true;
+          tab.term[r][n] = t;
+          tab.pair[r][n] = false;
+          ++n;
+        }
+      tab.cnt[r] = n;
+    }
+    return tab;
+  }
+  static constexpr Table tab = make();
+};
+
+template <int K, int T>
+__device__ __forceinline__ void pair_sum_if_used(const float2* w, float2* ps) {
+  if constexpr (PaleyCover<K>::tab.pair_used[T]) ps[T] = add2(w[T + 1], w[(T + 1) % Paley<K>::q + 1]);
+}
+
+template <int K, int... Ts>
+__device__ __forceinline__ void pair_sums(const float2* w, float2* ps, std::integer_sequence<int, Ts...>) {
+  (pair_sum_if_used<K, Ts>(w, ps), ...);
+}
+
+template <int K, int R, int J>
+__device__ __forceinline__ float2 cover_term(const float2* w, const float2* ps) {
+  constexpr int t = PaleyCover<K>::tab.term[R][J];
+  if constexpr (PaleyCover<K>::tab.pair[R][J]) return ps[t];
+  else return w[t + 1];
+}
+
+template <int K, int R, int... Js>
+__device__ __forceinline__ float2 cover_sum(const float2* w, const float2* ps, std::integer_sequence<int, Js...>) {
+  float2 acc = cover_term<K, R, 0>(w, ps);
+  ((acc = add2(acc, cover_term<K, R, Js + 1>(w, ps))), ...);
+  return acc;
+}
+
+// w[L] + ... + w[L + N - 1] as a balanced tree (short dependency chains).
+template <int L, int N>
+__device__ __forceinline__ float2 tree_sum(const float2* w) {
+  if constexpr (N == 1) return w[L];
+  else return add2(tree_sum<L, N / 2>(w), tree_sum<L + N / 2, N - N / 2>(w));
+}
+
+// Output pair I >= 1.  With a_i + b_i = 2 z_2i and b_i - a_i = -2 z_2i+1,
+//   y_I = w_0 + 2 P_I - F + w_I + (w_I.y, -w_I.x) = G + 2 (P_I + (z_2I, -z_2I+1)),
+// G = w_0 - F: two packed fused multiply-adds per pair.
+template <int K, int I, class Put>
+__device__ __forceinline__ void output_pair(const float* z, const float2* w, const float2* ps, float2 g, Put& put) {
+  const float2 p = cover_sum<K, I - 1>(w, ps, std::make_integer_sequence<int, PaleyCover<K>::tab.cnt[I - 1] - 1>{});
+  const float2 t = __ffma2_rn(make_float2(z[2 * I], z[2 * I + 1]), make_float2(1.f, -1.f), p);
+  const float2 y = __ffma2_rn(t, make_float2(2.f, 2.f), g);
+  put(2 * I, y.x);
+  put(2 * I + 1, y.y);
+}
+
+template <int K, class Put, int... Is>
+__device__ __forceinline__ void output_pairs(const float* z, const float2* w, const float2* ps, float2 g, Put& put,
+                                             std::integer_sequence<int, Is...>) {
+  (output_pair<K, Is + 1>(z, w, ps, g, put), ...);
+}
+
+// Compact form for the large orders (K >= 52), where keeping the inputs and
+// the pair sums live as well would spill registers: the residue sums taken
+// column by column, y_I = w_0 + 2 P_I - F + w_I + (w_I.y, -w_I.x).
 template <int K, int I, int T>
 __device__ __forceinline__ void add_if_plus(float2& acc, const float2* w) {
   if constexpr (Paley<K>::tab.plus[T][I - 1]) acc = add2(acc, w[T + 1]);
@@ -120,10 +218,8 @@ __device__ __forceinline__ float2 plus_sum(const float2* w, std::integer_sequenc
   return acc;
 }
 
-// Output pair I >= 1: y_I = w_0 + 2 P_I - F + w_I + (w_I.y, -w_I.x), written to
-// column-major rows 2I, 2I + 1 of the shared buffer through `put`.
 template <int K, int I, class Put>
-__device__ __forceinline__ void output_pair(const float2* w, float2 f, Put& put) {
+__device__ __forceinline__ void output_pair_compact(const float2* w, float2 f, Put& put) {
   const float2 pp = plus_sum<K, I>(w, std::make_integer_sequence<int, Paley<K>::q>{});
   float2 t = __ffma2_rn(pp, make_float2(2.f, 2.f), w[0]);
   t = sub2(t, f);
@@ -134,27 +230,46 @@ __device__ __forceinline__ void output_pair(const float2* w, float2 f, Put& put)
 }
 
 template <int K, class Put, int... Is>
-__device__ __forceinline__ void output_pairs(const float2* w, float2 f, Put& put, std::integer_sequence<int, Is...>) {
-  (output_pair<K, Is + 1>(w, f, put), ...);
+__device__ __forceinline__ void output_pairs_compact(const float2* w, float2 f, Put& put,
+                                                     std::integer_sequence<int, Is...>) {
+  (output_pair_compact<K, Is + 1>(w, f, put), ...);
 }
 
 // One column: z_k = get(k) for k < K; y = z . H_K written through put(k, y_k).
+// Every get happens before the first put, so get and put may address the
+// same storage.  Orders up to 36 share pair sums and use the two-FMA output
+// form; the large orders take the compact form.
 template <int K, class Get, class Put>
 __device__ __forceinline__ void kstage_column(Get& get, Put& put) {
   constexpr int q = Paley<K>::q;
-  float2 w[q + 1];
+  if constexpr (K >= 52) {
+    float2 w[q + 1];
 #pragma unroll
-  for (int i = 0; i <= q; ++i) {
-    const float a = get(2 * i), b = get(2 * i + 1);
-    w[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    for (int i = 0; i <= q; ++i) {
+      const float a = get(2 * i), b = get(2 * i + 1);
+      w[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+    const float2 f = tree_sum<1, q>(w);
+    const float2 y0 = add2(f, make_float2(w[0].y, -w[0].x));
+    put(0, y0.x);
+    put(1, y0.y);
+    output_pairs_compact<K>(w, f, put, std::make_integer_sequence<int, q>{});
+  } else {
+    float z[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) z[k] = get(k);
+    float2 w[q + 1];
+#pragma unroll
+    for (int i = 0; i <= q; ++i)
+      w[i] = make_float2(__fadd_rn(z[2 * i], z[2 * i + 1]), __fsub_rn(z[2 * i], z[2 * i + 1]));
+    const float2 f = tree_sum<1, q>(w);
+    float2 ps[q];
+    pair_sums<K>(w, ps, std::make_integer_sequence<int, q>{});
+    put(0, __fadd_rn(f.x, w[0].y));
+    put(1, __fsub_rn(f.y, w[0].x));
+    const float2 g = sub2(w[0], f);
+    output_pairs<K>(z, w, ps, g, put, std::make_integer_sequence<int, q>{});
   }
-  float2 f = w[1];
-#pragma unroll
-  for (int i = 2; i <= q; ++i) f = add2(f, w[i]);
-  const float2 y0 = add2(f, make_float2(w[0].y, -w[0].x));
-  put(0, y0.x);
-  put(1, y0.y);
-  output_pairs<K>(w, f, put, std::make_integer_sequence<int, q>{});
 }
 
 constexpr int kMaxThreads = 512;

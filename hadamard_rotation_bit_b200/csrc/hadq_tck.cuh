@@ -124,17 +124,29 @@ __device__ __forceinline__ void paley_mix(float (&z)[C], std::integer_sequence<i
 
 // The rest of the block rotation for one output index: z[c] = D[i', c] on
 // entry, the unnormalised y[c * 128 + i'] on exit.
+// Stages of stride d >= 2 pair neighbouring h and run as packed f32x2 adds.
 template <int K, int HI, int C>
 __device__ __forceinline__ void tck_finish(float (&z)[C]) {
 #pragma unroll
-  for (int d = 1; d < HI; d <<= 1) {
+  for (int d = 2; d < HI; d <<= 1) {
 #pragma unroll
-    for (int c = 0; c < C; ++c) {
+    for (int c = 0; c < C; c += 2) {
       if (((c % HI) & d) == 0) {
-        const float u = z[c], w = z[c + d];
-        z[c] = __fadd_rn(u, w);
-        z[c + d] = __fsub_rn(u, w);
+        const float2 u = make_float2(z[c], z[c + 1]), w = make_float2(z[c + d], z[c + d + 1]);
+        const float2 s = ksize::add2(u, w), t = ksize::sub2(u, w);
+        z[c] = s.x;
+        z[c + 1] = s.y;
+        z[c + d] = t.x;
+        z[c + d + 1] = t.y;
       }
+    }
+  }
+  if constexpr (HI > 1) {
+#pragma unroll
+    for (int c = 0; c < C; c += 2) {
+      const float u = z[c], w = z[c + 1];
+      z[c] = __fadd_rn(u, w);
+      z[c + 1] = __fsub_rn(u, w);
     }
   }
   paley_mix<K, HI>(z, std::make_integer_sequence<int, HI>{});

@@ -7,12 +7,14 @@ namespace hadq {
 namespace launch {
 namespace {
 
-// 4 stages of one block each, two epilogue groups (a thread holds up to 128
-// values plus the K-point mix's temporaries, so 10 warps of up to 204
-// registers), 8 blocks per CTA prefetched into L2 at entry.
+// 4 stages of one block each, 8 blocks per CTA prefetched into L2 at entry.
+// A thread holds one value per chunk plus the K-point mix's temporaries: two
+// epilogue groups (10 warps, at most 168 registers each) up to 96 chunks and
+// for 28 x 4; one group (6 warps, up to 255 registers) for the larger blocks,
+// where two groups would spill.
 template <int K, int HI, int MODE>
 TckVariant tck_variant() {
-  using C = tc::TckCfg<K, HI, 4, 2, 8>;
+  using C = tc::TckCfg<K, HI, 4, (K * HI > 96 && K != 28 ? 1 : 2), 8>;
   return TckVariant{&tc::tck_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::NP};
 }
 
