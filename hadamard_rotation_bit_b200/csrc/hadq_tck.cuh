@@ -19,19 +19,26 @@
 // 2-D tensor maps (columns beyond C hold whatever follows the block and are
 // never read).  Operands are exact in bf16; products accumulate in fp32 in
 // tensor memory.  TMEM lane i' then holds output index i' of every chunk of
-// the block, so the rest of the rotation runs in one thread's registers with
-// no data exchange: H_HI over h (Sylvester stages), then the Paley K-point
-// mix over k for each h (the compile-time residue table of hadq_ksize.cuh).
-// The thread's outputs y[c * 128 + i'] are one per chunk: for each chunk a
-// warp writes 32 consecutive outputs.
+// the block, so the rest of the rotation -- H_HI over h (Sylvester stages),
+// then the Paley K-point mix over k for each h (the compile-time residue table
+// of hadq_ksize.cuh) -- needs no data exchange between threads.  Each thread
+// works through its lane in passes, with tensor memory as scratch, so that
+// only one step's values are in registers at a time (at most K plus the
+// mix's temporaries, not K * HI): pass A, per window of 4 values of k, H_HI
+// and a write-back that puts each h's values in 4-column pieces; pass B, per
+// h, the K-point mix (rotation outputs leave from here); pass C, per-token
+// int8 only, after the row absmax is known, the codes.  The small register
+// footprint buys epilogue warps: up to four groups of 4, against two when a
+// thread held a value of every chunk.  A thread's outputs y[c * 128 + i'] are
+// one per chunk, so for each chunk a warp writes 32 consecutive outputs.
 //
 // Roles as in the block-128 kernel: warp 0 TMA producer, warp 1 TMEM
 // allocator and single-thread MMA issuer, then EPI_GROUPS groups of 4
-// epilogue warps (one TMEM lane quarter each) taking whole blocks round-robin.
-// Per-token int8 takes a whole row per block (b = n) and joins the row absmax
-// of the group's 4 warps in shared memory.  Every wait is bounded
-// (hadq_tc_fault), and thread 0 first asks L2 to prefetch the CTA's first
-// PREFETCH blocks.
+// epilogue warps (one TMEM lane quarter each) taking whole blocks round-robin,
+// each holding its block's accumulator until pass C has read it.  Per-token
+// int8 takes a whole row per block (b = n) and joins the row absmax of the
+// group's 4 warps in shared memory.  Every wait is bounded (hadq_tc_fault),
+// and thread 0 first asks L2 to prefetch the CTA's first PREFETCH blocks.
 #pragma once
 
 #include <utility>
@@ -109,47 +116,211 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&z)[C]) {
   if constexpr (R & 4) tmem_ld4(taddr + C32 + (R & 24), &z[C32 + (R & 24)]);
 }
 
-// H_K over k of the values z[k * HI + H] (one h = H).
-template <int K, int HI, int H, int C>
-__device__ __forceinline__ void paley_mix_h(float (&z)[C]) {
-  auto get = [&](int k) { return z[k * HI + H]; };
-  auto put = [&](int k, float v) { z[k * HI + H] = v; };
-  ksize::kstage_column<K>(get, put);   // reads every value before writing any
+// Tensor-memory stores of 4, 8 and 32 consecutive 32-bit columns of this
+// thread's lane (16: tmem_st16), and N-column loads and stores by size.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 
-template <int K, int HI, int C, int... Hs>
-__device__ __forceinline__ void paley_mix(float (&z)[C], std::integer_sequence<int, Hs...>) {
-  (paley_mix_h<K, HI, Hs>(z), ...);
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+               : "memory");
 }
 
-// The rest of the block rotation for one output index: z[c] = D[i', c] on
-// entry, the unnormalised y[c * 128 + i'] on exit.
-// Stages of stride d >= 2 pair neighbouring h and run as packed f32x2 adds.
-template <int K, int HI, int C>
-__device__ __forceinline__ void tck_finish(float (&z)[C]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  tmem_st16(taddr, r);
+  tmem_st16(taddr + 16, r + 16);
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float* v) {
+  static_assert(N == 4 || N == 8 || N == 16 || N == 32, "4, 8, 16 or 32 columns");
+  if constexpr (N == 4) tmem_ld4(taddr, v);
+  else if constexpr (N == 8) tmem_ld8(taddr, v);
+  else if constexpr (N == 16) tmem_ld16(taddr, v);
+  else tmem_ld32(taddr, v);
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t* r) {
+  static_assert(N == 4 || N == 8 || N == 16 || N == 32, "4, 8, 16 or 32 columns");
+  if constexpr (N == 4) tmem_st4(taddr, r);
+  else if constexpr (N == 8) tmem_st8(taddr, r);
+  else if constexpr (N == 16) tmem_st16(taddr, r);
+  else tmem_st32(taddr, r);
+}
+
+// Columns [0, C) of this thread's lane from registers, C a multiple of 4.
+template <int C>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float (&z)[C]) {
+  uint32_t r[C];
 #pragma unroll
-  for (int d = 2; d < HI; d <<= 1) {
+  for (int i = 0; i < C; ++i) r[i] = __float_as_uint(z[i]);
+  constexpr int C32 = C / 32 * 32;
 #pragma unroll
-    for (int c = 0; c < C; c += 2) {
-      if (((c % HI) & d) == 0) {
-        const float2 u = make_float2(z[c], z[c + 1]), w = make_float2(z[c + d], z[c + d + 1]);
-        const float2 s = ksize::add2(u, w), t = ksize::sub2(u, w);
-        z[c] = s.x;
-        z[c + 1] = s.y;
-        z[c + d] = t.x;
-        z[c + d + 1] = t.y;
+  for (int c = 0; c < C32; c += 32) tmem_st32(taddr + c, &r[c]);
+  constexpr int R = C - C32;
+  if constexpr (R & 16) tmem_st16(taddr + C32, &r[C32]);
+  if constexpr (R & 8) tmem_st8(taddr + C32 + (R & 16), &r[C32 + (R & 16)]);
+  if constexpr (R & 4) tmem_st4(taddr + C32 + (R & 24), &r[C32 + (R & 24)]);
+}
+
+// Scratch layout of the tensor-memory epilogue: with HI > 1 the columns are
+// windows of 4 values of k, each window holding its 4 * HI values h-major
+// (position j W + 4 h + kl for chunk (4 j + kl) HI + h, W = 4 HI); with HI = 1
+// position and chunk coincide.
+template <int HI>
+__host__ __device__ constexpr int scratch_chunk(int p) {
+  if (HI == 1) return p;
+  return (4 * (p / (4 * HI)) + (p % (4 * HI)) % 4) * HI + (p % (4 * HI)) / 4;
+}
+
+// Outputs of the values v[0, N) read from scratch positions P0 .. P0 + N - 1:
+// chunk c = scratch_chunk(P0 + i) goes to element e0 + 128 c.  Per-token int8
+// uses the arithmetic of the other kernels (codes rne(v * rn) by the
+// round-magic FMA; a tiny scale divides per element).
+template <int HI, int P0, int N, int MODE>
+__device__ __forceinline__ void tck_emit(const float* v, float norm, float s, float rn, bool tiny, void* out0,
+                                         int64_t e0) {
+  if constexpr (MODE < 0) {
+    uint8_t* codes = static_cast<uint8_t*>(out0) + e0;
+    if (!tiny) {
+      const float2 r2 = make_float2(rn, rn), m2 = make_float2(kRoundMagic, kRoundMagic);
+#pragma unroll
+      for (int i = 0; i < N; i += 2) {
+        const float2 q = __ffma2_rn(make_float2(v[i], v[i + 1]), r2, m2);
+        codes[128 * scratch_chunk<HI>(P0 + i)] = static_cast<uint8_t>(__float_as_uint(q.x) & 0xFFu);
+        codes[128 * scratch_chunk<HI>(P0 + i + 1)] = static_cast<uint8_t>(__float_as_uint(q.y) & 0xFFu);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const float q = fminf(fmaxf(__fdiv_rn(v[i] * norm, s), -127.f), 127.f);
+        codes[128 * scratch_chunk<HI>(P0 + i)] =
+            static_cast<uint8_t>((__float_as_uint(__fadd_rn(q, kRoundMagic)) - kRoundMagicBits) & 0xFFu);
+      }
+    }
+  } else if constexpr (MODE == OUT_BF16) {
+    uint16_t* o = static_cast<uint16_t*>(out0) + e0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) o[128 * scratch_chunk<HI>(P0 + i)] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i] * norm));
+  } else {
+    float* o = static_cast<float*>(out0) + e0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) o[128 * scratch_chunk<HI>(P0 + i)] = v[i] * norm;
+  }
+}
+
+// Pass C of the scratch epilogue: positions [P0, C) in pieces of up to 32.
+template <int HI, int C, int MODE, int P0>
+__device__ __forceinline__ void tck_emit_from(uint32_t tb, float norm, float s, float rn, bool tiny, void* out0,
+                                              int64_t e0) {
+  if constexpr (P0 < C) {
+    constexpr int L = C - P0;
+    constexpr int N = L >= 32 ? 32 : (L >= 16 ? 16 : (L >= 8 ? 8 : 4));
+    float v[N];
+    tmem_ldn<N>(tb + P0, v);
+    tmem_wait_ld();
+    tck_emit<HI, P0, N, MODE>(v, norm, s, rn, tiny, out0, e0);
+    tck_emit_from<HI, C, MODE, P0 + N>(tb, norm, s, rn, tiny, out0, e0);
+  }
+}
+
+// One block through tensor memory (tb = this thread's lane, first column of
+// the block's accumulator).  Pass A (HI > 1): per window of 4 values of k,
+// H_HI over h, written back h-major.  Pass B: per h, the K-point mix of the K
+// values of that h (one 4-column piece per window), written back; rotation
+// outputs leave from here.  Per-token int8 then joins the row absmax of the
+// group and, pass C, reads the block back and stores the codes.  Returns after
+// the last tensor-memory read of the block.
+template <int K, int HI, int MODE>
+__device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void* out0, void* out1, int64_t t,
+                                                  int64_t e0, int lane, int quarter, float* gred, int bar) {
+  constexpr int C = K * HI, W = 4 * HI;
+  if constexpr (HI > 1) {
+#pragma unroll 1
+    for (int j = 0; j < K / 4; ++j) {
+      float v[W];
+      tmem_ldn<W>(tb + j * W, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int d = 1; d < HI; d <<= 1) {
+#pragma unroll
+        for (int i = 0; i < W; ++i) {
+          if (((i % HI) & d) == 0) {
+            const float u = v[i], w = v[i + d];
+            v[i] = __fadd_rn(u, w);
+            v[i + d] = __fsub_rn(u, w);
+          }
+        }
+      }
+      uint32_t o[W];
+#pragma unroll
+      for (int kl = 0; kl < 4; ++kl)
+#pragma unroll
+        for (int h = 0; h < HI; ++h) o[4 * h + kl] = __float_as_uint(v[kl * HI + h]);
+      tmem_stn<W>(tb + j * W, o);
+    }
+    tmem_wait_st();
+  }
+  float mz = 0.f;
+#pragma unroll 1
+  for (int h = 0; h < HI; ++h) {
+    float z[K];
+    if constexpr (HI == 1) {
+      tmem_ld_cols<K>(tb, z);
+    } else {
+#pragma unroll
+      for (int j = 0; j < K / 4; ++j) tmem_ld4(tb + j * W + 4 * h, &z[4 * j]);
+    }
+    tmem_wait_ld();
+    auto get = [&](int k) { return z[k]; };
+    auto put = [&](int k, float v) { z[k] = v; };
+    ksize::kstage_column<K>(get, put);
+    if constexpr (MODE < 0) {
+      mz = fmaxf(mz, absmax_regs(z, 0, K));
+      if constexpr (HI == 1) {
+        tmem_st_cols<K>(tb, z);
+      } else {
+#pragma unroll
+        for (int j = 0; j < K / 4; ++j) {
+          const uint32_t r[4] = {__float_as_uint(z[4 * j]), __float_as_uint(z[4 * j + 1]), __float_as_uint(z[4 * j + 2]),
+                                 __float_as_uint(z[4 * j + 3])};
+          tmem_st4(tb + j * W + 4 * h, r);
+        }
+      }
+    } else {
+      // Value k of this h is chunk k HI + h.
+      float* of = static_cast<float*>(out0) + e0;
+      uint16_t* ob = static_cast<uint16_t*>(out0) + e0;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int64_t off = 128 * (static_cast<int64_t>(k) * HI + h);
+        if constexpr (MODE == OUT_BF16) ob[off] = __bfloat16_as_ushort(__float2bfloat16_rn(z[k] * norm));
+        else of[off] = z[k] * norm;
       }
     }
   }
-  if constexpr (HI > 1) {
+  if constexpr (MODE < 0) {
+    tmem_wait_st();
 #pragma unroll
-    for (int c = 0; c < C; c += 2) {
-      const float u = z[c], w = z[c + 1];
-      z[c] = __fadd_rn(u, w);
-      z[c + 1] = __fsub_rn(u, w);
-    }
+    for (int off = 16; off > 0; off >>= 1) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, off));
+    if (lane == 0) gred[quarter] = mz;
+    asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+    const float m = fmaxf(fmaxf(gred[0], gred[1]), fmaxf(gred[2], gred[3])) * norm;
+    asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");   // gred may be rewritten next block
+    const float s = int8_scale(m);
+    const bool tiny = s > 0.f && s < 1.0e-36f;
+    const float rn = (s >= 1.0e-36f && s <= 3.0e38f) ? code_factor(norm, s) : 0.f;
+    tck_emit_from<HI, C, MODE, 0>(tb, norm, s, rn, tiny, out0, e0);
+    if (quarter == 0 && lane == 0) static_cast<float*>(out1)[t] = s;
   }
-  paley_mix<K, HI>(z, std::make_integer_sequence<int, HI>{});
 }
 
 // MODE: OUT_F32 / OUT_BF16, or -1 for per-token int8 (one block = one row).
@@ -289,53 +460,11 @@ tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ C
           continue;
         }
         tc_fence_after();
-        float z[NC];
-        tmem_ld_cols<NC>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128, z);
-        tmem_wait_ld();
+        tck_block_scratch<C::K, C::HI, MODE>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128, norm,
+                                             out0, out1, t, t * kBlockElems + ip, lane, quarter, gred, bar);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        tck_finish<C::K, C::HI>(z);
-        const int64_t e0 = t * kBlockElems + ip;   // output of chunk c at e0 + 128 c
-        if constexpr (PER_TOKEN) {
-          float mz = absmax_regs(z, 0, NC);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mz = fmaxf(mz, __shfl_xor_sync(0xffffffffu, mz, off));
-          if (lane == 0) gred[quarter] = mz;
-          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
-          const float m = fmaxf(fmaxf(gred[0], gred[1]), fmaxf(gred[2], gred[3])) * norm;
-          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");   // gred may be rewritten next block
-          // The per-token int8 arithmetic of the other kernels: s = fp32(m / 127),
-          // codes rne(z * (norm / s)); a tiny scale divides per element.
-          const float s = int8_scale(m);
-          const bool tiny = s > 0.f && s < 1.0e-36f;
-          const float rn = (s >= 1.0e-36f && s <= 3.0e38f) ? code_factor(norm, s) : 0.f;
-          uint8_t* codes = static_cast<uint8_t*>(out0) + e0;
-          if (!tiny) {
-            const float2 r2 = make_float2(rn, rn), m2 = make_float2(kRoundMagic, kRoundMagic);
-#pragma unroll
-            for (int c = 0; c < NC; c += 2) {
-              const float2 p = __ffma2_rn(make_float2(z[c], z[c + 1]), r2, m2);
-              codes[128 * c] = static_cast<uint8_t>(__float_as_uint(p.x) & 0xFFu);
-              codes[128 * (c + 1)] = static_cast<uint8_t>(__float_as_uint(p.y) & 0xFFu);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-              const float q = fminf(fmaxf(__fdiv_rn(z[c] * norm, s), -127.f), 127.f);
-              codes[128 * c] = static_cast<uint8_t>((__float_as_uint(__fadd_rn(q, kRoundMagic)) - kRoundMagicBits) & 0xFFu);
-            }
-          }
-          if (ip == 0) static_cast<float*>(out1)[t] = s;
-        } else if constexpr (MODE == OUT_BF16) {
-          uint16_t* o = static_cast<uint16_t*>(out0) + e0;
-#pragma unroll
-          for (int c = 0; c < NC; ++c) o[128 * c] = __bfloat16_as_ushort(__float2bfloat16_rn(z[c] * norm));
-        } else {
-          float* o = static_cast<float*>(out0) + e0;
-#pragma unroll
-          for (int c = 0; c < NC; ++c) o[128 * c] = z[c] * norm;
-        }
       }
     }
   }

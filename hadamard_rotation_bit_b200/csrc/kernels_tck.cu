@@ -7,14 +7,21 @@ namespace hadq {
 namespace launch {
 namespace {
 
-// 4 stages of one block each, 8 blocks per CTA prefetched into L2 at entry.
-// A thread holds one value per chunk plus the K-point mix's temporaries: two
-// epilogue groups (10 warps, at most 168 registers each) up to 96 chunks and
-// for 28 x 4; one group (6 warps, up to 255 registers) for the larger blocks,
-// where two groups would spill.
+// 4 stages of one block each, 8 blocks per CTA prefetched into L2 at entry,
+// the epilogue through tensor memory.  Its widest step is the K-point mix of
+// one h (K values and the mix's temporaries in registers), so the number of
+// epilogue groups follows K: four (18 warps, at most 96 registers) up to
+// K = 28, three (14 warps, 128 registers) up to K = 60, one (6 warps) for
+// K = 108; fewer would leave warps idle, more would spill.  The accumulators
+// (4 x 128 TMEM columns) bound the groups at four.
+template <int K>
+constexpr int tck_groups() {
+  return K <= 28 ? 4 : (K <= 60 ? 3 : 1);
+}
+
 template <int K, int HI, int MODE>
 TckVariant tck_variant() {
-  using C = tc::TckCfg<K, HI, 4, (K * HI > 96 && K != 28 ? 1 : 2), 8>;
+  using C = tc::TckCfg<K, HI, 4, tck_groups<K>(), 8>;
   return TckVariant{&tc::tck_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::NP};
 }
 
