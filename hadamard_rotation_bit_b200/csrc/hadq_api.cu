@@ -350,6 +350,41 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                        "tensor-core block-128 kernel launch");
 }
 
+// RPBH at full size 4096, bf16 input, on the tensor cores (hadq_tcr.cuh): the
+// permutation and signs applied by gather warps in shared memory, then the
+// n = 4096 rotation and epilogue.  Rotation outputs, int4, MXFP4, NVFP4.
+bool tcr_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
+  return x_dtype == HADQ_BF16 && sh.kbase == 1 && sh.n == 4096 && sh.b == 4096 && mode >= 0 &&
+         mode != hadq::OUT_CODEBOOK;
+}
+
+hadq_status launch_tcr(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
+                       cudaStream_t stream, int sms, int dev, const int32_t* perm, const int8_t* signs) {
+  const hl::TcrVariant v = hl::tcr_kernel_for(mode);
+  if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no RPBH tensor-core kernel for this format");
+  constexpr int L = 32, R = 4;
+  if (sh.rows > (int64_t(1) << 31) - R) return fail(HADQ_ERR_UNSUPPORTED, "tensor-core path: too many rows");
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (encode == nullptr) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  CUtensorMap map;
+  cuuint64_t dims[3] = {L, 128, static_cast<cuuint64_t>(sh.rows)};
+  cuuint64_t strides[2] = {L * 2, static_cast<cuuint64_t>(sh.n) * 2};
+  cuuint32_t box[3] = {L, 128, R};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  int occ = 0;
+  hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
+  if (st != HADQ_OK) return st;
+  const int64_t tiles = (sh.rows + R - 1) / R;
+  const int64_t grid = std::min<int64_t>(tiles, sms);
+  return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, static_cast<const uint16_t*>(x), sh.rows,
+                                  static_cast<int>(sh.n), sh.norm, group, out0, out1, perm, signs),
+                       "RPBH tensor-core kernel launch");
+}
+
 // Blocks of b = K * 128 * hi bf16 elements on the tensor cores
 // (hadq_tck.cuh): H_128 on every 128-element chunk by one MMA, the H_hi and
 // Paley H_K factors in the registers of the thread that holds one output of
@@ -479,6 +514,9 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     seg_logs = std::min(sh.logs, std::max(std::max(sh.logb, ilog2(need)), 4));
   }
   (void)cudaGetLastError();   // launch errors below must be ours
+  if (ex.perm != nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
+      tcr_eligible(x_dtype, sh, mode))
+    return launch_tcr(x, sh, mode, group, out0, out1, stream, sms, dev, ex.perm, ex.rpbh_signs);
   if (ex.perm == nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
       tck_eligible(x_dtype, sh, mode, sg))
     return launch_tck(x, sh, mode, out0, out1, stream, sms, dev);

@@ -41,6 +41,13 @@ struct Tc128Variant {
 };
 
 using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, void*, void*);
+using TcrFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, const int32_t*,
+                       const int8_t*);
+
+struct TcrVariant {
+  TcrFn fn;
+  int threads, smem;
+};
 
 struct TckVariant {
   TckFn fn;
@@ -63,6 +70,7 @@ TeamRowFn team_row_kernel_bf16(int logb, bool sg);
 // per-token int8).
 TcVariant tc_kernel_for(int lo, int mode, int side);   // side: hadq::SignSide
 Tc128Variant tc128_kernel_for(int mode);   // signs of either side folded into B
+TcrVariant tcr_kernel_for(int mode);       // RPBH at full size 4096 (permutation gathered in shared memory)
 
 // Shared-memory staged kernels: blocks of K * 2^m elements (K a covered Paley
 // order 12 .. 108, or 1 with the RPBH permutation or the codebook quantizer);

@@ -1,0 +1,273 @@
+// Tensor-core variant of orbitquant's RPBH rotation at full size 4096, bf16
+// input ("orbitquant 0.2.0", Method Conformance: a random permutation of the
+// row's columns and one Rademacher sign per column, then the block Hadamard
+// rotation; here the block is the whole row).
+//
+// Row r of the output is y = H_4096 v / 64 with v_e = x[r][pi(e)] * s_e.  The
+// rotation is the n = 4096 tensor-core kernel's (hadq_tc.cuh): tiles of 4
+// rows, D = H_128 X_tile by one tcgen05 MMA per tile over the high 7 index
+// bits, the low 5 in the epilogue's registers.  The permutation moves data
+// across the whole row, so it cannot ride on the MMA operand or on the TMA
+// box; gather warps build each operand tile in shared memory instead:
+//
+//   TMA       the raw 4-row tile into one of RAW_STAGES raw stages;
+//   gather    for every output chunk of 8 columns e .. e + 7 of each row, 8
+//             16-bit loads from the raw tile at the swizzled places of
+//             pi(e) .. pi(e + 7), the signs applied by one XOR per pair, one
+//             16-byte store into a permuted stage laid out exactly as a TMA
+//             tile of v would be; then the raw stage goes back to the TMA
+//             producer and the permuted stage to the MMA;
+//   MMA       A = H_128 from tensor memory, B = the permuted stage;
+//   epilogue  as the n = 4096 kernel (LO = 5 register stages, quantizer).
+//
+// Each gather thread always owns the same two output chunks of every row, so
+// its 16 source offsets (two per word) and 8 sign words are computed once per
+// launch from the caller's permutation and signs.  Roles: warp 0 TMA
+// producer, warp 1 TMEM allocator and MMA issuer, warps 2..17 epilogue (one
+// row of each tile per group of 4), warps 18..25 gather.  Every wait is
+// bounded (hadq_tc_fault).
+#pragma once
+
+#include "hadq_tc.cuh"
+
+namespace hadq {
+namespace tc {
+
+struct TcrCfg {
+  static constexpr int LO = 5, L = 32, TILE_N = 128, R = 4, SPLIT = 4;
+  static constexpr int RAW_STAGES = 3, P_STAGES = 2;
+  static constexpr int PREFETCH = 2;                       // tiles per CTA prefetched into L2 at entry
+  static constexpr int GATHER_THREADS = 256;               // 2 output chunks of each row per thread
+  static constexpr int TILE_BYTES = 128 * TILE_N * 2;      // 4 rows of 4096 bf16
+  static constexpr int ROW_BYTES = TILE_BYTES / R;
+  static constexpr int ACC_BUFS = 3;                       // 3 x 128 TMEM columns, H_128 after them
+  static constexpr int A_COL = ACC_BUFS * TILE_N;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int FIRST_GATHER_WARP = 2 + 4 * SPLIT;
+  static constexpr int THREADS = 32 * FIRST_GATHER_WARP + GATHER_THREADS;
+  // kind::f16, fp32 accumulate, bf16 A and B, A K-major, B MN-major, N = 128, M = 128.
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                    (static_cast<uint32_t>(TILE_N >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+  static constexpr int SM_RAW = 0;
+  static constexpr int SM_P = SM_RAW + RAW_STAGES * TILE_BYTES;
+  static constexpr int SM_BARS = SM_P + P_STAGES * TILE_BYTES;
+  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * RAW_STAGES + 2 * P_STAGES + 2 * ACC_BUFS);
+  static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
+  static_assert(GATHER_THREADS * 2 * 8 == ROW_BYTES / 2, "two 8-column chunks of each row per gather thread");
+};
+
+// Byte offset within a row of the 64-byte-swizzled tile (the stage base is
+// 1024-byte aligned and a row is 8192 bytes, so only the in-row offset
+// decides the swizzle): 16-byte chunk bits 4..5 XOR address bits 7..8.
+__device__ __forceinline__ uint32_t swz64(uint32_t off) { return off ^ (((off >> 7) & 3u) << 4); }
+
+// MODE: an OutMode of tc_emit_row (rotation, int4, MXFP4, NVFP4).  perm: n
+// int32 source columns (entries outside [0, n) are clamped: memory-safe,
+// result unspecified); signs: n int8, negative = -1.
+template <int MODE>
+__global__ void __launch_bounds__(TcrCfg::THREADS, 1)
+tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
+               float norm, int group, void* __restrict__ out0, void* __restrict__ out1,
+               const int32_t* __restrict__ perm, const int8_t* __restrict__ signs) {
+  using C = TcrCfg;
+  constexpr int LO = C::LO, L = C::L, R = C::R;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);   // raw tile landed
+  uint64_t* empty = full + C::RAW_STAGES;                           // raw stage read by the gather
+  uint64_t* gathered = empty + C::RAW_STAGES;                       // permuted stage written
+  uint64_t* pfree = gathered + C::P_STAGES;                         // permuted stage read by the MMA
+  uint64_t* acc_full = pfree + C::P_STAGES;
+  uint64_t* acc_empty = acc_full + C::ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_SLOT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tiles = (rows + R - 1) / R;
+
+  if (threadIdx.x == 0) {
+    int64_t t = blockIdx.x;
+    for (int i = 0; i < C::PREFETCH && t < tiles; ++i, t += gridDim.x) {
+      const int64_t r1 = (t + 1) * R < rows ? (t + 1) * R : rows;
+      prefetch_l2(x + t * R * n, static_cast<uint32_t>((r1 - t * R) * n * 2));
+    }
+    for (int s = 0; s < C::RAW_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::GATHER_THREADS / 32);
+    }
+    for (int p = 0; p < C::P_STAGES; ++p) {
+      mbar_init(&gathered[p], C::GATHER_THREADS / 32);
+      mbar_init(&pfree[p], 1);
+    }
+    for (int b = 0; b < C::ACC_BUFS; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4 * C::SPLIT);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      grid_dependency_sync();
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int s = it % C::RAW_STAGES;
+        const uint32_t ph = (it / C::RAW_STAGES) & 1;
+        if (it >= C::RAW_STAGES && !mbar_wait(&empty[s], ph ^ 1)) {
+          atomicOr(&hadq_tc_fault, kFaultProducer);
+          drain_loads(full, C::RAW_STAGES, it);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], C::TILE_BYTES);
+        tma_load_3d(smem + C::SM_RAW + s * C::TILE_BYTES, &xmap, 0, 0, static_cast<int>(t * R), &full[s]);
+      }
+    }
+  } else if (warp >= C::FIRST_GATHER_WARP) {
+    // ----------------------------------------------------------------- gather
+    grid_dependency_sync();                  // the permutation and signs are caller memory
+    const int j = threadIdx.x - 32 * C::FIRST_GATHER_WARP;
+    uint32_t src[8], sgw[8], dst[2];   // src: two 13-bit in-row source offsets per word
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int c = j + C::GATHER_THREADS * q;   // output chunk: columns 8 c .. 8 c + 7
+      dst[q] = swz64(16u * static_cast<uint32_t>(c));
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const uint32_t p0 = min(static_cast<uint32_t>(__ldg(perm + 8 * c + i)), static_cast<uint32_t>(n - 1));
+        const uint32_t p1 = min(static_cast<uint32_t>(__ldg(perm + 8 * c + i + 1)), static_cast<uint32_t>(n - 1));
+        src[4 * q + i / 2] = swz64(2u * p0) | (swz64(2u * p1) << 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; i += 2)
+        sgw[4 * q + i / 2] = (__ldg(signs + 8 * c + i) < 0 ? 0x8000u : 0u) | (__ldg(signs + 8 * c + i + 1) < 0 ? 0x80000000u : 0u);
+    }
+    uint32_t it = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+      const int s = it % C::RAW_STAGES, p = it % C::P_STAGES;
+      const uint32_t sph = (it / C::RAW_STAGES) & 1, pph = (it / C::P_STAGES) & 1;
+      if (!mbar_wait(&full[s], sph) || (it >= C::P_STAGES && !mbar_wait(&pfree[p], pph ^ 1))) {
+        atomicOr(&hadq_tc_fault, kFaultSign);
+        break;
+      }
+      const uint8_t* raw = smem + C::SM_RAW + s * C::TILE_BYTES;
+      uint8_t* pb = smem + C::SM_P + p * C::TILE_BYTES;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t off = (i & 1) ? (src[4 * q + i / 2] >> 16) : (src[4 * q + i / 2] & 0xFFFFu);
+            v[i] = *reinterpret_cast<const uint16_t*>(raw + r * C::ROW_BYTES + off);
+          }
+          uint4 w;
+          w.x = __byte_perm(v[0], v[1], 0x5410) ^ sgw[4 * q + 0];
+          w.y = __byte_perm(v[2], v[3], 0x5410) ^ sgw[4 * q + 1];
+          w.z = __byte_perm(v[4], v[5], 0x5410) ^ sgw[4 * q + 2];
+          w.w = __byte_perm(v[6], v[7], 0x5410) ^ sgw[4 * q + 3];
+          *reinterpret_cast<uint4*>(pb + r * C::ROW_BYTES + dst[q]) = w;
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the permuted stage, to the tensor core
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&gathered[p]);
+        mbar_arrive(&empty[s]);
+      }
+    }
+  } else {
+    // Warps 1 .. FIRST_GATHER_WARP - 1: tensor memory, H_128, MMA, epilogue.
+    constexpr int kSetupThreads = 32 * (C::FIRST_GATHER_WARP - 1);
+    if (warp == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(kSetupThreads) : "memory");
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // H_128 into tensor memory (lane m = row m, column A_COL + c = the bf16
+    // pair k = 2c, 2c + 1), by the warps of the first epilogue group.
+    if (warp >= 2 && warp < 6) {
+      const int m = (warp & 3) * 32 + lane;
+      for (int c0 = 0; c0 < 64; c0 += 16) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k = 2 * (c0 + i);
+          w[i] = 0x3F803F80u | ((__popc(m & k) & 1u) << 15) | ((__popc(m & (k + 1)) & 1u) << 31);
+        }
+        tmem_st16(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::A_COL + c0, w);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(kSetupThreads) : "memory");
+    tc_fence_after();
+
+    if (warp == 1) {
+      // ------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        uint32_t it = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+          const int p = it % C::P_STAGES;
+          const uint32_t pph = (it / C::P_STAGES) & 1;
+          const int b = it % C::ACC_BUFS;
+          const uint32_t aph = (it / C::ACC_BUFS) & 1;
+          if (!mbar_wait(&gathered[p], pph) || (it >= C::ACC_BUFS && !mbar_wait(&acc_empty[b], aph ^ 1))) {
+            atomicOr(&hadq_tc_fault, kFaultMma);
+            drain_mmas(pfree, C::P_STAGES, it);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(smem + C::SM_P + p * C::TILE_BYTES);
+          const uint32_t d = tmem_base + b * C::TILE_N;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ta(d, tmem_base + C::A_COL + kk * 8, smem_desc(b_base + kk * 1024, 8192, 512, kSwizzle64),
+                        C::IDESC, kk > 0 ? 1u : 0u);
+          mma_commit(&pfree[p]);
+          mma_commit(&acc_full[b]);
+        }
+      }
+    } else {
+      // --------------------------------------------------------- epilogue
+      grid_dependency_sync();
+      const int quarter = warp & 3;
+      const int sub = (warp - 2) >> 2;         // row `sub` of every tile
+      const int hi = quarter * 32 + lane;
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int b = it % C::ACC_BUFS;
+        const uint32_t aph = (it / C::ACC_BUFS) & 1;
+        if (!mbar_wait(&acc_full[b], aph)) {
+          atomicOr(&hadq_tc_fault, kFaultEpilogue);
+          break;
+        }
+        tc_fence_after();
+        float z[L];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * C::TILE_N + sub * L, z);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        const int64_t row = t * R + sub;
+        tc_emit_row<LO, MODE, 0>(z, hi, row, row < rows, n, norm, group, out0, out1, nullptr);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+  }
+}
+
+}  // namespace tc
+}  // namespace hadq

@@ -3,6 +3,7 @@
 #include "hadq_launch.h"
 #include "hadq_tc.cuh"
 #include "hadq_tc128.cuh"
+#include "hadq_tcr.cuh"
 
 #include <type_traits>
 
@@ -53,6 +54,19 @@ Tc128Variant tc128_kernel_for(int mode) {
     default: break;
   }
   return Tc128Variant{fn, Tc128C::THREADS, Tc128C::SMEM_BYTES};
+}
+
+TcrVariant tcr_kernel_for(int mode) {
+  TcrFn fn = nullptr;
+  switch (mode) {
+    case OUT_F32: fn = &tc::tc_rpbh_kernel<OUT_F32>; break;
+    case OUT_BF16: fn = &tc::tc_rpbh_kernel<OUT_BF16>; break;
+    case OUT_INT4: fn = &tc::tc_rpbh_kernel<OUT_INT4>; break;
+    case OUT_MXFP4: fn = &tc::tc_rpbh_kernel<OUT_MXFP4>; break;
+    case OUT_NVFP4: fn = &tc::tc_rpbh_kernel<OUT_NVFP4>; break;
+    default: break;
+  }
+  return TcrVariant{fn, tc::TcrCfg::THREADS, tc::TcrCfg::SMEM_BYTES};
 }
 
 TcVariant tc_kernel_for(int lo, int mode, int side) {

@@ -128,3 +128,81 @@ def test_codebook_many_rows_grid_loops():
     torch.cuda.synchronize()
     _log("codebook4-rpbh-4096x4096", pc.check_codebook(x64, codes.cpu().numpy(), norms.cpu().numpy(), 4096, bits,
                                                        y=oracle.rpbh_rotate(x64, 4096, perm, signs)))
+
+
+# ------------------------------------------ RPBH on the tensor cores (n = 4096)
+
+@pytest.mark.parametrize("impl", ["tensor", "butterfly"])
+@pytest.mark.parametrize("fmt,group", [("int4", 128), ("int4", 32), ("mxfp4", 32), ("nvfp4", 16), ("f32", 0),
+                                       ("bf16", 0)])
+def test_rpbh_4096_tiles_both_impls(impl, fmt, group):
+    """Full-row RPBH at n = 4096: the gather-then-MMA kernel (tensor) and the
+    staged kernel (butterfly) on 1001 rows (251 tiles of 4 rows, the last one
+    ragged, more tiles than CTAs)."""
+    rows, n = 1001, 4096
+    stored, x64 = synth(rows, n, "bf16", seed=rows + len(fmt) + group, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
+    perm, signs, pd, sd = rpbh_args(n, 77 + group)
+    y = oracle.rpbh_rotate(x64, n, perm, signs)
+    old = H.hadq_set_impl(impl)
+    try:
+        if fmt in ("f32", "bf16"):
+            out = H.hadq_rotate_rpbh(to_dev(stored, "bf16"), pd, sd, n,
+                                     out_dtype=torch.float32 if fmt == "f32" else torch.bfloat16)
+            torch.cuda.synchronize()
+            if fmt == "f32":
+                _log(f"rpbh-{impl}-rot-{rows}x{n}", pc.check_rotation_f32(x64, out.cpu().numpy(), n, y=y))
+            else:
+                pc.check_rotation_bf16(x64, out.view(torch.int16).cpu().numpy().view(np.uint16), n, y=y)
+        else:
+            c, s = H.hadq_rotate_quant_rpbh(to_dev(stored, "bf16"), pd, sd, n, fmt, group)
+            torch.cuda.synchronize()
+            _log(f"rpbh-{impl}-{fmt}{group}-{rows}x{n}",
+                 pc.check(fmt, x64, c.cpu().numpy(), s.cpu().numpy(), n, group, y=y))
+    finally:
+        H.hadq_set_impl(old)
+
+
+def test_rpbh_4096_identity_matches_plain_tensor_kernel():
+    """Identity permutation and all-plus signs through the gather kernel: the
+    same codes as the plain n = 4096 tensor-core rotation, bit for bit (the
+    gather only moves data; the MMA and epilogue are the same arithmetic)."""
+    stored, _ = synth(37, 4096, "bf16", seed=6)
+    x = to_dev(stored, "bf16")
+    perm = torch.arange(4096, dtype=torch.int32, device="cuda")
+    ones = torch.ones(4096, dtype=torch.int8, device="cuda")
+    c0, s0 = H.hadq_rotate_quant(x, 0, "int4", 128)
+    c1, s1 = H.hadq_rotate_quant_rpbh(x, perm, ones, 4096, "int4", 128)
+    torch.cuda.synchronize()
+    assert torch.equal(c0, c1) and torch.equal(s0.view(torch.int16), s1.view(torch.int16))
+
+
+def test_rpbh_4096_guard_bytes():
+    rows, n = 9, 4096
+    stored, x64 = synth(rows, n, "bf16", seed=19)
+    perm, signs, pd, sd = rpbh_args(n, 19)
+    pad = 1024
+    cbuf = torch.full((rows * n // 2 + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((rows * n // 64 + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda")
+    codes = cbuf[pad:pad + rows * n // 2].view(rows, n // 2)
+    scales = sbuf[pad:pad + rows * n // 64].view(torch.float16).view(rows, n // 128)
+    H.hadq_rotate_quant_rpbh(to_dev(stored, "bf16"), pd, sd, n, "int4", 128, codes=codes, scales=scales)
+    torch.cuda.synchronize()
+    cb, sb = cbuf.cpu().numpy(), sbuf.cpu().numpy()
+    assert (cb[:pad] == 0xA5).all() and (cb[-pad:] == 0xA5).all()
+    assert (sb[:pad] == 0x5A).all() and (sb[-pad:] == 0x5A).all()
+    pc.check_int4(x64, codes.cpu().numpy(), scales.cpu().numpy(), n, 128, y=oracle.rpbh_rotate(x64, n, perm, signs))
+
+
+def test_config_c2p_full_size():
+    """The bench's c2p workload (4096 x 4096 bf16, its seeded permutation and
+    signs, int4 g128) in the launch the bench times; every row checked."""
+    from hadamard_rotation_bit_b200 import workloads as W
+    w = W.WORKLOADS["c2p"]
+    stored = W.generate("c2p")
+    perm, signs = W.generate_rpbh("c2p")
+    x64 = W.bits_to_float64(stored, "bf16")
+    c, s = H.hadq_rotate_quant_rpbh(to_dev(stored, "bf16"), torch.from_numpy(perm).cuda(),
+                                    torch.from_numpy(signs).cuda(), w.block, w.fmt, w.group)
+    torch.cuda.synchronize()
+    _log("c2p", pc.check_int4(x64, c.cpu().numpy(), s.cpu().numpy(), w.block, w.group,
+                              y=oracle.rpbh_rotate(x64, w.block, perm, signs)))
