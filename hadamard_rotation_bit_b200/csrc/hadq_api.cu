@@ -352,14 +352,15 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
 
 // RPBH at full size 4096, bf16 input, on the tensor cores (hadq_tcr.cuh): the
 // permutation and signs applied by gather warps in shared memory, then the
-// n = 4096 rotation and epilogue.  Rotation outputs, int4, MXFP4, NVFP4.
+// n = 4096 rotation and epilogue.  Rotation outputs, int4, MXFP4, NVFP4 and
+// the codebook quantizer.
 bool tcr_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
-  return x_dtype == HADQ_BF16 && sh.kbase == 1 && sh.n == 4096 && sh.b == 4096 && mode >= 0 &&
-         mode != hadq::OUT_CODEBOOK;
+  return x_dtype == HADQ_BF16 && sh.kbase == 1 && sh.n == 4096 && sh.b == 4096 && mode >= 0;
 }
 
 hadq_status launch_tcr(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
-                       cudaStream_t stream, int sms, int dev, const int32_t* perm, const int8_t* signs) {
+                       cudaStream_t stream, int sms, int dev, const int32_t* perm, const int8_t* signs,
+                       const double* thr) {
   const hl::TcrVariant v = hl::tcr_kernel_for(mode);
   if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no RPBH tensor-core kernel for this format");
   constexpr int L = 32, R = 4;
@@ -381,7 +382,7 @@ hadq_status launch_tcr(const void* x, const Shape& sh, int mode, int group, void
   const int64_t tiles = (sh.rows + R - 1) / R;
   const int64_t grid = std::min<int64_t>(tiles, sms);
   return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, map, static_cast<const uint16_t*>(x), sh.rows,
-                                  static_cast<int>(sh.n), sh.norm, group, out0, out1, perm, signs),
+                                  static_cast<int>(sh.n), sh.norm, group, out0, out1, perm, signs, thr),
                        "RPBH tensor-core kernel launch");
 }
 
@@ -516,7 +517,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
   (void)cudaGetLastError();   // launch errors below must be ours
   if (ex.perm != nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
       tcr_eligible(x_dtype, sh, mode))
-    return launch_tcr(x, sh, mode, group, out0, out1, stream, sms, dev, ex.perm, ex.rpbh_signs);
+    return launch_tcr(x, sh, mode, mode == hadq::OUT_CODEBOOK ? ex.bits : group, out0, out1, stream, sms, dev, ex.perm,
+                      ex.rpbh_signs, ex.thr);
   if (ex.perm == nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
       tck_eligible(x_dtype, sh, mode, sg))
     return launch_tck(x, sh, mode, out0, out1, stream, sms, dev);

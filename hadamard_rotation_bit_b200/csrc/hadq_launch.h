@@ -42,7 +42,7 @@ struct Tc128Variant {
 
 using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, void*, void*);
 using TcrFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, const int32_t*,
-                       const int8_t*);
+                       const int8_t*, const double*);
 
 struct TcrVariant {
   TcrFn fn;

@@ -21,7 +21,7 @@
 //   epilogue  as the n = 4096 kernel (LO = 5 register stages, quantizer).
 //
 // Each gather thread always owns the same two output chunks of every row, so
-// its 16 source offsets (two per word) and 8 sign words are computed once per
+// its 16 source offsets and signs (two of each per word) are computed once per
 // launch from the caller's permutation and signs.  Roles: warp 0 TMA
 // producer, warp 1 TMEM allocator and MMA issuer, warps 2..17 epilogue (one
 // row of each tile per group of 4), warps 18..25 gather.  Every wait is
@@ -51,7 +51,12 @@ struct TcrCfg {
   static constexpr int SM_RAW = 0;
   static constexpr int SM_P = SM_RAW + RAW_STAGES * TILE_BYTES;
   static constexpr int SM_BARS = SM_P + P_STAGES * TILE_BYTES;
-  static constexpr int SM_SLOT = SM_BARS + 8 * (2 * RAW_STAGES + 2 * P_STAGES + 2 * ACC_BUFS);
+  static constexpr int SM_RED = SM_BARS + 8 * (2 * RAW_STAGES + 2 * P_STAGES + 2 * ACC_BUFS);
+  // Codebook quantizer, per epilogue sub-group (one row of each tile): 4
+  // partial sums of squares (double) and up to 15 row thresholds (float).
+  static constexpr int SM_CB = SM_RED + 8 * 4 * SPLIT;   // 16-byte aligned (quartile loads)
+  static constexpr int SM_SLOT = SM_CB + 4 * 16 * SPLIT;
+  static_assert(SM_CB % 16 == 0, "quartile loads of the row thresholds are 16-byte loads");
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
   static_assert(GATHER_THREADS * 2 * 8 == ROW_BYTES / 2, "two 8-column chunks of each row per gather thread");
 };
@@ -61,14 +66,90 @@ struct TcrCfg {
 // decides the swizzle): 16-byte chunk bits 4..5 XOR address bits 7..8.
 __device__ __forceinline__ uint32_t swz64(uint32_t off) { return off ^ (((off >> 7) & 3u) << 4); }
 
-// MODE: an OutMode of tc_emit_row (rotation, int4, MXFP4, NVFP4).  perm: n
-// int32 source columns (entries outside [0, n) are clamped: memory-safe,
-// result unspecified); signs: n int8, negative = -1.
+// Codebook quantizer ("orbitquant 0.2.0", Method Conformance: per-token norm,
+// the normalised rotation, the nearest centroid of the unit-sphere Lloyd-Max
+// codebook) for one row; z holds the thread's 32 values of the row after the
+// tensor-core stage (output columns hi * 32 ..).  Every thread of the row's 4
+// warps calls it for every tile (work = false after a failed wait: the
+// barriers are still joined).  The code of u = y / ||y|| is the number of
+// unit thresholds t_j below u, i.e. of row thresholds tau_j = ||z|| t_j below
+// z; with h = fl(tau_j) and l = tau_j - h (double), z > tau_j exactly when
+// z >= g_j = (l < 0 ? h : the next float above h), so one float per
+// threshold decides exactly.  The norm is a double sum of squares.
+__device__ __forceinline__ void tcr_codebook_row(float (&z)[32], bool work, int quarter, int lane, int64_t e0,
+                                                 int64_t row, bool row_ok, float norm, int bits, const double* thr,
+                                                 double* red, float* gtab, int bar, uint8_t* codes, float* norms) {
+  double ss = 0.0;
+  if (work) {
+    fwht_bits<32, 0, 5>(z);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ss = fma(static_cast<double>(z[i]), static_cast<double>(z[i]), ss);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) red[quarter] = ss;
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+  const double zn = sqrt((red[0] + red[1]) + (red[2] + red[3]));
+  const int levels = 1 << bits;
+  if (quarter == 0 && lane < levels - 1) {
+    const double t = (zn > 0.0 ? zn : 1.0) * thr[lane];   // a zero row codes u = 0
+    const float h = __double2float_rn(t);
+    gtab[lane] = (t - static_cast<double>(h) < 0.0) ? h : nextafterf(h, INFINITY);
+  }
+  if (quarter == 0 && lane == 0 && row_ok && work) norms[row] = static_cast<float>(zn * static_cast<double>(norm));
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+  if (!work || !row_ok) return;
+  if (bits == 4) {
+    // The separators g_3, g_7, g_11 (registers) give the quartile Q of z; one
+    // 16-byte load of g_4Q .. g_4Q+2 and two more compares finish the search.
+    const float g3 = gtab[3], g7 = gtab[7], g11 = gtab[11];
+    const float4* quart = reinterpret_cast<const float4*>(gtab);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float v = z[8 * q + i];
+        const uint32_t b3 = v >= g7 ? 1u : 0u;
+        const uint32_t b2 = v >= (b3 ? g11 : g3) ? 1u : 0u;
+        const uint32_t Q = 2 * b3 + b2;
+        const float4 f = quart[Q];
+        const uint32_t b1 = v >= f.y ? 1u : 0u;
+        const uint32_t b0 = v >= (b1 ? f.z : f.x) ? 1u : 0u;
+        word |= (4 * Q + 2 * b1 + b0) << (4 * i);
+      }
+      w[q] = word;
+    }
+    *reinterpret_cast<uint4*>(codes + (e0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    const float g0 = gtab[0], g1 = gtab[1], g2 = gtab[2];
+    uint32_t w[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float v = z[16 * q + i];
+        const uint32_t b1 = v >= g1 ? 1u : 0u;
+        const uint32_t b0 = v >= (b1 ? g2 : g0) ? 1u : 0u;
+        word |= (2 * b1 + b0) << (2 * i);
+      }
+      w[q] = word;
+    }
+    *reinterpret_cast<uint2*>(codes + (e0 >> 2)) = make_uint2(w[0], w[1]);
+  }
+}
+
+// MODE: an OutMode of tc_emit_row (rotation, int4, MXFP4, NVFP4) or
+// OUT_CODEBOOK (group = bits, 2 or 4; thr = the 2^bits - 1 ascending unit
+// thresholds).  perm: n int32 source columns (entries outside [0, n) are
+// clamped: memory-safe, result unspecified); signs: n int8, negative = -1.
 template <int MODE>
 __global__ void __launch_bounds__(TcrCfg::THREADS, 1)
 tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t rows, int n,
                float norm, int group, void* __restrict__ out0, void* __restrict__ out1,
-               const int32_t* __restrict__ perm, const int8_t* __restrict__ signs) {
+               const int32_t* __restrict__ perm, const int8_t* __restrict__ signs, const double* __restrict__ thr) {
   using C = TcrCfg;
   constexpr int LO = C::LO, L = C::L, R = C::R;
   extern __shared__ uint8_t smem_raw[];
@@ -127,7 +208,10 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
     // ----------------------------------------------------------------- gather
     grid_dependency_sync();                  // the permutation and signs are caller memory
     const int j = threadIdx.x - 32 * C::FIRST_GATHER_WARP;
-    uint32_t src[8], sgw[8], dst[2];   // src: two 13-bit in-row source offsets per word
+    // src: per pair of output columns e, e + 1 the two 13-bit in-row source
+    // offsets (bits 0..12, 16..28) and their signs (bit 15, 31 set for -1),
+    // which are then exactly the XOR mask of the packed bf16 pair.
+    uint32_t src[8], dst[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int c = j + C::GATHER_THREADS * q;   // output chunk: columns 8 c .. 8 c + 7
@@ -136,11 +220,10 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
       for (int i = 0; i < 8; i += 2) {
         const uint32_t p0 = min(static_cast<uint32_t>(__ldg(perm + 8 * c + i)), static_cast<uint32_t>(n - 1));
         const uint32_t p1 = min(static_cast<uint32_t>(__ldg(perm + 8 * c + i + 1)), static_cast<uint32_t>(n - 1));
-        src[4 * q + i / 2] = swz64(2u * p0) | (swz64(2u * p1) << 16);
+        const uint32_t s0 = __ldg(signs + 8 * c + i) < 0 ? 0x8000u : 0u;
+        const uint32_t s1 = __ldg(signs + 8 * c + i + 1) < 0 ? 0x8000u : 0u;
+        src[4 * q + i / 2] = (swz64(2u * p0) | s0) | ((swz64(2u * p1) | s1) << 16);
       }
-#pragma unroll
-      for (int i = 0; i < 8; i += 2)
-        sgw[4 * q + i / 2] = (__ldg(signs + 8 * c + i) < 0 ? 0x8000u : 0u) | (__ldg(signs + 8 * c + i + 1) < 0 ? 0x80000000u : 0u);
     }
     uint32_t it = 0;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
@@ -159,14 +242,14 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
           uint32_t v[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const uint32_t off = (i & 1) ? (src[4 * q + i / 2] >> 16) : (src[4 * q + i / 2] & 0xFFFFu);
+            const uint32_t off = ((i & 1) ? (src[4 * q + i / 2] >> 16) : src[4 * q + i / 2]) & 0x1FFFu;
             v[i] = *reinterpret_cast<const uint16_t*>(raw + r * C::ROW_BYTES + off);
           }
           uint4 w;
-          w.x = __byte_perm(v[0], v[1], 0x5410) ^ sgw[4 * q + 0];
-          w.y = __byte_perm(v[2], v[3], 0x5410) ^ sgw[4 * q + 1];
-          w.z = __byte_perm(v[4], v[5], 0x5410) ^ sgw[4 * q + 2];
-          w.w = __byte_perm(v[6], v[7], 0x5410) ^ sgw[4 * q + 3];
+          w.x = __byte_perm(v[0], v[1], 0x5410) ^ (src[4 * q + 0] & 0x80008000u);
+          w.y = __byte_perm(v[2], v[3], 0x5410) ^ (src[4 * q + 1] & 0x80008000u);
+          w.z = __byte_perm(v[4], v[5], 0x5410) ^ (src[4 * q + 2] & 0x80008000u);
+          w.w = __byte_perm(v[6], v[7], 0x5410) ^ (src[4 * q + 3] & 0x80008000u);
           *reinterpret_cast<uint4*>(pb + r * C::ROW_BYTES + dst[q]) = w;
         }
       }
@@ -239,23 +322,34 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
       const int quarter = warp & 3;
       const int sub = (warp - 2) >> 2;         // row `sub` of every tile
       const int hi = quarter * 32 + lane;
+      double* red = reinterpret_cast<double*>(smem + C::SM_RED) + 4 * sub;
+      float* gtab = reinterpret_cast<float*>(smem + C::SM_CB) + 16 * sub;
       uint32_t it = 0;
+      bool failed = false;   // a wait ran out: skip the work (the codebook still joins its barriers)
       for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
         const int b = it % C::ACC_BUFS;
         const uint32_t aph = (it / C::ACC_BUFS) & 1;
-        if (!mbar_wait(&acc_full[b], aph)) {
+        if (!failed && !mbar_wait(&acc_full[b], aph)) {
           atomicOr(&hadq_tc_fault, kFaultEpilogue);
-          break;
+          failed = true;
         }
-        tc_fence_after();
+        if (failed && MODE != OUT_CODEBOOK) break;
         float z[L];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * C::TILE_N + sub * L, z);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[b]);
+        if (!failed) {
+          tc_fence_after();
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * C::TILE_N + sub * L, z);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
         const int64_t row = t * R + sub;
-        tc_emit_row<LO, MODE, 0>(z, hi, row, row < rows, n, norm, group, out0, out1, nullptr);
+        if constexpr (MODE == OUT_CODEBOOK) {
+          tcr_codebook_row(z, !failed, quarter, lane, row * n + static_cast<int64_t>(hi) * L, row, row < rows, norm,
+                           group, thr, red, gtab, 2 + sub, static_cast<uint8_t*>(out0), static_cast<float*>(out1));
+        } else {
+          tc_emit_row<LO, MODE, 0>(z, hi, row, row < rows, n, norm, group, out0, out1, nullptr);
+        }
       }
     }
   }

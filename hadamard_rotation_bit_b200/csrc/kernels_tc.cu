@@ -64,6 +64,7 @@ TcrVariant tcr_kernel_for(int mode) {
     case OUT_INT4: fn = &tc::tc_rpbh_kernel<OUT_INT4>; break;
     case OUT_MXFP4: fn = &tc::tc_rpbh_kernel<OUT_MXFP4>; break;
     case OUT_NVFP4: fn = &tc::tc_rpbh_kernel<OUT_NVFP4>; break;
+    case OUT_CODEBOOK: fn = &tc::tc_rpbh_kernel<OUT_CODEBOOK>; break;
     default: break;
   }
   return TcrVariant{fn, tc::TcrCfg::THREADS, tc::TcrCfg::SMEM_BYTES};

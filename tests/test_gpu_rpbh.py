@@ -134,18 +134,25 @@ def test_codebook_many_rows_grid_loops():
 
 @pytest.mark.parametrize("impl", ["tensor", "butterfly"])
 @pytest.mark.parametrize("fmt,group", [("int4", 128), ("int4", 32), ("mxfp4", 32), ("nvfp4", 16), ("f32", 0),
-                                       ("bf16", 0)])
+                                       ("bf16", 0), ("codebook", 4), ("codebook", 2)])
 def test_rpbh_4096_tiles_both_impls(impl, fmt, group):
     """Full-row RPBH at n = 4096: the gather-then-MMA kernel (tensor) and the
     staged kernel (butterfly) on 1001 rows (251 tiles of 4 rows, the last one
-    ragged, more tiles than CTAs)."""
+    ragged, more tiles than CTAs), every output format and the 2- and 4-bit
+    codebook quantizer."""
     rows, n = 1001, 4096
     stored, x64 = synth(rows, n, "bf16", seed=rows + len(fmt) + group, dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
     perm, signs, pd, sd = rpbh_args(n, 77 + group)
     y = oracle.rpbh_rotate(x64, n, perm, signs)
     old = H.hadq_set_impl(impl)
     try:
-        if fmt in ("f32", "bf16"):
+        if fmt == "codebook":
+            codes, norms = H.hadq_rotate_quant_codebook(to_dev(stored, "bf16"), group, _codebook_dev(n, group), n,
+                                                        perm=pd, signs=sd)
+            torch.cuda.synchronize()
+            _log(f"rpbh-{impl}-codebook{group}-{rows}x{n}",
+                 pc.check_codebook(x64, codes.cpu().numpy(), norms.cpu().numpy(), n, group, y=y))
+        elif fmt in ("f32", "bf16"):
             out = H.hadq_rotate_rpbh(to_dev(stored, "bf16"), pd, sd, n,
                                      out_dtype=torch.float32 if fmt == "f32" else torch.bfloat16)
             torch.cuda.synchronize()
