@@ -52,10 +52,11 @@ struct TcrCfg {
   static constexpr int SM_P = SM_RAW + RAW_STAGES * TILE_BYTES;
   static constexpr int SM_BARS = SM_P + P_STAGES * TILE_BYTES;
   static constexpr int SM_RED = SM_BARS + 8 * (2 * RAW_STAGES + 2 * P_STAGES + 2 * ACC_BUFS);
-  // Codebook quantizer, per epilogue sub-group (one row of each tile): 4
-  // partial sums of squares (double) and up to 15 row thresholds (float).
-  static constexpr int SM_CB = SM_RED + 8 * 4 * SPLIT;   // 16-byte aligned (quartile loads)
-  static constexpr int SM_SLOT = SM_CB + 4 * 16 * SPLIT;
+  // Codebook quantizer: per epilogue sub-group (one row of each tile) 2 x 4
+  // partial sums of squares (double; a buffer per tile parity), and per
+  // epilogue warp up to 15 row thresholds (float).
+  static constexpr int SM_CB = SM_RED + 8 * 2 * 4 * SPLIT;   // 16-byte aligned (quartile loads)
+  static constexpr int SM_SLOT = SM_CB + 4 * 16 * 4 * SPLIT;
   static_assert(SM_CB % 16 == 0, "quartile loads of the row thresholds are 16-byte loads");
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
   static_assert(GATHER_THREADS * 2 * 8 == ROW_BYTES / 2, "two 8-column chunks of each row per gather thread");
@@ -71,19 +72,26 @@ __device__ __forceinline__ uint32_t swz64(uint32_t off) { return off ^ (((off >>
 // codebook) for one row; z holds the thread's 32 values of the row after the
 // tensor-core stage (output columns hi * 32 ..).  Every thread of the row's 4
 // warps calls it for every tile (work = false after a failed wait: the
-// barriers are still joined).  The code of u = y / ||y|| is the number of
-// unit thresholds t_j below u, i.e. of row thresholds tau_j = ||z|| t_j below
-// z; with h = fl(tau_j) and l = tau_j - h (double), z > tau_j exactly when
+// barrier is still joined).  The code of u = y / ||y|| is the number of unit
+// thresholds t_j below u, i.e. of row thresholds tau_j = ||z|| t_j below z;
+// with h = fl(tau_j) and l = tau_j - h (double), z > tau_j exactly when
 // z >= g_j = (l < 0 ? h : the next float above h), so one float per
-// threshold decides exactly.  The norm is a double sum of squares.
+// threshold decides exactly.  The norm is a double sum of squares (four
+// accumulation chains), joined across the 4 warps by one named barrier; red
+// holds the partial sums of this tile (a buffer per tile parity: a warp can be
+// one tile ahead of the others when it writes, never two), and each warp
+// computes the thresholds into its own table gtab, so no second barrier is
+// needed.
 __device__ __forceinline__ void tcr_codebook_row(float (&z)[32], bool work, int quarter, int lane, int64_t e0,
                                                  int64_t row, bool row_ok, float norm, int bits, const double* thr,
                                                  double* red, float* gtab, int bar, uint8_t* codes, float* norms) {
   double ss = 0.0;
   if (work) {
     fwht_bits<32, 0, 5>(z);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ss = fma(static_cast<double>(z[i]), static_cast<double>(z[i]), ss);
+    for (int i = 0; i < 32; ++i) acc[i & 3] = fma(static_cast<double>(z[i]), static_cast<double>(z[i]), acc[i & 3]);
+    ss = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -91,13 +99,13 @@ __device__ __forceinline__ void tcr_codebook_row(float (&z)[32], bool work, int 
   asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
   const double zn = sqrt((red[0] + red[1]) + (red[2] + red[3]));
   const int levels = 1 << bits;
-  if (quarter == 0 && lane < levels - 1) {
+  if (lane < levels - 1) {
     const double t = (zn > 0.0 ? zn : 1.0) * thr[lane];   // a zero row codes u = 0
     const float h = __double2float_rn(t);
     gtab[lane] = (t - static_cast<double>(h) < 0.0) ? h : nextafterf(h, INFINITY);
   }
   if (quarter == 0 && lane == 0 && row_ok && work) norms[row] = static_cast<float>(zn * static_cast<double>(norm));
-  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+  __syncwarp();
   if (!work || !row_ok) return;
   if (bits == 4) {
     // The separators g_3, g_7, g_11 (registers) give the quartile Q of z; one
@@ -322,8 +330,8 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
       const int quarter = warp & 3;
       const int sub = (warp - 2) >> 2;         // row `sub` of every tile
       const int hi = quarter * 32 + lane;
-      double* red = reinterpret_cast<double*>(smem + C::SM_RED) + 4 * sub;
-      float* gtab = reinterpret_cast<float*>(smem + C::SM_CB) + 16 * sub;
+      double* red = reinterpret_cast<double*>(smem + C::SM_RED) + 8 * sub;      // [tile parity][quarter]
+      float* gtab = reinterpret_cast<float*>(smem + C::SM_CB) + 16 * (warp - 2);  // this warp's thresholds
       uint32_t it = 0;
       bool failed = false;   // a wait ran out: skip the work (the codebook still joins its barriers)
       for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
@@ -346,7 +354,8 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
         const int64_t row = t * R + sub;
         if constexpr (MODE == OUT_CODEBOOK) {
           tcr_codebook_row(z, !failed, quarter, lane, row * n + static_cast<int64_t>(hi) * L, row, row < rows, norm,
-                           group, thr, red, gtab, 2 + sub, static_cast<uint8_t*>(out0), static_cast<float*>(out1));
+                           group, thr, red + 4 * (it & 1), gtab, 2 + sub, static_cast<uint8_t*>(out0),
+                           static_cast<float*>(out1));
         } else {
           tc_emit_row<LO, MODE, 0>(z, hi, row, row < rows, n, norm, group, out0, out1, nullptr);
         }
