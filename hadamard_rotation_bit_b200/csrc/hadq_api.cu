@@ -148,20 +148,39 @@ hadq_status check_quant(hadq_fmt fmt, int64_t group, const Shape& sh, int* eff_g
       if (sh.n % 16 != 0) return fail(HADQ_ERR_INVALID_ARG, "NVFP4 needs n to be a multiple of 16");
       *eff_group = 16;
       return HADQ_OK;
+    case HADQ_MXFP4_BLOCKED:
+    case HADQ_NVFP4_BLOCKED: {
+      const int blk = fmt == HADQ_MXFP4_BLOCKED ? 32 : 16;
+      if (group != 0 && group != blk)
+        return fail(HADQ_ERR_INVALID_ARG, fmt == HADQ_MXFP4_BLOCKED ? "MXFP4 group must be 0 or 32"
+                                                                      : "NVFP4 group must be 0 or 16");
+      if (sh.n % (4 * blk) != 0)
+        return fail(HADQ_ERR_INVALID_ARG, "blocked scales need whole 4-column tiles: n a multiple of 4 x the block");
+      *eff_group = blk;
+      return HADQ_OK;
+    }
     default:
-      return fail(HADQ_ERR_INVALID_ARG, "fmt must be HADQ_INT4_SYM, HADQ_INT8_SYM, HADQ_MXFP4 or HADQ_NVFP4");
+      return fail(HADQ_ERR_INVALID_ARG,
+                  "fmt must be HADQ_INT4_SYM, HADQ_INT8_SYM, HADQ_MXFP4, HADQ_NVFP4 or a blocked FP4 format");
   }
 }
+
+bool blocked_fmt(hadq_fmt fmt) { return fmt == HADQ_MXFP4_BLOCKED || fmt == HADQ_NVFP4_BLOCKED; }
 
 int64_t codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt) {
   return fmt == HADQ_INT8_SYM ? rows * n : rows * n / 2;
 }
+
+// The tiled GEMM scale layout pads the rows to a multiple of 128.
+int64_t padded_scale_rows(int64_t rows) { return (rows + 127) / 128 * 128; }
 
 int64_t scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int group) {
   switch (fmt) {
     case HADQ_INT4_SYM: return rows * (n / group) * 2;
     case HADQ_INT8_SYM: return rows * 4;
     case HADQ_NVFP4: return rows * (n / 16);
+    case HADQ_MXFP4_BLOCKED: return padded_scale_rows(rows) * (n / 32);
+    case HADQ_NVFP4_BLOCKED: return padded_scale_rows(rows) * (n / 16);
     default: return rows * (n / 32);
   }
 }
@@ -673,6 +692,8 @@ int quant_mode(hadq_fmt fmt) {
     case HADQ_INT4_SYM: return hadq::OUT_INT4;
     case HADQ_MXFP4: return hadq::OUT_MXFP4;
     case HADQ_NVFP4: return hadq::OUT_NVFP4;
+    case HADQ_MXFP4_BLOCKED: return hadq::OUT_MXFP4_BLOCKED;
+    case HADQ_NVFP4_BLOCKED: return hadq::OUT_NVFP4_BLOCKED;
     default: return -1;
   }
 }
@@ -692,12 +713,27 @@ hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, i
   if (st != HADQ_OK || rows == 0) return st;
   // NVFP4 quantizes y / tensor_scale: fold the division into the rotation's
   // normalisation (one rounding, on the host, in double).
-  if (fmt == HADQ_NVFP4) sh.norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.b)) / tensor_scale);
+  if (fmt == HADQ_NVFP4 || fmt == HADQ_NVFP4_BLOCKED)
+    sh.norm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.b)) / tensor_scale);
   const Span outs[2] = {span(codes, codes_bytes(rows, n, fmt)), span(scales, scales_bytes(rows, n, fmt, g))};
   Signs sg{nullptr, hadq::SIGNS_NONE};
   Extra ex;
   st = perm != nullptr ? make_rpbh(perm, signs, sh, outs, 2, &ex) : make_signs(signs, side, sh, outs, 2, &sg);
   if (st != HADQ_OK) return st;
+  if (blocked_fmt(fmt)) {
+    // Only the tensor-core kernels write the tiled layout; the padding rows of
+    // the last 128-row tile are zeroed first (the kernel writes every other entry).
+    if (perm != nullptr || g_impl.load(std::memory_order_relaxed) == HADQ_IMPL_BUTTERFLY ||
+        !tc_eligible(x_dtype, sh, quant_mode(fmt)))
+      return fail(HADQ_ERR_UNSUPPORTED, "blocked FP4 scales: bf16 input at full size 4096 or 8192, tensor-core kernels");
+    if (rows % 128 != 0) {
+      const int64_t cols = n / g;   // scale columns per row
+      const int64_t tile_row_bytes = cols / 4 * 512;
+      const cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scales) + rows / 128 * tile_row_bytes, 0,
+                                            static_cast<size_t>(tile_row_bytes), static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, std::string("zero the scale padding: ") + cudaGetErrorString(e));
+    }
+  }
   return launch(x, x_dtype, sh, quant_mode(fmt), g, codes, scales, static_cast<cudaStream_t>(stream), sg, ex);
 }
 
@@ -900,7 +936,8 @@ hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtype x_dtype
 
 int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt) {
   if (rows < 0 || n <= 0 || n % 2 != 0) return 0;
-  if (fmt != HADQ_INT4_SYM && fmt != HADQ_INT8_SYM && fmt != HADQ_MXFP4 && fmt != HADQ_NVFP4) return 0;
+  if (fmt != HADQ_INT4_SYM && fmt != HADQ_INT8_SYM && fmt != HADQ_MXFP4 && fmt != HADQ_NVFP4 && !blocked_fmt(fmt))
+    return 0;
   return codes_bytes(rows, n, fmt);
 }
 
@@ -916,6 +953,10 @@ int64_t hadq_scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int64_t group) 
       return ((group == 0 || group == 32) && n % 32 == 0) ? rows * (n / 32) : 0;
     case HADQ_NVFP4:
       return ((group == 0 || group == 16) && n % 16 == 0) ? rows * (n / 16) : 0;
+    case HADQ_MXFP4_BLOCKED:
+      return ((group == 0 || group == 32) && n % 128 == 0) ? scales_bytes(rows, n, fmt, 32) : 0;
+    case HADQ_NVFP4_BLOCKED:
+      return ((group == 0 || group == 16) && n % 64 == 0) ? scales_bytes(rows, n, fmt, 16) : 0;
     default:
       return 0;
   }

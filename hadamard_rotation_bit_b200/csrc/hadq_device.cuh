@@ -15,7 +15,12 @@
 
 namespace hadq {
 
-enum OutMode : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3, OUT_NVFP4 = 4, OUT_CODEBOOK = 5 };
+// *_BLOCKED: MXFP4 / NVFP4 whose scales are written in the tiled layout that
+// block-scaled tensor-core GEMMs read (blocked_scale_offset).
+enum OutMode : int {
+  OUT_F32 = 0, OUT_BF16 = 1, OUT_INT4 = 2, OUT_MXFP4 = 3, OUT_NVFP4 = 4, OUT_CODEBOOK = 5,
+  OUT_MXFP4_BLOCKED = 6, OUT_NVFP4_BLOCKED = 7
+};
 
 // Random Hadamard signs ("Rotation Transform", section 1.5: H @ diag(+/-1) /
 // sqrt(N), the signs persisted as int8).  AFTER: output column j of every
@@ -604,8 +609,26 @@ __device__ __forceinline__ void store_int4_lanes(const float (&v)[N], float norm
   if (ok && (e0 & (group - 1)) == 0) scales[e0 >> (__ffs(group) - 1)] = s16;   // the group's first lane
 }
 
+// Offset of scale k (row-major index over rows x 2^LOG_C scale columns) in
+// the tiled scale layout of block-scaled tensor-core GEMMs (the "1D block
+// scaling factors" layout of NVIDIA's cuBLAS documentation): 128-row x
+// 4-column tiles of 512 bytes, row-block major; inside a tile, scale (r, c)
+// at (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.  LOG_C = 0: row-major (k).
+template <int LOG_C>
+__device__ __forceinline__ int64_t scale_offset(int64_t k) {
+  if constexpr (LOG_C == 0) {
+    return k;
+  } else {
+    static_assert(LOG_C >= 2, "whole 4-column tiles");
+    const int64_t r = k >> LOG_C;
+    const int c = static_cast<int>(k & ((int64_t(1) << LOG_C) - 1));
+    return (((r >> 7) << (LOG_C - 2)) + (c >> 2)) * 512 + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
+  }
+}
+
 // MXFP4: per 32 elements an E8M0 exponent e = clamp(floor(log2 m) - 2, -127, 127).
-template <bool PERM, int N>
+// LOG_C: the scale layout (scale_offset).
+template <bool PERM, int N, int LOG_C = 0>
 __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales, int64_t e0) {
   static_assert(N % 32 == 0, "MX groups are 32 elements");
@@ -631,7 +654,7 @@ __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uin
     } else {
       prev = w;
     }
-    scales[(e0 >> 5) + j] = static_cast<uint8_t>(byte);
+    scales[scale_offset<LOG_C>((e0 >> 5) + j)] = static_cast<uint8_t>(byte);
   }
 }
 
@@ -655,7 +678,7 @@ __device__ __forceinline__ float2 e4m3x2_values(uint16_t b) {
 // of v = z * nq (nq = the rotation's 1/sqrt(b) divided by the per-tensor
 // scale) and E2M1 codes of v / s; s == 0 gives codes 0.  Pairs of blocks
 // store 16 code bytes and 2 scale bytes at once.
-template <bool PERM, int N>
+template <bool PERM, int N, int LOG_C = 0>
 __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8_t* __restrict__ codes,
                                             uint8_t* __restrict__ scales, int64_t e0) {
   static_assert(N % 16 == 0, "NVFP4 blocks are 16 elements");
@@ -665,7 +688,7 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
     const float s = e4m3x2_values(b).x;
     const float f = s > 0.f ? code_factor(nq, s) : 0.f;
     reinterpret_cast<uint2*>(codes + (e0 >> 1))[0] = make_uint2(pack_e2m1x8<PERM>(v, 0, f), pack_e2m1x8<PERM>(v, 8, f));
-    scales[e0 >> 4] = static_cast<uint8_t>(b & 0xFFu);
+    scales[scale_offset<LOG_C>(e0 >> 4)] = static_cast<uint8_t>(b & 0xFFu);
   } else {
     static_assert(N % 32 == 0, "NVFP4 chunks above 16 elements come in pairs of blocks");
     uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of blocks 2j - 2, 2j - 1, stored with those of 2j, 2j + 1
@@ -686,7 +709,8 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
       } else {
         prev = w;
       }
-      reinterpret_cast<uint16_t*>(scales + ((e0 + 32 * j) >> 4))[0] = b;
+      // Scales 2i, 2i + 1 are neighbours in either layout (tile columns pair up).
+      reinterpret_cast<uint16_t*>(scales + scale_offset<LOG_C>((e0 + 32 * j) >> 4))[0] = b;
     }
   }
 }

@@ -305,10 +305,13 @@ __device__ __forceinline__ void tc_emit_row(float (&z)[1 << LO], int hi, int64_t
           static_cast<__half*>(out1)[(e0 + 32 * j) >> (__ffs(group) - 1)] = s16;
       }
     }
-  } else if constexpr (MODE == OUT_MXFP4) {
-    if (row_ok) store_mxfp4<false, L>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
-  } else if constexpr (MODE == OUT_NVFP4) {
-    if (row_ok) store_nvfp4<false, L>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+  } else if constexpr (MODE == OUT_MXFP4 || MODE == OUT_MXFP4_BLOCKED) {
+    // n = 2^(7 + LO): 2^(LO + 2) scales of 32 per row
+    constexpr int LOG_C = MODE == OUT_MXFP4_BLOCKED ? LO + 2 : 0;
+    if (row_ok) store_mxfp4<false, L, LOG_C>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+  } else if constexpr (MODE == OUT_NVFP4 || MODE == OUT_NVFP4_BLOCKED) {
+    constexpr int LOG_C = MODE == OUT_NVFP4_BLOCKED ? LO + 3 : 0;   // 2^(LO + 3) scales of 16 per row
+    if (row_ok) store_nvfp4<false, L, LOG_C>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
   } else if constexpr (MODE == OUT_BF16) {
     if (row_ok) store_rotated<false, L, true>(z, norm, out0, e0);
   } else {

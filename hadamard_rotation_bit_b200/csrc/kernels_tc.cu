@@ -34,6 +34,10 @@ TcVariant tc_pick(int lo, int mode) {
     case OUT_INT4: return lo == 5 ? tc_variant<C5, OUT_INT4, SIDE>() : tc_variant<C6H, OUT_INT4, SIDE>();
     case OUT_NVFP4: return lo == 5 ? tc_variant<C5, OUT_NVFP4, SIDE>() : tc_variant<C6, OUT_NVFP4, SIDE>();
     case OUT_MXFP4: return lo == 5 ? tc_variant<C5, OUT_MXFP4, SIDE>() : tc_variant<C6, OUT_MXFP4, SIDE>();
+    case OUT_MXFP4_BLOCKED:
+      return lo == 5 ? tc_variant<C5, OUT_MXFP4_BLOCKED, SIDE>() : tc_variant<C6, OUT_MXFP4_BLOCKED, SIDE>();
+    case OUT_NVFP4_BLOCKED:
+      return lo == 5 ? tc_variant<C5, OUT_NVFP4_BLOCKED, SIDE>() : tc_variant<C6, OUT_NVFP4_BLOCKED, SIDE>();
     default: return TcVariant{nullptr, 0, 0, 0};
   }
 }

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhadq.so"
 
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_F32, HADQ_BF16 = 0, 1
-FMTS = {"int4": 0, "int8": 1, "mxfp4": 2, "nvfp4": 3}
+FMTS = {"int4": 0, "int8": 1, "mxfp4": 2, "nvfp4": 3, "mxfp4_blocked": 4, "nvfp4_blocked": 5}
 HADQ_SIGNS_AFTER, HADQ_SIGNS_BEFORE = 0, 1
 SIDES = {"after": HADQ_SIGNS_AFTER, "before": HADQ_SIGNS_BEFORE}
 EXPORTS = (
@@ -211,6 +211,10 @@ def output_shapes(rows: int, n: int, fmt: str, group: int):
         return (rows, n // 2), torch.uint8, (rows, n // 32), torch.uint8
     if fmt == "nvfp4":
         return (rows, n // 2), torch.uint8, (rows, n // 16), torch.uint8
+    if fmt in ("mxfp4_blocked", "nvfp4_blocked"):
+        # the tiled GEMM scale layout: rows padded to 128, stored as 128 x 4 tiles
+        blk = 32 if fmt == "mxfp4_blocked" else 16
+        return (rows, n // 2), torch.uint8, ((rows + 127) // 128 * 128, n // blk), torch.uint8
     raise HadqError(HADQ_ERR_INVALID_ARG, f"unknown fmt {fmt!r}")
 
 

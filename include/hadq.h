@@ -71,7 +71,9 @@ typedef enum hadq_fmt {
   HADQ_INT4_SYM = 0,          /* symmetric int4 RTN per group, fp16 scales */
   HADQ_INT8_SYM = 1,          /* symmetric int8 RTN per token (row), fp32 scale */
   HADQ_MXFP4 = 2,             /* E2M1 codes, E8M0 shared exponent per 32 */
-  HADQ_NVFP4 = 3              /* E2M1 codes, FP8 E4M3 scale per 16 */
+  HADQ_NVFP4 = 3,             /* E2M1 codes, FP8 E4M3 scale per 16 */
+  HADQ_MXFP4_BLOCKED = 4,     /* HADQ_MXFP4, scales in the tiled GEMM layout */
+  HADQ_NVFP4_BLOCKED = 5      /* HADQ_NVFP4, scales in the tiled GEMM layout */
 } hadq_fmt;
 
 typedef enum hadq_sign_side {
@@ -131,6 +133,20 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  *                  s == 0 -> codes 0.
  *                  codes:  [rows x n/2] bytes, element 2i in the low nibble.
  *                  scales: [rows x n/16] E4M3 bytes.
+ *   HADQ_MXFP4_BLOCKED, HADQ_NVFP4_BLOCKED
+ *                  the same codes and scale values, the scales written in the
+ *                  layout block-scaled tensor-core GEMMs read, so the codes go
+ *                  straight into a W4A4 / MXFP4 product (the consumer after
+ *                  the rotation; reading: the "1D block scaling factors"
+ *                  layout of NVIDIA's public cuBLAS documentation).  With C
+ *                  scale columns per row (n/32 or n/16), rows padded to
+ *                  R = 128 * ceil(rows / 128): 128 x 4 tiles of 512 bytes in
+ *                  the order (row / 128, column / 4); inside a tile scale
+ *                  (r, c) at byte (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.
+ *                  scales: R x C bytes; the entries of the padding rows are
+ *                  written as 0.  Served by the tensor-core kernels: bf16
+ *                  input, full size n = 4096 or 8192 (HADQ_ERR_UNSUPPORTED
+ *                  otherwise, and under HADQ_IMPL_BUTTERFLY).
  *
  * Codes are computed from the fp32 rotation z (y = z / sqrt(b)) with the
  * stored scale s: the factor f = (1/sqrt(b)) / s is a correctly rounded fp32
@@ -303,7 +319,7 @@ HADQ_API hadq_status hadq_rotate_quant_host_static(const void* x_host, hadq_dtyp
 HADQ_API hadq_status hadq_codebook(int64_t d, int bits, double* centroids, double* thresholds);
 
 /* Bytes of the code and scale outputs of hadq_rotate_quant for these sizes
- * (0 for an invalid combination). */
+ * (0 for an invalid combination; the blocked formats count the padding rows). */
 HADQ_API int64_t hadq_codes_bytes(int64_t rows, int64_t n, hadq_fmt fmt);
 HADQ_API int64_t hadq_scales_bytes(int64_t rows, int64_t n, hadq_fmt fmt, int64_t group);
 

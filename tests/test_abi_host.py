@@ -211,7 +211,8 @@ def test_binding_checks_host_output_sizes(lib):
     binding allocates itself (output_shapes) are exactly the library's."""
     import torch
     for rows, n, fmt, group in [(5, 4096, "int4", 128), (5, 4096, "int4", 32), (3, 14336, "int8", 0),
-                                (7, 8192, "mxfp4", 32), (9, 48, "nvfp4", 16)]:
+                                (7, 8192, "mxfp4", 32), (9, 48, "nvfp4", 16), (5, 4096, "mxfp4_blocked", 32),
+                                (300, 8192, "nvfp4_blocked", 16)]:
         cs, cd, ss, sd = H.output_shapes(rows, n, fmt, group if fmt == "int4" else 32)
         codes, scales = torch.empty(cs, dtype=cd), torch.empty(ss, dtype=sd)
         assert codes.numel() * codes.element_size() == lib.hadq_codes_bytes(rows, n, H.FMTS[fmt])
@@ -275,3 +276,48 @@ def test_library_codebook_rejects_bad_arguments(lib):
     assert lib.hadq_codebook(64, 0, c.ctypes.data, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
     assert lib.hadq_codebook(64, 9, c.ctypes.data, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
     assert lib.hadq_codebook(64, 4, None, t.ctypes.data) == H.HADQ_ERR_INVALID_ARG
+
+
+def test_blocked_fp4_formats_sizes_and_checks(lib):
+    """The tiled-scale FP4 formats: scales padded to whole 128-row tiles, the
+    group rules of their base formats, whole 4-column tiles, and the
+    tensor-core path only (everything else HADQ_ERR_UNSUPPORTED, before any
+    CUDA call)."""
+    mxb, nvb = H.FMTS["mxfp4_blocked"], H.FMTS["nvfp4_blocked"]
+    assert lib.hadq_scales_bytes(5, 4096, mxb, 32) == 128 * 128
+    assert lib.hadq_scales_bytes(128, 4096, mxb, 0) == 128 * 128
+    assert lib.hadq_scales_bytes(129, 8192, nvb, 16) == 256 * 512
+    assert lib.hadq_scales_bytes(5, 4096 + 32, mxb, 32) == 0                        # 129 scale columns
+    assert lib.hadq_codes_bytes(5, 4096, mxb) == 5 * 2048
+    assert _q(lib, fmt=mxb, group=16) == H.HADQ_ERR_INVALID_ARG
+    assert _q(lib, fmt=nvb, group=32) == H.HADQ_ERR_INVALID_ARG
+    assert _q(lib, n=1056, fmt=mxb, group=32) == H.HADQ_ERR_INVALID_ARG              # 33 scale columns
+    assert _q(lib, fmt=6, group=32) == H.HADQ_ERR_INVALID_ARG                         # no such format
+    assert _q(lib, n=1024, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED               # not a tensor-core size
+    assert _q(lib, xd=0, n=4096, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED         # fp32 input
+    assert _q(lib, n=4096, block=128, fmt=nvb, group=16) == H.HADQ_ERR_UNSUPPORTED    # not the full row
+    assert lib.hadq_set_impl(1) == H.HADQ_OK                                          # butterfly kernels
+    try:
+        assert _q(lib, n=4096, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED
+    finally:
+        assert lib.hadq_set_impl(0) == H.HADQ_OK
+
+
+def test_tile_layout_map_matches_the_tiled_rearrangement():
+    """The GPU tests' index map of the tiled GEMM scale layout (offset
+    arithmetic) agrees with the layout written as a rearrangement: pad to
+    128-row x 4-column tiles, order the tiles row-block major, and inside a
+    tile put the four 32-row slabs side by side (r % 32 outermost, then the
+    slab, then the column)."""
+    from tests.test_gpu_blocked_gemm import tile_offsets
+    for rows, cols in [(128, 4), (300, 128), (5, 256), (257, 8)]:
+        pr, pc_ = (rows + 127) // 128 * 128, (cols + 3) // 4 * 4
+        m = np.zeros((pr, pc_), dtype=np.int64)
+        m[:rows, :cols] = np.arange(rows * cols).reshape(rows, cols) + 1
+        t = m.reshape(pr // 128, 128, pc_ // 4, 4).transpose(0, 2, 1, 3)          # tiles, row-block major
+        t = t.reshape(-1, 4, 32, 4).transpose(0, 2, 1, 3)                          # (slab, r % 32) -> (r % 32, slab)
+        ref = t.reshape(-1)
+        off = tile_offsets(pr, cols)
+        got = np.zeros(ref.size, dtype=np.int64)
+        got[off[:rows].reshape(-1)] = m[:rows, :cols].reshape(-1)
+        np.testing.assert_array_equal(got, ref)
