@@ -329,10 +329,14 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
 }
 
 // Block-128 rotations of bf16 rows on the tensor cores: every 128-element
-// block is a row of the MMA's A operand.  Per-token int8 takes one row per
+// chunk is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
-bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode) {
-  if (x_dtype != HADQ_BF16 || sh.kbase != 1 || sh.b != 128) return false;
+// Blocks of 256 .. 2048 (block or full size) take the same kernel with the
+// remaining stages across neighbouring lanes: unsigned, rotation outputs and
+// the grouped quantizers.
+bool tc128_eligible(hadq_dtype x_dtype, const Shape& sh, int mode, Signs sg) {
+  if (x_dtype != HADQ_BF16 || sh.kbase != 1 || sh.logb < 7 || sh.logb > 11) return false;
+  if (sh.logb > 7) return mode >= 0 && mode != hadq::OUT_CODEBOOK && sg.side == hadq::SIGNS_NONE;
   if (mode >= 0) return true;
   const int64_t bpr = sh.n >> 7;            // whole 8-row swizzle atoms per tile
   return bpr >= 32 && bpr <= 128 && bpr % 8 == 0;
@@ -357,7 +361,7 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(HADQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   }
-  const hl::Tc128Variant v = hl::tc128_kernel_for(mode);
+  const hl::Tc128Variant v = hl::tc128_kernel_for(mode, sh.logb - 7);
   if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no block-128 tensor-core kernel for this format");
   int occ = 0;
   hadq_status st = occupancy(reinterpret_cast<const void*>(v.fn), dev, v.threads, v.smem, &occ);
@@ -545,7 +549,8 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
     return launch_staged(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg, ex);
   if (g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY) {
     if (tc_eligible(x_dtype, sh, mode)) return launch_tc(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
-    if (tc128_eligible(x_dtype, sh, mode)) return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
+    if (tc128_eligible(x_dtype, sh, mode, sg))
+      return launch_tc128(x, sh, mode, group, out0, out1, stream, sms, dev, sg);
   }
   if (mode >= 0) {
     if (sh.b <= 128) {

@@ -69,7 +69,9 @@ TeamRowFn team_row_kernel_bf16(int logb, bool sg);
 // Tensor-core kernels: full size 2^(7 + lo), lo = 5 or 6; block 128 (mode -1 =
 // per-token int8).
 TcVariant tc_kernel_for(int lo, int mode, int side);   // side: hadq::SignSide
-Tc128Variant tc128_kernel_for(int mode);   // signs of either side folded into B
+// Block-128 kernel; e > 0: blocks of 2^e * 128 (1 <= e <= 4), the last e
+// stages across neighbouring lanes, no signs and no per-token int8.
+Tc128Variant tc128_kernel_for(int mode, int e);   // e = 0: signs of either side folded into B
 TcrVariant tcr_kernel_for(int mode);       // RPBH at full size 4096 (permutation gathered in shared memory)
 
 // Shared-memory staged kernels: blocks of K * 2^m elements (K a covered Paley

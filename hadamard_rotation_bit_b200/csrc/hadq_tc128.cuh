@@ -57,7 +57,13 @@ struct Tc128Cfg {
 
 // MODE: OUT_F32 / OUT_BF16 / OUT_INT4 / OUT_MXFP4 / OUT_NVFP4, or -1 for
 // per-token int8.  sg: none, or signs on either side (folded into B).
-template <class C, int MODE>
+// E > 0: blocks of b = 2^E * 128, H_b = H_(2^E) (x) H_128 over the element
+// index e = j * 128 + i.  The block's 2^E chunks j are 2^E neighbouring TMEM
+// lanes of one warp, so after the MMA the remaining E stages pair lanes by
+// shuffles (one shuffle and one fused multiply-add per value and stage); every
+// quantizer group still lies inside one chunk.  No signs and no per-token
+// int8 then (the host keeps those at b = 128).
+template <class C, int MODE, int E = 0>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
              const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
@@ -224,6 +230,17 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
+        if constexpr (E > 0) {
+          static_assert(MODE >= 0 && E <= 5, "blocks of up to 32 chunks, one warp");
+          // Chunk j = lane bits 0 .. E-1 of its block: the lower lane of each
+          // pair takes z + z', the upper z' - z.
+#pragma unroll
+          for (int d = 0; d < E; ++d) {
+            const float sgn = ((lane >> d) & 1) ? -1.f : 1.f;
+#pragma unroll
+            for (int i = 0; i < 128; ++i) z[i] = fmaf(z[i], sgn, __shfl_xor_sync(0xffffffffu, z[i], 1 << d));
+          }
+        }
         const int64_t blk = t * blocks_per_tile + m;
         const bool ok = m < blocks_per_tile && blk < blocks;
         const int64_t e0 = blk * 128;

@@ -46,15 +46,28 @@ using Tc128C = tc::Tc128Cfg<4, 2, 8>;
 
 }  // namespace
 
-Tc128Variant tc128_kernel_for(int mode) {
-  Tc128Fn fn = nullptr;
+namespace {
+template <int E>
+Tc128Fn tc128_fn(int mode) {
   switch (mode) {
-    case OUT_F32: fn = &tc::tc128_kernel<Tc128C, OUT_F32>; break;
-    case OUT_BF16: fn = &tc::tc128_kernel<Tc128C, OUT_BF16>; break;
-    case OUT_INT4: fn = &tc::tc128_kernel<Tc128C, OUT_INT4>; break;
-    case OUT_MXFP4: fn = &tc::tc128_kernel<Tc128C, OUT_MXFP4>; break;
-    case OUT_NVFP4: fn = &tc::tc128_kernel<Tc128C, OUT_NVFP4>; break;
-    case -1: fn = &tc::tc128_kernel<Tc128C, -1>; break;
+    case OUT_F32: return &tc::tc128_kernel<Tc128C, OUT_F32, E>;
+    case OUT_BF16: return &tc::tc128_kernel<Tc128C, OUT_BF16, E>;
+    case OUT_INT4: return &tc::tc128_kernel<Tc128C, OUT_INT4, E>;
+    case OUT_MXFP4: return &tc::tc128_kernel<Tc128C, OUT_MXFP4, E>;
+    case OUT_NVFP4: return &tc::tc128_kernel<Tc128C, OUT_NVFP4, E>;
+    default: return nullptr;
+  }
+}
+}  // namespace
+
+Tc128Variant tc128_kernel_for(int mode, int e) {
+  Tc128Fn fn = nullptr;
+  switch (e) {
+    case 0: fn = mode == -1 ? &tc::tc128_kernel<Tc128C, -1> : tc128_fn<0>(mode); break;
+    case 1: fn = tc128_fn<1>(mode); break;
+    case 2: fn = tc128_fn<2>(mode); break;
+    case 3: fn = tc128_fn<3>(mode); break;
+    case 4: fn = tc128_fn<4>(mode); break;
     default: break;
   }
   return Tc128Variant{fn, Tc128C::THREADS, Tc128C::SMEM_BYTES};

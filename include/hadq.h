@@ -343,7 +343,9 @@ HADQ_API int hadq_version(void);
  * the tensor-core kernels (tcgen05 MMA with H_128 for the high index bits,
  * operands staged by TMA) and the CUDA-core butterfly kernels.  The tensor-core
  * kernels cover bf16 input at full size 4096 / 8192 and at block 128 (every
- * format and sign variant), and blocks of K * 2^m with 2^m >= 128 and
+ * format and sign variant), blocks of 256 .. 2048 (block or full size; no
+ * signs, no per-token int8), RPBH at full size 4096, blocks of K * 2^m with
+ * 2^m >= 128 and
  * K * 2^m / 128 <= 128 chunks (no signs or permutation; rotation outputs, and
  * per-token int8 when the block is the whole row); every other call runs the
  * butterfly (staged) kernels whatever the choice.

@@ -222,3 +222,40 @@ def test_tc_nvfp4_configs(key):
     rng = np.random.default_rng(6)
     ids = np.unique(np.concatenate([np.arange(128), np.arange(rows - 128, rows), rng.choice(rows, 1024, replace=False)]))
     _log(f"tc-{key}", pc.check_nvfp4(W.bits_to_float64(stored[ids], "bf16"), codes[ids], scales[ids], w.block))
+
+
+# ------------------------- blocks of 256 .. 2048 on the block-128 kernel
+
+# (rows, n, block): block and full size, ragged chunk counts, tiles that loop
+BLK = [(37, 256, 0), (300, 4096, 256), (13, 512, 0), (129, 8192, 512), (5, 1024, 0), (77, 4096, 1024),
+       (3, 2048, 0), (65, 14336, 2048), (1000, 1024, 0)]
+
+
+@pytest.mark.parametrize("rows,n,block", BLK)
+def test_tc_blocks_rotate(rows, n, block):
+    stored, x64 = synth(rows, n, "bf16", seed=n + rows + block)
+    _log(f"tcb-rot-f32-{rows}x{n}-b{block}", pc.check_rotation_f32(x64, run_rotate(stored, "bf16", block, "f32"), block))
+    pc.check_rotation_bf16(x64, run_rotate(stored, "bf16", block, "bf16"), block)
+
+
+@pytest.mark.parametrize("rows,n,block", BLK)
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 128), ("mxfp4", 32), ("nvfp4", 16)])
+def test_tc_blocks_quant(rows, n, block, fmt, group):
+    stored, x64 = synth(rows, n, "bf16", seed=7 * n + rows + group + block,
+                        dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
+    codes, scales = run_quant(stored, "bf16", block, fmt, group)
+    _log(f"tcb-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, codes, scales, block, group))
+
+
+@pytest.mark.parametrize("n,block,fmt,group", [(8192, 256, "int4", 128), (1024, 0, "mxfp4", 32)])
+def test_tc_blocks_match_butterfly(n, block, fmt, group):
+    """The per-Linear shapes through both implementations: both pass the
+    oracle and agree on all but a few boundary codes."""
+    stored, x64 = synth(512, n, "bf16", seed=n + block + 1, dist="t")
+    c_tc, s_tc = run_quant(stored, "bf16", block, fmt, group)
+    H.hadq_set_impl("butterfly")
+    c_bf, s_bf = run_quant(stored, "bf16", block, fmt, group)
+    H.hadq_set_impl("tensor")
+    pc.check(fmt, x64, c_tc, s_tc, block, group)
+    pc.check(fmt, x64, c_bf, s_bf, block, group)
+    assert (c_tc != c_bf).sum() <= 32
