@@ -517,20 +517,27 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
           atomicOr(&hadq_tc_fault, kFaultSign);
           break;
         }
-        uint4* stage = reinterpret_cast<uint4*>(smem + C::SM_B + s * C::TILE_BYTES) + j;
+        // Shared-window addresses (ld/st.shared, not generic accesses).
+        const uint32_t stage = smem_u32(smem + C::SM_B + s * C::TILE_BYTES) + 16u * static_cast<uint32_t>(j);
         constexpr int kBatch = 8;              // loads in flight before the first store
 #pragma unroll
         for (int i0 = 0; i0 < kChunks; i0 += kBatch) {
           uint4 v[kBatch];
 #pragma unroll
-          for (int i = 0; i < kBatch; ++i) v[i] = stage[C::SIGN_THREADS * (i0 + i)];
+          for (int i = 0; i < kBatch; ++i)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                         : "r"(stage + 16u * C::SIGN_THREADS * (i0 + i)));
 #pragma unroll
           for (int i = 0; i < kBatch; ++i) {
             v[i].x ^= __byte_perm(q[i0 + i][0], 0u, 0x1404);
             v[i].y ^= __byte_perm(q[i0 + i][0], 0u, 0x3424);
             v[i].z ^= __byte_perm(q[i0 + i][1], 0u, 0x1404);
             v[i].w ^= __byte_perm(q[i0 + i][1], 0u, 0x3424);
-            stage[C::SIGN_THREADS * (i0 + i)] = v[i];
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                         ::"r"(stage + 16u * C::SIGN_THREADS * (i0 + i)), "r"(v[i].x), "r"(v[i].y), "r"(v[i].z),
+                           "r"(v[i].w)
+                         : "memory");
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
