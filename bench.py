@@ -67,7 +67,8 @@ SLEEP_CYCLES = 20_000_000      # ~10 ms of GPU sleep ahead of a timed region
 # launches below, in order.  c4 (R3) rotates Q to bf16 and quantizes K.
 STEP_PARTS = {"c1": ["c1"], "c2": ["c2"], "c3": ["c3"], "c4": ["c4q", "c4k"], "c5": ["c5"],
               "c2r": ["c2r"], "c2rb": ["c2rb"], "c2n": ["c2n"], "c5n": ["c5n"], "c3rb": ["c3rb"], "c5rb": ["c5rb"],
-              "c3k": ["c3k"], "c2p": ["c2p"], "c2q": ["c2q"], "pl256": ["pl256"], "pl1024": ["pl1024"]}
+              "c3k": ["c3k"], "c3km": ["c3km"], "c2p": ["c2p"], "c2q": ["c2q"], "pl256": ["pl256"],
+              "pl1024": ["pl1024"]}
 WORKLOAD = W.WORKLOADS["c2"]
 
 

@@ -411,19 +411,20 @@ hadq_status launch_tcr(const void* x, const Shape& sh, int mode, int group, void
 
 // Blocks of b = K * 128 * hi bf16 elements on the tensor cores
 // (hadq_tck.cuh): H_128 on every 128-element chunk by one MMA, the H_hi and
-// Paley H_K factors in the registers of the thread that holds one output of
-// every chunk, so K * hi <= 128.  Rotation outputs, and per-token int8 over
-// whole rows (b = n); signs, the RPBH permutation and the other quantizers
-// take the staged kernels.
+// Paley H_K factors by the thread that holds one output of every chunk
+// (through tensor memory), so K * hi <= 128.  Rotation outputs, int4, MXFP4,
+// NVFP4, and per-token int8 over whole rows (b = n); signs, the RPBH
+// permutation and the codebook take the staged kernels.
 bool tck_eligible(hadq_dtype x_dtype, const Shape& sh, int mode, Signs sg) {
   if (x_dtype != HADQ_BF16 || sh.kbase == 1 || sh.logk < 7 || sg.side != hadq::SIGNS_NONE) return false;
   if (static_cast<int64_t>(sh.kbase) << (sh.logk - 7) > 128) return false;
   if (mode < 0) return sh.b == sh.n;
-  return mode == hadq::OUT_F32 || mode == hadq::OUT_BF16;
+  return mode == hadq::OUT_F32 || mode == hadq::OUT_BF16 || mode == hadq::OUT_INT4 || mode == hadq::OUT_MXFP4 ||
+         mode == hadq::OUT_NVFP4;
 }
 
-hadq_status launch_tck(const void* x, const Shape& sh, int mode, void* out0, void* out1, cudaStream_t stream, int sms,
-                       int dev) {
+hadq_status launch_tck(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
+                       cudaStream_t stream, int sms, int dev) {
   const hl::TckVariant v = hl::tck_kernel_for(sh.kbase, 1 << (sh.logk - 7), mode);
   if (v.fn == nullptr) return fail(HADQ_ERR_UNSUPPORTED, "no K * 2^m tensor-core kernel for this size and format");
   const int64_t chunks = sh.rows * (sh.n >> 7);
@@ -450,7 +451,7 @@ hadq_status launch_tck(const void* x, const Shape& sh, int mode, void* out0, voi
   if (st != HADQ_OK) return st;
   const int64_t grid = std::min<int64_t>(blocks, sms);
   return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, maps[0], maps[1],
-                                  static_cast<const uint16_t*>(x), blocks, sh.norm, out0, out1),
+                                  static_cast<const uint16_t*>(x), blocks, sh.norm, group, out0, out1),
                        "K * 2^m tensor-core kernel launch");
 }
 
@@ -544,7 +545,7 @@ hadq_status launch(const void* x, hadq_dtype x_dtype, const Shape& sh, int mode,
                       ex.rpbh_signs, ex.thr);
   if (ex.perm == nullptr && g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY &&
       tck_eligible(x_dtype, sh, mode, sg))
-    return launch_tck(x, sh, mode, out0, out1, stream, sms, dev);
+    return launch_tck(x, sh, mode, group, out0, out1, stream, sms, dev);
   if (sh.kbase > 1 || ex.perm != nullptr || mode == hadq::OUT_CODEBOOK)
     return launch_staged(x, x_dtype, sh, mode, group, out0, out1, stream, sms, dev, sg, ex);
   if (g_impl.load(std::memory_order_relaxed) != HADQ_IMPL_BUTTERFLY) {

@@ -533,6 +533,29 @@ __device__ __forceinline__ void store_int4(const float (&v)[N], float norm, int 
   }
 }
 
+// Symmetric int4 codes of 32 consecutive outputs whose group (32, 64 or 128
+// elements, group-aligned) has the absmax mz of the unnormalised values,
+// joined by the caller; the arithmetic of store_int4.  The thread whose e0 is
+// the group's first element stores the scale.
+__device__ __forceinline__ void store_int4_piece32(const float (&v)[32], float norm, float mz, int group,
+                                                   uint8_t* __restrict__ codes, __half* __restrict__ scales,
+                                                   int64_t e0) {
+  const float m = mz * norm;
+  const __half s16 = __float2half_rn(int4_scale_f32(m));
+  const float s = __half2float(s16);
+  const float rn = (s > 0.f && s <= 65504.f) ? code_factor(norm, s) : 0.f;
+  uint4 w;
+  if (mz * rn < 7.25f) {
+    w = make_uint4(pack_int4x8<false>(v, 0, rn), pack_int4x8<false>(v, 8, rn), pack_int4x8<false>(v, 16, rn),
+                   pack_int4x8<false>(v, 24, rn));
+  } else {
+    w = make_uint4(pack_int4x8_clamped<false>(v, 0, rn), pack_int4x8_clamped<false>(v, 8, rn),
+                   pack_int4x8_clamped<false>(v, 16, rn), pack_int4x8_clamped<false>(v, 24, rn));
+  }
+  reinterpret_cast<uint4*>(codes + (e0 >> 1))[0] = w;
+  if ((e0 & (group - 1)) == 0) scales[e0 >> (__ffs(group) - 1)] = s16;
+}
+
 // Symmetric int4 with group 128 for a thread holding 64 consecutive outputs
 // (a group-aligned half when e0 % 128 == 0, the other half in lane ^ 1): the
 // group absmax is exchanged with that lane.  Every lane of the warp must call

@@ -40,7 +40,7 @@ struct Tc128Variant {
   int threads, smem;
 };
 
-using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, void*, void*);
+using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, int, void*, void*);
 using TcrFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, const int32_t*,
                        const int8_t*, const double*);
 
@@ -84,8 +84,8 @@ KsFn staged_kernel_f32(int k, int shi, int mode, int sgk);
 KsFn staged_kernel_bf16(int k, int shi, int mode, int sgk);
 
 // Tensor-core kernels for blocks of K * 128 * hi elements (K a Paley order,
-// K * hi <= 128 chunks of 128); mode OUT_F32 / OUT_BF16, or -1 = per-token
-// int8 (block = row).
+// K * hi <= 128 chunks of 128); mode OUT_F32 / OUT_BF16, -1 = per-token int8
+// (block = row), or OUT_INT4 / OUT_MXFP4 / OUT_NVFP4.
 TckVariant tck_kernel_for(int k, int hi, int mode);
 
 // The tensor-core kernels' sticky fault words (bounded waits that ran out),

@@ -49,8 +49,12 @@
 namespace hadq {
 namespace tc {
 
-template <int K_, int HI_, int STAGES_, int EPI_GROUPS_, int PREFETCH_>
+template <int K_, int HI_, int STAGES_, int EPI_GROUPS_, int PREFETCH_, bool GROUPED_ = false>
 struct TckCfg {
+  // GROUPED: the grouped quantizers (int4, MXFP4, NVFP4), which read the
+  // finished block back through a per-warp 32 x 32 transpose in shared
+  // memory (pass C) and join int4 group maxima of 64 / 128 across warps.
+  static constexpr bool GROUPED = GROUPED_;
   static constexpr int K = K_, HI = HI_, C = K * HI;   // chunks per block
   static constexpr int NP = (C + 15) / 16 * 16;         // MMA N
   static_assert(C % 4 == 0 && NP <= 128, "a thread holds one output of every chunk in registers");
@@ -68,8 +72,12 @@ struct TckCfg {
   static constexpr int SM_B = SM_A + kABytes;           // STAGES x TILE_BYTES
   static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
   static constexpr int SM_RED = SM_BARS + 8 * (2 * STAGES + 2 * ACC_BUFS);   // per-token row max
-  static constexpr int SM_SLOT = SM_RED + 4 * 4 * EPI_GROUPS;
+  static constexpr int TR_WORDS = 32 * 33;               // one warp's transpose tile (rows padded to 33 words)
+  static constexpr int SM_TR = SM_RED + 4 * 4 * EPI_GROUPS;
+  static constexpr int SM_GMAX = SM_TR + (GROUPED ? 4 * TR_WORDS * 4 * EPI_GROUPS : 0);   // [group][quarter][32]
+  static constexpr int SM_SLOT = SM_GMAX + (GROUPED ? 4 * 4 * 32 * EPI_GROUPS : 0);
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
   static_assert(PANEL_BYTES % 1024 == 0, "swizzle atoms of 8 chunks");
 };
 
@@ -239,10 +247,23 @@ __device__ __forceinline__ void tck_emit_from(uint32_t tb, float norm, float s, 
 // outputs leave from here.  Per-token int8 then joins the row absmax of the
 // group and, pass C, reads the block back and stores the codes.  Returns after
 // the last tensor-memory read of the block.
+// The grouped quantizers (int4, MXFP4, NVFP4) store the mixed values back as
+// per-token int8 does and, pass C, read them in batches of 32 positions: each
+// warp transposes its 32 lanes x 32 positions through its shared tile `tr`, so
+// that lane l holds the 32 consecutive outputs 32 quarter .. of the chunk at
+// position p0 + l -- one MXFP4 group, two NVFP4 groups, or 32 of an int4
+// group, whose absmax is joined across the group's warps through `gmax`.
+template <int MODE>
+__host__ __device__ constexpr bool tck_grouped() {
+  return MODE == OUT_INT4 || MODE == OUT_MXFP4 || MODE == OUT_NVFP4;
+}
+
 template <int K, int HI, int MODE>
 __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void* out0, void* out1, int64_t t,
-                                                  int64_t e0, int lane, int quarter, float* gred, int bar) {
+                                                  int64_t e0, int lane, int quarter, float* gred, int bar,
+                                                  float* tr, float* gmax, int group) {
   constexpr int C = K * HI, W = 4 * HI;
+  constexpr bool STORE_BACK = MODE < 0 || tck_grouped<MODE>();
   if constexpr (HI > 1) {
 #pragma unroll 1
     for (int j = 0; j < K / 4; ++j) {
@@ -283,8 +304,8 @@ __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void*
     auto get = [&](int k) { return z[k]; };
     auto put = [&](int k, float v) { z[k] = v; };
     ksize::kstage_column<K>(get, put);
-    if constexpr (MODE < 0) {
-      mz = fmaxf(mz, absmax_regs(z, 0, K));
+    if constexpr (STORE_BACK) {
+      if constexpr (MODE < 0) mz = fmaxf(mz, absmax_regs(z, 0, K));
       if constexpr (HI == 1) {
         tmem_st_cols<K>(tb, z);
       } else {
@@ -320,17 +341,54 @@ __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void*
     const float rn = (s >= 1.0e-36f && s <= 3.0e38f) ? code_factor(norm, s) : 0.f;
     tck_emit_from<HI, C, MODE, 0>(tb, norm, s, rn, tiny, out0, e0);
     if (quarter == 0 && lane == 0) static_cast<float*>(out1)[t] = s;
+  } else if constexpr (tck_grouped<MODE>()) {
+    tmem_wait_st();
+    const int64_t blk0 = t * (static_cast<int64_t>(C) * 128);
+    uint8_t* codes = static_cast<uint8_t*>(out0);
+#pragma unroll 1
+    for (int p0 = 0; p0 < C; p0 += 32) {
+      float v[32];
+      tmem_ld32(tb + p0, v);   // positions past C read unused accumulator columns and are not stored
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tr[j * 33 + lane] = v[j];
+      __syncwarp();
+      float u[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) u[k] = tr[lane * 33 + k];
+      __syncwarp();            // the tile is rewritten by the next batch
+      const int p = p0 + lane;
+      const bool ok = p < C;
+      const int64_t eo = blk0 + 128 * static_cast<int64_t>(scratch_chunk<HI>(ok ? p : 0)) + 32 * quarter;
+      if constexpr (MODE == OUT_MXFP4) {
+        if (ok) store_mxfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo);
+      } else if constexpr (MODE == OUT_NVFP4) {
+        if (ok) store_nvfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo);
+      } else {
+        float m32 = absmax_regs(u, 0, 32);
+        if (group > 32) {        // 64: this quarter and its neighbour; 128: all four
+          gmax[quarter * 32 + lane] = m32;
+          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+          m32 = group == 64 ? fmaxf(m32, gmax[(quarter ^ 1) * 32 + lane])
+                            : fmaxf(fmaxf(gmax[lane], gmax[32 + lane]), fmaxf(gmax[64 + lane], gmax[96 + lane]));
+          asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");   // gmax is rewritten by the next batch
+        }
+        if (ok) store_int4_piece32(u, norm, m32, group, codes, static_cast<__half*>(out1), eo);
+      }
+    }
   }
 }
 
-// MODE: OUT_F32 / OUT_BF16, or -1 for per-token int8 (one block = one row).
+// MODE: OUT_F32 / OUT_BF16, -1 for per-token int8 (one block = one row), or
+// a grouped quantizer (OUT_INT4 with `group`, OUT_MXFP4, OUT_NVFP4; C::GROUPED).
 template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
-           const uint16_t* __restrict__ x, int64_t blocks, float norm, void* __restrict__ out0,
+           const uint16_t* __restrict__ x, int64_t blocks, float norm, int group, void* __restrict__ out0,
            void* __restrict__ out1) {
   constexpr bool PER_TOKEN = MODE < 0;
-  static_assert(PER_TOKEN || MODE == OUT_F32 || MODE == OUT_BF16, "rotation or per-token int8");
+  static_assert(PER_TOKEN || MODE == OUT_F32 || MODE == OUT_BF16 || (tck_grouped<MODE>() && C::GROUPED),
+                "rotation, per-token int8 or a grouped quantizer with its shared tiles");
   constexpr int NC = C::C;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -444,6 +502,8 @@ tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ C
       bool failed = false;   // a wait ran out: skip the work, keep joining the group's barriers
       float* gred = red + 4 * group_id;
       const int bar = 2 + group_id;
+      float* tr = reinterpret_cast<float*>(smem + C::SM_TR) + (warp - 2) * C::TR_WORDS;   // grouped quantizers
+      float* gmax = reinterpret_cast<float*>(smem + C::SM_GMAX) + group_id * 128;
       for (int64_t t = blockIdx.x; t < blocks; t += gridDim.x, ++it) {
         if (static_cast<int>(it % C::EPI_GROUPS) != group_id) continue;
         const int b = it % C::ACC_BUFS;
@@ -456,12 +516,20 @@ tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ C
           if constexpr (PER_TOKEN) {
             asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
             asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+          } else if constexpr (MODE == OUT_INT4) {
+            if (group > 32) {
+              for (int p0 = 0; p0 < NC; p0 += 32) {
+                asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+                asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+              }
+            }
           }
           continue;
         }
         tc_fence_after();
         tck_block_scratch<C::K, C::HI, MODE>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128, norm,
-                                             out0, out1, t, t * kBlockElems + ip, lane, quarter, gred, bar);
+                                             out0, out1, t, t * kBlockElems + ip, lane, quarter, gred, bar, tr, gmax,
+                                             group);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);

@@ -21,7 +21,7 @@ constexpr int tck_groups() {
 
 template <int K, int HI, int MODE>
 TckVariant tck_variant() {
-  using C = tc::TckCfg<K, HI, 4, tck_groups<K>(), 8>;
+  using C = tc::TckCfg<K, HI, 4, tck_groups<K>(), 8, tc::tck_grouped<MODE>()>;
   return TckVariant{&tc::tck_kernel<C, MODE>, C::THREADS, C::SMEM_BYTES, C::NP};
 }
 
@@ -31,6 +31,9 @@ TckVariant tck_modes(int mode) {
     case OUT_F32: return tck_variant<K, HI, OUT_F32>();
     case OUT_BF16: return tck_variant<K, HI, OUT_BF16>();
     case -1: return tck_variant<K, HI, -1>();
+    case OUT_INT4: return tck_variant<K, HI, OUT_INT4>();
+    case OUT_MXFP4: return tck_variant<K, HI, OUT_MXFP4>();
+    case OUT_NVFP4: return tck_variant<K, HI, OUT_NVFP4>();
     default: return TckVariant{nullptr, 0, 0, 0};
   }
 }

@@ -37,10 +37,10 @@ permutation drawn from a ``seed + 1`` stream):
   on the butterfly kernels: the ``c5`` input with block 256 and int4 g128;
   131072 x 1024 bf16 ~ N(0, 1) with 1 % of the channels x50, rotated in full
   to MXFP4.
-* ``c3k``  the ``c3`` input rotated in full instead of by blocks of 128: the
-  14336-point rotation of a non-power-of-2 size ("Rotation Transform",
-  section 1.5: 14336 = 28 * 2^9, a base matrix of order 28 with a Sylvester
-  block); int8 per token.
+* ``c3k`` / ``c3km``  the ``c3`` input rotated in full instead of by blocks
+  of 128: the 14336-point rotation of a non-power-of-2 size ("Rotation
+  Transform", section 1.5: 14336 = 28 * 2^9, a base matrix of order 28 with a
+  Sylvester block); int8 per token / MXFP4.
 
 Values are drawn in float64, rounded to float32 (nearest even) and, for
 bf16 tensors, to bfloat16 (nearest even).
@@ -122,6 +122,8 @@ WORKLOADS = {
                      signs="before", base="c2"),
     "c3k": Workload("c3k", "R4 8192 tokens x intermediate 14336 bf16, full 14336-point Hadamard (K = 28 base "
                     "(x) 512-point Sylvester), int8 per token", 8192, 14336, 14336, "bf16", "int8", 0, base="c3"),
+    "c3km": Workload("c3km", "R4 8192 tokens x intermediate 14336 bf16, full 14336-point Hadamard (K = 28 base "
+                     "(x) 512-point Sylvester), MXFP4", 8192, 14336, 14336, "bf16", "mxfp4", 32, base="c3"),
     "c3rb": Workload("c3rb", "R4 8192 tokens x intermediate 14336 bf16, block 128 random Hadamard transpose "
                      "(signs before), int8 per token", 8192, 14336, 128, "bf16", "int8", 0, signs="before", base="c3"),
     "c2p": Workload("c2p", "R1 4096 tokens x hidden 4096 bf16, RPBH (random column permutation, n signs, full "

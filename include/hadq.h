@@ -346,8 +346,9 @@ HADQ_API int hadq_version(void);
  * format and sign variant), blocks of 256 .. 2048 (block or full size; no
  * signs, no per-token int8), RPBH at full size 4096, blocks of K * 2^m with
  * 2^m >= 128 and
- * K * 2^m / 128 <= 128 chunks (no signs or permutation; rotation outputs, and
- * per-token int8 when the block is the whole row); every other call runs the
+ * K * 2^m / 128 <= 128 chunks (no signs or permutation; rotation outputs,
+ * int4, MXFP4, NVFP4, and per-token int8 when the block is the whole row);
+ * every other call runs the
  * butterfly (staged) kernels whatever the choice.
  *   HADQ_IMPL_AUTO       the default: the tensor-core kernels wherever they apply
  *   HADQ_IMPL_TENSOR     the same (named for callers that want to say so)

@@ -5,9 +5,9 @@
 Each configuration runs through the C ABI at full size, in the default
 implementation choice (the launches bench.py times), and is compared element
 by element with the float64 oracle by tests/parity_check.py, the only
-checker.  The oracle sees every row of c1, c2, c3, c2r, c2rb, c3rb, c2n, c3k,
+checker.  The oracle sees every row of c1, c2, c3, c2r, c2rb, c3rb, c2n, c3k, c3km,
 c2p and c2q;
-for c4, c5, c5rb and c5n it sees a seeded row sample (first and last rows,
+for c4, c5, c5rb, c5n, pl256 and pl1024 it sees a seeded row sample (first and last rows,
 random rows and, for c5, the rows with the largest inputs), as the GPU tests
 do.  A failing comparison raises, so a written record means every compared
 element met the rule.
@@ -48,7 +48,8 @@ from hadamard_rotation_bit_b200 import workloads as W  # noqa: E402
 from tests import parity_check as pc  # noqa: E402
 
 NPROC = max(1, min(16, (os.cpu_count() or 2) // 2))
-CONFIGS = ["c1", "c2", "c3", "c4", "c5", "c2r", "c2rb", "c3rb", "c5rb", "c2n", "c5n", "c3k", "c2p", "c2q"]
+CONFIGS = ["c1", "c2", "c3", "c4", "c5", "c2r", "c2rb", "c3rb", "c5rb", "c2n", "c5n", "c3k", "c3km", "c2p", "c2q",
+           "pl256", "pl1024"]
 
 
 def _dev(stored, x_dtype):
@@ -133,7 +134,7 @@ def record(key):
         stored = W.generate(key, workers=NPROC)
         absmax = np.abs(W.bits_to_float64(stored[:, ::64], "bf16")).max(1)
         return {key: _record_part(key, _sample(w.rows, 5, absmax))}
-    if key == "c5rb":
+    if key in ("c5rb", "pl256", "pl1024"):
         return {key: _record_part(key, _sample(w.rows, 7))}
     return {key: _record_part(key)}
 

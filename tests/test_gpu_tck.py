@@ -139,3 +139,49 @@ def test_tck_involution():
     err = np.abs(back.cpu().numpy().astype(np.float64) - x64).max(axis=1) / np.linalg.norm(x64, axis=1)
     assert err.max() < 1e-6, err.max()
     assert oracle.resolve_block(52 * 256, 0) == 52 * 256
+
+
+# ------------------------------------------------ the grouped quantizers
+
+@pytest.mark.parametrize("k,hi", PAIRS)
+@pytest.mark.parametrize("fmt,group", [("int4", 32), ("int4", 64), ("int4", 128), ("mxfp4", 32), ("nvfp4", 16)])
+def test_tck_grouped_quant(k, hi, fmt, group):
+    n = k * 128 * hi
+    rows = 3 + (k * hi + group) % 6
+    stored, x64 = synth(rows, n, "bf16", seed=k * 1000 + hi * 10 + group,
+                        dist="t" if fmt in ("mxfp4", "nvfp4") else "normal")
+    codes, scales = run_quant(stored, "bf16", 0, fmt, group)
+    _log(f"tck-{fmt}{group}-{rows}x{n}", pc.check(fmt, x64, codes, scales, 0, group))
+
+
+@pytest.mark.parametrize("rows,n,block,fmt,group", [(5, 3 * 28 * 128, 28 * 128, "int4", 128),
+                                                    (3, 2 * 20 * 512, 20 * 512, "mxfp4", 32),
+                                                    (4, 5 * 12 * 128, 12 * 128, "nvfp4", 16),
+                                                    (301, 20 * 512, 0, "int4", 64),
+                                                    (149, 12 * 1024, 0, "mxfp4", 32)])
+def test_tck_grouped_blocks_and_grids(rows, n, block, fmt, group):
+    stored, x64 = synth(rows, n, "bf16", seed=rows + n + block + group)
+    codes, scales = run_quant(stored, "bf16", block, fmt, group)
+    _log(f"tck-{fmt}{group}-{rows}x{n}-b{block}", pc.check(fmt, x64, codes, scales, block, group))
+
+
+@pytest.mark.parametrize("fmt,group", [("int4", 128), ("mxfp4", 32), ("nvfp4", 16)])
+def test_tck_grouped_matches_staged(fmt, group):
+    stored, x64 = synth(64, 28 * 512, "bf16", seed=23 + group, dist="t")
+    c_tc, s_tc = run_quant(stored, "bf16", 0, fmt, group)
+    H.hadq_set_impl("butterfly")
+    c_st, s_st = run_quant(stored, "bf16", 0, fmt, group)
+    H.hadq_set_impl("tensor")
+    pc.check(fmt, x64, c_tc, s_tc, 0, group)
+    pc.check(fmt, x64, c_st, s_st, 0, group)
+    assert (c_tc != c_st).sum() <= 32
+
+
+def test_config_c3km_full_size():
+    """The bench's c3km workload: 8192 x 14336 bf16, H_28 (x) H_512, MXFP4,
+    every row checked."""
+    from hadamard_rotation_bit_b200 import workloads as W
+    w = W.WORKLOADS["c3km"]
+    stored = W.generate("c3km")
+    codes, scales = run_quant(stored, "bf16", w.block, w.fmt, w.group)
+    _log("c3km", pc.check_mxfp4(W.bits_to_float64(stored, "bf16"), codes, scales, w.block))
