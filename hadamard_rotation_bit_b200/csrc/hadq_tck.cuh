@@ -72,12 +72,13 @@ struct TckCfg {
   static constexpr int SM_B = SM_A + kABytes;           // STAGES x TILE_BYTES
   static constexpr int SM_BARS = SM_B + STAGES * TILE_BYTES;
   static constexpr int SM_RED = SM_BARS + 8 * (2 * STAGES + 2 * ACC_BUFS);   // per-token row max
-  static constexpr int TR_WORDS = 32 * 33;               // one warp's transpose tile (rows padded to 33 words)
+  static constexpr int TR_WORDS = 32 * 32;               // one warp's transpose tile (16-byte granules swizzled)
   static constexpr int SM_TR = SM_RED + 4 * 4 * EPI_GROUPS;
   static constexpr int SM_GMAX = SM_TR + (GROUPED ? 4 * TR_WORDS * 4 * EPI_GROUPS : 0);   // [group][quarter][32]
   static constexpr int SM_SLOT = SM_GMAX + (GROUPED ? 4 * 4 * 32 * EPI_GROUPS : 0);
   static constexpr int SMEM_BYTES = SM_SLOT + 16 + 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+  static_assert(SM_TR % 16 == 0, "16-byte reads of the transpose tiles");
   static_assert(PANEL_BYTES % 1024 == 0, "swizzle atoms of 8 chunks");
 };
 
@@ -350,12 +351,21 @@ __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void*
       float v[32];
       tmem_ld32(tb + p0, v);   // positions past C read unused accumulator columns and are not stored
       tmem_wait_ld();
+      // Row j of the tile holds position p0 + j; its 16-byte granules are
+      // XOR-swizzled by j % 8, so both the column writes and the row reads
+      // (8 x 16 bytes) are free of bank conflicts.
 #pragma unroll
-      for (int j = 0; j < 32; ++j) tr[j * 33 + lane] = v[j];
+      for (int j = 0; j < 32; ++j) tr[j * 32 + ((((lane >> 2) ^ j) & 7) << 2) + (lane & 3)] = v[j];
       __syncwarp();
       float u[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) u[k] = tr[lane * 33 + k];
+      for (int g = 0; g < 8; ++g) {
+        const float4 q = *reinterpret_cast<const float4*>(tr + lane * 32 + ((g ^ (lane & 7)) << 2));
+        u[4 * g] = q.x;
+        u[4 * g + 1] = q.y;
+        u[4 * g + 2] = q.z;
+        u[4 * g + 3] = q.w;
+      }
       __syncwarp();            // the tile is rewritten by the next batch
       const int p = p0 + lane;
       const bool ok = p < C;
