@@ -328,6 +328,13 @@ hadq_status launch_tc(const void* x, const Shape& sh, int mode, int group, void*
                        "tensor-core kernel launch");
 }
 
+// Scale columns per row of the tiled-scale FP4 formats (0 otherwise).
+int tiled_scale_cols(const Shape& sh, int mode) {
+  if (mode == hadq::OUT_MXFP4_BLOCKED) return static_cast<int>(sh.n / 32);
+  if (mode == hadq::OUT_NVFP4_BLOCKED) return static_cast<int>(sh.n / 16);
+  return 0;
+}
+
 // Block-128 rotations of bf16 rows on the tensor cores: every 128-element
 // chunk is a row of the MMA's A operand.  Per-token int8 takes one row per
 // tile and so needs 32 <= n / 128 <= 128 with n / 128 a multiple of 8.
@@ -369,7 +376,8 @@ hadq_status launch_tc128(const void* x, const Shape& sh, int mode, int group, vo
   const int64_t tiles = (blocks + bpt - 1) / bpt;
   const int64_t grid = std::min<int64_t>(tiles, sms);
   return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, maps[0], maps[1],
-                                  static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1, sg),
+                                  static_cast<const uint16_t*>(x), blocks, bpt, sh.norm, group, out0, out1, sg,
+                                  tiled_scale_cols(sh, mode)),
                        "tensor-core block-128 kernel launch");
 }
 
@@ -420,8 +428,9 @@ bool tck_eligible(hadq_dtype x_dtype, const Shape& sh, int mode, Signs sg) {
   if (static_cast<int64_t>(sh.kbase) << (sh.logk - 7) > 128) return false;
   if (mode < 0) return sh.b == sh.n;
   return mode == hadq::OUT_F32 || mode == hadq::OUT_BF16 || mode == hadq::OUT_INT4 || mode == hadq::OUT_MXFP4 ||
-         mode == hadq::OUT_NVFP4;
+         mode == hadq::OUT_NVFP4 || mode == hadq::OUT_MXFP4_BLOCKED || mode == hadq::OUT_NVFP4_BLOCKED;
 }
+
 
 hadq_status launch_tck(const void* x, const Shape& sh, int mode, int group, void* out0, void* out1,
                        cudaStream_t stream, int sms, int dev) {
@@ -451,7 +460,8 @@ hadq_status launch_tck(const void* x, const Shape& sh, int mode, int group, void
   if (st != HADQ_OK) return st;
   const int64_t grid = std::min<int64_t>(blocks, sms);
   return launch_result(launch_pdl(v.fn, grid, v.threads, v.smem, stream, maps[0], maps[1],
-                                  static_cast<const uint16_t*>(x), blocks, sh.norm, group, out0, out1),
+                                  static_cast<const uint16_t*>(x), blocks, sh.norm, group, out0, out1,
+                                  tiled_scale_cols(sh, mode)),
                        "K * 2^m tensor-core kernel launch");
 }
 
@@ -729,9 +739,10 @@ hadq_status rotate_quant_impl(const void* x, hadq_dtype x_dtype, int64_t rows, i
   if (blocked_fmt(fmt)) {
     // Only the tensor-core kernels write the tiled layout; the padding rows of
     // the last 128-row tile are zeroed first (the kernel writes every other entry).
+    const int qm = quant_mode(fmt);
     if (perm != nullptr || g_impl.load(std::memory_order_relaxed) == HADQ_IMPL_BUTTERFLY ||
-        !tc_eligible(x_dtype, sh, quant_mode(fmt)))
-      return fail(HADQ_ERR_UNSUPPORTED, "blocked FP4 scales: bf16 input at full size 4096 or 8192, tensor-core kernels");
+        !(tc_eligible(x_dtype, sh, qm) || tc128_eligible(x_dtype, sh, qm, sg) || tck_eligible(x_dtype, sh, qm, sg)))
+      return fail(HADQ_ERR_UNSUPPORTED, "blocked FP4 scales: bf16 input on a tensor-core shape (no RPBH)");
     if (rows % 128 != 0) {
       const int64_t cols = n / g;   // scale columns per row
       const int64_t tile_row_bytes = cols / 4 * 512;

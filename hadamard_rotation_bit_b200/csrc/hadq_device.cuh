@@ -649,11 +649,33 @@ __device__ __forceinline__ int64_t scale_offset(int64_t k) {
   }
 }
 
+// The same tiled offset for a run-time number of scale columns per row
+// (a multiple of 4): scale k = row * cols + column.  One 32-bit division per
+// call; callers use it once per thread and chunk.
+struct TiledScales {
+  int64_t r;   // row of the first scale of the chunk
+  int c;       // its column
+  int cols;    // scale columns per row
+  __device__ __forceinline__ TiledScales(int64_t k, int cols_) : cols(cols_) {
+    // k < 2^32: a scale per 16 elements or more, and fewer than 2^36 elements
+    // of 2 bytes or more fit any device memory
+    const uint32_t q = static_cast<uint32_t>(k) / static_cast<uint32_t>(cols_);
+    r = q;
+    c = static_cast<int>(static_cast<uint32_t>(k) - q * static_cast<uint32_t>(cols_));
+  }
+  // Offset of scale k + j, j small enough to stay in the row.
+  __device__ __forceinline__ int64_t operator()(int j) const {
+    const int cj = c + j;
+    return ((r >> 7) * (cols >> 2) + (cj >> 2)) * 512 + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (cj & 3);
+  }
+};
+
 // MXFP4: per 32 elements an E8M0 exponent e = clamp(floor(log2 m) - 2, -127, 127).
-// LOG_C: the scale layout (scale_offset).
+// LOG_C: the scale layout (scale_offset); tiled_cols > 0: the tiled layout
+// with that many scale columns per row (TiledScales).
 template <bool PERM, int N, int LOG_C = 0>
 __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uint8_t* __restrict__ codes,
-                                            uint8_t* __restrict__ scales, int64_t e0) {
+                                            uint8_t* __restrict__ scales, int64_t e0, int tiled_cols = 0) {
   static_assert(N % 32 == 0, "MX groups are 32 elements");
   uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of sub-block j - 1, stored with those of j
 #pragma unroll
@@ -677,7 +699,8 @@ __device__ __forceinline__ void store_mxfp4(const float (&v)[N], float norm, uin
     } else {
       prev = w;
     }
-    scales[scale_offset<LOG_C>((e0 >> 5) + j)] = static_cast<uint8_t>(byte);
+    if (tiled_cols > 0) scales[TiledScales(e0 >> 5, tiled_cols)(j)] = static_cast<uint8_t>(byte);
+    else scales[scale_offset<LOG_C>((e0 >> 5) + j)] = static_cast<uint8_t>(byte);
   }
 }
 
@@ -703,7 +726,7 @@ __device__ __forceinline__ float2 e4m3x2_values(uint16_t b) {
 // store 16 code bytes and 2 scale bytes at once.
 template <bool PERM, int N, int LOG_C = 0>
 __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8_t* __restrict__ codes,
-                                            uint8_t* __restrict__ scales, int64_t e0) {
+                                            uint8_t* __restrict__ scales, int64_t e0, int tiled_cols = 0) {
   static_assert(N % 16 == 0, "NVFP4 blocks are 16 elements");
   if constexpr (N == 16) {
     const float m = absmax_regs(v, 0, 16) * nq;
@@ -711,7 +734,8 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
     const float s = e4m3x2_values(b).x;
     const float f = s > 0.f ? code_factor(nq, s) : 0.f;
     reinterpret_cast<uint2*>(codes + (e0 >> 1))[0] = make_uint2(pack_e2m1x8<PERM>(v, 0, f), pack_e2m1x8<PERM>(v, 8, f));
-    scales[scale_offset<LOG_C>(e0 >> 4)] = static_cast<uint8_t>(b & 0xFFu);
+    if (tiled_cols > 0) scales[TiledScales(e0 >> 4, tiled_cols)(0)] = static_cast<uint8_t>(b & 0xFFu);
+    else scales[scale_offset<LOG_C>(e0 >> 4)] = static_cast<uint8_t>(b & 0xFFu);
   } else {
     static_assert(N % 32 == 0, "NVFP4 chunks above 16 elements come in pairs of blocks");
     uint4 prev = make_uint4(0u, 0u, 0u, 0u);   // codes of blocks 2j - 2, 2j - 1, stored with those of 2j, 2j + 1
@@ -733,7 +757,9 @@ __device__ __forceinline__ void store_nvfp4(const float (&v)[N], float nq, uint8
         prev = w;
       }
       // Scales 2i, 2i + 1 are neighbours in either layout (tile columns pair up).
-      reinterpret_cast<uint16_t*>(scales + scale_offset<LOG_C>((e0 + 32 * j) >> 4))[0] = b;
+      const int64_t off = tiled_cols > 0 ? TiledScales(e0 >> 4, tiled_cols)(2 * j)
+                                         : scale_offset<LOG_C>((e0 + 32 * j) >> 4);
+      reinterpret_cast<uint16_t*>(scales + off)[0] = b;
     }
   }
 }

@@ -22,7 +22,7 @@ using TeamFn = void (*)(const void*, int64_t, float, int, void*, void*, Signs);
 using TeamRowFn = void (*)(const void*, int64_t, int64_t, float, int8_t*, float*, Signs);
 using TcFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, Signs);
 using Tc128Fn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*,
-                         Signs);
+                         Signs, int);
 }  // namespace launch
 namespace ksize {
 struct StageArgs;
@@ -40,7 +40,7 @@ struct Tc128Variant {
   int threads, smem;
 };
 
-using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, int, void*, void*);
+using TckFn = void (*)(const CUtensorMap, const CUtensorMap, const uint16_t*, int64_t, float, int, void*, void*, int);
 using TcrFn = void (*)(const CUtensorMap, const uint16_t*, int64_t, int, float, int, void*, void*, const int32_t*,
                        const int8_t*, const double*);
 

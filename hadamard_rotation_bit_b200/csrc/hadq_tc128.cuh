@@ -67,7 +67,7 @@ template <class C, int MODE, int E = 0>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
              const uint16_t* __restrict__ x, int64_t blocks, int blocks_per_tile, float norm, int group,
-             void* __restrict__ out0, void* __restrict__ out1, Signs sg) {
+             void* __restrict__ out0, void* __restrict__ out1, Signs sg, int scale_cols) {
   constexpr bool PER_TOKEN = MODE < 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -257,10 +257,15 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
           if (m == 0) static_cast<float*>(out1)[t] = int8_scale(mrow);
         } else if constexpr (MODE == OUT_INT4) {
           if (ok) store_int4<false, 128>(z, norm, group, static_cast<uint8_t*>(out0), static_cast<__half*>(out1), e0);
-        } else if constexpr (MODE == OUT_MXFP4) {
-          if (ok) store_mxfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
-        } else if constexpr (MODE == OUT_NVFP4) {
-          if (ok) store_nvfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0);
+        } else if constexpr (MODE == OUT_MXFP4 || MODE == OUT_MXFP4_BLOCKED) {
+          // the tiled GEMM scale layout: scale_cols = n / 32 columns per row
+          if (ok)
+            store_mxfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0,
+                                    MODE == OUT_MXFP4_BLOCKED ? scale_cols : 0);
+        } else if constexpr (MODE == OUT_NVFP4 || MODE == OUT_NVFP4_BLOCKED) {
+          if (ok)
+            store_nvfp4<false, 128>(z, norm, static_cast<uint8_t*>(out0), static_cast<uint8_t*>(out1), e0,
+                                    MODE == OUT_NVFP4_BLOCKED ? scale_cols : 0);
         } else if constexpr (MODE == OUT_BF16) {
           if (ok) store_rotated<false, 128, true>(z, norm, out0, e0);
         } else {

@@ -256,13 +256,14 @@ __device__ __forceinline__ void tck_emit_from(uint32_t tb, float norm, float s, 
 // group, whose absmax is joined across the group's warps through `gmax`.
 template <int MODE>
 __host__ __device__ constexpr bool tck_grouped() {
-  return MODE == OUT_INT4 || MODE == OUT_MXFP4 || MODE == OUT_NVFP4;
+  return MODE == OUT_INT4 || MODE == OUT_MXFP4 || MODE == OUT_NVFP4 || MODE == OUT_MXFP4_BLOCKED ||
+         MODE == OUT_NVFP4_BLOCKED;
 }
 
 template <int K, int HI, int MODE>
 __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void* out0, void* out1, int64_t t,
                                                   int64_t e0, int lane, int quarter, float* gred, int bar,
-                                                  float* tr, float* gmax, int group) {
+                                                  float* tr, float* gmax, int group, int scale_cols) {
   constexpr int C = K * HI, W = 4 * HI;
   constexpr bool STORE_BACK = MODE < 0 || tck_grouped<MODE>();
   if constexpr (HI > 1) {
@@ -370,10 +371,14 @@ __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void*
       const int p = p0 + lane;
       const bool ok = p < C;
       const int64_t eo = blk0 + 128 * static_cast<int64_t>(scratch_chunk<HI>(ok ? p : 0)) + 32 * quarter;
-      if constexpr (MODE == OUT_MXFP4) {
-        if (ok) store_mxfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo);
-      } else if constexpr (MODE == OUT_NVFP4) {
-        if (ok) store_nvfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo);
+      if constexpr (MODE == OUT_MXFP4 || MODE == OUT_MXFP4_BLOCKED) {
+        if (ok)
+          store_mxfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo,
+                                 MODE == OUT_MXFP4_BLOCKED ? scale_cols : 0);
+      } else if constexpr (MODE == OUT_NVFP4 || MODE == OUT_NVFP4_BLOCKED) {
+        if (ok)
+          store_nvfp4<false, 32>(u, norm, codes, static_cast<uint8_t*>(out1), eo,
+                                 MODE == OUT_NVFP4_BLOCKED ? scale_cols : 0);
       } else {
         float m32 = absmax_regs(u, 0, 32);
         if (group > 32) {        // 64: this quarter and its neighbour; 128: all four
@@ -390,12 +395,13 @@ __device__ __forceinline__ void tck_block_scratch(uint32_t tb, float norm, void*
 }
 
 // MODE: OUT_F32 / OUT_BF16, -1 for per-token int8 (one block = one row), or
-// a grouped quantizer (OUT_INT4 with `group`, OUT_MXFP4, OUT_NVFP4; C::GROUPED).
+// a grouped quantizer (OUT_INT4 with `group`, OUT_MXFP4, OUT_NVFP4 and their
+// tiled-scale forms with scale_cols scale columns per row; C::GROUPED).
 template <class C, int MODE>
 __global__ void __launch_bounds__(C::THREADS, 1)
 tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ CUtensorMap map_p1,
            const uint16_t* __restrict__ x, int64_t blocks, float norm, int group, void* __restrict__ out0,
-           void* __restrict__ out1) {
+           void* __restrict__ out1, int scale_cols) {
   constexpr bool PER_TOKEN = MODE < 0;
   static_assert(PER_TOKEN || MODE == OUT_F32 || MODE == OUT_BF16 || (tck_grouped<MODE>() && C::GROUPED),
                 "rotation, per-token int8 or a grouped quantizer with its shared tiles");
@@ -539,7 +545,7 @@ tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ C
         tc_fence_after();
         tck_block_scratch<C::K, C::HI, MODE>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128, norm,
                                              out0, out1, t, t * kBlockElems + ip, lane, quarter, gred, bar, tr, gmax,
-                                             group);
+                                             group, scale_cols);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);

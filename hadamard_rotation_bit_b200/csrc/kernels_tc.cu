@@ -55,6 +55,8 @@ Tc128Fn tc128_fn(int mode) {
     case OUT_INT4: return &tc::tc128_kernel<Tc128C, OUT_INT4, E>;
     case OUT_MXFP4: return &tc::tc128_kernel<Tc128C, OUT_MXFP4, E>;
     case OUT_NVFP4: return &tc::tc128_kernel<Tc128C, OUT_NVFP4, E>;
+    case OUT_MXFP4_BLOCKED: return &tc::tc128_kernel<Tc128C, OUT_MXFP4_BLOCKED, E>;
+    case OUT_NVFP4_BLOCKED: return &tc::tc128_kernel<Tc128C, OUT_NVFP4_BLOCKED, E>;
     default: return nullptr;
   }
 }

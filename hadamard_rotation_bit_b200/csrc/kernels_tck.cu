@@ -34,6 +34,8 @@ TckVariant tck_modes(int mode) {
     case OUT_INT4: return tck_variant<K, HI, OUT_INT4>();
     case OUT_MXFP4: return tck_variant<K, HI, OUT_MXFP4>();
     case OUT_NVFP4: return tck_variant<K, HI, OUT_NVFP4>();
+    case OUT_MXFP4_BLOCKED: return tck_variant<K, HI, OUT_MXFP4_BLOCKED>();
+    case OUT_NVFP4_BLOCKED: return tck_variant<K, HI, OUT_NVFP4_BLOCKED>();
     default: return TckVariant{nullptr, 0, 0, 0};
   }
 }

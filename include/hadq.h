@@ -145,8 +145,10 @@ HADQ_API hadq_status hadq_rotate_inverse(const void* x, hadq_dtype x_dtype, int6
  *                  (r, c) at byte (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.
  *                  scales: R x C bytes; the entries of the padding rows are
  *                  written as 0.  Served by the tensor-core kernels: bf16
- *                  input, full size n = 4096 or 8192 (HADQ_ERR_UNSUPPORTED
- *                  otherwise, and under HADQ_IMPL_BUTTERFLY).
+ *                  input at full size 4096 or 8192, blocks of 128 .. 2048
+ *                  (unsigned above 128), and blocks of K * 2^m with
+ *                  2^m >= 128 (unsigned); HADQ_ERR_UNSUPPORTED otherwise,
+ *                  with RPBH, and under HADQ_IMPL_BUTTERFLY.
  *
  * Codes are computed from the fp32 rotation z (y = z / sqrt(b)) with the
  * stored scale s: the factor f = (1/sqrt(b)) / s is a correctly rounded fp32

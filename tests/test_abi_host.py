@@ -281,7 +281,7 @@ def test_library_codebook_rejects_bad_arguments(lib):
 def test_blocked_fp4_formats_sizes_and_checks(lib):
     """The tiled-scale FP4 formats: scales padded to whole 128-row tiles, the
     group rules of their base formats, whole 4-column tiles, and the
-    tensor-core path only (everything else HADQ_ERR_UNSUPPORTED, before any
+    tensor-core shapes only (everything else HADQ_ERR_UNSUPPORTED, before any
     CUDA call)."""
     mxb, nvb = H.FMTS["mxfp4_blocked"], H.FMTS["nvfp4_blocked"]
     assert lib.hadq_scales_bytes(5, 4096, mxb, 32) == 128 * 128
@@ -293,9 +293,9 @@ def test_blocked_fp4_formats_sizes_and_checks(lib):
     assert _q(lib, fmt=nvb, group=32) == H.HADQ_ERR_INVALID_ARG
     assert _q(lib, n=1056, fmt=mxb, group=32) == H.HADQ_ERR_INVALID_ARG              # 33 scale columns
     assert _q(lib, fmt=6, group=32) == H.HADQ_ERR_INVALID_ARG                         # no such format
-    assert _q(lib, n=1024, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED               # not a tensor-core size
+    assert _q(lib, n=1024, block=64, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED     # not a tensor-core size
     assert _q(lib, xd=0, n=4096, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED         # fp32 input
-    assert _q(lib, n=4096, block=128, fmt=nvb, group=16) == H.HADQ_ERR_UNSUPPORTED    # not the full row
+    assert _q(lib, xd=0, n=4096, block=128, fmt=nvb, group=16) == H.HADQ_ERR_UNSUPPORTED   # fp32 blocks
     assert lib.hadq_set_impl(1) == H.HADQ_OK                                          # butterfly kernels
     try:
         assert _q(lib, n=4096, fmt=mxb, group=32) == H.HADQ_ERR_UNSUPPORTED

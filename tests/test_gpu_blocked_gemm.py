@@ -64,12 +64,16 @@ def decode_fp4(codes_packed: np.ndarray, scales: np.ndarray, fmt: str) -> np.nda
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
-@pytest.mark.parametrize("rows,n", [(256, 4096), (300, 4096), (5, 8192), (129, 8192)])
-def test_blocked_scales_match_row_major(fmt, rows, n):
-    stored, x64 = synth(rows, n, "bf16", seed=rows + n, dist="t")
+@pytest.mark.parametrize("rows,n,block", [(256, 4096, 0), (300, 4096, 0), (5, 8192, 0), (129, 8192, 0),
+                                          (300, 14336, 128), (129, 8192, 256), (37, 2048, 0), (130, 14336, 0),
+                                          (5, 28 * 256, 0)])
+def test_blocked_scales_match_row_major(fmt, rows, n, block):
+    """Every tensor-core shape: full 4096 / 8192, blocks of 128 .. 2048, K * 2^m
+    (14336 = 28 * 512, 7168 = 28 * 256)."""
+    stored, x64 = synth(rows, n, "bf16", seed=rows + n + block, dist="t")
     x = to_dev(stored, "bf16")
-    c_rm, s_rm = H.hadq_rotate_quant(x, 0, fmt, 32 if fmt == "mxfp4" else 16)
-    c_bl, s_bl = H.hadq_rotate_quant(x, 0, fmt + "_blocked", 32 if fmt == "mxfp4" else 16)
+    c_rm, s_rm = H.hadq_rotate_quant(x, block, fmt, 32 if fmt == "mxfp4" else 16)
+    c_bl, s_bl = H.hadq_rotate_quant(x, block, fmt + "_blocked", 32 if fmt == "mxfp4" else 16)
     torch.cuda.synchronize()
     cols = n // (32 if fmt == "mxfp4" else 16)
     assert s_bl.shape == ((rows + 127) // 128 * 128, cols)
@@ -79,8 +83,8 @@ def test_blocked_scales_match_row_major(fmt, rows, n):
     pad = np.ones(flat.size, dtype=bool)
     pad[tile_offsets((rows + 127) // 128 * 128, cols)[:rows].reshape(-1)] = False
     assert not flat[pad].any(), "padding rows are zero"
-    _log(f"blocked-{fmt}-{rows}x{n}", pc.check(fmt, x64, c_bl.cpu().numpy(), unblock(flat, rows, cols), 0,
-                                                32 if fmt == "mxfp4" else 16))
+    _log(f"blocked-{fmt}-{rows}x{n}-b{block}", pc.check(fmt, x64, c_bl.cpu().numpy(), unblock(flat, rows, cols), block,
+                                                         32 if fmt == "mxfp4" else 16))
 
 
 def _scaled_mm(a_codes, a_scales, w_codes, w_scales, fmt, k):
@@ -97,17 +101,19 @@ def _scaled_mm(a_codes, a_scales, w_codes, w_scales, fmt, k):
     return F.scaled_mm(a, b, sa, recipe, sb, recipe, sw, sw, output_dtype=torch.bfloat16)
 
 
-@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
-def test_w4a4_gemm_on_blocked_outputs(fmt):
-    """x (256 x 4096 bf16, outlier channels) and W (512 x 4096 bf16) rotated
-    and quantized by the library; their codes and tiled scales go straight
-    into a block-scaled GEMM."""
-    m, nw, k = 256, 512, 4096
+@pytest.mark.parametrize("fmt,k,block", [("mxfp4", 4096, 0), ("nvfp4", 4096, 0), ("mxfp4", 14336, 128),
+                                         ("mxfp4", 14336, 0)])
+def test_w4a4_gemm_on_blocked_outputs(fmt, k, block):
+    """x (256 x K bf16, outlier channels) and W (512 x K bf16) rotated and
+    quantized by the library (R1 at K = 4096; the down_proj input at
+    K = 14336, by blocks of 128 or in full); their codes and tiled scales go
+    straight into a block-scaled GEMM."""
+    m, nw = 256, 512
     blk = 32 if fmt == "mxfp4" else 16
     xs, x64 = synth(m, k, "bf16", seed=41)
     ws, w64 = synth(nw, k, "bf16", seed=42, outliers=False)
-    cx, sx = H.hadq_rotate_quant(to_dev(xs, "bf16"), 0, fmt + "_blocked", blk)
-    cw, sw = H.hadq_rotate_quant(to_dev(ws, "bf16"), 0, fmt + "_blocked", blk)
+    cx, sx = H.hadq_rotate_quant(to_dev(xs, "bf16"), block, fmt + "_blocked", blk)
+    cw, sw = H.hadq_rotate_quant(to_dev(ws, "bf16"), block, fmt + "_blocked", blk)
     torch.cuda.synchronize()
     try:
         y = _scaled_mm(cx, sx, cw, sw, fmt, k)
@@ -122,14 +128,14 @@ def test_w4a4_gemm_on_blocked_outputs(fmt):
     bound = 1e-2 * np.abs(ref) + 1e-4 * (np.abs(a) @ np.abs(w).T)   # bf16 output, fp32 accumulation
     assert (np.abs(y - ref) <= bound).all(), float((np.abs(y - ref) / bound).max())
     # the library's codes are the oracle's (boundary cases aside)
-    pc.check(fmt, x64, cx.cpu().numpy(), unblock(sx.cpu().numpy(), m, k // blk), 0, blk)
+    pc.check(fmt, x64, cx.cpu().numpy(), unblock(sx.cpu().numpy(), m, k // blk), block, blk)
     # the W4A4 product approximates x W^T, better with the rotation than without
     exact = x64 @ w64.T
     err_rot = np.linalg.norm(y - exact) / np.linalg.norm(exact)
     _, cxn, sxn = oracle.quantize(x64, fmt, blk)
     _, cwn, swn = oracle.quantize(w64, fmt, blk)
     err_plain = np.linalg.norm(decode_fp4(cxn, sxn, fmt) @ decode_fp4(cwn, swn, fmt).T - exact) / np.linalg.norm(exact)
-    _log(f"w4a4-{fmt}", {"rel_err_rotated": err_rot, "rel_err_unrotated": err_plain})
+    _log(f"w4a4-{fmt}-k{k}-b{block}", {"rel_err_rotated": err_rot, "rel_err_unrotated": err_plain})
     assert err_rot < 0.2, err_rot
     if fmt == "mxfp4":
         # one power-of-2 scale per 32 elements: outlier channels cost the other
