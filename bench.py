@@ -361,6 +361,39 @@ def _device_input(key, seed, dev, workers, rows=None):
     return stored, torch.from_numpy(stored).to(dev)
 
 
+def _two_stream_interval(step, steps, warm, stream, side, dev, dist):
+    """Max-over-ranks seconds of K steps alternating between two streams."""
+    s1 = torch.cuda.Stream(device=dev)
+    t2_start = torch.cuda.Event(enable_timing=True, external=True)
+    t2_end = torch.cuda.Event(enable_timing=True, external=True)
+    ev_fork2 = torch.cuda.Event()
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        for i in range(warm):
+            step(steps + i)
+        ev_fork2.record(stream)
+        side.wait_event(ev_fork2)
+        t2_start.record(side)
+        s1.wait_event(ev_fork2)
+        for i in range(steps):
+            step(i, stream if i % 2 == 0 else s1)
+        stream.wait_stream(s1)
+        stream.wait_stream(side)
+        t2_end.record(stream)
+    with torch.cuda.stream(stream):
+        g2.replay()
+    stream.synchronize()
+    barrier(dist)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(SLEEP_CYCLES)
+        g2.replay()
+    stream.synchronize()
+    barrier(dist)
+    elapsed = max_over_ranks(dist, t2_start.elapsed_time(t2_end) / 1e3)
+    del g2
+    return elapsed
+
+
 def run_hadq(args):
     from hadamard_rotation_bit_b200 import hadq as H
     dist, rank, world, local = dist_setup()
@@ -413,9 +446,9 @@ def run_hadq(args):
     bytes_step = step_bytes(cfg, args.rows)
     stream = torch.cuda.Stream(device=dev)
 
-    def step(i):
+    def step(i, st=None):
         for j in range(len(keys)):
-            launch(j, i, stream, outs)
+            launch(j, i, stream if st is None else st, outs)
 
     with torch.cuda.stream(stream):
         for i in range(warm):
@@ -481,6 +514,16 @@ def run_hadq(args):
     stream.synchronize()
     barrier(dist)
     host_submit_max = max_over_ranks(dist, h_start.elapsed_time(h_end) / 1e3)
+
+    # Diagnostic: the same K steps with consecutive steps on two streams.  The
+    # steps are independent batches, so a step need not wait for the one
+    # before it on the other stream, and its CTAs start as the other step's
+    # CTAs leave; each stream's steps keep their programmatic launch on the
+    # step before them on that stream.  Events and warm-up as in the timed graph.
+    # Consecutive steps write different buffer sets only when there are two.
+    two_streams = None
+    if nbuf >= 2:
+        two_streams = _two_stream_interval(step, steps, warm, stream, side, dev, dist)
 
     # Diagnostic: an event pair around each step, all queued behind a sleep
     # kernel so the steps run back to back without host gaps.
@@ -580,7 +623,10 @@ def run_hadq(args):
                                      "warm-up step's completion, end at the K-th step's)",
                          "step_interval_us": interval_max * 1e6,
                          "step_interval_us_host_submit": host_submit_max / steps * 1e6,
-                         "step_us_event_pairs_median": step_ev * 1e6},
+                         "step_us_event_pairs_median": step_ev * 1e6,
+                         "two_streams": None if two_streams is None else
+                         {"step_interval_us": two_streams / steps * 1e6,
+                          "frac": bytes_step / (two_streams / steps) / 1e9 / peak}},
             "e2e": e2e,
             "gpu_launches": steps * len(keys),
             "clocks": clocks.summary(),

@@ -105,6 +105,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory rounded up to a 1024-byte boundary (what the
+// 128-byte swizzle atoms need), as an offset from the __shared__ array
+// itself: the compiler then still knows every pointer derived from it to be
+// shared memory and emits shared loads and stores (an integer round trip
+// through uintptr_t would leave generic accesses, which take the longer
+// global-memory path through the load/store unit).
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
@@ -334,7 +344,7 @@ tc_rotate_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __res
   constexpr int T = tc_threads<C, SIDE>();
   constexpr int kFirstSignWarp = 2 + 4 * C::SPLIT;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;

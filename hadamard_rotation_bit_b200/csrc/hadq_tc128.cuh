@@ -70,7 +70,7 @@ tc128_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__
              void* __restrict__ out0, void* __restrict__ out1, Signs sg, int scale_cols) {
   constexpr bool PER_TOKEN = MODE < 0;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;

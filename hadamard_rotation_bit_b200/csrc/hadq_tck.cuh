@@ -407,7 +407,7 @@ tck_kernel(const __grid_constant__ CUtensorMap map_p0, const __grid_constant__ C
                 "rotation, per-token int8 or a grouped quantizer with its shared tiles");
   constexpr int NC = C::C;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;

@@ -161,7 +161,7 @@ tc_rpbh_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restr
   using C = TcrCfg;
   constexpr int LO = C::LO, L = C::L, R = C::R;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);   // raw tile landed
   uint64_t* empty = full + C::RAW_STAGES;                           // raw stage read by the gather
   uint64_t* gathered = empty + C::RAW_STAGES;                       // permuted stage written
