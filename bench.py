@@ -21,8 +21,9 @@ host's submission or the graph's launch latency.  `value` = bytes of all ranks /
 `roofline.achieved` = bytes per launch / mean launch interval (kernel plus
 inter-kernel gap).  Beside it the line reports a K-step replay with host-side
 events recorded while the host submits the graph (the window then also holds
-the submission and graph-launch latency) and a median over per-launch event
-pairs.
+the submission and graph-launch latency), a median over per-launch event
+pairs, and (`roofline.two_streams`) the same K steps with consecutive steps
+on two streams, as independent batches can be scheduled.
 `e2e` repeats the metric through hadq_rotate_quant_host (pinned host input,
 copies in and out inside the timed region).
 
