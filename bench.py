@@ -119,8 +119,11 @@ def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
-    except (OSError, KeyError, ValueError):
+            v = json.load(f)["hbm_gbs"]
+        if isinstance(v, dict):            # {"value": ...} form
+            v = v.get("value", v.get("gbs"))
+        return float(v), "measured"
+    except (OSError, KeyError, ValueError, TypeError):
         return FALLBACK_HBM_GBS, "fallback"
 
 
